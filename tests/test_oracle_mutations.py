@@ -1,0 +1,176 @@
+"""Plant plausible mistakes in a private copy of the CPU oracle and check that
+at least one pin fails for each.  Shows the pins are strong enough to catch
+a dropped term, a wrong sign or index, a transposed operand, a reversed tie
+rule, a missing bias or mask, or a wrong head-to-group mapping.  CPU only;
+the real oracle module is never modified."""
+import importlib.util
+import math
+import os
+
+import pytest
+import torch
+
+from tests import oracle_pins as P
+
+ORACLE_SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                          "oracle", "msa_oracle.py")
+
+
+def fresh_oracle(tag):
+    spec = importlib.util.spec_from_file_location(f"_oracle_copy_{tag}", ORACLE_SRC)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _mut_causal_off_by_one(o):
+    orig = o.pooled_scores
+
+    def pooled_scores(q, k, pos, block, n_blocks):
+        out = orig(q, k, max(pos - 1, 0), block, n_blocks)
+        return out
+    o.pooled_scores = pooled_scores
+
+
+def _mut_no_causal_mask(o):
+    def pooled_scores(q, k, pos, block, n_blocks):
+        s = o.token_scores(q, k)
+        out = torch.full((n_blocks,), float("-inf"), dtype=torch.float64)
+        for b in range(o.n_visible_blocks(pos, block)):
+            out[b] = s[b * block:(b + 1) * block].max()
+        return out
+    o.pooled_scores = pooled_scores
+
+
+def _mut_tie_higher_index(o):
+    def ranked_blocks(row, pos, block):
+        nvis = o.n_visible_blocks(pos, block)
+        return sorted(range(nvis), key=lambda b: (-float(row[b]), -b))
+    o.ranked_blocks = ranked_blocks
+
+
+def _mut_no_bias(o):
+    o.LOCAL_BIAS = 0.0
+
+    orig = o.block_scores
+
+    def block_scores(idx_q, idx_k, qs, qp, block, local_bias=0.0):
+        return orig(idx_q, idx_k, qs, qp, block, 0.0)
+    o.block_scores = block_scores
+
+
+def _mut_gqa_modulo(o):
+    def sparse_attention(q, k_cache, v_cache, sel, q_stream, q_pos, block, scale=None, queries=None):
+        n_q, Hq, D = q.shape
+        G = k_cache.shape[1]
+        scale = 1.0 / math.sqrt(D) if scale is None else scale
+        out = torch.empty((n_q, Hq, D), dtype=torch.float64)
+        for i in range(n_q):
+            s, p = int(q_stream[i]), int(q_pos[i])
+            for h in range(Hq):
+                g = h % G
+                rows = torch.tensor(o.attended_rows(sel[i, g].tolist(), p, block))
+                K = k_cache[s, g, rows].double()
+                V = v_cache[s, g, rows].double()
+                w = torch.softmax(K @ q[i, h].double() * scale, 0)
+                out[i, h] = w @ V
+        return out
+    o.sparse_attention = sparse_attention
+
+
+def _mut_no_scale(o):
+    orig = o.sparse_attention
+
+    def sparse_attention(q, k, v, sel, qs, qp, block, scale=None, queries=None):
+        return orig(q, k, v, sel, qs, qp, block, 1.0, queries)
+    o.sparse_attention = sparse_attention
+
+
+def _mut_nvis_off_by_one(o):
+    o.n_visible_blocks = lambda pos, block: max(pos // block, 1)
+
+
+def _mut_transposed_scores(o):
+    def token_scores(q, rows):
+        rows = rows.double()
+        # uses the key's coordinates in reverse order
+        return rows.flip(-1) @ q.double()
+    o.token_scores = token_scores
+
+
+def _mut_dropped_term(o):
+    def token_scores(q, rows):
+        return rows.double()[:, :-1] @ q.double()[:-1]
+    o.token_scores = token_scores
+
+
+def _mut_future_rows(o):
+    def attended_rows(sel_ids, pos, block):
+        rows = []
+        for b in sel_ids:
+            if int(b) >= 0:
+                rows.extend(range(int(b) * block, (int(b) + 1) * block))
+        return rows
+    o.attended_rows = attended_rows
+
+
+def _mut_sign(o):
+    orig = o.sparse_attention
+
+    def sparse_attention(q, k, v, sel, qs, qp, block, scale=None, queries=None):
+        D = q.shape[-1]
+        return orig(q, k, v, sel, qs, qp, block, -1.0 / math.sqrt(D), queries)
+    o.sparse_attention = sparse_attention
+
+
+def _mut_k_minus_one(o):
+    def select_one(row, pos, block, top_k):
+        return sorted(o.ranked_blocks(row, pos, block)[:max(top_k - 1, 1)])
+    o.select_one = select_one
+
+
+def _mut_unsorted_ids(o):
+    def select_one(row, pos, block, top_k):
+        return o.ranked_blocks(row, pos, block)[:top_k]
+    o.select_one = select_one
+
+
+def _mut_lowest_scores(o):
+    def ranked_blocks(row, pos, block):
+        nvis = o.n_visible_blocks(pos, block)
+        loc = pos // block
+        rest = sorted((b for b in range(nvis) if b != loc), key=lambda b: (float(row[b]), b))
+        return [loc] + rest
+    o.ranked_blocks = ranked_blocks
+
+
+def _mut_append_swapped(o):
+    def indexer_append(cache, new, ts, tp):
+        out = cache.clone()
+        for t in range(ts.numel()):
+            out[int(ts[t]), :, int(tp[t])] = new[ts.numel() - 1 - t]
+        return out
+    o.indexer_append = indexer_append
+
+
+MUTATIONS = [_mut_causal_off_by_one, _mut_no_causal_mask, _mut_tie_higher_index, _mut_no_bias,
+             _mut_gqa_modulo, _mut_no_scale, _mut_nvis_off_by_one, _mut_transposed_scores,
+             _mut_dropped_term, _mut_future_rows, _mut_sign, _mut_k_minus_one,
+             _mut_unsorted_ids, _mut_lowest_scores, _mut_append_swapped]
+
+
+@pytest.mark.parametrize("mut", MUTATIONS, ids=lambda f: f.__name__[5:])
+def test_mutation_is_caught(mut):
+    o = fresh_oracle(mut.__name__)
+    mut(o)
+    failed = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(o)
+        except Exception:        # AssertionError, or a crash the mistake causes
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught {mut.__name__}"
+
+
+def test_unmutated_copy_passes():
+    P.run_all(fresh_oracle("clean"))

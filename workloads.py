@@ -1,0 +1,207 @@
+"""Seeded synthetic inputs for MiniMax Sparse Attention (MSA) workloads.
+
+This module only draws random numbers and lays them out; it holds none of the
+method's arithmetic.  Both the CPU oracle (tests, CPU baseline) and the CUDA
+path (tests, bench) take their inputs from here, so both sides always see the
+same bytes.
+
+Geometry follows the head layout stated in the llama.cpp pull request "Add
+MiniMax-M3 (MSA: MiniMax Sparse Attention) support" (review comment with the
+random-init test model): head_dim 128, 4 KV heads = 4 indexer groups, indexer
+dim 128, block 128, top-k 16; 64 query heads (16 per group).
+
+Recipe (identical for every workload):
+  * torch CPU ``Generator`` seeded with ``seed`` (default 0);
+  * draw order: indexer keys, K, V (each stream in turn, shape [G][L][dim]),
+    then indexer queries, then Q;
+  * indexer values are float32 N(0,1)/sqrt(idx_dim); with ``quantize_idx`` they
+    are rounded to the nearest multiple of 1/8 (torch.round, half to even) so
+    that equal block scores occur;
+  * K, V and Q are float32 N(0,1) draws rounded to bfloat16 (round to nearest
+    even).
+Positions [0, L_existing) are in the cache before the step; positions
+[L_existing, L_total) are the step's new tokens (appended by the step);
+capacity is L_total rounded up to a multiple of the block size, and slots past
+L_total are zero.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+N_Q_HEADS = 64
+N_KV_HEADS = 4
+HEAD_DIM = 128
+IDX_DIM = 128
+BLOCK = 128
+TOP_K = 16
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shape of one synthetic MSA step.
+
+    ``queries`` selects which positions issue a query: "last" (one decode
+    query per stream at L_total-1) or "new" (every appended token queries,
+    as in prefill).
+    """
+    name: str
+    n_streams: int
+    l_existing: int
+    l_total: int
+    queries: str = "last"
+    quantize_idx: bool = False
+    n_q_heads: int = N_Q_HEADS
+    n_kv_heads: int = N_KV_HEADS
+    head_dim: int = HEAD_DIM
+    idx_dim: int = IDX_DIM
+    block: int = BLOCK
+    top_k: int = TOP_K
+    description: str = ""
+
+    @property
+    def capacity(self) -> int:
+        return -(-self.l_total // self.block) * self.block
+
+    @property
+    def n_new(self) -> int:
+        return self.l_total - self.l_existing
+
+    @property
+    def n_queries(self) -> int:
+        per = 1 if self.queries == "last" else self.n_new
+        return self.n_streams * per
+
+
+# The five workloads of the benchmark plan (names say what they are).
+DECODE_4K = Workload("decode_1x4k", 1, 4095, 4096, "last",
+                     description="1 stream, 4096-token context, one query at 4095")
+DECODE_32K_X32 = Workload("decode_32x32k", 32, 32767, 32768, "last",
+                          description="32 streams x 32768-token context, one query each at 32767")
+PREFILL_16K = Workload("prefill_1x16k", 1, 0, 16384, "new",
+                       description="16384 tokens appended to an empty cache, every token queries")
+DECODE_128K_X8 = Workload("decode_8x128k", 8, 131071, 131072, "last",
+                          description="8 streams x 131072-token context, one query each")
+CHUNKED_PREFILL_TIES = Workload("chunked_prefill_4x2k_on_64k_ties", 4, 65536, 67584, "new",
+                                quantize_idx=True,
+                                description="4 streams append 2048 tokens to a 65536-token cache; "
+                                            "indexer values quantised to 1/8")
+WORKLOADS = {w.name: w for w in (DECODE_4K, DECODE_32K_X32, PREFILL_16K, DECODE_128K_X8,
+                                 CHUNKED_PREFILL_TIES)}
+
+
+@dataclass
+class Inputs:
+    """All tensors of one step, on the CPU, in the library's layouts.
+
+    idx_k_cache [S][G][cap][Di] f32, k_cache/v_cache [S][G][cap][D] bf16 hold
+    the existing tokens only (new slots are zero).  The new tokens are
+    idx_k_new [n_tok][G][Di] f32, k_new/v_new [n_tok][G][D] bf16 with
+    tok_stream/tok_pos [n_tok] int32.  Queries: q_stream/q_pos [n_q] int32,
+    idx_q [n_q][G][Di] f32, q [n_q][Hq][D] bf16.
+    """
+    w: Workload
+    idx_k_cache: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    tok_stream: torch.Tensor
+    tok_pos: torch.Tensor
+    idx_k_new: torch.Tensor
+    k_new: torch.Tensor
+    v_new: torch.Tensor
+    q_stream: torch.Tensor
+    q_pos: torch.Tensor
+    idx_q: torch.Tensor
+    q: torch.Tensor
+    extra: dict = field(default_factory=dict)
+
+
+def _idx_draw(g: torch.Generator, shape, idx_dim: int, quantize: bool) -> torch.Tensor:
+    x = torch.randn(shape, generator=g, dtype=torch.float32) / math.sqrt(idx_dim)
+    if quantize:
+        x = torch.round(x * 8.0) / 8.0
+    return x
+
+
+def _bf16_draw(g: torch.Generator, shape) -> torch.Tensor:
+    return torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_inputs(w: Workload, seed: int = 0, streams: range | None = None) -> Inputs:
+    """Draw the inputs of workload ``w``.
+
+    ``streams`` restricts the draw to a sub-range of streams (a bounded sample
+    for CPU timing); the generator is seeded per stream block so that a
+    sampled stream gets the same values it has in the full draw.
+    """
+    S = w.n_streams
+    streams = range(S) if streams is None else streams
+    G, Di, D, Hq = w.n_kv_heads, w.idx_dim, w.head_dim, w.n_q_heads
+    cap, L, L0 = w.capacity, w.l_total, w.l_existing
+    ns = len(streams)
+
+    idx_full = torch.zeros((ns, G, cap, Di), dtype=torch.float32)
+    k_full = torch.zeros((ns, G, cap, D), dtype=torch.bfloat16)
+    v_full = torch.zeros((ns, G, cap, D), dtype=torch.bfloat16)
+    nq_per = 1 if w.queries == "last" else w.n_new
+    idx_q = torch.empty((ns * nq_per, G, Di), dtype=torch.float32)
+    q = torch.empty((ns * nq_per, Hq, D), dtype=torch.bfloat16)
+
+    for i, s in enumerate(streams):
+        # one independent generator per stream: a stream's values do not
+        # depend on which other streams are drawn
+        g = torch.Generator().manual_seed(seed * 1_000_003 + s)
+        idx_full[i, :, :L] = _idx_draw(g, (G, L, Di), Di, w.quantize_idx)
+        k_full[i, :, :L] = _bf16_draw(g, (G, L, D))
+        v_full[i, :, :L] = _bf16_draw(g, (G, L, D))
+        idx_q[i * nq_per:(i + 1) * nq_per] = _idx_draw(g, (nq_per, G, Di), Di, w.quantize_idx)
+        q[i * nq_per:(i + 1) * nq_per] = _bf16_draw(g, (nq_per, Hq, D))
+
+    # split into existing cache + new tokens
+    new_pos = torch.arange(L0, L, dtype=torch.int32)
+    tok_stream = torch.repeat_interleave(torch.arange(ns, dtype=torch.int32), len(new_pos))
+    tok_pos = new_pos.repeat(ns)
+    idx_k_new = idx_full[:, :, L0:L].permute(0, 2, 1, 3).reshape(-1, G, Di).contiguous()
+    k_new = k_full[:, :, L0:L].permute(0, 2, 1, 3).reshape(-1, G, D).contiguous()
+    v_new = v_full[:, :, L0:L].permute(0, 2, 1, 3).reshape(-1, G, D).contiguous()
+    idx_full[:, :, L0:L] = 0
+    k_full[:, :, L0:L] = 0
+    v_full[:, :, L0:L] = 0
+
+    if w.queries == "last":
+        q_stream = torch.arange(ns, dtype=torch.int32)
+        q_pos = torch.full((ns,), L - 1, dtype=torch.int32)
+    else:
+        q_stream = tok_stream.clone()
+        q_pos = tok_pos.clone()
+    return Inputs(w, idx_full, k_full, v_full, tok_stream, tok_pos, idx_k_new, k_new, v_new,
+                  q_stream, q_pos, idx_q, q)
+
+
+def make_custom(n_streams: int, capacity: int, lengths, q_positions, *, seed: int = 0,
+                n_q_heads: int = N_Q_HEADS, n_kv_heads: int = N_KV_HEADS,
+                head_dim: int = HEAD_DIM, idx_dim: int = IDX_DIM, quantize_idx: bool = False,
+                kv_dtype=torch.bfloat16):
+    """Caches already holding ``lengths[s]`` tokens per stream and an explicit
+    list of (stream, position) queries.  Used for ragged / edge-case tests.
+
+    Returns (idx_k_cache, k_cache, v_cache, q_stream, q_pos, idx_q, q).
+    """
+    g = torch.Generator().manual_seed(seed)
+    G = n_kv_heads
+    idx = torch.zeros((n_streams, G, capacity, idx_dim), dtype=torch.float32)
+    k = torch.zeros((n_streams, G, capacity, head_dim), dtype=kv_dtype)
+    v = torch.zeros((n_streams, G, capacity, head_dim), dtype=kv_dtype)
+    for s in range(n_streams):
+        L = lengths[s]
+        idx[s, :, :L] = _idx_draw(g, (G, L, idx_dim), idx_dim, quantize_idx)
+        k[s, :, :L] = torch.randn((G, L, head_dim), generator=g).to(kv_dtype)
+        v[s, :, :L] = torch.randn((G, L, head_dim), generator=g).to(kv_dtype)
+    q_stream = torch.tensor([sp[0] for sp in q_positions], dtype=torch.int32)
+    q_pos = torch.tensor([sp[1] for sp in q_positions], dtype=torch.int32)
+    n_q = len(q_positions)
+    idx_q = _idx_draw(g, (n_q, G, idx_dim), idx_dim, quantize_idx)
+    q = torch.randn((n_q, n_q_heads, head_dim), generator=g).to(kv_dtype)
+    return idx, k, v, q_stream, q_pos, idx_q, q
