@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA decode step: tokens/s at 32K context x 32 streams on
+one B200 (or N replicas, one per GPU, for --gpus N), and the achieved HBM
+bandwidth of the step and of its dominant kernel.
+
+A step is one pass of the whole hot path over one batch of decode queries:
+append the new token's indexer key and K/V rows, fused block scores
+(score + causal mask + maxpool + local bias), top-16 selection and the
+block-sparse attention, all through the C ABI.  Every step re-appends the
+token at the last slot and queries there, so each step is the same work.
+Inputs (2.1 GB of F32 indexer keys + 2.1 GB of bf16 K/V per GPU) are larger
+than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) shard independent
+streams: each rank holds its own 32 streams (weak scaling, no collective on
+the data path; one all-reduce of the timing at the end).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MSA decode tokens/s @32K ctx x32 streams; achieved HBM GB/s vs peak"
+WORKLOAD = W.DECODE_32K_X32
+
+# DRAM traffic of one block-scores launch on this workload, from the ncu
+# capture summarised in profiles/, valid only for the kernel source it was
+# taken on (sha256 prefix of msa_scores_gemv.cuh).
+SCORES_TRAFFIC = {"source_sha": None, "bytes_per_launch": None}
+
+
+def scores_source_sha() -> str:
+    p = os.path.join(ROOT, "block_sparse_attention_maxpool_b200", "csrc", "msa_scores_gemv.cuh")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+def scores_bytes(w) -> int:
+    """Bytes the block-score kernel must move per launch: every visible
+    indexer key once (512 B per key per group), the indexer queries, and the
+    block-score output."""
+    G, Di = w.n_kv_heads, w.idx_dim
+    n_q = w.n_queries
+    keys = n_q * G * w.l_total * Di * 4           # decode: each query sees l_total keys
+    return keys + n_q * G * Di * 4 + n_q * G * (w.capacity // w.block) * 4
+
+
+def step_bytes(w) -> int:
+    """Bytes one decode step must move: visible indexer keys, the 16 selected
+    K/V blocks per group, the query and the output (the plan's per-stream
+    count: 67,108,864 + 4,194,304 + 34,816 at 32K context)."""
+    G, D = w.n_kv_heads, w.head_dim
+    idx = w.l_total * G * w.idx_dim * 4
+    kv = min(w.top_k, w.l_total // w.block + 1) * w.block * G * D * 2 * 2
+    qo = w.n_q_heads * D * 2 * 2 + G * w.idx_dim * 4
+    return (idx + kv + qo) * w.n_streams
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi every 200 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.rows = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def mark(self):
+        return len(self.rows)
+
+    def stop(self, since: int = 0) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [r for r in self.rows[since:] if len(r) >= 8] or [r for r in self.rows if len(r) >= 8]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, dev):
+    import block_sparse_attention_maxpool_b200 as msa
+    from block_sparse_attention_maxpool_b200 import build as msa_build
+
+    if rank == 0:
+        msa_build.build()
+    if world > 1:
+        torch.distributed.barrier(device_ids=[dev])
+    w = WORKLOAD
+    shape = msa.Shape(n_streams=w.n_streams, capacity=w.capacity)
+    inp = W.make_inputs(w, seed=rank)                    # each rank: its own 32 streams
+    d = {n: getattr(inp, n).to(dev) for n in ("idx_k_cache", "k_cache", "v_cache", "tok_stream",
+                                               "tok_pos", "idx_k_new", "k_new", "v_new",
+                                               "q_stream", "q_pos", "idx_q", "q")}
+    del inp
+    n_q = w.n_queries
+    G = w.n_kv_heads
+    bufs = {
+        "block_scores": torch.empty((n_q, G, shape.n_blocks), dtype=torch.float32, device=dev),
+        "sel": torch.empty((n_q, G, shape.top_k), dtype=torch.int32, device=dev),
+        "n_sel": torch.empty((n_q, G), dtype=torch.int32, device=dev),
+        "out": torch.empty((n_q, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=dev),
+    }
+    ws = msa.msa_workspace_bytes(shape, n_q, msa.MODE_DECODE)
+    bufs["workspace"] = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
+    launches_per_step = 5 + (1 if ws > 0 else 0)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(shape.head_dim)
+
+    def step(ev=None):
+        msa.msa_indexer_append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], stream)
+        msa.msa_kv_append(shape, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
+                          d["tok_pos"], stream)
+        if ev is not None:
+            ev[0].record(stream)
+        msa.msa_block_scores(shape, d["idx_q"], d["idx_k_cache"], d["q_stream"], d["q_pos"],
+                             bufs["block_scores"], stream)
+        if ev is not None:
+            ev[1].record(stream)
+        msa.msa_select_topk(shape, bufs["block_scores"], d["q_pos"], bufs["sel"], bufs["n_sel"], stream)
+        msa.msa_sparse_attn_decode(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"],
+                                   d["q_pos"], scale, bufs["out"], bufs["workspace"], stream)
+
+    clocks = ClockSampler(dev) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if msa.msa_get_device_error(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- device-resident timing -------------------------------------------
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier(device_ids=[dev])
+    torch.cuda.synchronize(dev)
+    mark = clocks.mark() if clocks else 0
+    t0.record(stream)
+    for i in range(args.steps):
+        step(kev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier(device_ids=[dev])
+    ms = t0.elapsed_time(t1) / args.steps
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+
+    # ---- end to end: host inputs in, host output out, every step ------------
+    host_names = ("tok_stream", "tok_pos", "idx_k_new", "k_new", "v_new", "q_stream", "q_pos", "idx_q", "q")
+    host = {n: d[n].cpu().pin_memory() for n in host_names}
+    h_out = torch.empty(bufs["out"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = max(3, min(args.steps, 200))
+    for _ in range(3):
+        for n in host_names:
+            d[n].copy_(host[n], non_blocking=True)
+        step()
+        h_out.copy_(bufs["out"], non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for n in host_names:
+            d[n].copy_(host[n], non_blocking=True)
+        step()
+        h_out.copy_(bufs["out"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if msa.msa_get_device_error(stream) != 0:
+        raise RuntimeError("device error during timing")
+    clk = clocks.stop(mark) if clocks else None
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms, k_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms, k_ms = t.tolist()
+    if rank != 0:
+        return None
+
+    peaks = load_peaks()
+    tokens = w.n_streams * world
+    sbytes = scores_bytes(w)
+    achieved = sbytes / (k_ms * 1e-3) / 1e9
+    traffic = SCORES_TRAFFIC["bytes_per_launch"] if SCORES_TRAFFIC["source_sha"] == scores_source_sha() else None
+    step_gbs = step_bytes(w) / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32 indexer / bf16 attention (f32 accumulate)",
+        "data": "synthetic (seeded N(0,1) K/V/Q bf16, indexer N(0,1)/sqrt(128) f32)",
+        "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "context": w.l_total,
+                   "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                   "block": w.block, "top_k": w.top_k, "parallelism": f"replicas{world}",
+                   "l2": "inputs 4.2 GB per GPU > 126 MB L2, no flush"},
+        "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peaks["hbm_gbs"],
+                     "frac": step_gbs / peaks["hbm_gbs"], "bytes_per_step": step_bytes(w)},
+        "roofline": {"kernel": "block_scores_gemv", "bound": "hbm", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic, "algorithmic_bytes": sbytes, "ms_per_launch": k_ms,
+                     "peak_src": peaks["src"]},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(n_streams: int, seed: int = 0):
+    import oracle
+    w = WORKLOAD
+    inp = W.make_inputs(w, seed=seed, streams=range(n_streams))
+    caches = [oracle.indexer_append(c, n, inp.tok_stream, inp.tok_pos)
+              for c, n in ((inp.idx_k_cache, inp.idx_k_new), (inp.k_cache, inp.k_new), (inp.v_cache, inp.v_new))]
+
+    def run():
+        oracle.msa_step(caches[0], caches[1], caches[2], inp.idx_q, inp.q, inp.q_stream, inp.q_pos,
+                        w.block, w.top_k)
+    return run
+
+
+def cpu_baseline(budget_s: float = 10.0, n_streams: int = 8) -> dict:
+    run = oracle_sample(n_streams)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": reps * n_streams / el, "unit": "tokens/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{n_streams} of the 32 streams of {WORKLOAD.name}, all steps (append, FP64 block "
+                      f"scores, selection, attention), repeated {reps}x over {el:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    run = oracle_sample(1)
+    for _ in range(args.warmup):
+        run()
+    budget = 120.0
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t)
+        if sum(times) > budget:
+            break
+    ms = 1e3 * sum(times) / len(times)
+    value = 1.0 / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": len(times), "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD.name, "streams_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": f"1 of 32 streams of {WORKLOAD.name} per step (FP64 CPU oracle)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, rank, world, local)
+        if line is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

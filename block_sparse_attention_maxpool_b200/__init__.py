@@ -1,0 +1,269 @@
+"""MiniMax Sparse Attention (MSA) hot path on B200: Python binding.
+
+Thin ctypes layer over ``libmsa.so`` (the C ABI declared in include/msa.h):
+it checks tensor dtypes, devices and shapes, passes raw device pointers and
+the current CUDA stream, and turns a non-zero status into ``MsaError``.  All
+computation runs in the library's CUDA kernels; there is no fallback.  If the
+library has not been built, every call raises.
+
+Build:  python -m block_sparse_attention_maxpool_b200.build
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_block_scores",
+           "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
+           "msa_workspace_bytes", "msa_get_device_error", "msa_version", "library", "LIB_PATH",
+           "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
+MODE_DECODE = 0
+MODE_PREFILL = 1
+LOCAL_BIAS = 2.0 ** 100
+
+STATUS = {0: "MSA_OK", -1: "MSA_ERR_NULL", -2: "MSA_ERR_ALIGN", -3: "MSA_ERR_SHAPE",
+          -4: "MSA_ERR_RANGE", -5: "MSA_ERR_WORKSPACE", -6: "MSA_ERR_CUDA"}
+DEVERR = {0x1: "QUERY_RANGE", 0x2: "TOKEN_RANGE", 0x4: "SEL_RANGE", 0x8: "TIMEOUT"}
+
+
+class MsaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class CShape(ctypes.Structure):
+    _fields_ = [("n_streams", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+
+@dataclass(frozen=True)
+class Shape:
+    """Geometry of one MSA layer's caches (msa_shape)."""
+    n_streams: int
+    capacity: int
+    n_q_heads: int = 64
+    n_kv_heads: int = 4
+    head_dim: int = 128
+    idx_dim: int = 128
+    block: int = 128
+    top_k: int = 16
+
+    @property
+    def n_blocks(self) -> int:
+        return self.capacity // self.block
+
+    def c(self) -> CShape:
+        return CShape(self.n_streams, self.capacity, self.n_q_heads, self.n_kv_heads,
+                      self.head_dim, self.idx_dim, self.block, self.top_k)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_SIGS = {
+    "msa_indexer_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P]),
+    "msa_kv_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I, _P]),
+    "msa_block_scores": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P]),
+    "msa_select_topk": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I, _P, _P, _P]),
+    "msa_sparse_attn_decode": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
+                                              ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_sparse_attn_prefill": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
+                                               ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(CShape), _I, _I]),
+    "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "msa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
+    "msa_version": (ctypes.c_int, []),
+}
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libmsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "'python -m block_sparse_attention_maxpool_b200.build'")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None, dtype, shape, name: str) -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise MsaError(fn, status)
+
+
+def _n(t: torch.Tensor, name: str) -> int:
+    if t.dim() != 1:
+        raise ValueError(f"{name} must be 1-D")
+    return t.shape[0]
+
+
+def msa_indexer_append(shape: Shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, stream=None):
+    n = _n(tok_stream, "tok_stream")
+    s = shape.c()
+    _check("msa_indexer_append", library().msa_indexer_append(
+        ctypes.byref(s),
+        _ptr(idx_k_cache, torch.float32, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
+        _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
+        _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+        n, _stream(stream)))
+
+
+def msa_kv_append(shape: Shape, k_cache, v_cache, k_new, v_new, tok_stream, tok_pos, stream=None):
+    n = _n(tok_stream, "tok_stream")
+    cs = (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.head_dim)
+    ns = (n, shape.n_kv_heads, shape.head_dim)
+    s = shape.c()
+    _check("msa_kv_append", library().msa_kv_append(
+        ctypes.byref(s), _ptr(k_cache, torch.bfloat16, cs, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, cs, "v_cache"), _ptr(k_new, torch.bfloat16, ns, "k_new"),
+        _ptr(v_new, torch.bfloat16, ns, "v_new"), _ptr(tok_stream, torch.int32, (n,), "tok_stream"),
+        _ptr(tok_pos, torch.int32, (n,), "tok_pos"), n, _stream(stream)))
+
+
+def msa_block_scores(shape: Shape, idx_q, idx_k_cache, q_stream, q_pos, block_scores=None, stream=None):
+    n = _n(q_pos, "q_pos")
+    if block_scores is None:
+        block_scores = torch.empty((n, shape.n_kv_heads, shape.n_blocks), dtype=torch.float32,
+                                   device=idx_q.device)
+    s = shape.c()
+    _check("msa_block_scores", library().msa_block_scores(
+        ctypes.byref(s), _ptr(idx_q, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_q"),
+        _ptr(idx_k_cache, torch.float32, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
+        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+        _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
+        _stream(stream)))
+    return block_scores
+
+
+def msa_select_topk(shape: Shape, block_scores, q_pos, sel=None, n_sel=None, stream=None):
+    n = _n(q_pos, "q_pos")
+    dev = block_scores.device
+    if sel is None:
+        sel = torch.empty((n, shape.n_kv_heads, shape.top_k), dtype=torch.int32, device=dev)
+    if n_sel is None:
+        n_sel = torch.empty((n, shape.n_kv_heads), dtype=torch.int32, device=dev)
+    s = shape.c()
+    _check("msa_select_topk", library().msa_select_topk(
+        ctypes.byref(s),
+        _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
+        _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+        _ptr(sel, torch.int32, (n, shape.n_kv_heads, shape.top_k), "sel"),
+        _ptr(n_sel, torch.int32, (n, shape.n_kv_heads), "n_sel"), _stream(stream)))
+    return sel, n_sel
+
+
+def msa_workspace_bytes(shape: Shape, n_q: int, mode: int) -> int:
+    s = shape.c()
+    v = library().msa_workspace_bytes(ctypes.byref(s), n_q, mode)
+    if v == ctypes.c_size_t(-1).value:
+        raise MsaError("msa_workspace_bytes", -3)
+    return v
+
+
+def _attn(fn_name: str, mode: int, shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos,
+          softmax_scale=None, out=None, workspace=None, stream=None):
+    n = _n(q_pos, "q_pos")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(shape.head_dim)
+    if out is None:
+        out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=q.device)
+    need = msa_workspace_bytes(shape, n, mode)
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        ws_ptr = _ptr(workspace, torch.uint8, None, "workspace")
+        ws_bytes = workspace.numel()
+    cs = (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.head_dim)
+    s = shape.c()
+    _check(fn_name, getattr(library(), fn_name)(
+        ctypes.byref(s), _ptr(q, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
+        _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+        _ptr(sel, torch.int32, (n, shape.n_kv_heads, shape.top_k), "sel"),
+        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+        float(softmax_scale), _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"),
+        ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def msa_sparse_attn_decode(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos, softmax_scale=None,
+                           out=None, workspace=None, stream=None):
+    return _attn("msa_sparse_attn_decode", MODE_DECODE, shape, q, k_cache, v_cache, sel, q_stream,
+                 q_pos, softmax_scale, out, workspace, stream)
+
+
+def msa_sparse_attn_prefill(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos, softmax_scale=None,
+                            out=None, workspace=None, stream=None):
+    return _attn("msa_sparse_attn_prefill", MODE_PREFILL, shape, q, k_cache, v_cache, sel, q_stream,
+                 q_pos, softmax_scale, out, workspace, stream)
+
+
+def msa_get_device_error(stream=None) -> int:
+    """Wait for the stream, then read and clear the device error word."""
+    v = ctypes.c_uint32(0)
+    _check("msa_get_device_error", library().msa_get_device_error(ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+def msa_version() -> int:
+    return library().msa_version()
+
+
+def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None, stream=None,
+                prefill: bool = False):
+    """One MSA step through the C ABI: append the new tokens' indexer keys
+    and K/V rows, score blocks, select the top-k and attend.
+
+    caches: idx_k_cache, k_cache, v_cache (device); new: tok_stream, tok_pos,
+    idx_k_new, k_new, v_new, q_stream, q_pos, idx_q, q (device).  ``bufs`` may
+    hold preallocated block_scores / sel / n_sel / out / workspace.
+    Returns (out, sel, n_sel, block_scores).
+    """
+    b = bufs or {}
+    msa_indexer_append(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"],
+                       new["tok_pos"], stream)
+    msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
+                  new["tok_stream"], new["tok_pos"], stream)
+    bs = msa_block_scores(shape, new["idx_q"], caches["idx_k_cache"], new["q_stream"], new["q_pos"],
+                          b.get("block_scores"), stream)
+    sel, n_sel = msa_select_topk(shape, bs, new["q_pos"], b.get("sel"), b.get("n_sel"), stream)
+    attn = msa_sparse_attn_prefill if prefill else msa_sparse_attn_decode
+    out = attn(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
+               new["q_pos"], None, b.get("out"), b.get("workspace"), stream)
+    return out, sel, n_sel, bs

@@ -1,0 +1,314 @@
+// C ABI of the MSA hot path (declarations and contracts in include/msa.h).
+// Host-side argument checks, launch configuration and TMA descriptors; the
+// kernels live in the msa_*.cuh headers included below (one translation
+// unit, so the per-device error word needs no relocatable device code).
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "msa.h"
+#include "msa_append.cuh"
+#include "msa_attn_decode.cuh"
+#include "msa_common.cuh"
+#include "msa_scores_gemv.cuh"
+#include "msa_select.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kScoreStages = 4;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(const msa_shape* sh) {
+  if (sh == nullptr) return MSA_ERR_NULL;
+  if (sh->n_streams <= 0 || sh->capacity <= 0 || sh->block != 128 || sh->capacity % 128 != 0 ||
+      sh->head_dim != 128 || sh->idx_dim != 128 || sh->top_k != 16 || sh->n_kv_heads < 1 ||
+      sh->n_kv_heads > 16 || sh->n_q_heads != 16 * sh->n_kv_heads)
+    return MSA_ERR_SHAPE;
+  // every cache row index must fit a signed 32-bit TMA coordinate
+  if (static_cast<int64_t>(sh->n_streams) * sh->n_kv_heads * sh->capacity >= (int64_t{1} << 31))
+    return MSA_ERR_SHAPE;
+  return MSA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+int current_device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MSA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MSA_ERR_CUDA;
+  return MSA_OK;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename Kernel>
+int ensure_smem(Kernel kernel, size_t bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MSA_ERR_CUDA;
+  const uint64_t bit = uint64_t{1} << (dev & 63);
+  if (done_mask.load(std::memory_order_acquire) & bit) return MSA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess)
+    return MSA_ERR_CUDA;
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return MSA_OK;
+}
+
+// ---- TMA descriptors ----------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// A [rows][128] bf16 cache viewed as 2-D; boxes of 128 rows x 64 columns
+// (128 bytes, the widest box the 128-byte swizzle allows).
+int make_kv_map(CUtensorMap* m, const void* base, int64_t rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return MSA_ERR_CUDA;
+  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
+// Split-K factor of the attention kernel: few (query, group) pairs are
+// spread over more CTAs so the selected blocks of a decode step are read by
+// many SMs at once.  Depends only on the pair count, so the workspace size
+// query and the launch always agree.
+int attn_splits(int64_t n_pairs, int mode) {
+  if (mode == MSA_MODE_PREFILL) return 1;
+  if (n_pairs >= 512) return 1;
+  if (n_pairs >= 256) return 2;
+  if (n_pairs >= 96) return 4;
+  if (n_pairs >= 32) return 8;
+  return 16;
+}
+
+size_t attn_workspace(int64_t n_pairs, int n_split) {
+  if (n_split <= 1) return 0;
+  const size_t slots = static_cast<size_t>(n_pairs) * n_split * msa::attn::kHpg;
+  return slots * (msa::attn::kD + 2) * sizeof(float);
+}
+
+int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache, const msa_bf16* v_cache,
+                const int32_t* sel, const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                float softmax_scale, msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream,
+                int mode) {
+  int st = check_shape(sh);
+  if (st != MSA_OK) return st;
+  if (n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0) return MSA_OK;
+  if (!q || !k_cache || !v_cache || !sel || !q_stream || !q_pos || !out) return MSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(sel) || !aligned16(out))
+    return MSA_ERR_ALIGN;
+  if (!std::isfinite(softmax_scale)) return MSA_ERR_RANGE;
+  const int G = sh->n_kv_heads;
+  const int64_t n_pairs = static_cast<int64_t>(n_q) * G;
+  const int n_split = attn_splits(n_pairs, mode);
+  if (n_pairs * n_split >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const size_t need = attn_workspace(n_pairs, n_split);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need) return MSA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MSA_ERR_ALIGN;
+  }
+  const int64_t rows = static_cast<int64_t>(sh->n_streams) * G * sh->capacity;
+  CUtensorMap tm_k, tm_v;
+  if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
+  if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
+  static std::atomic<uint64_t> smem_done{0};
+  if ((st = ensure_smem(msa::attn::sparse_attn_kernel, msa::attn::kSmemBytes, smem_done)) != MSA_OK) return st;
+
+  msa::attn::Params P;
+  P.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  P.sel = sel;
+  P.q_stream = q_stream;
+  P.q_pos = q_pos;
+  P.out = reinterpret_cast<__nv_bfloat16*>(out);
+  P.ws_o = need > 0 ? static_cast<float*>(workspace) : nullptr;
+  P.ws_ml = need > 0 ? P.ws_o + static_cast<size_t>(n_pairs) * n_split * msa::attn::kHpg * msa::attn::kD : nullptr;
+  P.n_q = n_q;
+  P.G = G;
+  P.n_streams = sh->n_streams;
+  P.capacity = sh->capacity;
+  P.n_split = n_split;
+  P.blocks_per_split = msa::attn::kTopK / n_split;
+  P.scale_log2 = softmax_scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  msa::attn::sparse_attn_kernel<<<static_cast<unsigned>(n_pairs * n_split), msa::attn::kThreads,
+                                  msa::attn::kSmemBytes, s>>>(tm_k, tm_v, P);
+  if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
+  if (n_split > 1) {
+    const int64_t warps = n_pairs * msa::attn::kHpg;
+    const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
+    msa::attn::attn_combine_kernel<<<grid, 256, 0, s>>>(P.ws_o, P.ws_ml, P.out, static_cast<int>(n_pairs), n_split);
+    if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
+  }
+  return MSA_OK;
+}
+
+int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache1, const void* src1,
+                const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, int row_bytes,
+                void* stream) {
+  int st = check_shape(sh);
+  if (st != MSA_OK) return st;
+  if (n_tok < 0) return MSA_ERR_RANGE;
+  if (n_tok == 0) return MSA_OK;
+  if (!cache0 || !src0 || !tok_stream || !tok_pos) return MSA_ERR_NULL;
+  if (!aligned16(cache0) || !aligned16(src0) || (cache1 && !aligned16(cache1)) || (src1 && !aligned16(src1)))
+    return MSA_ERR_ALIGN;
+  const int64_t warps = static_cast<int64_t>(n_tok) * sh->n_kv_heads;
+  if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
+  msa::append_rows_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(cache0), static_cast<const uint8_t*>(src0), static_cast<uint8_t*>(cache1),
+      static_cast<const uint8_t*>(src1), tok_stream, tok_pos, n_tok, sh->n_streams, sh->n_kv_heads,
+      sh->capacity, row_bytes);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+int msa_indexer_append(const msa_shape* shape, float* idx_k_cache, const float* idx_k_new,
+                       const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
+  return append_rows(shape, idx_k_cache, idx_k_new, nullptr, nullptr, tok_stream, tok_pos, n_tok,
+                     128 * static_cast<int>(sizeof(float)), stream);
+}
+
+int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, const msa_bf16* k_new,
+                  const msa_bf16* v_new, const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok,
+                  void* stream) {
+  if (n_tok > 0 && (!v_cache || !v_new)) return MSA_ERR_NULL;
+  return append_rows(shape, k_cache, k_new, v_cache, v_new, tok_stream, tok_pos, n_tok,
+                     128 * static_cast<int>(sizeof(msa_bf16)), stream);
+}
+
+int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
+                     const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
+                     void* stream) {
+  int st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0) return MSA_OK;
+  if (!idx_q || !idx_k_cache || !q_stream || !q_pos || !block_scores) return MSA_ERR_NULL;
+  if (!aligned16(idx_q) || !aligned16(idx_k_cache) || !aligned16(block_scores)) return MSA_ERR_ALIGN;
+  using namespace msa::gemv;
+  Params P;
+  P.idx_q = idx_q;
+  P.idx_k = idx_k_cache;
+  P.q_stream = q_stream;
+  P.q_pos = q_pos;
+  P.bs = block_scores;
+  P.n_q = n_q;
+  P.G = shape->n_kv_heads;
+  P.n_streams = shape->n_streams;
+  P.capacity = shape->capacity;
+  P.nblk = shape->capacity / 128;
+  P.n_tasks = static_cast<long long>(n_q) * P.G * P.nblk;
+  int sms = 0;
+  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+  const size_t smem = sizeof(Smem<kScoreStages>);
+  static std::atomic<uint64_t> smem_done{0};
+  if ((st = ensure_smem(block_scores_gemv_kernel<kScoreStages>, smem, smem_done)) != MSA_OK) return st;
+  const long long grid = std::min<long long>(sms, P.n_tasks);
+  block_scores_gemv_kernel<kScoreStages>
+      <<<static_cast<unsigned>(grid), kThreads, smem, static_cast<cudaStream_t>(stream)>>>(P);
+  return cuda_status(cudaGetLastError());
+}
+
+int msa_select_topk(const msa_shape* shape, const float* block_scores, const int32_t* q_pos, int32_t n_q,
+                    int32_t* sel, int32_t* n_sel, void* stream) {
+  int st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0) return MSA_OK;
+  if (!block_scores || !q_pos || !sel) return MSA_ERR_NULL;
+  if (!aligned16(block_scores) || !aligned16(sel)) return MSA_ERR_ALIGN;
+  const int G = shape->n_kv_heads;
+  const int nblk = shape->capacity / 128;
+  const int64_t warps = static_cast<int64_t>(n_q) * G;
+  if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (nblk <= 32 * 8) {
+    msa::sel::select_topk_kernel<8><<<grid, 256, 0, s>>>(block_scores, q_pos, n_q, G, nblk, shape->capacity,
+                                                          sel, n_sel);
+  } else if (nblk <= 32 * 32) {
+    msa::sel::select_topk_kernel<32><<<grid, 256, 0, s>>>(block_scores, q_pos, n_q, G, nblk, shape->capacity,
+                                                           sel, n_sel);
+  } else {
+    msa::sel::select_topk_kernel<0><<<grid, 256, 0, s>>>(block_scores, q_pos, n_q, G, nblk, shape->capacity,
+                                                          sel, n_sel);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
+                           const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
+                           const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_DECODE);
+}
+
+int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
+                            const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
+                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_PREFILL);
+}
+
+size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {
+  if (check_shape(shape) != MSA_OK || n_q < 0 || (mode != MSA_MODE_DECODE && mode != MSA_MODE_PREFILL))
+    return static_cast<size_t>(-1);
+  const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
+  return attn_workspace(n_pairs, attn_splits(n_pairs, mode));
+}
+
+const char* msa_status_string(int status) {
+  switch (status) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_NULL: return "MSA_ERR_NULL: a required pointer is NULL";
+    case MSA_ERR_ALIGN: return "MSA_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case MSA_ERR_SHAPE: return "MSA_ERR_SHAPE: unsupported geometry";
+    case MSA_ERR_RANGE: return "MSA_ERR_RANGE: count or value out of range";
+    case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace missing or too small";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA: CUDA launch or query failed";
+    default: return "unknown MSA status";
+  }
+}
+
+int msa_get_device_error(uint32_t* flags, void* stream) {
+  if (flags == nullptr) return MSA_ERR_NULL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MSA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, msa::g_dev_error, sizeof(v)) != cudaSuccess) return MSA_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(msa::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return MSA_ERR_CUDA;
+  *flags = v;
+  return MSA_OK;
+}
+
+int msa_version(void) { return kVersion; }
+
+}  // extern "C"

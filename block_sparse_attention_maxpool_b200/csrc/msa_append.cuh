@@ -1,0 +1,45 @@
+// Cache append: copies new tokens' rows into a [S][G][cap][row] cache.
+// Used for the F32 indexer-key cache (row = 128 floats = 512 B) and the
+// bf16 K/V caches (row = 128 bf16 = 256 B).  Pure data movement: one warp
+// per (token, group) row, 16-byte vector loads and stores.
+#pragma once
+
+#include "msa_common.cuh"
+
+namespace msa {
+
+// rows_bytes: bytes of one row (a multiple of 16, at most 512).
+// Up to two caches (K and V) are written by the same launch; cache1/src1
+// may be null.
+__global__ void __launch_bounds__(256) append_rows_kernel(
+    uint8_t* __restrict__ cache0, const uint8_t* __restrict__ src0, uint8_t* __restrict__ cache1,
+    const uint8_t* __restrict__ src1, const int32_t* __restrict__ tok_stream,
+    const int32_t* __restrict__ tok_pos, int n_tok, int n_streams, int n_groups, int capacity,
+    int row_bytes) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_tok * n_groups) return;
+  const int t = warp / n_groups;
+  const int g = warp - t * n_groups;
+  const int s = tok_stream[t];
+  const int p = tok_pos[t];
+  if (s < 0 || s >= n_streams || p < 0 || p >= capacity) {
+    if (g == 0 && lane == 0) raise_error(MSA_DEVERR_TOKEN_RANGE);
+    return;
+  }
+  const size_t dst_row = (static_cast<size_t>(s) * n_groups + g) * capacity + p;
+  const size_t src_row = static_cast<size_t>(t) * n_groups + g;
+  const int vecs = row_bytes >> 4;
+  if (lane < vecs) {
+    const int4* a = reinterpret_cast<const int4*>(src0 + src_row * row_bytes) + lane;
+    int4* b = reinterpret_cast<int4*>(cache0 + dst_row * row_bytes) + lane;
+    *b = __ldg(a);
+    if (cache1 != nullptr) {
+      const int4* c = reinterpret_cast<const int4*>(src1 + src_row * row_bytes) + lane;
+      int4* d = reinterpret_cast<int4*>(cache1 + dst_row * row_bytes) + lane;
+      *d = __ldg(c);
+    }
+  }
+}
+
+}  // namespace msa

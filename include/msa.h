@@ -1,0 +1,186 @@
+/*
+ * msa.h - C ABI of the MiniMax Sparse Attention (MSA) hot path for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The method (llama.cpp pull request "Add MiniMax-M3 (MSA: MiniMax Sparse
+ * Attention) support", sections "Overview" and "Implementation"): for every
+ * query, one indexer head per GQA group scores each causally visible key as
+ * idx_q . idx_k, the scores are max-pooled over 128-slot key blocks, the
+ * query's own (local) block gets a large positive bias so it is always kept,
+ * and the top-16 blocks are selected.  Attention then runs over only those
+ * 16 x 128 = 2048 K/V rows, shared by the group's 16 query heads.
+ *
+ * Conventions for every call
+ *  - All tensor pointers are DEVICE pointers into caller-owned memory,
+ *    contiguous in the layout stated, 16-byte aligned.  The library never
+ *    allocates, frees or keeps a pointer after a call returns.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and returns MSA_OK or a negative MSA_ERR_* code.  On an
+ *    error nothing is launched and no output is written.
+ *  - Conditions only the device can see (a position or stream id outside the
+ *    cache, a selected block id that is not visible) set a bit in a per-device
+ *    error word and skip the affected work; kernels never trap.  Read and
+ *    clear the word with msa_get_device_error().
+ *  - Block scores, selection and attention read rows j <= q_pos of the query's
+ *    stream: append a token's indexer key and K/V row before scoring or
+ *    attending a query at that position (the query sees its own token).
+ *  - Supported geometry of the CUDA kernels: head_dim = idx_dim = block = 128,
+ *    top_k = 16, n_q_heads = 16 * n_kv_heads, 1 <= n_kv_heads <= 16,
+ *    capacity a positive multiple of 128 (the KV length is a multiple of 128,
+ *    as the MSA branch asserts).  Other shapes return MSA_ERR_SHAPE.
+ *
+ * Layouts (S streams, G = n_kv_heads groups, cap = capacity, nblk = cap/128,
+ * Hq = n_q_heads, D = head_dim, Di = idx_dim):
+ *   idx_k_cache   [S][G][cap][Di]  float32   indexer-key cache
+ *   k_cache       [S][G][cap][D]   bfloat16  K cache (non-transposed)
+ *   v_cache       [S][G][cap][D]   bfloat16  V cache (non-transposed)
+ *   idx_q         [n_q][G][Di]     float32   one indexer query per group
+ *   q             [n_q][Hq][D]     bfloat16  head h belongs to group h / 16
+ *   q_stream, q_pos [n_q]          int32     stream and absolute slot
+ *   block_scores  [n_q][G][nblk]   float32
+ *   sel           [n_q][G][top_k]  int32     ascending block ids, -1 padded
+ *   n_sel         [n_q][G]         int32
+ *   out           [n_q][Hq][D]     bfloat16
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define MSA_OK             0
+#define MSA_ERR_NULL      (-1)  /* a required pointer is NULL                  */
+#define MSA_ERR_ALIGN     (-2)  /* a pointer is not 16-byte aligned            */
+#define MSA_ERR_SHAPE     (-3)  /* geometry not supported (see above)          */
+#define MSA_ERR_RANGE     (-4)  /* a count is negative or too large            */
+#define MSA_ERR_WORKSPACE (-5)  /* workspace missing or smaller than required  */
+#define MSA_ERR_CUDA      (-6)  /* a CUDA launch or query failed               */
+
+/* ---- device error word bits (msa_get_device_error) -------------------- */
+#define MSA_DEVERR_QUERY_RANGE 0x1u /* q_stream/q_pos outside [0,S) x [0,cap): query skipped */
+#define MSA_DEVERR_TOKEN_RANGE 0x2u /* tok_stream/tok_pos outside the cache: token skipped   */
+#define MSA_DEVERR_SEL_RANGE   0x4u /* sel id not a visible block: that block skipped       */
+#define MSA_DEVERR_TIMEOUT     0x8u /* a bounded wait on a copy gave up: output incomplete  */
+
+/* The local-force bias added to the score of each query's own block
+ * ("a large positive bias on each query's local block", MSA pull request,
+ * section "Implementation").  2^100 exceeds twice any finite score the
+ * indexer can produce in practice, so the local block always ranks first;
+ * in float32 the biased score is exactly 2^100. */
+#define MSA_LOCAL_BIAS 0x1p100f
+
+/* Bit pattern of an IEEE bfloat16 value. */
+typedef uint16_t msa_bf16;
+
+typedef struct msa_shape {
+  int32_t n_streams;   /* S: independent sequences, one cache region each      */
+  int32_t capacity;    /* slots per stream, a multiple of block                */
+  int32_t n_q_heads;   /* Hq: 64 for the MiniMax-M3 attention layers           */
+  int32_t n_kv_heads;  /* G: KV heads = GQA groups = indexer heads (4)         */
+  int32_t head_dim;    /* D: 128                                               */
+  int32_t idx_dim;     /* Di: indexer dimension, 128                           */
+  int32_t block;       /* key block size of the max-pool, 128                  */
+  int32_t top_k;       /* blocks kept per query and group, 16                  */
+} msa_shape;
+
+/* msa_indexer_append - write new tokens' indexer keys into the F32 cache.
+ * The indexer keeps its own per-layer F32 key cache beside K/V, one region
+ * per stream (MSA pull request, section "Implementation").
+ *   idx_k_new [n_tok][G][Di] f32; token t goes to idx_k_cache[tok_stream[t]]
+ *   [g][tok_pos[t]][:] for every group g.  Tokens with an out-of-range
+ *   stream or slot are skipped and set MSA_DEVERR_TOKEN_RANGE.  Two tokens
+ *   naming the same slot race.  n_tok == 0 is a no-op. */
+MSA_API int msa_indexer_append(const msa_shape* shape, float* idx_k_cache, const float* idx_k_new,
+                       const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok,
+                       void* stream);
+
+/* msa_kv_append - write new tokens' K and V rows ([n_tok][G][D] bf16 each)
+ * into the bf16 caches at (tok_stream[t], tok_pos[t]); same rules as
+ * msa_indexer_append.  The main K/V cache keeps the non-transposed V layout
+ * (MSA pull request, section "Requirements and fallbacks"). */
+MSA_API int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache,
+                  const msa_bf16* k_new, const msa_bf16* v_new, const int32_t* tok_stream,
+                  const int32_t* tok_pos, int32_t n_tok, void* stream);
+
+/* msa_block_scores - fused indexer score, causal mask, max-pool and local
+ * bias: block_scores[i][g][b] = max over slots j of block b with j <= q_pos[i]
+ * of idx_q[i][g] . idx_k_cache[q_stream[i]][g][j], accumulated in float32
+ * ("force F32 indexer score accum", MSA branch commit message); blocks with
+ * no visible slot are -inf; the local block q_pos[i]/128 gets
+ * + MSA_LOCAL_BIAS (MSA pull request, section "Implementation":
+ * bs = maxpool_128(idx_q*idx_k^T + causal mask) plus the local-force bias).
+ * NaN scores are treated as -inf.  An out-of-range query writes -inf
+ * everywhere and sets MSA_DEVERR_QUERY_RANGE. */
+MSA_API int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
+                     const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                     float* block_scores, void* stream);
+
+/* msa_select_topk - top-k block selection per (query, group).
+ * Ranks the visible blocks b <= q_pos/128 by (score descending, block index
+ * ascending) and keeps the first min(top_k, q_pos/128 + 1): with fewer
+ * visible blocks than top_k every visible block is taken (MSA pull request,
+ * RADV review comment: k = min(indexer_top_k, n_blocks)).  Ids are written
+ * ascending into sel, padded with -1; n_sel (may be NULL) gets the count.
+ * Equal scores go to the lower block index; NaN ranks as -inf.  A q_pos
+ * outside [0, capacity) writes an empty selection and sets
+ * MSA_DEVERR_QUERY_RANGE. */
+MSA_API int msa_select_topk(const msa_shape* shape, const float* block_scores, const int32_t* q_pos,
+                    int32_t n_q, int32_t* sel, int32_t* n_sel, void* stream);
+
+/* msa_sparse_attn_decode - block-sparse GQA attention for a few queries
+ * (decode: one new token per stream).  For query i and head h (group
+ * g = h/16): out[i][h] = softmax(softmax_scale * q[i][h] . K_j) . V_j over
+ * rows j of the blocks in sel[i][g] with j <= q_pos[i] (MSA pull request,
+ * section "Overview": attention runs only over the selected blocks; the
+ * token-level causal mask applies inside the local block).  Softmax and
+ * accumulation in float32, output rounded to bf16 (nearest even).  A query
+ * with no attended row writes zeros.  `workspace` holds split partial results
+ * and must be at least msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE)
+ * bytes (it may be NULL when that is 0). */
+MSA_API int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
+                           const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
+                           const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* msa_sparse_attn_prefill - the same computation as msa_sparse_attn_decode,
+ * for batches of many queries (prefill: every appended token is a query).
+ * MSA pull request, "Implementation", batch case: the query's block-level
+ * selection combined with the token-level causal mask.  Workspace:
+ * msa_workspace_bytes(shape, n_q, MSA_MODE_PREFILL). */
+MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
+                            const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
+                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+#define MSA_MODE_DECODE  0
+#define MSA_MODE_PREFILL 1
+
+/* Bytes of workspace the attention call of `mode` needs for n_q queries
+ * (0 when none).  Returns (size_t)-1 for an unsupported shape. */
+MSA_API size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode);
+
+/* Human-readable name of a status code (static string). */
+MSA_API const char* msa_status_string(int status);
+
+/* Wait for `stream`, then read and clear the calling thread's current
+ * device's error word into *flags (MSA_DEVERR_* bits). */
+MSA_API int msa_get_device_error(uint32_t* flags, void* stream);
+
+/* Library version, major*10000 + minor*100 + patch. */
+MSA_API int msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H */

@@ -1,0 +1,151 @@
+"""Helpers shared by the GPU parity tests: run MSA steps through the C ABI on
+seeded inputs and compare them with the CPU oracle.
+
+Comparison rules
+  * cache append, selection from identical float32 scores: bit-exact;
+  * block scores (float32 on the GPU vs float64 in the oracle): the float32
+    dot product of 128 terms, formed as 4-term FMA chains summed over a 32-lane
+    tree, rounds each term at most ~9 times, so |err| <= 9 u sum_d |q_d k_d|
+    (u = 2^-24).  The test allows 16 u times the largest such sum in the
+    block, plus exact agreement of -inf and of the local bias;
+  * end-to-end selection: ids bit-exact, except (q, g) pairs whose oracle
+    ranks top_k and top_k+1 are within 1e-5 relative (and not exactly equal);
+    those are counted and the attention is checked with the GPU's selection;
+  * attention (bf16 out vs float64): elementwise |got - bf16(want)| <=
+    max(4e-3, one bf16 ulp of want), and mean |got - want| <= 5e-4.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+import block_sparse_attention_maxpool_b200 as msa
+import oracle
+from tests.oracle_pins import near_tie_excused
+
+U32 = 2.0 ** -24
+ATTN_MAX_ABS = 4e-3
+ATTN_MEAN_ABS = 5e-4
+
+
+def shape_of(w) -> msa.Shape:
+    return msa.Shape(n_streams=w.n_streams, capacity=w.capacity, n_q_heads=w.n_q_heads,
+                     n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, idx_dim=w.idx_dim,
+                     block=w.block, top_k=w.top_k)
+
+
+def to_dev(inp, dev="cuda"):
+    names = ["idx_k_cache", "k_cache", "v_cache", "tok_stream", "tok_pos", "idx_k_new", "k_new",
+             "v_new", "q_stream", "q_pos", "idx_q", "q"]
+    return {n: getattr(inp, n).to(dev).contiguous() for n in names}
+
+
+def run_step(shape, d, prefill=False):
+    caches = {k: d[k] for k in ("idx_k_cache", "k_cache", "v_cache")}
+    out, sel, n_sel, bs = msa.decode_step(shape, caches, d, prefill=prefill)
+    err = msa.msa_get_device_error()
+    return out, sel, n_sel, bs, err
+
+
+def oracle_caches(inp):
+    idx = oracle.indexer_append(inp.idx_k_cache, inp.idx_k_new, inp.tok_stream, inp.tok_pos)
+    k = oracle.indexer_append(inp.k_cache, inp.k_new, inp.tok_stream, inp.tok_pos)
+    v = oracle.indexer_append(inp.v_cache, inp.v_new, inp.tok_stream, inp.tok_pos)
+    return idx, k, v
+
+
+def score_bounds(idx_q, idx_k_cache, q_stream, q_pos, block):
+    """Per (query, group, block): 16 u max_j sum_d |q_d k_jd| over visible j."""
+    n_q, G = idx_q.shape[0], idx_q.shape[1]
+    nblk = idx_k_cache.shape[2] // block
+    out = torch.zeros((n_q, G, nblk), dtype=torch.float64)
+    for i in range(n_q):
+        s, p = int(q_stream[i]), int(q_pos[i])
+        for g in range(G):
+            a = idx_k_cache[s, g, :p + 1].double().abs() @ idx_q[i, g].double().abs()
+            nb = p // block + 1
+            pad = torch.full((nb * block,), 0.0, dtype=torch.float64)
+            pad[:p + 1] = a
+            out[i, g, :nb] = 16 * U32 * pad.view(nb, block).amax(dim=1)
+    return out
+
+
+def check_scores(bs_gpu, bs_orc, bounds):
+    g = bs_gpu.double()
+    inf_g, inf_o = torch.isinf(g) & (g < 0), torch.isinf(bs_orc) & (bs_orc < 0)
+    assert torch.equal(inf_g, inf_o), "-inf pattern differs"
+    fin = ~inf_o
+    big = bs_orc >= oracle.LOCAL_BIAS / 2
+    assert torch.equal(g[big], bs_orc[big]), "local bias differs"
+    small = fin & ~big
+    err = (g[small] - bs_orc[small]).abs()
+    ok = err <= bounds[small] + 1e-30
+    assert bool(ok.all()), f"block score error {err.max():.3e} above bound"
+    return float(err.max()) if err.numel() else 0.0
+
+
+def check_selection(sel_gpu, nsel_gpu, bs_orc, q_pos, block, top_k):
+    """Returns (merged sel for the attention check, number of excused near-ties)."""
+    sel_o, nsel_o = oracle.select_blocks(bs_orc, q_pos, block, top_k)
+    merged = sel_o.clone()
+    excused = 0
+    n_q, G = sel_o.shape[0], sel_o.shape[1]
+    mism = (sel_gpu != sel_o).any(dim=2) | (nsel_gpu != nsel_o)
+    for i, g in mism.nonzero().tolist():
+        p = int(q_pos[i])
+        got = [b for b in sel_gpu[i, g].tolist() if b >= 0]
+        want = [b for b in sel_o[i, g].tolist() if b >= 0]
+        bnd = oracle.boundary_scores(bs_orc[i, g], p, block, top_k)
+        assert near_tie_excused(bnd, bs_orc[i, g], got, want), \
+            f"selection differs at query {i} group {g}: gpu {got} oracle {want} boundary {bnd}"
+        assert len(got) == len(want) and got == sorted(got)
+        merged[i, g] = sel_gpu[i, g]
+        excused += 1
+    return merged, excused
+
+
+def bf16_ulp(x: torch.Tensor) -> torch.Tensor:
+    a = x.abs().clamp_min(2.0 ** -126)
+    return torch.exp2(torch.floor(torch.log2(a)) - 7)
+
+
+def check_attention(out_gpu, out_orc, rows=None):
+    g = out_gpu.double()
+    w = out_orc
+    if rows is not None:
+        g, w = g[rows], w[rows]
+    w_bf = w.to(torch.bfloat16).double()
+    tol = torch.maximum(torch.full_like(w, ATTN_MAX_ABS), bf16_ulp(w))
+    d = (g - w_bf).abs()
+    bad = d > tol
+    assert not bool(bad.any()), f"attention max err {d.max():.3e} (tol {tol[bad].min():.3e}) at {bad.nonzero()[0].tolist()}"
+    mean = float((g - w).abs().mean())
+    assert mean <= ATTN_MEAN_ABS, f"attention mean abs err {mean:.3e}"
+    return float((g - w).abs().max()), mean
+
+
+def full_parity(inp, queries=None, prefill=False, dev="cuda"):
+    """Run one step on the GPU and compare every part with the oracle on the
+    query indices ``queries`` (all when None).  Returns a small report."""
+    w = inp.w
+    shape = shape_of(w)
+    d = to_dev(inp, dev)
+    out, sel, n_sel, bs, err = run_step(shape, d, prefill)
+    assert err == 0, f"device error word {err:#x}"
+    idx_o, k_o, v_o = oracle_caches(inp)
+    assert torch.equal(d["idx_k_cache"].cpu(), idx_o), "indexer cache after append"
+    assert torch.equal(d["k_cache"].cpu(), k_o) and torch.equal(d["v_cache"].cpu(), v_o), "K/V append"
+    n_q = inp.q_pos.numel()
+    qsub = torch.arange(n_q) if queries is None else torch.as_tensor(queries, dtype=torch.long)
+    qs, qp = inp.q_stream[qsub], inp.q_pos[qsub]
+    bs_o = oracle.block_scores(inp.idx_q[qsub], idx_o, qs, qp, w.block)
+    bounds = score_bounds(inp.idx_q[qsub], idx_o, qs, qp, w.block)
+    bs_g, sel_g, nsel_g, out_g = bs.cpu()[qsub], sel.cpu()[qsub], n_sel.cpu()[qsub], out.cpu()[qsub]
+    max_score_err = check_scores(bs_g, bs_o, bounds)
+    merged, excused = check_selection(sel_g, nsel_g, bs_o, qp, w.block, w.top_k)
+    out_o = oracle.sparse_attention(inp.q[qsub], k_o, v_o, merged, qs, qp, w.block,
+                                    1.0 / math.sqrt(w.head_dim))
+    max_err, mean_err = check_attention(out_g, out_o)
+    return dict(queries=len(qsub), near_ties=excused, max_score_err=max_score_err,
+                attn_max_abs=max_err, attn_mean_abs=mean_err)

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/msa.h declares, and rejects bad arguments with the
+documented status codes before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_maxpool_b200 as msa
+from block_sparse_attention_maxpool_b200 import build as msa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    msa_build.build()
+    return msa.library()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MSA_API\s+[\w\s\*]+?\b(msa_\w+)\s*\(", text)))
+
+
+def header_constants():
+    text = open(HEADER).read()
+    return {m[0]: int(m[1]) for m in re.findall(r"#define\s+(MSA_(?:OK|ERR_\w+))\s+\(?(-?\d+)\)?", text)}
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ("msa_indexer_append", "msa_block_scores", "msa_select_topk",
+                 "msa_sparse_attn_decode", "msa_sparse_attn_prefill"):
+        assert name in fns
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_status_table_matches_header():
+    consts = header_constants()
+    for name, value in consts.items():
+        assert msa.STATUS[value] == name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.msa_version() >= 100
+    assert lib.msa_status_string(0) == b"MSA_OK"
+    assert lib.msa_status_string(-5).startswith(b"MSA_ERR_WORKSPACE")
+
+
+GOOD = msa.Shape(n_streams=2, capacity=1024)
+FAKE = 0x10000          # a 16-byte aligned address that is never dereferenced
+
+
+def call_scores(lib, shape, n_q=4, **over):
+    a = dict(idx_q=FAKE, idx_k=FAKE, qs=FAKE, qp=FAKE, bs=FAKE)
+    a.update(over)
+    s = shape.c()
+    return lib.msa_block_scores(ctypes.byref(s), a["idx_q"], a["idx_k"], a["qs"], a["qp"], n_q,
+                                a["bs"], None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(capacity=1000), dict(capacity=0), dict(n_streams=0), dict(head_dim=64), dict(idx_dim=64),
+    dict(block=64), dict(top_k=8), dict(n_q_heads=32), dict(n_kv_heads=0), dict(n_kv_heads=17, n_q_heads=272),
+    dict(n_streams=4096, capacity=1 << 20),
+])
+def test_shape_rejected(lib, bad):
+    sh = msa.Shape(**{**GOOD.__dict__, **bad})
+    assert call_scores(lib, sh) == -3
+
+
+def test_null_and_alignment(lib):
+    assert lib.msa_block_scores(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == -1
+    assert call_scores(lib, GOOD, idx_k=0) == -1
+    assert call_scores(lib, GOOD, bs=0) == -1
+    assert call_scores(lib, GOOD, idx_q=FAKE + 4) == -2
+    assert call_scores(lib, GOOD, n_q=-1) == -4
+    assert call_scores(lib, GOOD, n_q=0, idx_q=0, idx_k=0) == 0      # empty batch is a no-op
+
+
+def test_select_and_append_validation(lib):
+    s = GOOD.c()
+    assert lib.msa_select_topk(ctypes.byref(s), FAKE, FAKE, 3, 0, 0, None) == -1
+    assert lib.msa_select_topk(ctypes.byref(s), FAKE + 8, FAKE, 3, FAKE, 0, None) == -2
+    assert lib.msa_select_topk(ctypes.byref(s), FAKE, FAKE, 0, 0, 0, None) == 0
+    assert lib.msa_indexer_append(ctypes.byref(s), FAKE, FAKE, FAKE, 0, 2, None) == -1
+    assert lib.msa_indexer_append(ctypes.byref(s), FAKE + 4, FAKE, FAKE, FAKE, 2, None) == -2
+    assert lib.msa_indexer_append(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, -2, None) == -4
+    assert lib.msa_kv_append(ctypes.byref(s), FAKE, 0, FAKE, FAKE, FAKE, FAKE, 2, None) == -1
+    assert lib.msa_kv_append(ctypes.byref(s), 0, 0, 0, 0, 0, 0, 0, None) == 0
+
+
+def test_attention_validation_and_workspace(lib):
+    s = GOOD.c()
+    # decode with 2 queries x 4 groups = 8 pairs needs split workspace
+    need = lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_DECODE)
+    assert need == 8 * 16 * 16 * 130 * 4
+    assert lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_PREFILL) == 0
+    assert lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_DECODE) == 0
+    bad = msa.Shape(n_streams=2, capacity=1000).c()
+    assert lib.msa_workspace_bytes(ctypes.byref(bad), 2, 0) == ctypes.c_size_t(-1).value
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, ctypes.c_float(0.088), FAKE]
+    assert lib.msa_sparse_attn_decode(ctypes.byref(s), *args, 0, 0, None) == -5
+    assert lib.msa_sparse_attn_decode(ctypes.byref(s), *args, FAKE, need - 1, None) == -5
+    assert lib.msa_sparse_attn_decode(ctypes.byref(s), *args, FAKE + 4, need, None) == -2
+    nan_args = list(args)
+    nan_args[7] = ctypes.c_float(float("nan"))
+    assert lib.msa_sparse_attn_decode(ctypes.byref(s), *nan_args, FAKE, need, None) == -4
+    null_args = list(args)
+    null_args[1] = 0
+    assert lib.msa_sparse_attn_prefill(ctypes.byref(s), *null_args, 0, 0, None) == -1
+    assert lib.msa_sparse_attn_prefill(ctypes.byref(s), *args[:6], 0, args[7], FAKE, 0, 0, None) == 0
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    sh = msa.Shape(n_streams=1, capacity=128)
+    with pytest.raises(ValueError):
+        msa.msa_select_topk(sh, torch.zeros((1, 4, 1)), torch.zeros(1, dtype=torch.int32),
+                            sel=torch.zeros((1, 4, 16), dtype=torch.int32),
+                            n_sel=torch.zeros((1, 4), dtype=torch.int32), stream=0)

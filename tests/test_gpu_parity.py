@@ -1,0 +1,251 @@
+"""GPU parity of every step of the MSA hot path against the CPU oracle, through
+the C ABI: cache append, block scores, top-k selection, block-sparse
+attention, and the whole step on small ragged cases and on the five
+benchmark workloads (full size, sampled where the oracle would be slow)."""
+import math
+
+import pytest
+import torch
+
+import block_sparse_attention_maxpool_b200 as msa
+import oracle
+import workloads as W
+from block_sparse_attention_maxpool_b200 import build as msa_build
+from tests import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    msa_build.build()
+    msa.msa_get_device_error()          # clear leftovers
+    yield
+    torch.cuda.synchronize()
+
+
+def report(name, rep):
+    print(f"\n[parity] {name}: {rep}")
+
+
+# ---------------------------------------------------------------------------
+# step by step
+# ---------------------------------------------------------------------------
+def test_append_bit_exact_and_range_errors():
+    g = torch.Generator().manual_seed(11)
+    sh = msa.Shape(n_streams=3, capacity=384, n_kv_heads=2, n_q_heads=32)
+    idx = torch.randn((3, 2, 384, 128), generator=g)
+    k = torch.randn((3, 2, 384, 128), generator=g).to(torch.bfloat16)
+    v = torch.randn((3, 2, 384, 128), generator=g).to(torch.bfloat16)
+    n = 50
+    ts = torch.randint(0, 3, (n,), generator=g, dtype=torch.int32)
+    tp = torch.randperm(384, generator=g)[:n].to(torch.int32)
+    new_i = torch.randn((n, 2, 128), generator=g)
+    new_k = torch.randn((n, 2, 128), generator=g).to(torch.bfloat16)
+    new_v = torch.randn((n, 2, 128), generator=g).to(torch.bfloat16)
+    di, dk, dv = idx.cuda(), k.cuda(), v.cuda()
+    msa.msa_indexer_append(sh, di, new_i.cuda(), ts.cuda(), tp.cuda())
+    msa.msa_kv_append(sh, dk, dv, new_k.cuda(), new_v.cuda(), ts.cuda(), tp.cuda())
+    assert msa.msa_get_device_error() == 0
+    assert torch.equal(di.cpu(), oracle.indexer_append(idx, new_i, ts, tp))
+    assert torch.equal(dk.cpu(), oracle.indexer_append(k, new_k, ts, tp))
+    assert torch.equal(dv.cpu(), oracle.indexer_append(v, new_v, ts, tp))
+    # out-of-range tokens are skipped and reported
+    bad_s = torch.tensor([3, 0], dtype=torch.int32).cuda()
+    bad_p = torch.tensor([0, 384], dtype=torch.int32).cuda()
+    before = di.clone()
+    msa.msa_indexer_append(sh, di, new_i[:2].cuda(), bad_s, bad_p)
+    assert msa.msa_get_device_error() & 0x2
+    assert torch.equal(di, before)
+
+
+def _rand_scores(g, n_q, G, nblk, q_pos, ties):
+    bs = torch.randn((n_q, G, nblk), generator=g)
+    if ties:
+        bs = torch.round(bs * 2) / 2          # many exact ties, both signs of zero
+    for i in range(n_q):
+        p = int(q_pos[i])
+        bs[i, :, p // 128 + 1:] = float("-inf")
+        bs[i, :, p // 128] += 2.0 ** 100
+    return bs
+
+
+@pytest.mark.parametrize("nblk", [1, 9, 200, 256, 600, 1024, 1500])
+@pytest.mark.parametrize("ties", [False, True])
+def test_select_bit_exact_from_identical_scores(nblk, ties):
+    g = torch.Generator().manual_seed(nblk * 2 + ties)
+    cap = nblk * 128
+    G, n_q = 4, 40
+    q_pos = torch.randint(0, cap, (n_q,), generator=g, dtype=torch.int32)
+    q_pos[0], q_pos[1] = cap - 1, 0
+    q_pos[2] = min(cap - 1, 15 * 128 + 5)     # exactly 16 visible blocks
+    q_pos[3] = min(cap - 1, 16 * 128)         # 17 visible blocks
+    bs = _rand_scores(g, n_q, G, nblk, q_pos, ties)
+    sh = msa.Shape(n_streams=1, capacity=cap)
+    sel, n_sel = msa.msa_select_topk(sh, bs.cuda(), q_pos.cuda())
+    assert msa.msa_get_device_error() == 0
+    sel_o, nsel_o = oracle.select_blocks(bs.double(), q_pos, 128, 16)
+    assert torch.equal(sel.cpu(), sel_o)
+    assert torch.equal(n_sel.cpu(), nsel_o)
+
+
+def test_select_nan_ranks_last_and_bad_positions():
+    sh = msa.Shape(n_streams=1, capacity=128 * 40)
+    bs = torch.zeros((2, 4, 40))
+    bs[:, :, 0] = float("nan")
+    bs[:, :, 39] += 2.0 ** 100
+    q_pos = torch.tensor([128 * 40 - 1, 128 * 40], dtype=torch.int32)   # second is out of range
+    sel, n_sel = msa.msa_select_topk(sh, bs.cuda(), q_pos.cuda())
+    assert msa.msa_get_device_error() & 0x1
+    sel = sel.cpu()
+    assert 0 not in sel[0, 0].tolist()             # the NaN block loses to every finite one
+    assert sel[0, 0].tolist() == list(range(1, 16)) + [39]
+    assert sel[1].eq(-1).all() and n_sel.cpu()[1].eq(0).all()
+
+
+def _random_selection(g, q_pos, G, top_k=16):
+    n_q = q_pos.numel()
+    sel = torch.full((n_q, G, top_k), -1, dtype=torch.int32)
+    for i in range(n_q):
+        p = int(q_pos[i])
+        nvis = p // 128 + 1
+        for gg in range(G):
+            k = int(torch.randint(1, min(top_k, nvis) + 1, (1,), generator=g))
+            others = torch.randperm(nvis - 1, generator=g)[:k - 1].tolist() if nvis > 1 else []
+            ids = sorted(set(others) | {nvis - 1})
+            sel[i, gg, :len(ids)] = torch.tensor(ids, dtype=torch.int32)
+    return sel
+
+
+@pytest.mark.parametrize("n_q,mode", [(1, "decode"), (3, "decode"), (20, "decode"), (40, "decode"),
+                                      (70, "decode"), (150, "decode"), (37, "prefill")])
+def test_attention_given_selection(n_q, mode):
+    g = torch.Generator().manual_seed(n_q)
+    S, cap, G = 3, 128 * 24, 4
+    lengths = [cap, 1000, 129]
+    qpos = []
+    for i in range(n_q):
+        s = i % S
+        qpos.append((s, int(torch.randint(0, lengths[s], (1,), generator=g))))
+    qpos[0] = (0, cap - 1)
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, lengths, qpos, seed=n_q)
+    sel = _random_selection(g, qp, G)
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    fn = msa.msa_sparse_attn_decode if mode == "decode" else msa.msa_sparse_attn_prefill
+    out = fn(sh, q.cuda(), k.cuda(), v.cuda(), sel.cuda(), qs.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() == 0
+    want = oracle.sparse_attention(q, k, v, sel, qs, qp, 128, 1 / math.sqrt(128))
+    report(f"attention n_q={n_q} {mode}", PT.check_attention(out.cpu(), want))
+
+
+def test_attention_empty_and_invalid_selection():
+    S, cap = 1, 512
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, [512], [(0, 300), (0, 100)], seed=5)
+    sel = torch.full((2, 4, 16), -1, dtype=torch.int32)
+    sel[0, :, 0] = 2
+    sel[0, 1, 1] = 3                 # block 3 starts past position 300: invalid, skipped
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    out = msa.msa_sparse_attn_decode(sh, q.cuda(), k.cuda(), v.cuda(), sel.cuda(), qs.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() & 0x4
+    sel_clean = sel.clone()
+    sel_clean[0, 1, 1] = -1
+    want = oracle.sparse_attention(q, k, v, sel_clean, qs, qp, 128)
+    want[1] = 0.0                    # query 1 has an empty selection: zeros
+    PT.check_attention(out.cpu(), want)
+
+
+def test_block_scores_ragged_multi_stream():
+    S, cap = 3, 128 * 10
+    lengths = [cap, 700, 129]
+    qpos = [(0, 0), (0, 127), (0, 128), (0, 129), (0, cap - 1), (1, 699), (1, 383), (2, 128), (2, 5),
+            (1, 256), (0, 640), (0, 1000)]
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, lengths, qpos, seed=3)
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    bs = msa.msa_block_scores(sh, iq.cuda(), idx.cuda(), qs.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() == 0
+    bs_o = oracle.block_scores(iq, idx, qs, qp, 128)
+    PT.check_scores(bs.cpu(), bs_o, PT.score_bounds(iq, idx, qs, qp, 128))
+
+
+def test_block_scores_out_of_range_query():
+    sh = msa.Shape(n_streams=1, capacity=256)
+    idx, k, v, qs, qp, iq, q = W.make_custom(1, 256, [256], [(0, 10), (0, 10)], seed=4)
+    qs[1] = 1                        # stream 1 does not exist
+    bs = msa.msa_block_scores(sh, iq.cuda(), idx.cuda(), qs.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() & 0x1
+    bs = bs.cpu()
+    assert torch.isinf(bs[1]).all() and (bs[1] < 0).all()
+    assert torch.isfinite(bs[0, :, 0]).all()
+
+
+# ---------------------------------------------------------------------------
+# whole step
+# ---------------------------------------------------------------------------
+def test_step_small_prefill_ragged_tail():
+    w = W.Workload("prefill_1x2500", 1, 0, 2500, "new")
+    inp = W.make_inputs(w, seed=1)
+    q = list(range(0, 2500, 7)) + [2047, 2048, 2049, 2499]
+    report(w.name, PT.full_parity(inp, queries=q, prefill=True))
+
+
+def test_step_small_chunked_prefill_with_ties():
+    w = W.Workload("chunk_2x600_on_2000_ties", 2, 2000, 2600, "new", quantize_idx=True)
+    inp = W.make_inputs(w, seed=2)
+    rep = PT.full_parity(inp, prefill=True)
+    report(w.name, rep)
+    assert rep["near_ties"] == 0          # quantised scores are exact in float32: no excuses
+
+
+def test_step_decode_mixed_streams():
+    w = W.Workload("decode_6x3000", 6, 2999, 3000, "last")
+    report(w.name, PT.full_parity(W.make_inputs(w, seed=3)))
+
+
+def test_step_is_deterministic():
+    w = W.Workload("decode_4x2200", 4, 2199, 2200, "last")
+    inp = W.make_inputs(w, seed=4)
+    sh = PT.shape_of(w)
+    outs = []
+    for _ in range(2):
+        d = PT.to_dev(inp)
+        out, sel, n_sel, bs, err = PT.run_step(sh, d)
+        outs.append((out.cpu(), sel.cpu(), bs.cpu()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# the five benchmark workloads at full size
+# ---------------------------------------------------------------------------
+def test_workload_decode_1x4k_full():
+    report(W.DECODE_4K.name, PT.full_parity(W.make_inputs(W.DECODE_4K)))
+
+
+def test_workload_decode_32x32k_sampled():
+    inp = W.make_inputs(W.DECODE_32K_X32)
+    report(W.DECODE_32K_X32.name, PT.full_parity(inp, queries=[0, 7, 19, 31]))
+
+
+def test_workload_decode_8x128k_sampled():
+    inp = W.make_inputs(W.DECODE_128K_X8)
+    report(W.DECODE_128K_X8.name, PT.full_parity(inp, queries=[0, 5]))
+
+
+def test_workload_prefill_16k_sampled():
+    inp = W.make_inputs(W.PREFILL_16K)
+    g = torch.Generator().manual_seed(7)
+    q = sorted(set([0, 1, 2, 127, 128, 129, 2046, 2047, 2048, 2049, 4095, 4096, 8191, 16383]
+                   + torch.randint(0, 16384, (36,), generator=g).tolist()))
+    report(W.PREFILL_16K.name, PT.full_parity(inp, queries=q, prefill=True))
+
+
+def test_workload_chunked_prefill_ties_sampled():
+    inp = W.make_inputs(W.CHUNKED_PREFILL_TIES)
+    g = torch.Generator().manual_seed(8)
+    q = sorted(set([0, 1, 2047, 2048, 4095, 6143, 8191]
+                   + torch.randint(0, 8192, (25,), generator=g).tolist()))
+    rep = PT.full_parity(inp, queries=q, prefill=True)
+    report(W.CHUNKED_PREFILL_TIES.name, rep)
+    assert rep["near_ties"] == 0
