@@ -41,10 +41,13 @@ import workloads as W  # noqa: E402
 METRIC = "MSA decode tokens/s @32K ctx x32 streams; achieved HBM GB/s vs peak"
 WORKLOAD = W.DECODE_32K_X32
 
-# DRAM traffic of one block-scores launch on this workload, from the ncu
-# capture summarised in profiles/, valid only for the kernel source it was
-# taken on (sha256 prefix of msa_scores_gemv.cuh).
-SCORES_TRAFFIC = {"source_sha": None, "bytes_per_launch": None}
+# DRAM traffic of one block-scores launch on the 32-stream workload, from
+# the ncu capture summarised in profiles/block_scores_gemv_decode_8x32k.md:
+# 536,909,056 B read + 4,248,576 B written on 8 streams, scaled by 4 to 32
+# streams (the reads grow in proportion to the keys scanned).  Valid only
+# for the kernel source it was taken on (sha256 prefix of
+# msa_scores_gemv.cuh); any other source reports null.
+SCORES_TRAFFIC = {"source_sha": "c741d20f2bada528", "bytes_per_launch": 4 * (536_909_056 + 4_248_576)}
 
 
 def scores_source_sha() -> str:
@@ -145,6 +148,8 @@ def run_ours(args, rank, world, dev):
     if world > 1:
         torch.distributed.barrier(device_ids=[dev])
     w = WORKLOAD
+    if args.streams != w.n_streams:      # smaller case for profiler captures
+        w = W.Workload(f"decode_{args.streams}x32k", args.streams, w.l_existing, w.l_total, "last")
     shape = msa.Shape(n_streams=w.n_streams, capacity=w.capacity)
     inp = W.make_inputs(w, seed=rank)                    # each rank: its own 32 streams
     d = {n: getattr(inp, n).to(dev) for n in ("idx_k_cache", "k_cache", "v_cache", "tok_stream",
@@ -260,7 +265,7 @@ def run_ours(args, rank, world, dev):
         "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "context": w.l_total,
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                    "block": w.block, "top_k": w.top_k, "parallelism": f"replicas{world}",
-                   "l2": "inputs 4.2 GB per GPU > 126 MB L2, no flush"},
+                   "l2": f"inputs {2 * w.n_streams * w.capacity * w.n_kv_heads * 512 / 1e9:.1f} GB per GPU > 126 MB L2, no flush"},
         "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peaks["hbm_gbs"],
                      "frac": step_gbs / peaks["hbm_gbs"], "bytes_per_step": step_bytes(w)},
         "roofline": {"kernel": "block_scores_gemv", "bound": "hbm", "achieved": achieved,
@@ -340,6 +345,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--streams", type=int, default=WORKLOAD.n_streams,
+                    help="decode streams per GPU (32 = the benchmark workload; fewer for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
