@@ -19,7 +19,7 @@ import torch
 
 __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_block_scores",
            "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
-           "msa_workspace_bytes", "msa_get_device_error", "msa_version", "library", "LIB_PATH",
+           "msa_workspace_bytes", "msa_get_device_error", "msa_sparse_attn_decode_noalloc", "msa_version", "library", "LIB_PATH",
            "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
@@ -78,6 +78,8 @@ _SIGS = {
                                               ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "msa_sparse_attn_prefill": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
                                                ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_sparse_attn_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P,
+                                                      _I, ctypes.c_float, _P, _P]),
     "msa_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(CShape), _I, _I]),
     "msa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "msa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -232,6 +234,33 @@ def msa_sparse_attn_prefill(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_
                             out=None, workspace=None, stream=None):
     return _attn("msa_sparse_attn_prefill", MODE_PREFILL, shape, q, k_cache, v_cache, sel, q_stream,
                  q_pos, softmax_scale, out, workspace, stream)
+
+
+NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def msa_sparse_attn_decode_noalloc(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos,
+                                   softmax_scale=None, out=None, stream=None):
+    """Decode attention for callers that cannot allocate device memory: the
+    split partials go to the library's fixed 8 MiB device buffer instead of
+    a workspace.  ``out`` is still the caller's (allocated here only when
+    None, for convenience).  Calls sharing the buffer at the same time on the
+    GPU race; see include/msa.h."""
+    n = _n(q_pos, "q_pos")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(shape.head_dim)
+    if out is None:
+        out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=q.device)
+    cs = (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.head_dim)
+    s = shape.c()
+    _check("msa_sparse_attn_decode_noalloc", library().msa_sparse_attn_decode_noalloc(
+        ctypes.byref(s), _ptr(q, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
+        _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+        _ptr(sel, torch.int32, (n, shape.n_kv_heads, shape.top_k), "sel"),
+        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+        float(softmax_scale), _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"),
+        _stream(stream)))
+    return out
 
 
 def msa_get_device_error(stream=None) -> int:

@@ -278,6 +278,54 @@ int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, const msa
                      workspace_bytes, stream, MSA_MODE_PREFILL);
 }
 
+// ---- attention without a caller workspace ----------------------------------
+// File-scope scratch for msa_sparse_attn_decode_noalloc.  In host code the
+// name is only a stand-in for the symbol: its device address is looked up
+// once per device with cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MSA_NOALLOC_SCRATCH_BYTES];
+
+}  // extern "C"
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {};
+
+int noalloc_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return MSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
+                                   const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
+                                   const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
+                                   void* stream) {
+  const int st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0) return MSA_OK;
+  const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
+  const size_t need = attn_workspace(n_pairs, attn_splits(n_pairs, MSA_MODE_DECODE));
+  if (need > MSA_NOALLOC_SCRATCH_BYTES) return MSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    const int s2 = noalloc_scratch(&scratch);
+    if (s2 != MSA_OK) return s2;
+  }
+  return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, scratch,
+                     MSA_NOALLOC_SCRATCH_BYTES, stream, MSA_MODE_DECODE);
+}
+
 size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {
   if (check_shape(shape) != MSA_OK || n_q < 0 || (mode != MSA_MODE_DECODE && mode != MSA_MODE_PREFILL))
     return static_cast<size_t>(-1);

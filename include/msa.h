@@ -166,6 +166,34 @@ MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, c
 #define MSA_MODE_DECODE  0
 #define MSA_MODE_PREFILL 1
 
+/* Size of the fixed device buffer used by msa_sparse_attn_decode_noalloc. */
+#define MSA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/* msa_sparse_attn_decode_noalloc - msa_sparse_attn_decode without a
+ * caller-provided workspace.  The pages describe no such call; it exists for
+ * callers that cannot allocate device memory when they run attention, for
+ * example a runtime whose device memory is all handed out by a pool sized at
+ * start-up, or a program driving the C ABI from a language that has no CUDA
+ * allocator of its own.  Such a caller still owns q, the caches, sel and out.
+ *
+ * The split partial results go to one file-scope device buffer of
+ * MSA_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
+ * the process exits.  A call whose msa_workspace_bytes(shape, n_q,
+ * MSA_MODE_DECODE) exceeds that size is rejected with MSA_ERR_WORKSPACE
+ * (with 4 groups only n_q = 127 needs more).  The first call on each
+ * device looks up the buffer's device address (with that device current);
+ * make that first call before any stream capture.  All calls share the
+ * buffer: calls that can run at the same time on the GPU (different streams,
+ * or different host threads on one device) race and must be serialised by
+ * the caller.  Nothing in the buffer needs to start at zero: every call
+ * writes each partial it reads.  Allocates nothing, on the host or the
+ * device. */
+MSA_API int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf16* q,
+                                           const msa_bf16* k_cache, const msa_bf16* v_cache,
+                                           const int32_t* sel, const int32_t* q_stream,
+                                           const int32_t* q_pos, int32_t n_q, float softmax_scale,
+                                           msa_bf16* out, void* stream);
+
 /* Bytes of workspace the attention call of `mode` needs for n_q queries
  * (0 when none).  Returns (size_t)-1 for an unsupported shape. */
 MSA_API size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode);

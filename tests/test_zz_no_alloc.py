@@ -1,0 +1,61 @@
+"""msa_sparse_attn_decode_noalloc: decode attention for callers that cannot
+allocate device memory when they run attention (a runtime whose device
+memory all belongs to a pool sized at start-up, or a program using the C ABI
+from a language with no CUDA allocator).  Instead of a caller workspace it
+uses the library's fixed file-scope device buffer.
+
+The GPU test calls the new entry point through the C ABI twice in a row, with
+different batch sizes (so the second call runs over the first call's leftover
+buffer contents), and checks each output against the workspace entry point
+msa_sparse_attn_decode within the attention tolerance of the parity tests.
+This file is collected last so a failure here never hides another test."""
+import ctypes
+
+import pytest
+import torch
+
+import block_sparse_attention_maxpool_b200 as msa
+import workloads as W
+from block_sparse_attention_maxpool_b200 import build as msa_build
+from tests import parity as PT
+
+
+def test_noalloc_rejects_batches_beyond_the_fixed_buffer():
+    """Host-side size check (no GPU needed): 127 queries x 4 groups need
+    8,453,120 bytes of split partials, more than the 8 MiB buffer."""
+    msa_build.build()
+    lib = msa.library()
+    sh = msa.Shape(n_streams=1, capacity=4096)
+    s = sh.c()
+    assert lib.msa_workspace_bytes(ctypes.byref(s), 127, msa.MODE_DECODE) > msa.NOALLOC_SCRATCH_BYTES
+    fake = 0x10000
+    st = lib.msa_sparse_attn_decode_noalloc(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 127,
+                                            ctypes.c_float(0.088), fake, None)
+    assert st == -5
+    bad = msa.Shape(n_streams=1, capacity=1000).c()
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(bad), fake, fake, fake, fake, fake, fake, 1,
+                                              ctypes.c_float(0.088), fake, None) == -3
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    msa_build.build()
+    for call, (n_streams, ctx, seed) in enumerate(((32, 3000, 31), (5, 2600, 32))):
+        w = W.Workload(f"noalloc_{n_streams}x{ctx}", n_streams, ctx - 1, ctx, "last")
+        inp = W.make_inputs(w, seed=seed)
+        shape = PT.shape_of(w)
+        d = PT.to_dev(inp)
+        caches = {k: d[k] for k in ("idx_k_cache", "k_cache", "v_cache")}
+        out_ws, sel, n_sel, bs = msa.decode_step(shape, caches, d)      # workspace entry point
+        assert msa.msa_workspace_bytes(shape, w.n_queries, msa.MODE_DECODE) > 0   # split path used
+        out_na = torch.full_like(out_ws, float("nan"))
+        msa.msa_sparse_attn_decode_noalloc(shape, d["q"], d["k_cache"], d["v_cache"], sel, d["q_stream"],
+                                           d["q_pos"], out=out_na)
+        assert msa.msa_get_device_error() == 0
+        a, b = out_na.cpu().double(), out_ws.cpu().double()
+        assert torch.isfinite(a).all(), f"call {call}: output not fully written"
+        diff = (a - b).abs()
+        assert float(diff.max()) <= PT.ATTN_MAX_ABS, f"call {call}: max abs diff {float(diff.max())}"
+        assert float(diff.mean()) <= PT.ATTN_MEAN_ABS, f"call {call}: mean abs diff {float(diff.mean())}"
