@@ -147,9 +147,11 @@ def run_ours(args, rank, world, dev):
         msa_build.build()
     if world > 1:
         torch.distributed.barrier(device_ids=[dev])
-    w = WORKLOAD
-    if args.streams != w.n_streams:      # smaller case for profiler captures
-        w = W.Workload(f"decode_{args.streams}x32k", args.streams, w.l_existing, w.l_total, "last")
+    w = W.WORKLOADS[args.workload]
+    if args.streams is not None and args.streams != w.n_streams:    # smaller case for profiler captures
+        w = W.Workload(f"{w.name}_{args.streams}streams", args.streams, w.l_existing, w.l_total, w.queries,
+                       quantize_idx=w.quantize_idx)
+    prefill = w.queries == "new"
     shape = msa.Shape(n_streams=w.n_streams, capacity=w.capacity)
     inp = W.make_inputs(w, seed=rank)                    # each rank: its own 32 streams
     d = {n: getattr(inp, n).to(dev) for n in ("idx_k_cache", "k_cache", "v_cache", "tok_stream",
@@ -164,7 +166,8 @@ def run_ours(args, rank, world, dev):
         "n_sel": torch.empty((n_q, G), dtype=torch.int32, device=dev),
         "out": torch.empty((n_q, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=dev),
     }
-    ws = msa.msa_workspace_bytes(shape, n_q, msa.MODE_DECODE)
+    mode = msa.MODE_PREFILL if prefill else msa.MODE_DECODE
+    ws = msa.msa_workspace_bytes(shape, n_q, mode)
     bufs["workspace"] = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
     launches_per_step = 5 + (1 if ws > 0 else 0)
     stream = torch.cuda.current_stream(dev)
@@ -177,12 +180,13 @@ def run_ours(args, rank, world, dev):
         if ev is not None:
             ev[0].record(stream)
         msa.msa_block_scores(shape, d["idx_q"], d["idx_k_cache"], d["q_stream"], d["q_pos"],
-                             bufs["block_scores"], stream)
+                             bufs["block_scores"], stream, bufs["workspace"])
         if ev is not None:
             ev[1].record(stream)
         msa.msa_select_topk(shape, bufs["block_scores"], d["q_pos"], bufs["sel"], bufs["n_sel"], stream)
-        msa.msa_sparse_attn_decode(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"],
-                                   d["q_pos"], scale, bufs["out"], bufs["workspace"], stream)
+        attn = msa.msa_sparse_attn_prefill if prefill else msa.msa_sparse_attn_decode
+        attn(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"], d["q_pos"], scale,
+             bufs["out"], bufs["workspace"], stream)
 
     clocks = ClockSampler(dev) if rank == 0 else None
     for _ in range(args.warmup):
@@ -215,7 +219,7 @@ def run_ours(args, rank, world, dev):
     h_out = torch.empty(bufs["out"].shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = h_out.numel() * h_out.element_size()
-    e2e_steps = max(3, min(args.steps, 200))
+    e2e_steps = max(3, min(args.steps, 200 if not prefill else 20))
     for _ in range(3):
         for n in host_names:
             d[n].copy_(host[n], non_blocking=True)
@@ -244,6 +248,8 @@ def run_ours(args, rank, world, dev):
         return None
 
     peaks = load_peaks()
+    if prefill:
+        return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks)
     tokens = w.n_streams * world
     sbytes = scores_bytes(w)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
@@ -278,6 +284,43 @@ def run_ours(args, rank, world, dev):
         "clocks": clk,
     }
     return line
+
+
+def prefill_flops(w) -> tuple[int, int]:
+    """Algorithmic FLOPs of one prefill step: the indexer contraction over
+    each query's visible keys (2 * Di per key per group) and the attention
+    over each query's attended rows (QK and PV: 4 * D per row per head)."""
+    ind = att = 0
+    for p in range(w.l_existing, w.l_total):
+        nvis = p // w.block + 1
+        rows = p + 1 if nvis <= w.top_k else (w.top_k - 1) * w.block + p % w.block + 1
+        ind += 2 * w.idx_dim * w.n_kv_heads * (p + 1)
+        att += 4 * w.head_dim * w.n_q_heads * rows
+    return ind * w.n_streams, att * w.n_streams
+
+
+def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks):
+    ind, att = prefill_flops(w)
+    tokens = w.n_queries * world
+    tf = (ind + att) / (ms * 1e-3) / 1e12
+    ktf = ind / (k_ms * 1e-3) / 1e12
+    return {
+        "metric": f"MSA prefill tokens/s ({w.name}); achieved TFLOP/s vs bf16 peak",
+        "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 indexer / bf16 attention (f32 accumulate)", "data": "synthetic",
+        "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "new_tokens": w.n_new,
+                   "context": w.l_total, "parallelism": f"replicas{world}"},
+        "step_tensor": {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
+                        "frac": tf / peaks["bf16_tflops"], "indexer_flops": ind, "attention_flops": att},
+        "roofline": {"kernel": "block_scores", "bound": "tensor", "achieved": ktf, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": ktf / peaks["bf16_tflops"], "traffic": None,
+                     "ms_per_launch": k_ms, "peak_src": peaks["src"]},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -345,8 +388,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--streams", type=int, default=WORKLOAD.n_streams,
-                    help="decode streams per GPU (32 = the benchmark workload; fewer for profiler captures)")
+    ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD.name,
+                    help="workload to time (default: the 32-stream 32K decode benchmark)")
+    ap.add_argument("--streams", type=int, default=None,
+                    help="override the workload's stream count (smaller cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -369,7 +414,7 @@ def main():
     try:
         line = run_ours(args, rank, world, local)
         if line is not None:
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name:
                 line["cpu_baseline"] = cpu_baseline()
             print(json.dumps(line), flush=True)
     finally:

@@ -72,7 +72,8 @@ _I = ctypes.c_int32
 _SIGS = {
     "msa_indexer_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P]),
     "msa_kv_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I, _P]),
-    "msa_block_scores": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P]),
+    "msa_block_scores": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t,
+                                        _P]),
     "msa_select_topk": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I, _P, _P, _P]),
     "msa_sparse_attn_decode": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
                                               ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
@@ -158,18 +159,30 @@ def msa_kv_append(shape: Shape, k_cache, v_cache, k_new, v_new, tok_stream, tok_
         _ptr(tok_pos, torch.int32, (n,), "tok_pos"), n, _stream(stream)))
 
 
-def msa_block_scores(shape: Shape, idx_q, idx_k_cache, q_stream, q_pos, block_scores=None, stream=None):
+def _workspace(shape: Shape, n: int, mode: int, workspace, device):
+    """(pointer, bytes) of the caller's workspace, allocating one if needed."""
+    need = msa_workspace_bytes(shape, n, mode)
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=device)
+    if workspace is None:
+        return 0, 0, None
+    return _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), workspace
+
+
+def msa_block_scores(shape: Shape, idx_q, idx_k_cache, q_stream, q_pos, block_scores=None, stream=None,
+                     workspace=None):
     n = _n(q_pos, "q_pos")
     if block_scores is None:
         block_scores = torch.empty((n, shape.n_kv_heads, shape.n_blocks), dtype=torch.float32,
                                    device=idx_q.device)
+    ws_ptr, ws_bytes, _keep = _workspace(shape, n, MODE_DECODE, workspace, idx_q.device)
     s = shape.c()
     _check("msa_block_scores", library().msa_block_scores(
         ctypes.byref(s), _ptr(idx_q, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_q"),
         _ptr(idx_k_cache, torch.float32, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
         _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
         _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
-        _stream(stream)))
+        ws_ptr, ws_bytes, _stream(stream)))
     return block_scores
 
 
@@ -205,13 +218,7 @@ def _attn(fn_name: str, mode: int, shape: Shape, q, k_cache, v_cache, sel, q_str
         softmax_scale = 1.0 / math.sqrt(shape.head_dim)
     if out is None:
         out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=q.device)
-    need = msa_workspace_bytes(shape, n, mode)
-    if workspace is None and need > 0:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
-    ws_ptr, ws_bytes = 0, 0
-    if workspace is not None:
-        ws_ptr = _ptr(workspace, torch.uint8, None, "workspace")
-        ws_bytes = workspace.numel()
+    ws_ptr, ws_bytes, _keep = _workspace(shape, n, mode, workspace, q.device)
     cs = (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.head_dim)
     s = shape.c()
     _check(fn_name, getattr(library(), fn_name)(
@@ -289,8 +296,13 @@ def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None,
                        new["tok_pos"], stream)
     msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
                   new["tok_stream"], new["tok_pos"], stream)
+    n = new["q_pos"].shape[0]
+    mode = MODE_PREFILL if prefill else MODE_DECODE
+    if b.get("workspace") is None and msa_workspace_bytes(shape, n, mode) > 0:
+        b = dict(b, workspace=torch.empty((msa_workspace_bytes(shape, n, mode),), dtype=torch.uint8,
+                                          device=new["q"].device))
     bs = msa_block_scores(shape, new["idx_q"], caches["idx_k_cache"], new["q_stream"], new["q_pos"],
-                          b.get("block_scores"), stream)
+                          b.get("block_scores"), stream, b.get("workspace"))
     sel, n_sel = msa_select_topk(shape, bs, new["q_pos"], b.get("sel"), b.get("n_sel"), stream)
     attn = msa_sparse_attn_prefill if prefill else msa_sparse_attn_decode
     out = attn(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],

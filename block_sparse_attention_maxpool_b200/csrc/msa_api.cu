@@ -2,6 +2,7 @@
 // Host-side argument checks, launch configuration and TMA descriptors; the
 // kernels live in the msa_*.cuh headers included below (one translation
 // unit, so the per-device error word needs no relocatable device code).
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -12,6 +13,7 @@
 #include "msa_attn_decode.cuh"
 #include "msa_common.cuh"
 #include "msa_scores_gemv.cuh"
+#include "msa_scores_tc.cuh"
 #include "msa_select.cuh"
 
 namespace {
@@ -74,19 +76,36 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// A [rows][128] bf16 cache viewed as 2-D; boxes of 128 rows x 64 columns
-// (128 bytes, the widest box the 128-byte swizzle allows).
-int make_kv_map(CUtensorMap* m, const void* base, int64_t rows) {
+// A [rows][128] tensor of 16-bit elements viewed as 2-D; boxes of 128 rows x
+// 64 columns (128 bytes, the widest box the 128-byte swizzle allows).
+int make_map_16bit(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, int64_t rows) {
   EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return MSA_ERR_CUDA;
   const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {128 * 2};
   const cuuint32_t box[2] = {64, 128};
   const cuuint32_t estride[2] = {1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estride,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
+int make_kv_map(CUtensorMap* m, const void* base, int64_t rows) {
+  return make_map_16bit(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rows);
+}
+
+// Block scores take the tensor-core tile path for prefill-shaped batches:
+// at least 256 queries and on average at least 64 per stream (so tiles of
+// 128 consecutive queries mostly share a stream).  A function of the shape
+// and the count only, so the workspace query and the call agree.
+bool scores_use_tiles(const msa_shape* sh, int32_t n_q) {
+  return n_q >= 256 && static_cast<int64_t>(n_q) >= int64_t{64} * sh->n_streams;
+}
+
+size_t scores_workspace(const msa_shape* sh, int32_t n_q) {
+  if (!scores_use_tiles(sh, n_q)) return 0;
+  return msa::tc::workspace_layout(n_q, sh->n_kv_heads, sh->n_streams, sh->capacity).total;
 }
 
 // Split-K factor of the attention kernel: few (query, group) pairs are
@@ -204,13 +223,26 @@ int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, 
 
 int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
                      const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
-                     void* stream) {
+                     void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_shape(shape);
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
   if (n_q == 0) return MSA_OK;
   if (!idx_q || !idx_k_cache || !q_stream || !q_pos || !block_scores) return MSA_ERR_NULL;
   if (!aligned16(idx_q) || !aligned16(idx_k_cache) || !aligned16(block_scores)) return MSA_ERR_ALIGN;
+  const bool tiles = scores_use_tiles(shape, n_q);
+  const size_t need = scores_workspace(shape, n_q);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need) return MSA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MSA_ERR_ALIGN;
+  }
+  int sms = 0;
+  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int G = shape->n_kv_heads;
+  const int S = shape->n_streams;
+  const int cap = shape->capacity;
+
   using namespace msa::gemv;
   Params P;
   P.idx_q = idx_q;
@@ -219,19 +251,72 @@ int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* id
   P.q_pos = q_pos;
   P.bs = block_scores;
   P.n_q = n_q;
-  P.G = shape->n_kv_heads;
-  P.n_streams = shape->n_streams;
-  P.capacity = shape->capacity;
-  P.nblk = shape->capacity / 128;
-  P.n_tasks = static_cast<long long>(n_q) * P.G * P.nblk;
-  int sms = 0;
-  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+  P.G = G;
+  P.n_streams = S;
+  P.capacity = cap;
+  P.nblk = cap / 128;
+  P.n_tasks = static_cast<long long>(n_q) * G * P.nblk;
+  P.q_list = nullptr;
+  P.q_count = nullptr;
   const size_t smem = sizeof(Smem<kScoreStages>);
   static std::atomic<uint64_t> smem_done{0};
   if ((st = ensure_smem(block_scores_gemv_kernel<kScoreStages>, smem, smem_done)) != MSA_OK) return st;
+
+  if (tiles) {
+    namespace T = msa::tc;
+    const T::Workspace L = T::workspace_layout(n_q, G, S, cap);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    T::Params Q;
+    Q.idx_q = idx_q;
+    Q.idx_k = idx_k_cache;
+    Q.q_stream = q_stream;
+    Q.q_pos = q_pos;
+    Q.bs = block_scores;
+    Q.n_q = n_q;
+    Q.G = G;
+    Q.n_streams = S;
+    Q.capacity = cap;
+    Q.nblk = cap / 128;
+    Q.n_tiles = L.n_tiles;
+    Q.n_q_pad = L.n_q_pad;
+    Q.n_chunks = (Q.nblk + T::kChunk - 1) / T::kChunk;
+    Q.counters = reinterpret_cast<int*>(ws + L.counters);
+    Q.tile_stream = reinterpret_cast<int*>(ws + L.tile_stream);
+    Q.tile_nb = reinterpret_cast<int*>(ws + L.tile_nb);
+    Q.leftover = reinterpret_cast<int*>(ws + L.leftover);
+    Q.qscale = reinterpret_cast<float*>(ws + L.qscale);
+    Q.qhi = reinterpret_cast<__half*>(ws + L.qhi);
+    Q.qlo = reinterpret_cast<__half*>(ws + L.qlo);
+    Q.kscale = reinterpret_cast<float*>(ws + L.kscale);
+    Q.khi = reinterpret_cast<__half*>(ws + L.khi);
+    Q.klo = reinterpret_cast<__half*>(ws + L.klo);
+    const int64_t key_rows = static_cast<int64_t>(S) * G * cap;
+    const int64_t q_rows = static_cast<int64_t>(G) * L.n_q_pad;
+    CUtensorMap m_qhi, m_qlo, m_khi, m_klo;
+    if ((st = make_map_16bit(&m_qhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Q.qhi, q_rows)) != MSA_OK) return st;
+    if ((st = make_map_16bit(&m_qlo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Q.qlo, q_rows)) != MSA_OK) return st;
+    if ((st = make_map_16bit(&m_khi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Q.khi, key_rows)) != MSA_OK) return st;
+    if ((st = make_map_16bit(&m_klo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Q.klo, key_rows)) != MSA_OK) return st;
+    static std::atomic<uint64_t> tc_smem_done{0};
+    if ((st = ensure_smem(T::block_scores_tc_kernel, T::SmemLayout::kBytes, tc_smem_done)) != MSA_OK) return st;
+
+    T::tc_init_kernel<<<1, 256, 0, cs>>>(Q.counters, 1 + S);
+    T::tc_tile_info_kernel<<<(L.n_tiles * 32 + 255) / 256, 256, 0, cs>>>(Q);
+    T::tc_split_queries_kernel<<<static_cast<unsigned>((q_rows * 32 + 255) / 256), 256, 0, cs>>>(Q);
+    T::tc_split_keys_kernel<<<static_cast<unsigned>((key_rows * 32 + 255) / 256), 256, 0, cs>>>(Q);
+    const int n_tasks = G * Q.n_chunks * Q.n_tiles;
+    T::block_scores_tc_kernel<<<static_cast<unsigned>(std::min(sms, n_tasks)), T::kThreads,
+                                T::SmemLayout::kBytes, cs>>>(m_qhi, m_qlo, m_khi, m_klo, Q);
+    if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
+    // queries of mixed-stream tiles: streaming kernel over the leftover list
+    P.q_list = Q.leftover;
+    P.q_count = Q.counters;
+    block_scores_gemv_kernel<kScoreStages><<<static_cast<unsigned>(sms), kThreads, smem, cs>>>(P);
+    return cuda_status(cudaGetLastError());
+  }
+
   const long long grid = std::min<long long>(sms, P.n_tasks);
-  block_scores_gemv_kernel<kScoreStages>
-      <<<static_cast<unsigned>(grid), kThreads, smem, static_cast<cudaStream_t>(stream)>>>(P);
+  block_scores_gemv_kernel<kScoreStages><<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(P);
   return cuda_status(cudaGetLastError());
 }
 
@@ -330,7 +415,7 @@ size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {
   if (check_shape(shape) != MSA_OK || n_q < 0 || (mode != MSA_MODE_DECODE && mode != MSA_MODE_PREFILL))
     return static_cast<size_t>(-1);
   const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
-  return attn_workspace(n_pairs, attn_splits(n_pairs, mode));
+  return std::max(scores_workspace(shape, n_q), attn_workspace(n_pairs, attn_splits(n_pairs, mode)));
 }
 
 const char* msa_status_string(int status) {

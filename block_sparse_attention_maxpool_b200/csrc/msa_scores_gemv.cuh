@@ -48,8 +48,19 @@ struct Params {
   const int32_t* q_pos;
   float* bs;             // [n_q][G][nblk]
   int n_q, G, n_streams, capacity, nblk;
-  long long n_tasks;     // n_q * G * nblk
+  long long n_tasks;     // n_q * G * nblk (ignored in list mode)
+  const int32_t* q_list;   // list mode: score only these query indices ...
+  const int32_t* q_count;  // ... of which there are *q_count (device memory)
 };
+
+// Task t -> (query, group, block); in list mode the query comes from q_list.
+__device__ __forceinline__ void task_coords(const Params& P, long long t, int& qi, int& g, int& b) {
+  b = static_cast<int>(t % P.nblk);
+  const long long qg = t / P.nblk;
+  g = static_cast<int>(qg % P.G);
+  const int i = static_cast<int>(qg / P.G);
+  qi = P.q_list != nullptr ? P.q_list[i] : i;
+}
 
 // Visible blocks of query qi (0 for an out-of-range query).
 __device__ __forceinline__ int query_visible(const Params& P, int qi, int& s, int& p) {
@@ -90,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
   Smem<kStages>& sm = *reinterpret_cast<Smem<kStages>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long T = P.n_tasks;
+  const long long T = P.q_list != nullptr ? static_cast<long long>(*P.q_count) * P.G * P.nblk : P.n_tasks;
   const long long t_begin = T * blockIdx.x / gridDim.x;
   const long long t_end = T * (blockIdx.x + 1) / gridDim.x;
 
@@ -111,10 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
     bool ok = true;
     int k = 0;
     for (long long t = t_begin; t < t_end && ok; ++t) {
-      const int b = static_cast<int>(t % P.nblk);
-      const long long qg = t / P.nblk;
-      const int g = static_cast<int>(qg % P.G);
-      const int qi = static_cast<int>(qg / P.G);
+      int qi, g, b;
+      task_coords(P, t, qi, g, b);
       int s, p;
       const int nvis = query_visible(P, qi, s, p);
       if (b >= nvis) continue;
@@ -145,15 +154,15 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
   int k = 0;
   int par = 0;
   for (long long t = t_begin; t < t_end; ++t) {
-    const int b = static_cast<int>(t % P.nblk);
-    const long long qg = t / P.nblk;
-    const int g = static_cast<int>(qg % P.G);
-    const int qi = static_cast<int>(qg / P.G);
+    int qi, g, b;
+    task_coords(P, t, qi, g, b);
+    const long long qg = static_cast<long long>(qi) * P.G + g;
+    const size_t out = static_cast<size_t>(qg) * P.nblk + b;
     int s, p;
     const int nvis = query_visible(P, qi, s, p);
     if (b >= nvis) {
       if (warp == 0 && lane == 0) {
-        P.bs[t] = -INFINITY;
+        P.bs[out] = -INFINITY;
         if (nvis == 0 && b == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
       }
       continue;
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
 #pragma unroll
       for (int w = 1; w < kConsumerWarps; ++w) mm = fmaxf(mm, sm.red[par][w]);
       if (b == p / kBlock) mm += MSA_LOCAL_BIAS;
-      P.bs[t] = mm;
+      P.bs[out] = mm;
     }
     par ^= 1;
   }

@@ -121,10 +121,22 @@ MSA_API int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v
  * + MSA_LOCAL_BIAS (MSA pull request, section "Implementation":
  * bs = maxpool_128(idx_q*idx_k^T + causal mask) plus the local-force bias).
  * NaN scores are treated as -inf.  An out-of-range query writes -inf
- * everywhere and sets MSA_DEVERR_QUERY_RANGE. */
+ * everywhere and sets MSA_DEVERR_QUERY_RANGE.
+ *
+ * Two kernels implement it.  Decode-shaped batches (fewer than 256 queries,
+ * or fewer than 64 per stream on average) stream the F32 keys through a
+ * GEMV; they need no workspace.  Prefill-shaped batches run tiles of 128
+ * consecutive queries against 128-key blocks on the tcgen05 tensor cores:
+ * each F32 row is split exactly as 2^-e (hi + lo) with fp16 hi, lo and three
+ * MMAs (hi.hi + hi.lo + lo.hi) accumulate in F32, which keeps the score within
+ * about 2^-21 of sum |q_d k_d|.  Tiles whose queries span several streams
+ * fall back to the GEMV for the queries of the other streams.  The tile path
+ * needs `workspace` of at least msa_workspace_bytes(shape, n_q, mode) bytes,
+ * 256-byte aligned (its contents need not be initialised). */
 MSA_API int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
                      const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
-                     float* block_scores, void* stream);
+                     float* block_scores, void* workspace, size_t workspace_bytes,
+                     void* stream);
 
 /* msa_select_topk - top-k block selection per (query, group).
  * Ranks the visible blocks b <= q_pos/128 by (score descending, block index
@@ -194,8 +206,10 @@ MSA_API int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf1
                                            const int32_t* q_pos, int32_t n_q, float softmax_scale,
                                            msa_bf16* out, void* stream);
 
-/* Bytes of workspace the attention call of `mode` needs for n_q queries
- * (0 when none).  Returns (size_t)-1 for an unsupported shape. */
+/* Bytes of workspace that msa_block_scores and the attention call of `mode`
+ * need for n_q queries (the larger of the two; one buffer serves both calls
+ * of a step, since they run in stream order).  0 when neither needs any.
+ * Returns (size_t)-1 for an unsupported shape. */
 MSA_API size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode);
 
 /* Human-readable name of a status code (static string). */

@@ -3,11 +3,16 @@ seeded inputs and compare them with the CPU oracle.
 
 Comparison rules
   * cache append, selection from identical float32 scores: bit-exact;
-  * block scores (float32 on the GPU vs float64 in the oracle): the float32
-    dot product of 128 terms, formed as 4-term FMA chains summed over a 32-lane
-    tree, rounds each term at most ~9 times, so |err| <= 9 u sum_d |q_d k_d|
-    (u = 2^-24).  The test allows 16 u times the largest such sum in the
-    block, plus exact agreement of -inf and of the local bias;
+  * block scores (float32 on the GPU vs float64 in the oracle).  Streaming
+    kernel: the float32 dot product of 128 terms, formed as 4-term FMA chains
+    summed over a 32-lane tree, rounds each term at most ~9 times, so
+    |err| <= 9 u sum_d |q_d k_d| (u = 2^-24).  Tensor-core tile kernel: each
+    factor is split exactly as 2^-e (hi + lo) in fp16, so hi + lo differs
+    from it by at most 2^-23 of the row scale, the dropped lo.lo product is
+    at most 2^-22 |q_d k_d|, and the float32 accumulation of 24 partial
+    products adds at most 24 u of the running sum: together below 56 u sum_d
+    |q_d k_d|.  The test allows 64 u times the largest such sum in the block,
+    plus exact agreement of -inf and of the local bias;
   * end-to-end selection: ids bit-exact, except (q, g) pairs whose oracle
     ranks top_k and top_k+1 are within 1e-5 relative (and not exactly equal);
     those are counted and the attention is checked with the GPU's selection;
@@ -56,7 +61,7 @@ def oracle_caches(inp):
 
 
 def score_bounds(idx_q, idx_k_cache, q_stream, q_pos, block):
-    """Per (query, group, block): 16 u max_j sum_d |q_d k_jd| over visible j."""
+    """Per (query, group, block): 64 u max_j sum_d |q_d k_jd| over visible j."""
     n_q, G = idx_q.shape[0], idx_q.shape[1]
     nblk = idx_k_cache.shape[2] // block
     out = torch.zeros((n_q, G, nblk), dtype=torch.float64)
@@ -67,7 +72,7 @@ def score_bounds(idx_q, idx_k_cache, q_stream, q_pos, block):
             nb = p // block + 1
             pad = torch.full((nb * block,), 0.0, dtype=torch.float64)
             pad[:p + 1] = a
-            out[i, g, :nb] = 16 * U32 * pad.view(nb, block).amax(dim=1)
+            out[i, g, :nb] = 64 * U32 * pad.view(nb, block).amax(dim=1)
     return out
 
 

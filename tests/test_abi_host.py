@@ -59,11 +59,11 @@ FAKE = 0x10000          # a 16-byte aligned address that is never dereferenced
 
 
 def call_scores(lib, shape, n_q=4, **over):
-    a = dict(idx_q=FAKE, idx_k=FAKE, qs=FAKE, qp=FAKE, bs=FAKE)
+    a = dict(idx_q=FAKE, idx_k=FAKE, qs=FAKE, qp=FAKE, bs=FAKE, ws=0, ws_bytes=0)
     a.update(over)
     s = shape.c()
     return lib.msa_block_scores(ctypes.byref(s), a["idx_q"], a["idx_k"], a["qs"], a["qp"], n_q,
-                                a["bs"], None)
+                                a["bs"], a["ws"], a["ws_bytes"], None)
 
 
 @pytest.mark.parametrize("bad", [
@@ -77,12 +77,22 @@ def test_shape_rejected(lib, bad):
 
 
 def test_null_and_alignment(lib):
-    assert lib.msa_block_scores(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, None) == -1
+    assert lib.msa_block_scores(None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, 0, 0, None) == -1
     assert call_scores(lib, GOOD, idx_k=0) == -1
     assert call_scores(lib, GOOD, bs=0) == -1
     assert call_scores(lib, GOOD, idx_q=FAKE + 4) == -2
     assert call_scores(lib, GOOD, n_q=-1) == -4
     assert call_scores(lib, GOOD, n_q=0, idx_q=0, idx_k=0) == 0      # empty batch is a no-op
+
+
+def test_tile_path_requires_workspace(lib):
+    sh = msa.Shape(n_streams=1, capacity=4096)
+    s = sh.c()
+    need = lib.msa_workspace_bytes(ctypes.byref(s), 512, msa.MODE_PREFILL)
+    assert need > 0
+    assert call_scores(lib, sh, n_q=512) == -5                               # none given
+    assert call_scores(lib, sh, n_q=512, ws=FAKE, ws_bytes=need - 1) == -5   # too small
+    assert call_scores(lib, sh, n_q=512, ws=FAKE + 16, ws_bytes=need) == -2  # not 256-B aligned
 
 
 def test_select_and_append_validation(lib):
@@ -103,7 +113,12 @@ def test_attention_validation_and_workspace(lib):
     need = lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_DECODE)
     assert need == 8 * 16 * 16 * 130 * 4
     assert lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_PREFILL) == 0
-    assert lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_DECODE) == 0
+    # 4096 queries over 2 streams: prefill-shaped, the block scores take the tile path
+    big = lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_DECODE)
+    assert big > 0 and big == lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_PREFILL)
+    # 600 decode queries over 600 streams stay on the streaming kernel and split-free attention
+    many = msa.Shape(n_streams=600, capacity=1024).c()
+    assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_DECODE) == 0
     bad = msa.Shape(n_streams=2, capacity=1000).c()
     assert lib.msa_workspace_bytes(ctypes.byref(bad), 2, 0) == ctypes.c_size_t(-1).value
     args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, ctypes.c_float(0.088), FAKE]

@@ -169,6 +169,38 @@ def test_block_scores_ragged_multi_stream():
     PT.check_scores(bs.cpu(), bs_o, PT.score_bounds(iq, idx, qs, qp, 128))
 
 
+def test_block_scores_tile_path_mixed_streams_and_padding():
+    """A prefill-shaped batch (tensor-core tiles): 3 streams, queries in
+    stream-contiguous runs that do not align with the 128-query tiles (so
+    mixed tiles send some queries to the streaming kernel), unsorted
+    positions, a padded last tile, 40 key blocks (two 32-block chunks) and
+    two invalid queries."""
+    S, cap = 3, 128 * 40
+    lengths = [cap, 4000, 3000]
+    g = torch.Generator().manual_seed(12)
+    qpos = []
+    for s, n in ((0, 300), (1, 200), (2, 150)):
+        pos = torch.randint(0, lengths[s], (n,), generator=g).tolist()
+        qpos += [(s, p) for p in pos]
+    qpos[5] = (0, cap - 1)
+    qpos[301] = (1, 0)
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, lengths, qpos, seed=12)
+    qs_bad, qp_bad = qs.clone(), qp.clone()
+    qs_bad[10] = 7                   # no such stream
+    qp_bad[400] = cap                # past the capacity
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    assert msa.msa_workspace_bytes(sh, len(qpos), msa.MODE_PREFILL) > 0     # tile path
+    bs = msa.msa_block_scores(sh, iq.cuda(), idx.cuda(), qs_bad.cuda(), qp_bad.cuda())
+    assert msa.msa_get_device_error() & 0x1
+    bs = bs.cpu()
+    for bad in (10, 400):
+        assert torch.isinf(bs[bad]).all() and (bs[bad] < 0).all()
+    good = [i for i in range(len(qpos)) if i not in (10, 400)]
+    bs_o = oracle.block_scores(iq[good], idx, qs[good], qp[good], 128)
+    err = PT.check_scores(bs[good], bs_o, PT.score_bounds(iq[good], idx, qs[good], qp[good], 128))
+    report("tile path scores", {"queries": len(good), "max_err": err})
+
+
 def test_block_scores_out_of_range_query():
     sh = msa.Shape(n_streams=1, capacity=256)
     idx, k, v, qs, qp, iq, q = W.make_custom(1, 256, [256], [(0, 10), (0, 10)], seed=4)
