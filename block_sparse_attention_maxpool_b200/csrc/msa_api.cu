@@ -11,6 +11,7 @@
 #include "msa.h"
 #include "msa_append.cuh"
 #include "msa_attn_decode.cuh"
+#include "msa_attn_prefill_tc.cuh"
 #include "msa_common.cuh"
 #include "msa_scores_gemv.cuh"
 #include "msa_scores_tc.cuh"
@@ -78,12 +79,13 @@ EncodeTiledFn encode_tiled() {
 
 // A [rows][128] tensor of 16-bit elements viewed as 2-D; boxes of 128 rows x
 // 64 columns (128 bytes, the widest box the 128-byte swizzle allows).
-int make_map_16bit(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, int64_t rows) {
+int make_map_16bit(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, int64_t rows,
+                   uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return MSA_ERR_CUDA;
   const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {128 * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   const CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estride,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -152,6 +154,34 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   CUtensorMap tm_k, tm_v;
   if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
   if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (mode == MSA_MODE_PREFILL) {
+    // tensor-core kernel, one persistent CTA per SM
+    CUtensorMap tm_q;
+    if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q,
+                             static_cast<int64_t>(n_q) * sh->n_q_heads, 16)) != MSA_OK)
+      return st;
+    static std::atomic<uint64_t> tc_smem_done{0};
+    if ((st = ensure_smem(msa::pattn::sparse_attn_prefill_tc_kernel, msa::pattn::Layout::kBytes, tc_smem_done)) !=
+        MSA_OK)
+      return st;
+    int sms = 0;
+    if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+    msa::pattn::Params Q;
+    Q.sel = sel;
+    Q.q_stream = q_stream;
+    Q.q_pos = q_pos;
+    Q.out = reinterpret_cast<__nv_bfloat16*>(out);
+    Q.n_q = n_q;
+    Q.G = G;
+    Q.n_streams = sh->n_streams;
+    Q.capacity = sh->capacity;
+    Q.scale_log2 = softmax_scale * 1.4426950408889634f;
+    const int64_t grid = std::min<int64_t>(sms, n_pairs);
+    msa::pattn::sparse_attn_prefill_tc_kernel<<<static_cast<unsigned>(grid), msa::pattn::kThreads,
+                                                msa::pattn::Layout::kBytes, s>>>(tm_q, tm_k, tm_v, Q);
+    return cuda_status(cudaGetLastError());
+  }
   static std::atomic<uint64_t> smem_done{0};
   if ((st = ensure_smem(msa::attn::sparse_attn_kernel, msa::attn::kSmemBytes, smem_done)) != MSA_OK) return st;
 
@@ -170,7 +200,6 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   P.n_split = n_split;
   P.blocks_per_split = msa::attn::kTopK / n_split;
   P.scale_log2 = softmax_scale * 1.4426950408889634f;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   msa::attn::sparse_attn_kernel<<<static_cast<unsigned>(n_pairs * n_split), msa::attn::kThreads,
                                   msa::attn::kSmemBytes, s>>>(tm_k, tm_v, P);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
