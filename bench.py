@@ -88,6 +88,30 @@ def step_bytes(w) -> int:
 
 
 # ---------------------------------------------------------------------------
+# multi-GPU: replicas over disjoint streams, timing reduced by max
+# ---------------------------------------------------------------------------
+def shard_streams(streams_per_rank: int, rank: int) -> range:
+    """Global ids of the decode streams rank `rank` owns: each rank holds its
+    own contiguous run of independent streams (no data crosses GPUs)."""
+    return range(rank * streams_per_rank, (rank + 1) * streams_per_rank)
+
+
+def max_over_ranks(values, device=None) -> list[float]:
+    """Element-wise maximum of per-rank timings (slowest rank decides)."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(streams_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job decode throughput: one token per stream per step on every rank."""
+    return streams_per_rank * world / (ms_per_step * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -153,7 +177,7 @@ def run_ours(args, rank, world, dev):
                        quantize_idx=w.quantize_idx)
     prefill = w.queries == "new"
     shape = msa.Shape(n_streams=w.n_streams, capacity=w.capacity)
-    inp = W.make_inputs(w, seed=rank)                    # each rank: its own 32 streams
+    inp = W.make_inputs(w, streams=shard_streams(w.n_streams, rank))   # this rank's own streams
     d = {n: getattr(inp, n).to(dev) for n in ("idx_k_cache", "k_cache", "v_cache", "tok_stream",
                                                "tok_pos", "idx_k_new", "k_new", "v_new",
                                                "q_stream", "q_pos", "idx_q", "q")}
@@ -240,24 +264,20 @@ def run_ours(args, rank, world, dev):
         raise RuntimeError("device error during timing")
     clk = clocks.stop(mark) if clocks else None
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms, k_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms, k_ms = t.tolist()
+    ms, e2e_ms, k_ms = max_over_ranks([ms, e2e_ms, k_ms], device=dev)
     if rank != 0:
         return None
 
     peaks = load_peaks()
     if prefill:
         return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks)
-    tokens = w.n_streams * world
     sbytes = scores_bytes(w)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     traffic = SCORES_TRAFFIC["bytes_per_launch"] if SCORES_TRAFFIC["source_sha"] == scores_source_sha() else None
     step_gbs = step_bytes(w) / (ms * 1e-3) / 1e9
     line = {
         "metric": METRIC,
-        "value": tokens / (ms * 1e-3),
+        "value": job_tokens_per_s(w.n_streams, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -278,8 +298,8 @@ def run_ours(args, rank, world, dev):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "algorithmic_bytes": sbytes, "ms_per_launch": k_ms,
                      "peak_src": peaks["src"]},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "e2e": {"value": job_tokens_per_s(w.n_streams, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
