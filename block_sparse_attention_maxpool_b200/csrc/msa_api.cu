@@ -10,7 +10,7 @@
 
 #include "msa.h"
 #include "msa_append.cuh"
-#include "msa_attn_decode.cuh"
+#include "msa_attn_decode_sk.cuh"
 #include "msa_attn_prefill_tc.cuh"
 #include "msa_common.cuh"
 #include "msa_scores_gemv.cuh"
@@ -110,23 +110,14 @@ size_t scores_workspace(const msa_shape* sh, int32_t n_q) {
   return msa::tc::workspace_layout(n_q, sh->n_kv_heads, sh->n_streams, sh->capacity).total;
 }
 
-// Split-K factor of the attention kernel: few (query, group) pairs are
-// spread over more CTAs so the selected blocks of a decode step are read by
-// many SMs at once.  Depends only on the pair count, so the workspace size
-// query and the launch always agree.
-int attn_splits(int64_t n_pairs, int mode) {
-  if (mode == MSA_MODE_PREFILL) return 1;
-  if (n_pairs >= 512) return 1;
-  if (n_pairs >= 256) return 2;
-  if (n_pairs >= 96) return 4;
-  if (n_pairs >= 32) return 8;
-  return 16;
-}
-
-size_t attn_workspace(int64_t n_pairs, int n_split) {
-  if (n_split <= 1) return 0;
-  const size_t slots = static_cast<size_t>(n_pairs) * n_split * msa::attn::kHpg;
-  return slots * (msa::attn::kD + 2) * sizeof(float);
+// Decode attention workspace: two partial results per CTA of the persistent
+// grid (at most kMaxCtas CTAs, at most one per unit).  Depends only on the
+// pair count, so the workspace query and the launch always agree.
+size_t attn_workspace(int64_t n_pairs, int mode) {
+  if (mode == MSA_MODE_PREFILL || n_pairs == 0) return 0;
+  const int64_t units = n_pairs * msa::dattn::kTopK;
+  const int64_t ctas = std::min<int64_t>(units, msa::dattn::kMaxCtas);
+  return static_cast<size_t>(ctas) * 2 * msa::dattn::kPartial * sizeof(float);
 }
 
 int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache, const msa_bf16* v_cache,
@@ -143,9 +134,8 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   if (!std::isfinite(softmax_scale)) return MSA_ERR_RANGE;
   const int G = sh->n_kv_heads;
   const int64_t n_pairs = static_cast<int64_t>(n_q) * G;
-  const int n_split = attn_splits(n_pairs, mode);
-  if (n_pairs * n_split >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
-  const size_t need = attn_workspace(n_pairs, n_split);
+  if (n_pairs * msa::dattn::kTopK >= (int64_t{1} << 40)) return MSA_ERR_RANGE;
+  const size_t need = attn_workspace(n_pairs, mode);
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need) return MSA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MSA_ERR_ALIGN;
@@ -155,6 +145,8 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
   if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int sms = 0;
+  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
   if (mode == MSA_MODE_PREFILL) {
     // tensor-core kernel, one persistent CTA per SM
     CUtensorMap tm_q;
@@ -165,8 +157,6 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     if ((st = ensure_smem(msa::pattn::sparse_attn_prefill_tc_kernel, msa::pattn::Layout::kBytes, tc_smem_done)) !=
         MSA_OK)
       return st;
-    int sms = 0;
-    if ((st = current_device_sms(&sms)) != MSA_OK) return st;
     msa::pattn::Params Q;
     Q.sel = sel;
     Q.q_stream = q_stream;
@@ -182,34 +172,32 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
                                                 msa::pattn::Layout::kBytes, s>>>(tm_q, tm_k, tm_v, Q);
     return cuda_status(cudaGetLastError());
   }
+  // decode: persistent stream-K grid over (pair, selected block) units
   static std::atomic<uint64_t> smem_done{0};
-  if ((st = ensure_smem(msa::attn::sparse_attn_kernel, msa::attn::kSmemBytes, smem_done)) != MSA_OK) return st;
-
-  msa::attn::Params P;
+  if ((st = ensure_smem(msa::dattn::sparse_attn_decode_sk_kernel, msa::dattn::Layout::kBytes, smem_done)) !=
+      MSA_OK)
+    return st;
+  msa::dattn::Params P;
   P.q = reinterpret_cast<const __nv_bfloat16*>(q);
   P.sel = sel;
   P.q_stream = q_stream;
   P.q_pos = q_pos;
   P.out = reinterpret_cast<__nv_bfloat16*>(out);
-  P.ws_o = need > 0 ? static_cast<float*>(workspace) : nullptr;
-  P.ws_ml = need > 0 ? P.ws_o + static_cast<size_t>(n_pairs) * n_split * msa::attn::kHpg * msa::attn::kD : nullptr;
+  P.ws = static_cast<float*>(workspace);
   P.n_q = n_q;
   P.G = G;
   P.n_streams = sh->n_streams;
   P.capacity = sh->capacity;
-  P.n_split = n_split;
-  P.blocks_per_split = msa::attn::kTopK / n_split;
+  P.n_units = n_pairs * msa::dattn::kTopK;
+  P.n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), P.n_units,
+                                                static_cast<int64_t>(msa::dattn::kMaxCtas)}));
   P.scale_log2 = softmax_scale * 1.4426950408889634f;
-  msa::attn::sparse_attn_kernel<<<static_cast<unsigned>(n_pairs * n_split), msa::attn::kThreads,
-                                  msa::attn::kSmemBytes, s>>>(tm_k, tm_v, P);
+  msa::dattn::sparse_attn_decode_sk_kernel<<<static_cast<unsigned>(P.n_cta), msa::dattn::kThreads,
+                                             msa::dattn::Layout::kBytes, s>>>(tm_k, tm_v, P);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
-  if (n_split > 1) {
-    const int64_t warps = n_pairs * msa::attn::kHpg;
-    const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
-    msa::attn::attn_combine_kernel<<<grid, 256, 0, s>>>(P.ws_o, P.ws_ml, P.out, static_cast<int>(n_pairs), n_split);
-    if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
-  }
-  return MSA_OK;
+  const int64_t warps = n_pairs * msa::dattn::kHpg;
+  msa::dattn::attn_sk_combine_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(P);
+  return cuda_status(cudaGetLastError());
 }
 
 int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache1, const void* src1,
@@ -428,8 +416,13 @@ int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf16* q, co
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
   if (n_q == 0) return MSA_OK;
+  // argument errors are reported before the one-time device set-up below
+  if (!q || !k_cache || !v_cache || !sel || !q_stream || !q_pos || !out) return MSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(sel) || !aligned16(out))
+    return MSA_ERR_ALIGN;
+  if (!std::isfinite(softmax_scale)) return MSA_ERR_RANGE;
   const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
-  const size_t need = attn_workspace(n_pairs, attn_splits(n_pairs, MSA_MODE_DECODE));
+  const size_t need = attn_workspace(n_pairs, MSA_MODE_DECODE);
   if (need > MSA_NOALLOC_SCRATCH_BYTES) return MSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (need > 0) {
@@ -444,7 +437,7 @@ size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {
   if (check_shape(shape) != MSA_OK || n_q < 0 || (mode != MSA_MODE_DECODE && mode != MSA_MODE_PREFILL))
     return static_cast<size_t>(-1);
   const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
-  return std::max(scores_workspace(shape, n_q), attn_workspace(n_pairs, attn_splits(n_pairs, mode)));
+  return std::max(scores_workspace(shape, n_q), attn_workspace(n_pairs, mode));
 }
 
 const char* msa_status_string(int status) {

@@ -1,0 +1,374 @@
+// Block-sparse GQA attention for decode batches: persistent, stream-K style.
+//
+// MSA pull request "Add MiniMax-M3 (MSA) support", section "Overview": each
+// query attends to the rows of its selected blocks only (16 x 128 = 2048
+// keys), shared by the 16 heads of its GQA group; the token-level causal mask
+// applies inside the local block.
+//
+// A decode step has few (query, group) pairs, each reading 16 blocks of K and
+// V (1 MB).  The work units are (pair, selected block); every CTA of a
+// persistent grid (at most one per SM) takes one contiguous, equal share of
+// the units, so all SMs stream K/V for the whole kernel with no wave tail.
+// One producer thread TMA-loads each unit's K and V tiles (four 16 KB boxes,
+// 128-byte swizzle) into a two-stage ring; eight consumer warps each own 16
+// key rows of the block and compute S = Q K^T (16 heads x 16 rows) and
+// O += P V with bf16 m16n8k16 MMAs, fp32 accumulation and a streaming base-2
+// softmax.  Consecutive units of one pair accumulate in registers; when the
+// pair changes the eight warps merge through shared memory.  A pair whose
+// units all lie in one CTA's share is written out directly; a pair cut by a
+// share boundary leaves one partial (max, sum, unnormalised O) per CTA,
+// merged by attn_sk_combine_kernel.
+#pragma once
+
+#include "msa_common.cuh"
+
+namespace msa {
+namespace dattn {
+
+constexpr int kD = 128;
+constexpr int kBlock = 128;
+constexpr int kHpg = 16;
+constexpr int kTopK = 16;
+constexpr int kWarps = 8;                           // consumer warps
+constexpr int kThreads = (kWarps + 1) * 32;         // + one producer warp
+constexpr int kRowsPerWarp = kBlock / kWarps;       // 16
+constexpr uint32_t kTileBytes = kBlock * 64 * 2;    // [128 rows][64 dims] bf16 = 16 KB
+constexpr uint32_t kStageBytes = 4 * kTileBytes;    // K lo, K hi, V lo, V hi
+constexpr int kStages = 2;
+constexpr int kOStride = kD + 4;                    // padded fp32 row of the merge buffer
+constexpr int kMaxCtas = 256;                       // grid cap (bounds the workspace)
+constexpr int kPartial = kHpg * (kD + 2);           // floats of one partial: O[16][128], m[16], l[16]
+
+struct Layout {
+  static constexpr uint32_t kStageOff = 0;
+  static constexpr uint32_t kMergeOff = kStages * kStageBytes;
+  static constexpr uint32_t kMlOff = kMergeOff + kWarps * kHpg * kOStride * 4;
+  static constexpr uint32_t kBarOff = kMlOff + kWarps * kHpg * 2 * 4;
+  static constexpr uint32_t kEnd = kBarOff + 64;
+  static constexpr size_t kBytes = kEnd + 1024;
+};
+
+struct Params {
+  const __nv_bfloat16* q;     // [n_q][Hq][D]
+  const int32_t* sel;         // [n_q][G][16]
+  const int32_t* q_stream;
+  const int32_t* q_pos;
+  __nv_bfloat16* out;         // [n_q][Hq][D]
+  float* ws;                  // [n_cta][2][kPartial]
+  int n_q, G, n_streams, capacity, n_cta;
+  long long n_units;          // n_q * G * 16
+  float scale_log2;
+};
+
+__host__ __device__ inline long long unit_begin(long long U, int C, int c) { return U * c / C; }
+
+// The CTA whose share holds unit u.
+__device__ inline int cta_of(long long U, int C, long long u) {
+  int c = static_cast<int>(u * C / U);
+  while (c + 1 < C && unit_begin(U, C, c + 1) <= u) ++c;
+  while (c > 0 && unit_begin(U, C, c) > u) --c;
+  return c;
+}
+
+// Cache row of unit u's block, or -1 when the unit has nothing to attend
+// (padding, an invalid selection or an invalid query).  p: query position.
+__device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, bool report) {
+  const long long pair = u / kTopK;
+  const int j = static_cast<int>(u - pair * kTopK);
+  const int qi = static_cast<int>(pair / P.G);
+  const int g = static_cast<int>(pair - static_cast<long long>(qi) * P.G);
+  const int s = P.q_stream[qi];
+  p = P.q_pos[qi];
+  if (s < 0 || s >= P.n_streams || p < 0 || p >= P.capacity) {
+    if (report && j == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
+    return -1;
+  }
+  const int b = P.sel[pair * kTopK + j];
+  if (b < 0) return -1;
+  if (b > p / kBlock) {
+    if (report) raise_error(MSA_DEVERR_SEL_RANGE);
+    return -1;
+  }
+  return (s * P.G + g) * P.capacity + b * kBlock;
+}
+
+// Merge the eight warps' states of one pair and write the output rows (or
+// this CTA's partial for a pair shared with a neighbouring CTA).
+__device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long long pair, long long u0,
+                                           long long u1, int slot_cta, float (&o)[16][4], float (&m_run)[2],
+                                           float (&l_run)[2], int warp, int lane) {
+  const int gr = lane >> 2, tq = lane & 3;
+  const int tid = warp * 32 + lane;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+  }
+  float* so = reinterpret_cast<float*>(smem + Layout::kMergeOff);   // [8][16][kOStride]
+  float* sml = reinterpret_cast<float*>(smem + Layout::kMlOff);     // [8][16][2]
+  named_barrier_sync(1, kWarps * 32);                                 // previous merge fully read
+  {
+    float* ow = so + warp * kHpg * kOStride;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      const int col = n * 8 + tq * 2;
+      *reinterpret_cast<float2*>(ow + gr * kOStride + col) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(ow + (gr + 8) * kOStride + col) = make_float2(o[n][2], o[n][3]);
+    }
+    if (tq == 0) {
+      sml[(warp * kHpg + gr) * 2 + 0] = m_run[0];
+      sml[(warp * kHpg + gr) * 2 + 1] = l_run[0];
+      sml[(warp * kHpg + gr + 8) * 2 + 0] = m_run[1];
+      sml[(warp * kHpg + gr + 8) * 2 + 1] = l_run[1];
+    }
+  }
+  named_barrier_sync(1, kWarps * 32);
+  const int head = tid >> 4;            // 16 heads x 16 threads
+  const int d0 = (tid & 15) * 8;        // 8 dims per thread
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sml[(w * kHpg + head) * 2]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  float L = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float sc = exp2f(sml[(w * kHpg + head) * 2] - Mu);
+    L += sml[(w * kHpg + head) * 2 + 1] * sc;
+    const float4* src = reinterpret_cast<const float4*>(so + (w * kHpg + head) * kOStride + d0);
+    const float4 a = src[0], b = src[1];
+    acc[0] += a.x * sc; acc[1] += a.y * sc; acc[2] += a.z * sc; acc[3] += a.w * sc;
+    acc[4] += b.x * sc; acc[5] += b.y * sc; acc[6] += b.z * sc; acc[7] += b.w * sc;
+  }
+  const bool complete = pair * kTopK >= u0 && pair * kTopK + kTopK <= u1;
+  if (complete) {
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint32_t pk[4];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) pk[d] = pack_bf16(acc[2 * d] * inv, acc[2 * d + 1] * inv);
+    __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + d0;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  } else {
+    const int slot = pair * kTopK < u0 ? 0 : 1;
+    float* part = P.ws + (static_cast<size_t>(slot_cta) * 2 + slot) * kPartial;
+    float* dst = part + head * kD + d0;
+    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    if ((tid & 15) == 0) {
+      part[kHpg * kD + head] = M;
+      part[kHpg * kD + kHpg + head] = L;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                                 const Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Layout::kBarOff);
+  uint64_t* empty = full + kStages;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long U = P.n_units;
+  const long long u0 = unit_begin(U, P.n_cta, blockIdx.x);
+  const long long u1 = unit_begin(U, P.n_cta, blockIdx.x + 1);
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kWarps);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // -------------------------------- producer --------------------------------
+    if (lane != 0) return;
+    int k = 0;
+    bool ok = true;
+    for (long long u = u0; u < u1 && ok; ++u) {
+      int p;
+      const int row = unit_row(P, u, p, false);
+      if (row < 0) continue;
+      const int st = k % kStages;
+      const int use = k / kStages;
+      if (use > 0) ok = mbar_wait(&empty[st], (use - 1) & 1);
+      if (!ok) break;
+      uint8_t* dst = smem + Layout::kStageOff + st * kStageBytes;
+      mbar_arrive_expect_tx(&full[st], kStageBytes);
+      tma_load_2d(dst, &tm_k, 0, row, &full[st]);
+      tma_load_2d(dst + kTileBytes, &tm_k, 64, row, &full[st]);
+      tma_load_2d(dst + 2 * kTileBytes, &tm_v, 0, row, &full[st]);
+      tma_load_2d(dst + 3 * kTileBytes, &tm_v, 64, row, &full[st]);
+      ++k;
+    }
+    // no copy may still be landing when the CTA exits
+    for (int j = max(0, k - kStages); j < k; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
+    return;
+  }
+
+  // -------------------------------- consumers --------------------------------
+  const int gr = lane >> 2;   // fragment row group
+  const int tq = lane & 3;    // thread in quad
+  const int wr = warp * kRowsPerWarp;
+  uint32_t qa[8][4];
+  float o[16][4];
+  float m_run[2], l_run[2];
+  long long cur = -1;
+  int k = 0;
+  bool ok = true;
+  for (long long u = u0; u < u1; ++u) {
+    const long long pair = u / kTopK;
+    if (pair != cur) {
+      if (cur >= 0) flush_pair(P, smem, cur, u0, u1, blockIdx.x, o, m_run, l_run, warp, lane);
+      cur = pair;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      m_run[0] = m_run[1] = -INFINITY;
+      l_run[0] = l_run[1] = 0.f;
+      // Q of the pair's 16 heads as the A operand, straight from global memory
+      const __nv_bfloat16* qb = P.q + static_cast<size_t>(pair) * kHpg * kD;
+      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qb + gr * kD);
+      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qb + (gr + 8) * kD);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int c = ks * 8 + tq;   // 32-bit word of dims 16ks + 2tq
+        qa[ks][0] = __ldg(r0 + c);
+        qa[ks][1] = __ldg(r1 + c);
+        qa[ks][2] = __ldg(r0 + c + 4);
+        qa[ks][3] = __ldg(r1 + c + 4);
+      }
+    }
+    int p;
+    const int row = unit_row(P, u, p, warp == 0 && lane == 0);
+    if (row < 0) continue;
+    const int st = k % kStages;
+    if (ok) ok = mbar_wait(&full[st], (k / kStages) & 1);
+    if (ok) {
+      const uint32_t kbase = smem_addr(smem + Layout::kStageOff + st * kStageBytes);
+      const uint32_t vbase = kbase + 2 * kTileBytes;
+      // S = Q K^T: two n-tiles of 8 key rows
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int half = ks >> 2;
+        const int c0 = (ks & 3) * 2;
+        const int mi = lane >> 3;
+        const int r = wr + (mi >> 1) * 8 + (lane & 7);
+        const int ch = c0 + (mi & 1);
+        uint32_t b[4];
+        ldmatrix_x4(b, kbase + half * kTileBytes + swz128(r, ch));
+        mma_bf16_16816(sacc[0], qa[ks], b[0], b[1]);
+        mma_bf16_16816(sacc[1], qa[ks], b[2], b[3]);
+      }
+      // causal mask inside the block, base-2 scaling, online softmax
+      const int jb = (row % P.capacity) + wr;    // absolute slot of this warp's first key
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = jb + nt * 8 + tq * 2 + (e & 1);
+          const float x = j <= p ? sacc[nt][e] * P.scale_log2 : -INFINITY;
+          sacc[nt][e] = x;
+          mx[e >> 1] = fmaxf(mx[e >> 1], x);
+        }
+      }
+      float alpha[2], m_use[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+        const float m_new = fmaxf(m_run[h], mx[h]);
+        m_use[h] = m_new == -INFINITY ? 0.f : m_new;
+        alpha[h] = exp2f(m_run[h] - m_use[h]);
+        m_run[h] = m_new;
+      }
+      float rs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pe = exp2f(sacc[nt][e] - m_use[e >> 1]);
+          sacc[nt][e] = pe;
+          rs[e >> 1] += pe;
+        }
+      }
+      l_run[0] = l_run[0] * alpha[0] + rs[0];
+      l_run[1] = l_run[1] * alpha[1] + rs[1];
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[0];
+        o[n][2] *= alpha[1];
+        o[n][3] *= alpha[1];
+      }
+      // O += P V: P (16 heads x 16 rows) is the A operand of one k-step
+      uint32_t pa[4];
+      pa[0] = pack_bf16(sacc[0][0], sacc[0][1]);
+      pa[1] = pack_bf16(sacc[0][2], sacc[0][3]);
+      pa[2] = pack_bf16(sacc[1][0], sacc[1][1]);
+      pa[3] = pack_bf16(sacc[1][2], sacc[1][3]);
+#pragma unroll
+      for (int jn = 0; jn < 8; ++jn) {
+        const int half = jn >> 2;
+        const int c = (jn & 3) * 2;
+        const int mi = lane >> 3;
+        const int r = wr + (mi & 1) * 8 + (lane & 7);
+        const int ch = c + (mi >> 1);
+        uint32_t v[4];
+        ldmatrix_x4_trans(v, vbase + half * kTileBytes + swz128(r, ch));
+        const int nt = half * 8 + c;
+        mma_bf16_16816(o[nt], pa, v[0], v[1]);
+        mma_bf16_16816(o[nt + 1], pa, v[2], v[3]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+    ++k;
+  }
+  if (cur >= 0) flush_pair(P, smem, cur, u0, u1, blockIdx.x, o, m_run, l_run, warp, lane);
+}
+
+// Pairs cut by a share boundary: merge the partials of every CTA whose share
+// touches the pair.  One warp per (pair, head), four dims per lane.
+__global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long n_pairs = P.n_units / kTopK;
+  if (w >= n_pairs * kHpg) return;
+  const long long pair = w / kHpg;
+  const int head = static_cast<int>(w - pair * kHpg);
+  const long long U = P.n_units;
+  const int c_lo = cta_of(U, P.n_cta, pair * kTopK);
+  const int c_hi = cta_of(U, P.n_cta, pair * kTopK + kTopK - 1);
+  if (c_lo == c_hi) return;                              // written directly by its CTA
+  float M = -INFINITY;
+  for (int c = c_lo; c <= c_hi; ++c) {
+    const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
+    M = fmaxf(M, P.ws[(static_cast<size_t>(c) * 2 + slot) * kPartial + kHpg * kD + head]);
+  }
+  const float Mu = M == -INFINITY ? 0.f : M;
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = c_lo; c <= c_hi; ++c) {
+    const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
+    const float* part = P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial;
+    const float sc = exp2f(part[kHpg * kD + head] - Mu);
+    L += part[kHpg * kD + kHpg + head] * sc;
+    const float4 v = *reinterpret_cast<const float4*>(part + head * kD + lane * 4);
+    acc.x += v.x * sc;
+    acc.y += v.y * sc;
+    acc.z += v.z * sc;
+    acc.w += v.w * sc;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + lane * 4;
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+}
+
+}  // namespace dattn
+}  // namespace msa

@@ -157,9 +157,10 @@ MSA_API int msa_select_topk(const msa_shape* shape, const float* block_scores, c
  * section "Overview": attention runs only over the selected blocks; the
  * token-level causal mask applies inside the local block).  Softmax and
  * accumulation in float32, output rounded to bf16 (nearest even).  A query
- * with no attended row writes zeros.  `workspace` holds split partial results
- * and must be at least msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE)
- * bytes (it may be NULL when that is 0). */
+ * with no attended row writes zeros.  A persistent grid splits the (pair,
+ * selected block) units evenly over the SMs; `workspace` holds the partial
+ * results of pairs cut between two CTAs (at most 2 per CTA, 256 CTAs) and
+ * must be at least msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE) bytes. */
 MSA_API int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
                            const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
@@ -188,11 +189,12 @@ MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, c
  * start-up, or a program driving the C ABI from a language that has no CUDA
  * allocator of its own.  Such a caller still owns q, the caches, sel and out.
  *
- * The split partial results go to one file-scope device buffer of
+ * The partial results go to one file-scope device buffer of
  * MSA_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
  * the process exits.  A call whose msa_workspace_bytes(shape, n_q,
- * MSA_MODE_DECODE) exceeds that size is rejected with MSA_ERR_WORKSPACE
- * (with 4 groups only n_q = 127 needs more).  The first call on each
+ * MSA_MODE_DECODE) exceeded that size would be rejected with
+ * MSA_ERR_WORKSPACE; the decode partials need at most 256 CTAs x 2 x 8320
+ * bytes = 4,259,840 bytes, so every batch fits.  The first call on each
  * device looks up the buffer's device address (with that device current);
  * make that first call before any stream capture.  All calls share the
  * buffer: calls that can run at the same time on the GPU (different streams,

@@ -109,16 +109,20 @@ def test_select_and_append_validation(lib):
 
 def test_attention_validation_and_workspace(lib):
     s = GOOD.c()
-    # decode with 2 queries x 4 groups = 8 pairs needs split workspace
+    # decode: 2 partials (16 heads x (128 + 2) floats) per CTA, one CTA per
+    # (pair, block) unit at most, 256 CTAs at most
     need = lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_DECODE)
-    assert need == 8 * 16 * 16 * 130 * 4
+    assert need == min(2 * 4 * 16, 256) * 2 * 16 * 130 * 4
+    assert lib.msa_workspace_bytes(ctypes.byref(s), 1000, msa.MODE_DECODE) >= 256 * 2 * 16 * 130 * 4
     assert lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_PREFILL) == 0
     # 4096 queries over 2 streams: prefill-shaped, the block scores take the tile path
     big = lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_DECODE)
     assert big > 0 and big == lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_PREFILL)
-    # 600 decode queries over 600 streams stay on the streaming kernel and split-free attention
+    # 600 decode queries over 600 streams keep the streaming score kernel (no
+    # score workspace): only the attention partials remain
     many = msa.Shape(n_streams=600, capacity=1024).c()
-    assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_DECODE) == 0
+    assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_DECODE) == 256 * 2 * 16 * 130 * 4
+    assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_PREFILL) == 0
     bad = msa.Shape(n_streams=2, capacity=1000).c()
     assert lib.msa_workspace_bytes(ctypes.byref(bad), 2, 0) == ctypes.c_size_t(-1).value
     args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, ctypes.c_float(0.088), FAKE]

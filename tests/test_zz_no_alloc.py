@@ -20,18 +20,23 @@ from block_sparse_attention_maxpool_b200 import build as msa_build
 from tests import parity as PT
 
 
-def test_noalloc_rejects_batches_beyond_the_fixed_buffer():
-    """Host-side size check (no GPU needed): 127 queries x 4 groups need
-    8,453,120 bytes of split partials, more than the 8 MiB buffer."""
+def test_noalloc_buffer_covers_every_batch_and_checks_shapes():
+    """Host-side checks (no GPU needed): the decode partials of any batch fit
+    the fixed buffer (at most 256 CTAs x 2 partials), and bad arguments are
+    rejected before any device work."""
     msa_build.build()
     lib = msa.library()
+    # many streams: decode-shaped batches, so the query measures the attention partials only
+    many = msa.Shape(n_streams=20000, capacity=128).c()
+    for n_q in (1, 3, 127, 128, 4096, 1 << 20):
+        assert 0 < lib.msa_workspace_bytes(ctypes.byref(many), n_q, msa.MODE_DECODE) <= msa.NOALLOC_SCRATCH_BYTES
     sh = msa.Shape(n_streams=1, capacity=4096)
     s = sh.c()
-    assert lib.msa_workspace_bytes(ctypes.byref(s), 127, msa.MODE_DECODE) > msa.NOALLOC_SCRATCH_BYTES
     fake = 0x10000
-    st = lib.msa_sparse_attn_decode_noalloc(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 127,
-                                            ctypes.c_float(0.088), fake, None)
-    assert st == -5
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(s), fake, fake, fake, fake, fake, fake, -1,
+                                              ctypes.c_float(0.088), fake, None) == -4
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(s), 0, fake, fake, fake, fake, fake, 3,
+                                              ctypes.c_float(0.088), fake, None) == -1
     bad = msa.Shape(n_streams=1, capacity=1000).c()
     assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(bad), fake, fake, fake, fake, fake, fake, 1,
                                               ctypes.c_float(0.088), fake, None) == -3
