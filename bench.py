@@ -43,11 +43,11 @@ WORKLOAD = W.DECODE_32K_X32
 
 # DRAM traffic of one block-scores launch on the 32-stream workload, from
 # the ncu capture summarised in profiles/block_scores_gemv_decode_8x32k.md:
-# 536,909,056 B read + 4,248,576 B written on 8 streams, scaled by 4 to 32
+# 536,910,848 B read + 6,198,016 B written on 8 streams, scaled by 4 to 32
 # streams (the reads grow in proportion to the keys scanned).  Valid only
 # for the kernel source it was taken on (sha256 prefix of
 # msa_scores_gemv.cuh); any other source reports null.
-SCORES_TRAFFIC = {"source_sha": "c741d20f2bada528", "bytes_per_launch": 4 * (536_909_056 + 4_248_576)}
+SCORES_TRAFFIC = {"source_sha": "38974ffe0b0592f0", "bytes_per_launch": 4 * (536_910_848 + 6_198_016)}
 
 
 def scores_source_sha() -> str:
