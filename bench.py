@@ -193,24 +193,36 @@ def run_ours(args, rank, world, dev):
     mode = msa.MODE_PREFILL if prefill else msa.MODE_DECODE
     ws = msa.msa_workspace_bytes(shape, n_q, mode)
     bufs["workspace"] = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
-    launches_per_step = 5 + (1 if ws > 0 else 0)
+    # kernels per step: 2 appends, block scores (1 streaming kernel, or 6 on the
+    # tensor-core tile path of prefill batches), select, attention (+ combine in decode)
+    tiles = n_q >= 256 and n_q >= 64 * w.n_streams
+    launches_per_step = 2 + (6 if tiles else 1) + 1 + (1 if prefill else 2)
     stream = torch.cuda.current_stream(dev)
     scale = 1.0 / math.sqrt(shape.head_dim)
 
-    def step(ev=None):
-        msa.msa_indexer_append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], stream)
+    def part_append(st):
+        msa.msa_indexer_append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st)
         msa.msa_kv_append(shape, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
-                          d["tok_pos"], stream)
-        if ev is not None:
-            ev[0].record(stream)
+                          d["tok_pos"], st)
+
+    def part_scores(st):
         msa.msa_block_scores(shape, d["idx_q"], d["idx_k_cache"], d["q_stream"], d["q_pos"],
-                             bufs["block_scores"], stream, bufs["workspace"])
-        if ev is not None:
-            ev[1].record(stream)
-        msa.msa_select_topk(shape, bufs["block_scores"], d["q_pos"], bufs["sel"], bufs["n_sel"], stream)
+                             bufs["block_scores"], st, bufs["workspace"])
+
+    def part_attend(st):
+        msa.msa_select_topk(shape, bufs["block_scores"], d["q_pos"], bufs["sel"], bufs["n_sel"], st)
         attn = msa.msa_sparse_attn_prefill if prefill else msa.msa_sparse_attn_decode
         attn(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"], d["q_pos"], scale,
-             bufs["out"], bufs["workspace"], stream)
+             bufs["out"], bufs["workspace"], st)
+
+    def step(ev=None):
+        part_append(stream)
+        if ev is not None:
+            ev[0].record(stream)
+        part_scores(stream)
+        if ev is not None:
+            ev[1].record(stream)
+        part_attend(stream)
 
     clocks = ClockSampler(dev) if rank == 0 else None
     for _ in range(args.warmup):
@@ -218,6 +230,28 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     if msa.msa_get_device_error(stream) != 0:
         raise RuntimeError("device error during warm-up")
+    graphs = None
+    if not args.no_graph:
+        # The step's launches captured once and replayed: the same kernels on
+        # the same buffers, without per-launch host work.  Three graphs, so
+        # events between them still time the block-score kernel on its own.
+        graphs = [torch.cuda.CUDAGraph() for _ in range(3)]
+        for g, part in zip(graphs, (part_append, part_scores, part_attend)):
+            with torch.cuda.graph(g):
+                part(None)
+        torch.cuda.synchronize(dev)
+
+        def step(ev=None):                                   # noqa: F811  (graph replay)
+            graphs[0].replay()
+            if ev is not None:
+                ev[0].record(stream)
+            graphs[1].replay()
+            if ev is not None:
+                ev[1].record(stream)
+            graphs[2].replay()
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
 
     # ---- device-resident timing -------------------------------------------
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -244,10 +278,15 @@ def run_ours(args, rank, world, dev):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = h_out.numel() * h_out.element_size()
     e2e_steps = max(3, min(args.steps, 200 if not prefill else 20))
+    def api_step():
+        part_append(stream)
+        part_scores(stream)
+        part_attend(stream)
+
     for _ in range(3):
         for n in host_names:
             d[n].copy_(host[n], non_blocking=True)
-        step()
+        api_step()
         h_out.copy_(bufs["out"], non_blocking=True)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -255,7 +294,7 @@ def run_ours(args, rank, world, dev):
     for _ in range(e2e_steps):
         for n in host_names:
             d[n].copy_(host[n], non_blocking=True)
-        step()
+        api_step()
         h_out.copy_(bufs["out"], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -270,10 +309,13 @@ def run_ours(args, rank, world, dev):
 
     peaks = load_peaks()
     if prefill:
-        return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks)
+        return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks,
+                            graphs)
     sbytes = scores_bytes(w)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
-    traffic = SCORES_TRAFFIC["bytes_per_launch"] if SCORES_TRAFFIC["source_sha"] == scores_source_sha() else None
+    traffic = None
+    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD:   # measured for this workload only
+        traffic = SCORES_TRAFFIC["bytes_per_launch"]
     step_gbs = step_bytes(w) / (ms * 1e-3) / 1e9
     line = {
         "metric": METRIC,
@@ -289,6 +331,7 @@ def run_ours(args, rank, world, dev):
         "dtype": "f32 indexer / bf16 attention (f32 accumulate)",
         "data": "synthetic (seeded N(0,1) K/V/Q bf16, indexer N(0,1)/sqrt(128) f32)",
         "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "context": w.l_total,
+                   "launch": "cuda graphs" if graphs is not None else "direct",
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                    "block": w.block, "top_k": w.top_k, "parallelism": f"replicas{world}",
                    "l2": f"inputs {2 * w.n_streams * w.capacity * w.n_kv_heads * 512 / 1e9:.1f} GB per GPU > 126 MB L2, no flush"},
@@ -319,7 +362,8 @@ def prefill_flops(w) -> tuple[int, int]:
     return ind * w.n_streams, att * w.n_streams
 
 
-def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks):
+def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks,
+                 graphs=None):
     ind, att = prefill_flops(w)
     tokens = w.n_queries * world
     tf = (ind + att) / (ms * 1e-3) / 1e12
@@ -330,7 +374,8 @@ def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 indexer / bf16 attention (f32 accumulate)", "data": "synthetic",
         "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "new_tokens": w.n_new,
-                   "context": w.l_total, "parallelism": f"replicas{world}"},
+                   "context": w.l_total, "parallelism": f"replicas{world}",
+                   "launch": "cuda graphs" if graphs is not None else "direct"},
         "step_tensor": {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
                         "frac": tf / peaks["bf16_tflops"], "indexer_flops": ind, "attention_flops": att},
         "roofline": {"kernel": "block_scores", "bound": "tensor", "achieved": ktf, "peak": peaks["bf16_tflops"],
@@ -408,6 +453,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel from Python in the timed loop instead of replaying CUDA graphs")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD.name,
                     help="workload to time (default: the 32-stream 32K decode benchmark)")
     ap.add_argument("--streams", type=int, default=None,

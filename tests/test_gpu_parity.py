@@ -120,7 +120,7 @@ def _random_selection(g, q_pos, G, top_k=16):
 
 
 @pytest.mark.parametrize("n_q,mode", [(1, "decode"), (3, "decode"), (20, "decode"), (40, "decode"),
-                                      (70, "decode"), (150, "decode"), (37, "prefill")])
+                                      (70, "decode"), (150, "decode"), (300, "decode"), (37, "prefill")])
 def test_attention_given_selection(n_q, mode):
     g = torch.Generator().manual_seed(n_q)
     S, cap, G = 3, 128 * 24, 4
@@ -233,6 +233,43 @@ def test_step_small_chunked_prefill_with_ties():
 def test_step_decode_mixed_streams():
     w = W.Workload("decode_6x3000", 6, 2999, 3000, "last")
     report(w.name, PT.full_parity(W.make_inputs(w, seed=3)))
+
+
+@pytest.mark.parametrize("G", [1, 2, 8])
+def test_step_other_group_counts(G):
+    """1, 2 or 8 KV/indexer groups (16 query heads each): decode across
+    streams, and a prefill batch that takes the tensor-core tile path."""
+    dec = W.Workload(f"decode_3x1500_g{G}", 3, 1499, 1500, "last", n_kv_heads=G, n_q_heads=16 * G)
+    report(dec.name, PT.full_parity(W.make_inputs(dec, seed=20 + G)))
+    pre = W.Workload(f"prefill_1x700_g{G}", 1, 0, 700, "new", n_kv_heads=G, n_q_heads=16 * G)
+    report(pre.name, PT.full_parity(W.make_inputs(pre, seed=30 + G), prefill=True))
+
+
+def test_step_single_block_capacity():
+    """Capacity of one 128-slot block: every query sees one (partial) block."""
+    w = W.Workload("prefill_2x100_cap128", 2, 0, 100, "new")
+    report(w.name, PT.full_parity(W.make_inputs(w, seed=9), prefill=True))
+    d = W.Workload("decode_5x128", 5, 127, 128, "last")
+    report(d.name, PT.full_parity(W.make_inputs(d, seed=10)))
+
+
+def test_decode_attention_invalid_query_in_shared_pair():
+    """An invalid query among valid ones in the stream-K decode kernel: its
+    pairs write zeros and set the error bit, the others stay exact."""
+    S, cap = 2, 128 * 20
+    qpos = [(0, cap - 1), (1, 1700), (0, 900)]
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, [cap, 1800], qpos, seed=14)
+    g = torch.Generator().manual_seed(14)
+    sel = _random_selection(g, qp, 4)
+    qs_bad = qs.clone()
+    qs_bad[1] = 5                      # stream 5 does not exist
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    out = msa.msa_sparse_attn_decode(sh, q.cuda(), k.cuda(), v.cuda(), sel.cuda(), qs_bad.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() & 0x1
+    out = out.cpu()
+    assert out[1].eq(0).all()
+    want = oracle.sparse_attention(q, k, v, sel, qs, qp, 128, queries=[0, 2])
+    PT.check_attention(out[[0, 2]], want[[0, 2]])
 
 
 def test_step_is_deterministic():
