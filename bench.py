@@ -43,11 +43,11 @@ WORKLOAD = W.DECODE_32K_X32
 
 # DRAM traffic of one block-scores launch on the 32-stream workload, from
 # the ncu capture summarised in profiles/block_scores_gemv_decode_8x32k.md:
-# 536,910,848 B read + 6,198,016 B written on 8 streams, scaled by 4 to 32
+# 536,910,848 B read + 3,630,336 B written on 8 streams, scaled by 4 to 32
 # streams (the reads grow in proportion to the keys scanned).  Valid only
 # for the kernel source it was taken on (sha256 prefix of
 # msa_scores_gemv.cuh); any other source reports null.
-SCORES_TRAFFIC = {"source_sha": "38974ffe0b0592f0", "bytes_per_launch": 4 * (536_910_848 + 6_198_016)}
+SCORES_TRAFFIC = {"source_sha": "f1bdebf997a9634d", "bytes_per_launch": 4 * (536_910_848 + 3_630_336)}
 
 
 def scores_source_sha() -> str:
@@ -66,22 +66,22 @@ def load_peaks() -> dict:
 # ---------------------------------------------------------------------------
 # algorithmic bytes
 # ---------------------------------------------------------------------------
-def scores_bytes(w) -> int:
+def scores_bytes(w, key_bytes: int = 4) -> int:
     """Bytes the block-score kernel must move per launch: every visible
-    indexer key once (512 B per key per group), the indexer queries, and the
-    block-score output."""
+    indexer key once (512 B per key per group; 256 B with the F16 cache),
+    the indexer queries, and the block-score output."""
     G, Di = w.n_kv_heads, w.idx_dim
     n_q = w.n_queries
-    keys = n_q * G * w.l_total * Di * 4           # decode: each query sees l_total keys
+    keys = n_q * G * w.l_total * Di * key_bytes   # decode: each query sees l_total keys
     return keys + n_q * G * Di * 4 + n_q * G * (w.capacity // w.block) * 4
 
 
-def step_bytes(w) -> int:
+def step_bytes(w, key_bytes: int = 4) -> int:
     """Bytes one decode step must move: visible indexer keys, the 16 selected
     K/V blocks per group, the query and the output (the plan's per-stream
     count: 67,108,864 + 4,194,304 + 34,816 at 32K context)."""
     G, D = w.n_kv_heads, w.head_dim
-    idx = w.l_total * G * w.idx_dim * 4
+    idx = w.l_total * G * w.idx_dim * key_bytes
     kv = min(w.top_k, w.l_total // w.block + 1) * w.block * G * D * 2 * 2
     qo = w.n_q_heads * D * 2 * 2 + G * w.idx_dim * 4
     return (idx + kv + qo) * w.n_streams
@@ -182,6 +182,9 @@ def run_ours(args, rank, world, dev):
                                                "tok_pos", "idx_k_new", "k_new", "v_new",
                                                "q_stream", "q_pos", "idx_q", "q")}
     del inp
+    if args.idx_f16:
+        d["idx_k_cache"] = d["idx_k_cache"].half()         # F16 indexer-key cache variant
+    key_bytes = 2 if args.idx_f16 else 4
     n_q = w.n_queries
     G = w.n_kv_heads
     bufs = {
@@ -201,7 +204,8 @@ def run_ours(args, rank, world, dev):
     scale = 1.0 / math.sqrt(shape.head_dim)
 
     def part_append(st):
-        msa.msa_indexer_append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st)
+        append = msa.msa_indexer_append_f16 if args.idx_f16 else msa.msa_indexer_append
+        append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st)
         msa.msa_kv_append(shape, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
                           d["tok_pos"], st)
 
@@ -311,14 +315,14 @@ def run_ours(args, rank, world, dev):
     if prefill:
         return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks,
                             graphs)
-    sbytes = scores_bytes(w)
+    sbytes = scores_bytes(w, key_bytes)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     traffic = None
-    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD:   # measured for this workload only
-        traffic = SCORES_TRAFFIC["bytes_per_launch"]
-    step_gbs = step_bytes(w) / (ms * 1e-3) / 1e9
+    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD and not args.idx_f16:
+        traffic = SCORES_TRAFFIC["bytes_per_launch"]          # measured for this workload only
+    step_gbs = step_bytes(w, key_bytes) / (ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC,
+        "metric": METRIC if not args.idx_f16 else METRIC.replace("x32 streams", "x32 streams, F16 indexer cache"),
         "value": job_tokens_per_s(w.n_streams, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -328,7 +332,7 @@ def run_ours(args, rank, world, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32 indexer / bf16 attention (f32 accumulate)",
+        "dtype": ("f16" if args.idx_f16 else "f32") + " indexer / bf16 attention (f32 accumulate)",
         "data": "synthetic (seeded N(0,1) K/V/Q bf16, indexer N(0,1)/sqrt(128) f32)",
         "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "context": w.l_total,
                    "launch": "cuda graphs" if graphs is not None else "direct",
@@ -336,7 +340,7 @@ def run_ours(args, rank, world, dev):
                    "block": w.block, "top_k": w.top_k, "parallelism": f"replicas{world}",
                    "l2": f"inputs {2 * w.n_streams * w.capacity * w.n_kv_heads * 512 / 1e9:.1f} GB per GPU > 126 MB L2, no flush"},
         "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peaks["hbm_gbs"],
-                     "frac": step_gbs / peaks["hbm_gbs"], "bytes_per_step": step_bytes(w)},
+                     "frac": step_gbs / peaks["hbm_gbs"], "bytes_per_step": step_bytes(w, key_bytes)},
         "roofline": {"kernel": "block_scores_gemv", "bound": "hbm", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "algorithmic_bytes": sbytes, "ms_per_launch": k_ms,
@@ -453,6 +457,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--idx-f16", action="store_true",
+                    help="decode with the F16 indexer-key cache variant instead of the F32 cache")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from Python in the timed loop instead of replaying CUDA graphs")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD.name,
@@ -481,7 +487,7 @@ def main():
     try:
         line = run_ours(args, rank, world, local)
         if line is not None:
-            if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name:
+            if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name and not args.idx_f16:
                 line["cpu_baseline"] = cpu_baseline()
             print(json.dumps(line), flush=True)
     finally:

@@ -18,6 +18,7 @@ from dataclasses import dataclass
 import torch
 
 __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_block_scores",
+           "msa_indexer_append_f16",
            "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
            "msa_workspace_bytes", "msa_get_device_error", "msa_sparse_attn_decode_noalloc", "msa_version", "library", "LIB_PATH",
            "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step"]
@@ -74,6 +75,9 @@ _SIGS = {
     "msa_kv_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I, _P]),
     "msa_block_scores": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t,
                                         _P]),
+    "msa_block_scores_f16": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P,
+                                            ctypes.c_size_t, _P]),
+    "msa_indexer_append_f16": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P]),
     "msa_select_topk": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I, _P, _P, _P]),
     "msa_sparse_attn_decode": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
                                               ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
@@ -169,17 +173,36 @@ def _workspace(shape: Shape, n: int, mode: int, workspace, device):
     return _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), workspace
 
 
+def msa_indexer_append_f16(shape: Shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, stream=None):
+    """F16 indexer-key cache variant of msa_indexer_append (float16 cache;
+    the new F32 keys are rounded to fp16 as they are written)."""
+    n = _n(tok_stream, "tok_stream")
+    s = shape.c()
+    _check("msa_indexer_append_f16", library().msa_indexer_append_f16(
+        ctypes.byref(s),
+        _ptr(idx_k_cache, torch.float16, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
+        _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
+        _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+        n, _stream(stream)))
+
+
 def msa_block_scores(shape: Shape, idx_q, idx_k_cache, q_stream, q_pos, block_scores=None, stream=None,
                      workspace=None):
+    """Block scores over the F32 indexer-key cache, or over the F16 cache
+    variant when idx_k_cache is a float16 tensor."""
     n = _n(q_pos, "q_pos")
+    if idx_k_cache.dtype == torch.float16:
+        fn, kdt = "msa_block_scores_f16", torch.float16
+    else:
+        fn, kdt = "msa_block_scores", torch.float32
     if block_scores is None:
         block_scores = torch.empty((n, shape.n_kv_heads, shape.n_blocks), dtype=torch.float32,
                                    device=idx_q.device)
     ws_ptr, ws_bytes, _keep = _workspace(shape, n, MODE_DECODE, workspace, idx_q.device)
     s = shape.c()
-    _check("msa_block_scores", library().msa_block_scores(
+    _check(fn, getattr(library(), fn)(
         ctypes.byref(s), _ptr(idx_q, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_q"),
-        _ptr(idx_k_cache, torch.float32, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
+        _ptr(idx_k_cache, kdt, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
         _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
         _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
         ws_ptr, ws_bytes, _stream(stream)))
@@ -286,14 +309,15 @@ def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None,
     """One MSA step through the C ABI: append the new tokens' indexer keys
     and K/V rows, score blocks, select the top-k and attend.
 
-    caches: idx_k_cache, k_cache, v_cache (device); new: tok_stream, tok_pos,
+    caches: idx_k_cache (float32, or float16 for the F16 cache variant),
+    k_cache, v_cache (device); new: tok_stream, tok_pos,
     idx_k_new, k_new, v_new, q_stream, q_pos, idx_q, q (device).  ``bufs`` may
     hold preallocated block_scores / sel / n_sel / out / workspace.
     Returns (out, sel, n_sel, block_scores).
     """
     b = bufs or {}
-    msa_indexer_append(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"],
-                       new["tok_pos"], stream)
+    append = msa_indexer_append_f16 if caches["idx_k_cache"].dtype == torch.float16 else msa_indexer_append
+    append(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"], new["tok_pos"], stream)
     msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
                   new["tok_stream"], new["tok_pos"], stream)
     n = new["q_pos"].shape[0]

@@ -4,6 +4,7 @@
 // unit, so the per-device error word needs no relocatable device code).
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -220,27 +221,12 @@ int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache
   return cuda_status(cudaGetLastError());
 }
 
-}  // namespace
-
-extern "C" {
-
-int msa_indexer_append(const msa_shape* shape, float* idx_k_cache, const float* idx_k_new,
-                       const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
-  return append_rows(shape, idx_k_cache, idx_k_new, nullptr, nullptr, tok_stream, tok_pos, n_tok,
-                     128 * static_cast<int>(sizeof(float)), stream);
-}
-
-int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, const msa_bf16* k_new,
-                  const msa_bf16* v_new, const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok,
-                  void* stream) {
-  if (n_tok > 0 && (!v_cache || !v_new)) return MSA_ERR_NULL;
-  return append_rows(shape, k_cache, k_new, v_cache, v_new, tok_stream, tok_pos, n_tok,
-                     128 * static_cast<int>(sizeof(msa_bf16)), stream);
-}
-
-int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
-                     const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+template <typename KeyT>
+int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* idx_k_cache,
+                      const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  constexpr bool kF16 = std::is_same<KeyT, __half>::value;
+  constexpr int kStagesT = kScoreStages;                              // 32 KB stages for either key type
   int st = check_shape(shape);
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
@@ -261,7 +247,7 @@ int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* id
   const int cap = shape->capacity;
 
   using namespace msa::gemv;
-  Params P;
+  Params<KeyT> P;
   P.idx_q = idx_q;
   P.idx_k = idx_k_cache;
   P.q_stream = q_stream;
@@ -275,9 +261,9 @@ int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* id
   P.n_tasks = static_cast<long long>(n_q) * G * P.nblk;
   P.q_list = nullptr;
   P.q_count = nullptr;
-  const size_t smem = sizeof(Smem<kScoreStages>);
+  const size_t smem = sizeof(Smem<KeyT, kStagesT>);
   static std::atomic<uint64_t> smem_done{0};
-  if ((st = ensure_smem(block_scores_gemv_kernel<kScoreStages>, smem, smem_done)) != MSA_OK) return st;
+  if ((st = ensure_smem(block_scores_gemv_kernel<KeyT, kStagesT>, smem, smem_done)) != MSA_OK) return st;
 
   if (tiles) {
     namespace T = msa::tc;
@@ -285,7 +271,8 @@ int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* id
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     T::Params Q;
     Q.idx_q = idx_q;
-    Q.idx_k = idx_k_cache;
+    Q.idx_k = kF16 ? nullptr : reinterpret_cast<const float*>(idx_k_cache);
+    Q.idx_k16 = kF16 ? reinterpret_cast<const __half*>(idx_k_cache) : nullptr;
     Q.q_stream = q_stream;
     Q.q_pos = q_pos;
     Q.bs = block_scores;
@@ -328,12 +315,61 @@ int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* id
     // queries of mixed-stream tiles: streaming kernel over the leftover list
     P.q_list = Q.leftover;
     P.q_count = Q.counters;
-    block_scores_gemv_kernel<kScoreStages><<<static_cast<unsigned>(sms), kThreads, smem, cs>>>(P);
+    block_scores_gemv_kernel<KeyT, kStagesT><<<static_cast<unsigned>(sms), kThreads, smem, cs>>>(P);
     return cuda_status(cudaGetLastError());
   }
 
   const long long grid = std::min<long long>(sms, P.n_tasks);
-  block_scores_gemv_kernel<kScoreStages><<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(P);
+  block_scores_gemv_kernel<KeyT, kStagesT><<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(P);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+int msa_indexer_append(const msa_shape* shape, float* idx_k_cache, const float* idx_k_new,
+                       const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
+  return append_rows(shape, idx_k_cache, idx_k_new, nullptr, nullptr, tok_stream, tok_pos, n_tok,
+                     128 * static_cast<int>(sizeof(float)), stream);
+}
+
+int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, const msa_bf16* k_new,
+                  const msa_bf16* v_new, const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok,
+                  void* stream) {
+  if (n_tok > 0 && (!v_cache || !v_new)) return MSA_ERR_NULL;
+  return append_rows(shape, k_cache, k_new, v_cache, v_new, tok_stream, tok_pos, n_tok,
+                     128 * static_cast<int>(sizeof(msa_bf16)), stream);
+}
+
+int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
+                     const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return block_scores_impl<float>(shape, idx_q, idx_k_cache, q_stream, q_pos, n_q, block_scores, workspace,
+                                  workspace_bytes, stream);
+}
+
+int msa_block_scores_f16(const msa_shape* shape, const float* idx_q, const msa_f16* idx_k_cache,
+                         const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return block_scores_impl<__half>(shape, idx_q, reinterpret_cast<const __half*>(idx_k_cache), q_stream, q_pos,
+                                   n_q, block_scores, workspace, workspace_bytes, stream);
+}
+
+int msa_indexer_append_f16(const msa_shape* shape, msa_f16* idx_k_cache, const float* idx_k_new,
+                           const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
+  int st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_tok < 0) return MSA_ERR_RANGE;
+  if (n_tok == 0) return MSA_OK;
+  if (!idx_k_cache || !idx_k_new || !tok_stream || !tok_pos) return MSA_ERR_NULL;
+  if (!aligned16(idx_k_cache) || !aligned16(idx_k_new)) return MSA_ERR_ALIGN;
+  const int64_t warps = static_cast<int64_t>(n_tok) * shape->n_kv_heads;
+  if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
+  msa::append_idx_f16_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<__half*>(idx_k_cache), idx_k_new, tok_stream, tok_pos, n_tok, shape->n_streams,
+      shape->n_kv_heads, shape->capacity);
   return cuda_status(cudaGetLastError());
 }
 

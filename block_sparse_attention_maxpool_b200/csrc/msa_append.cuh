@@ -4,6 +4,8 @@
 // per (token, group) row, 16-byte vector loads and stores.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -40,6 +42,34 @@ __global__ void __launch_bounds__(256) append_rows_kernel(
       *d = __ldg(c);
     }
   }
+}
+
+// F16 indexer-key cache variant: each F32 key of 128 values is rounded to
+// fp16 (nearest even) as it is written.  One warp per (token, group) row,
+// four values per lane.
+__global__ void __launch_bounds__(256) append_idx_f16_kernel(__half* __restrict__ cache,
+                                                             const float* __restrict__ src,
+                                                             const int32_t* __restrict__ tok_stream,
+                                                             const int32_t* __restrict__ tok_pos, int n_tok,
+                                                             int n_streams, int n_groups, int capacity) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_tok * n_groups) return;
+  const int t = warp / n_groups;
+  const int g = warp - t * n_groups;
+  const int s = tok_stream[t];
+  const int p = tok_pos[t];
+  if (s < 0 || s >= n_streams || p < 0 || p >= capacity) {
+    if (g == 0 && lane == 0) raise_error(MSA_DEVERR_TOKEN_RANGE);
+    return;
+  }
+  const float4 x = __ldg(reinterpret_cast<const float4*>(src + (static_cast<size_t>(t) * n_groups + g) * 128) + lane);
+  const __half2 a = __floats2half2_rn(x.x, x.y);
+  const __half2 b = __floats2half2_rn(x.z, x.w);
+  uint2 out;
+  out.x = *reinterpret_cast<const uint32_t*>(&a);
+  out.y = *reinterpret_cast<const uint32_t*>(&b);
+  *(reinterpret_cast<uint2*>(cache + ((static_cast<size_t>(s) * n_groups + g) * capacity + p) * 128) + lane) = out;
 }
 
 }  // namespace msa

@@ -84,7 +84,8 @@ __host__ inline Workspace workspace_layout(int n_q, int G, int S, int cap) {
 
 struct Params {
   const float* idx_q;       // [n_q][G][Di]
-  const float* idx_k;       // [S][G][cap][Di]
+  const float* idx_k;       // [S][G][cap][Di] F32 cache (null when idx_k16 is used)
+  const __half* idx_k16;    // [S][G][cap][Di] F16 cache variant (null for the F32 cache)
   const int32_t* q_stream;
   const int32_t* q_pos;
   float* bs;                // [n_q][G][nblk]
@@ -221,7 +222,15 @@ __global__ void __launch_bounds__(256) tc_split_keys_kernel(const Params P) {
   const int j = static_cast<int>(w % P.capacity);
   const int s = static_cast<int>(w / (static_cast<long long>(P.G) * P.capacity));
   if (j >= P.counters[1 + s] * kBlock) return;
-  const float4 x = __ldcs(reinterpret_cast<const float4*>(P.idx_k + w * kDi) + lane);
+  float4 x;
+  if (P.idx_k16 != nullptr) {
+    const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(P.idx_k16 + w * kDi) + lane);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+    x = make_float4(a.x, a.y, b.x, b.y);
+  } else {
+    x = __ldcs(reinterpret_cast<const float4*>(P.idx_k + w * kDi) + lane);
+  }
   __half2 hi[2], lo[2];
   const int e = split_row4(x, hi, lo);
   *reinterpret_cast<uint2*>(P.khi + w * kDi + lane * 4) =

@@ -83,6 +83,9 @@ extern "C" {
 /* Bit pattern of an IEEE bfloat16 value. */
 typedef uint16_t msa_bf16;
 
+/* Bit pattern of an IEEE binary16 (fp16) value. */
+typedef uint16_t msa_f16;
+
 typedef struct msa_shape {
   int32_t n_streams;   /* S: independent sequences, one cache region each      */
   int32_t capacity;    /* slots per stream, a multiple of block                */
@@ -137,6 +140,25 @@ MSA_API int msa_block_scores(const msa_shape* shape, const float* idx_q, const f
                      const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
                      float* block_scores, void* workspace, size_t workspace_bytes,
                      void* stream);
+
+/* F16 indexer-key cache variant.  The MSA pull request keeps the indexer
+ * cache in F32 by default ("set default cache type to F32", MSA branch
+ * commit message) and its review thread compares F16 against F32 indexer
+ * precision (IF16 vs IF32 KL divergence); these two calls are the F16 cache
+ * type: keys are stored as fp16, which halves the bytes a decode step
+ * streams.  msa_indexer_append_f16 rounds each F32 key value to fp16
+ * (nearest even) as it writes idx_k_cache [S][G][cap][Di] (fp16 bits);
+ * msa_block_scores_f16 computes exactly what msa_block_scores computes on the
+ * fp16 keys (each converted exactly to F32, F32 accumulation, same pooling,
+ * bias, layouts, workspace and errors).  Selection and attention calls are
+ * unchanged. */
+MSA_API int msa_indexer_append_f16(const msa_shape* shape, msa_f16* idx_k_cache, const float* idx_k_new,
+                                   const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok,
+                                   void* stream);
+MSA_API int msa_block_scores_f16(const msa_shape* shape, const float* idx_q, const msa_f16* idx_k_cache,
+                                 const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                                 float* block_scores, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /* msa_select_topk - top-k block selection per (query, group).
  * Ranks the visible blocks b <= q_pos/128 by (score descending, block index

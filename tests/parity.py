@@ -40,10 +40,13 @@ def shape_of(w) -> msa.Shape:
                      block=w.block, top_k=w.top_k)
 
 
-def to_dev(inp, dev="cuda"):
+def to_dev(inp, dev="cuda", idx_f16=False):
     names = ["idx_k_cache", "k_cache", "v_cache", "tok_stream", "tok_pos", "idx_k_new", "k_new",
              "v_new", "q_stream", "q_pos", "idx_q", "q"]
-    return {n: getattr(inp, n).to(dev).contiguous() for n in names}
+    d = {n: getattr(inp, n).to(dev).contiguous() for n in names}
+    if idx_f16:
+        d["idx_k_cache"] = d["idx_k_cache"].half()
+    return d
 
 
 def run_step(shape, d, prefill=False):
@@ -53,8 +56,13 @@ def run_step(shape, d, prefill=False):
     return out, sel, n_sel, bs, err
 
 
-def oracle_caches(inp):
-    idx = oracle.indexer_append(inp.idx_k_cache, inp.idx_k_new, inp.tok_stream, inp.tok_pos)
+def oracle_caches(inp, idx_f16=False):
+    """The caches after the step's append.  With the F16 indexer-cache variant
+    the keys are the F32 keys rounded to fp16 by torch (nearest even)."""
+    if idx_f16:
+        idx = oracle.indexer_append(inp.idx_k_cache.half(), inp.idx_k_new.half(), inp.tok_stream, inp.tok_pos)
+    else:
+        idx = oracle.indexer_append(inp.idx_k_cache, inp.idx_k_new, inp.tok_stream, inp.tok_pos)
     k = oracle.indexer_append(inp.k_cache, inp.k_new, inp.tok_stream, inp.tok_pos)
     v = oracle.indexer_append(inp.v_cache, inp.v_new, inp.tok_stream, inp.tok_pos)
     return idx, k, v
@@ -130,15 +138,15 @@ def check_attention(out_gpu, out_orc, rows=None):
     return float((g - w).abs().max()), mean
 
 
-def full_parity(inp, queries=None, prefill=False, dev="cuda"):
+def full_parity(inp, queries=None, prefill=False, dev="cuda", idx_f16=False):
     """Run one step on the GPU and compare every part with the oracle on the
     query indices ``queries`` (all when None).  Returns a small report."""
     w = inp.w
     shape = shape_of(w)
-    d = to_dev(inp, dev)
+    d = to_dev(inp, dev, idx_f16)
     out, sel, n_sel, bs, err = run_step(shape, d, prefill)
     assert err == 0, f"device error word {err:#x}"
-    idx_o, k_o, v_o = oracle_caches(inp)
+    idx_o, k_o, v_o = oracle_caches(inp, idx_f16)
     assert torch.equal(d["idx_k_cache"].cpu(), idx_o), "indexer cache after append"
     assert torch.equal(d["k_cache"].cpu(), k_o) and torch.equal(d["v_cache"].cpu(), v_o), "K/V append"
     n_q = inp.q_pos.numel()

@@ -272,6 +272,23 @@ def test_decode_attention_invalid_query_in_shared_pair():
     PT.check_attention(out[[0, 2]], want[[0, 2]])
 
 
+@pytest.mark.parametrize("case", ["decode", "prefill", "ties"])
+def test_step_f16_indexer_cache(case):
+    """F16 indexer-key cache variant: append rounds keys to fp16 (bit-exact
+    with torch's rounding), block scores on fp16 keys within the float32
+    bound, selection and attention as for the F32 cache."""
+    if case == "decode":
+        w, kw = W.Workload("decode_5x2600_f16", 5, 2599, 2600, "last"), {}
+    elif case == "prefill":
+        w, kw = W.Workload("prefill_1x1500_f16", 1, 0, 1500, "new"), {"prefill": True}
+    else:
+        w, kw = W.Workload("chunk_2x400_on_1600_ties_f16", 2, 1600, 2000, "new", quantize_idx=True), {"prefill": True}
+    rep = PT.full_parity(W.make_inputs(w, seed=41), idx_f16=True, **kw)
+    report(w.name, rep)
+    if case == "ties":
+        assert rep["near_ties"] == 0 and rep["max_score_err"] == 0.0
+
+
 def test_step_is_deterministic():
     w = W.Workload("decode_4x2200", 4, 2199, 2200, "last")
     inp = W.make_inputs(w, seed=4)
@@ -295,6 +312,7 @@ def test_workload_decode_1x4k_full():
 def test_workload_decode_32x32k_sampled():
     inp = W.make_inputs(W.DECODE_32K_X32)
     report(W.DECODE_32K_X32.name, PT.full_parity(inp, queries=[0, 7, 19, 31]))
+    report(W.DECODE_32K_X32.name + " f16 indexer cache", PT.full_parity(inp, queries=[3, 30], idx_f16=True))
 
 
 def test_workload_decode_8x128k_sampled():
