@@ -41,13 +41,14 @@ import workloads as W  # noqa: E402
 METRIC = "MSA decode tokens/s @32K ctx x32 streams; achieved HBM GB/s vs peak"
 WORKLOAD = W.DECODE_32K_X32
 
-# DRAM traffic of one block-scores launch on the 32-stream workload, from
-# the ncu capture summarised in profiles/block_scores_gemv_decode_8x32k.md:
-# 536,910,848 B read + 3,630,336 B written on 8 streams, scaled by 4 to 32
-# streams (the reads grow in proportion to the keys scanned).  Valid only
-# for the kernel source it was taken on (sha256 prefix of
-# msa_scores_gemv.cuh); any other source reports null.
-SCORES_TRAFFIC = {"source_sha": "f1bdebf997a9634d", "bytes_per_launch": 4 * (536_910_848 + 3_630_336)}
+# DRAM traffic of one block-scores launch on the 32-stream workload, per key
+# type, from the ncu captures summarised in
+# profiles/block_scores_gemv_decode_8x32k.md: bytes read + written on 8
+# streams, scaled by 4 to 32 streams (the reads grow in proportion to the
+# keys scanned).  Valid only for the kernel source it was taken on (sha256
+# prefix of msa_scores_gemv.cuh); any other source reports null.
+SCORES_TRAFFIC = {"source_sha": "7065233549d01316",
+                  "bytes_per_launch": {"f32": 4 * (536_908_544 + 3_283_712), "f16": 4 * (268_472_832 + 3_113_984)}}
 
 
 def scores_source_sha() -> str:
@@ -318,8 +319,8 @@ def run_ours(args, rank, world, dev):
     sbytes = scores_bytes(w, key_bytes)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     traffic = None
-    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD and not args.idx_f16:
-        traffic = SCORES_TRAFFIC["bytes_per_launch"]          # measured for this workload only
+    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD:
+        traffic = SCORES_TRAFFIC["bytes_per_launch"]["f16" if args.idx_f16 else "f32"]   # this workload only
     step_gbs = step_bytes(w, key_bytes) / (ms * 1e-3) / 1e9
     line = {
         "metric": METRIC if not args.idx_f16 else METRIC.replace("x32 streams", "x32 streams, F16 indexer cache"),

@@ -21,7 +21,6 @@
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
-constexpr int kScoreStages = 4;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -226,7 +225,7 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
                       const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
                       void* workspace, size_t workspace_bytes, void* stream) {
   constexpr bool kF16 = std::is_same<KeyT, __half>::value;
-  constexpr int kStagesT = kScoreStages;                              // 32 KB stages for either key type
+  using Cfg = msa::gemv::Config<KeyT>;
   int st = check_shape(shape);
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
@@ -261,9 +260,11 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
   P.n_tasks = static_cast<long long>(n_q) * G * P.nblk;
   P.q_list = nullptr;
   P.q_count = nullptr;
-  const size_t smem = sizeof(Smem<KeyT, kStagesT>);
+  const size_t smem = sizeof(Smem<KeyT, Cfg::kStages, Cfg::kWarps>);
+  const auto kernel = block_scores_gemv_kernel<KeyT, Cfg::kStages, Cfg::kWarps, Cfg::kCtasPerSm>;
+  constexpr int kThreads = (Cfg::kWarps + 1) * 32;
   static std::atomic<uint64_t> smem_done{0};
-  if ((st = ensure_smem(block_scores_gemv_kernel<KeyT, kStagesT>, smem, smem_done)) != MSA_OK) return st;
+  if ((st = ensure_smem(kernel, smem, smem_done)) != MSA_OK) return st;
 
   if (tiles) {
     namespace T = msa::tc;
@@ -315,12 +316,12 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
     // queries of mixed-stream tiles: streaming kernel over the leftover list
     P.q_list = Q.leftover;
     P.q_count = Q.counters;
-    block_scores_gemv_kernel<KeyT, kStagesT><<<static_cast<unsigned>(sms), kThreads, smem, cs>>>(P);
+    kernel<<<static_cast<unsigned>(Cfg::kCtasPerSm * sms), kThreads, smem, cs>>>(P);
     return cuda_status(cudaGetLastError());
   }
 
-  const long long grid = std::min<long long>(sms, P.n_tasks);
-  block_scores_gemv_kernel<KeyT, kStagesT><<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(P);
+  const long long grid = std::min<long long>(static_cast<long long>(Cfg::kCtasPerSm) * sms, P.n_tasks);
+  kernel<<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(P);
   return cuda_status(cudaGetLastError());
 }
 

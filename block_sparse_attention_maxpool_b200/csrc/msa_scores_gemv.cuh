@@ -14,7 +14,8 @@
 // each take 8 rows of a chunk (one 16-byte load per lane per row, so a row
 // is one conflict-free 512-byte shared-memory read) and reduce the 8 partial
 // dot products across the warp with a transposed butterfly (9 shuffles for
-// 8 rows).  Rows past the query position are masked, the per-block maximum
+// 8 rows).  The F16 cache variant runs two CTAs per SM, each with a 3-stage
+// ring, and reduces half-warp row pairs the same way.  Rows past the query position are masked, the per-block maximum
 // is combined across warps and the local block gets MSA_LOCAL_BIAS.
 #pragma once
 
@@ -28,33 +29,42 @@ namespace gemv {
 constexpr int kDi = 128;                                 // indexer dim
 constexpr int kBlock = 128;                              // key block
 constexpr uint32_t kStageBytes = 32 * 1024;              // one chunk of key rows
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
 
-// KeyT: float (the F32 cache) or __half (the F16 cache variant).  A 32 KB
-// chunk holds 64 F32 key rows or 128 F16 key rows (one block).
+// Launch shape per key type: consumer warps, ring stages and resident CTAs
+// per SM (the grid is that many CTAs per SM, each with the ring in shared
+// memory).
 template <typename KeyT>
-struct Rows {
-  static constexpr int kPerStage = kStageBytes / (kDi * sizeof(KeyT));
-  static constexpr int kPerWarp = kPerStage / kConsumerWarps;   // 8 (F32) or 16 (F16)
+struct Config;
+template <>
+struct Config<float> {
+  static constexpr int kWarps = 8, kStages = 4, kCtasPerSm = 1;
+};
+template <>
+struct Config<__half> {   // twice the blocks per byte: two independent rings per SM hide the per-block joins
+  static constexpr int kWarps = 8, kStages = 3, kCtasPerSm = 2;
 };
 
-template <typename KeyT, int kStages>
+// KeyT: float (the F32 cache) or __half (the F16 cache variant).  A 32 KB
+// chunk holds 64 F32 key rows or 128 F16 key rows (one block).  An F32 row
+// spans the warp (4 values per lane); an F16 row spans a half-warp (8 values
+// per lane), so one 16-byte load per lane covers two rows.
+template <typename KeyT, int kWarps>
+struct Rows {
+  static constexpr int kPerStage = kStageBytes / (kDi * sizeof(KeyT));
+  static constexpr int kPerWarp = kPerStage / kWarps;
+  static constexpr int kPerLoad = sizeof(KeyT) == 2 ? 2 : 1;
+  static constexpr int kPartials = kPerWarp / kPerLoad;   // dot products per lane per chunk
+  static constexpr int kLanesPerRow = 32 / kPerLoad;
+  static_assert(kPerWarp * kWarps == kPerStage && kPartials >= 1, "rows must split evenly over warps");
+};
+
+template <typename KeyT, int kStages, int kWarps>
 struct Smem {
   KeyT stage[kStages][kStageBytes / sizeof(KeyT)];
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  float red[2][kConsumerWarps];
+  float red[2][kWarps];
 };
-
-// Four consecutive key elements as float.
-__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ float4 load4(const __half* p) {
-  const uint2 raw = *reinterpret_cast<const uint2*>(p);
-  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-  return make_float4(a.x, a.y, b.x, b.y);
-}
 
 template <typename KeyT>
 struct Params {
@@ -69,84 +79,95 @@ struct Params {
   const int32_t* q_count;  // ... of which there are *q_count (device memory)
 };
 
-// Task t -> (query, group, block); in list mode the query comes from q_list.
+// Walks the task space (query slot, group, block) in order, block fastest,
+// without a division per task; the query's stream, position and visible
+// block count are re-read only when the query slot changes.
 template <typename KeyT>
-__device__ __forceinline__ void task_coords(const Params<KeyT>& P, long long t, int& qi, int& g, int& b) {
-  b = static_cast<int>(t % P.nblk);
-  const long long qg = t / P.nblk;
-  g = static_cast<int>(qg % P.G);
-  const int i = static_cast<int>(qg / P.G);
-  qi = P.q_list != nullptr ? P.q_list[i] : i;
-}
-
-// Visible blocks of query qi (0 for an out-of-range query).
-template <typename KeyT>
-__device__ __forceinline__ int query_visible(const Params<KeyT>& P, int qi, int& s, int& p) {
-  s = P.q_stream[qi];
-  p = P.q_pos[qi];
-  if (s < 0 || s >= P.n_streams || p < 0 || p >= P.capacity) return 0;
-  return p / kBlock + 1;
-}
-
-// Sum over the warp of 8 per-lane partial dot products (rows 0..7); the
-// result for row (lane >> 2) lands in every lane of that quad.
-__device__ __forceinline__ float reduce8_rows(const float (&v)[8], int lane) {
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-  float q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float send = b4 ? v[i] : v[i + 4];
-    const float keep = b4 ? v[i + 4] : v[i];
-    q[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+struct Cursor {
+  int i, g, b;      // query slot (index into q_list in list mode), group, block
+  int qi, s, p, nvis;
+  __device__ __forceinline__ void load_query(const Params<KeyT>& P) {
+    qi = P.q_list != nullptr ? P.q_list[i] : i;
+    s = P.q_stream[qi];
+    p = P.q_pos[qi];
+    nvis = (s < 0 || s >= P.n_streams || p < 0 || p >= P.capacity) ? 0 : p / kBlock + 1;
   }
-  float r[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float send = b3 ? q[i] : q[i + 2];
-    const float keep = b3 ? q[i + 2] : q[i];
-    r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  __device__ __forceinline__ void start(const Params<KeyT>& P, long long t, long long t_end) {
+    b = static_cast<int>(t % P.nblk);
+    const long long qg = t / P.nblk;
+    g = static_cast<int>(qg % P.G);
+    i = static_cast<int>(qg / P.G);
+    if (t < t_end) load_query(P);
   }
-  const float send = b2 ? r[0] : r[1];
-  float t = (b2 ? r[1] : r[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
-  t += __shfl_xor_sync(0xffffffffu, t, 2);
-  t += __shfl_xor_sync(0xffffffffu, t, 1);
+  // Advance to task t + 1 (t + 1 < t_end).
+  __device__ __forceinline__ void next(const Params<KeyT>& P) {
+    if (++b < P.nblk) return;
+    b = 0;
+    if (++g < P.G) return;
+    g = 0;
+    ++i;
+    load_query(P);
+  }
+};
+
+// Sum over groups of kLanes lanes of kN per-lane partials (kN <= kLanes, both
+// powers of two).  Each halving step trades half of the partials with the
+// lane kLanes/2, kLanes/4, ... away, so after log2(kN) steps every lane holds
+// one partially summed index; the remaining steps finish the sum.  Partial
+// partial_index<kN, kLanes>(lane) ends in the lane (every lane of the group
+// whose bits select that index holds it).
+template <int kN, int kLanes>
+__device__ __forceinline__ float transposed_sum(float (&v)[kN], int lane) {
+  static_assert(kN >= 1 && kN <= kLanes && (kN & (kN - 1)) == 0 && (kLanes & (kLanes - 1)) == 0, "bad shape");
+  int off = kLanes / 2;
+#pragma unroll
+  for (int n = kN; n > 1; n /= 2, off /= 2) {
+    const bool upper = lane & off;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = upper ? v[i] : v[i + n / 2];
+      const float keep = upper ? v[i + n / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (; off >= 1; off /= 2) t += __shfl_xor_sync(0xffffffffu, t, off);
   return t;
 }
 
-// F16 rows: each half-warp holds one row of a row pair (lane >> 4 picks the
-// row), each lane 8 of its 128 values.  Sum over each half-warp of 8 per-lane
-// partial dot products (row pairs 0..7); the result for pair
-// 4*b3 + 2*b2 + b1 (bits of the lane index) lands in both lanes of that pair.
-__device__ __forceinline__ float reduce8_pairs(const float (&v)[8], int lane) {
-  const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-  float q[4];
+template <int kN, int kLanes>
+__device__ __forceinline__ int partial_index(int lane) {
+  int idx = 0, off = kLanes / 2;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float send = b3 ? v[i] : v[i + 4];
-    const float keep = b3 ? v[i + 4] : v[i];
-    q[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-  }
-  float r[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float send = b2 ? q[i] : q[i + 2];
-    const float keep = b2 ? q[i + 2] : q[i];
-    r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-  const float send = b1 ? r[0] : r[1];
-  float t = (b1 ? r[1] : r[0]) + __shfl_xor_sync(0xffffffffu, send, 2);
-  t += __shfl_xor_sync(0xffffffffu, t, 1);
-  return t;
+  for (int n = kN; n > 1; n /= 2, off /= 2)
+    if (lane & off) idx += n / 2;
+  return idx;
 }
 
-template <typename KeyT, int kStages>
-__global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Params<KeyT> P) {
+// Dot product of 8 F16 key values (one 16-byte word) with 8 query values.
+__device__ __forceinline__ float dot8_f16(const uint4 raw, const float4 qa, const float4 qb) {
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+  const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.z));
+  const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&raw.w));
+  float acc = qa.x * a.x;
+  acc = fmaf(qa.y, a.y, acc);
+  acc = fmaf(qa.z, b.x, acc);
+  acc = fmaf(qa.w, b.y, acc);
+  acc = fmaf(qb.x, c.x, acc);
+  acc = fmaf(qb.y, c.y, acc);
+  acc = fmaf(qb.z, d.x, acc);
+  return fmaf(qb.w, d.y, acc);
+}
+
+template <typename KeyT, int kStages, int kWarps, int kMinCtas>
+__global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv_kernel(const Params<KeyT> P) {
   constexpr bool kF16 = sizeof(KeyT) == 2;
-  constexpr int kRowsPerStage = Rows<KeyT>::kPerStage;
-  constexpr int kRowsPerWarp = Rows<KeyT>::kPerWarp;
-  constexpr int kStageElems = kRowsPerStage * kDi;
+  using R = Rows<KeyT, kWarps>;
+  constexpr int kStageElems = R::kPerStage * kDi;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem<KeyT, kStages>& sm = *reinterpret_cast<Smem<KeyT, kStages>*>(smem_raw);
+  Smem<KeyT, kStages, kWarps>& sm = *reinterpret_cast<Smem<KeyT, kStages, kWarps>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long T = P.q_list != nullptr ? static_cast<long long>(*P.q_count) * P.G * P.nblk : P.n_tasks;
@@ -157,27 +178,27 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
 #pragma unroll
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kConsumerWarps);
+      mbar_init(&sm.empty[s], kWarps);
     }
     mbar_fence_init();
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
+  Cursor<KeyT> cur;
+  cur.start(P, t_begin, t_end);
+
+  if (warp == kWarps) {
     // ---------------- producer: one thread issues every chunk copy --------
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
     bool ok = true;
     int k = 0;
     for (long long t = t_begin; t < t_end && ok; ++t) {
-      int qi, g, b;
-      task_coords(P, t, qi, g, b);
-      int s, p;
-      const int nvis = query_visible(P, qi, s, p);
-      if (b >= nvis) continue;
-      const int n_chunks = min(p - b * kBlock, kBlock - 1) / kRowsPerStage + 1;
-      const KeyT* src =
-          P.idx_k + ((static_cast<size_t>(s) * P.G + g) * P.capacity + static_cast<size_t>(b) * kBlock) * kDi;
+      if (t > t_begin) cur.next(P);
+      if (cur.b >= cur.nvis) continue;
+      const int n_chunks = min(cur.p - cur.b * kBlock, kBlock - 1) / R::kPerStage + 1;
+      const KeyT* src = P.idx_k + ((static_cast<size_t>(cur.s) * P.G + cur.g) * P.capacity +
+                                   static_cast<size_t>(cur.b) * kBlock) * kDi;
       for (int c = 0; c < n_chunks; ++c, ++k) {
         const int st = k % kStages;
         const uint32_t use = static_cast<uint32_t>(k / kStages);
@@ -196,6 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
   }
 
   // ---------------- consumers ------------------------------------------------
+  // Lane layout within a chunk: this warp owns rows [warp * kPerWarp, +kPerWarp);
+  // partial r of a lane covers row r * kPerLoad + (lane / kLanesPerRow) of them.
+  const int part_row = partial_index<R::kPartials, R::kLanesPerRow>(lane) * R::kPerLoad + lane / R::kLanesPerRow;
+  const int lane_in_row = lane % R::kLanesPerRow;
   bool ok = true;
   long long cur_qg = -1;
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -203,85 +228,62 @@ __global__ void __launch_bounds__(kThreads, 1) block_scores_gemv_kernel(const Pa
   int k = 0;
   int par = 0;
   for (long long t = t_begin; t < t_end; ++t) {
-    int qi, g, b;
-    task_coords(P, t, qi, g, b);
-    const long long qg = static_cast<long long>(qi) * P.G + g;
+    if (t > t_begin) cur.next(P);
+    const int b = cur.b, p = cur.p;
+    const long long qg = static_cast<long long>(cur.qi) * P.G + cur.g;
     const size_t out = static_cast<size_t>(qg) * P.nblk + b;
-    int s, p;
-    const int nvis = query_visible(P, qi, s, p);
-    if (b >= nvis) {
+    if (b >= cur.nvis) {
       if (warp == 0 && lane == 0) {
         P.bs[out] = -INFINITY;
-        if (nvis == 0 && b == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
+        if (cur.nvis == 0 && b == 0 && cur.g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
       }
       continue;
     }
     if (qg != cur_qg) {
       cur_qg = qg;
-      if constexpr (kF16) {   // dims 8j .. 8j+7, j = lane & 15
-        const float4* qp = reinterpret_cast<const float4*>(P.idx_q + static_cast<size_t>(qg) * kDi) + 2 * (lane & 15);
-        qv = __ldg(qp);
-        qv2 = __ldg(qp + 1);
-      } else {
-        qv = __ldg(reinterpret_cast<const float4*>(P.idx_q + static_cast<size_t>(qg) * kDi) + lane);
+      const float4* qp = reinterpret_cast<const float4*>(P.idx_q + static_cast<size_t>(qg) * kDi);
+      if constexpr (kF16) {   // dims 8j .. 8j+7, j = lane_in_row
+        qv = __ldg(qp + 2 * lane_in_row);
+        qv2 = __ldg(qp + 2 * lane_in_row + 1);
+      } else {                // dims 4 * lane .. +3
+        qv = __ldg(qp + lane_in_row);
       }
     }
     float m = -INFINITY;
-    const int n_chunks = min(p - b * kBlock, kBlock - 1) / kRowsPerStage + 1;
+    const int n_chunks = min(p - b * kBlock, kBlock - 1) / R::kPerStage + 1;
     for (int c = 0; c < n_chunks; ++c, ++k) {
       const int st = k % kStages;
       if (ok) ok = mbar_wait(&sm.full[st], (k / kStages) & 1);
       if (ok) {
-        if constexpr (kF16) {
-          // 16 rows per warp as 8 row pairs; one 16-byte load covers 8 values
-          const KeyT* base = sm.stage[st] + (warp * kRowsPerWarp + (lane >> 4)) * kDi + 8 * (lane & 15);
-          float part[8];
+        const KeyT* base = sm.stage[st] + (warp * R::kPerWarp + lane / R::kLanesPerRow) * kDi;
+        float part[R::kPartials];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(base + 2 * i * kDi);
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-            const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-            const float2 cc = __half22float2(*reinterpret_cast<const __half2*>(&raw.z));
-            const float2 dd = __half22float2(*reinterpret_cast<const __half2*>(&raw.w));
-            float acc = qv.x * a.x;
-            acc = fmaf(qv.y, a.y, acc);
-            acc = fmaf(qv.z, bb.x, acc);
-            acc = fmaf(qv.w, bb.y, acc);
-            acc = fmaf(qv2.x, cc.x, acc);
-            acc = fmaf(qv2.y, cc.y, acc);
-            acc = fmaf(qv2.z, dd.x, acc);
-            part[i] = fmaf(qv2.w, dd.y, acc);
-          }
-          const float dot = reduce8_pairs(part, lane);
-          const int ip = ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-          const int j = b * kBlock + c * kRowsPerStage + warp * kRowsPerWarp + 2 * ip + (lane >> 4);
-          if (j <= p) m = fmaxf(m, dot);
-        } else {
-          const KeyT* base = sm.stage[st] + warp * kRowsPerWarp * kDi + lane * 4;
-          float part[kRowsPerWarp];
-#pragma unroll
-          for (int r = 0; r < kRowsPerWarp; ++r) {
-            const float4 kv = load4(base + r * kDi);
+        for (int r = 0; r < R::kPartials; ++r) {
+          const KeyT* row = base + r * R::kPerLoad * kDi;
+          if constexpr (kF16) {
+            part[r] = dot8_f16(*reinterpret_cast<const uint4*>(row + 8 * lane_in_row), qv, qv2);
+          } else {
+            const float4 kv = *reinterpret_cast<const float4*>(row + 4 * lane_in_row);
             part[r] = fmaf(qv.w, kv.w, fmaf(qv.z, kv.z, fmaf(qv.y, kv.y, qv.x * kv.x)));
           }
-          const float dot = reduce8_rows(part, lane);
-          const int j = b * kBlock + c * kRowsPerStage + warp * kRowsPerWarp + (lane >> 2);
-          if (j <= p) m = fmaxf(m, dot);  // fmaxf drops NaN: a NaN score ranks as -inf
         }
+        const float dot = transposed_sum<R::kPartials, R::kLanesPerRow>(part, lane);
+        const int j = b * kBlock + c * R::kPerStage + warp * R::kPerWarp + part_row;
+        if (j <= p) m = fmaxf(m, dot);  // fmaxf drops NaN: a NaN score ranks as -inf
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[st]);
     }
-    if constexpr (kF16) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    // lanes that differ only below bit kSame hold the same row
+    constexpr int kSame = R::kLanesPerRow / R::kPartials;
+#pragma unroll
+    for (int off = kSame; off < 32; off *= 2) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (lane == 0) sm.red[par][warp] = m;
-    named_barrier_sync(1, kConsumerWarps * 32);
+    named_barrier_sync(1, kWarps * 32);
     if (warp == 0 && lane == 0) {
       float mm = sm.red[par][0];
 #pragma unroll
-      for (int w = 1; w < kConsumerWarps; ++w) mm = fmaxf(mm, sm.red[par][w]);
+      for (int w = 1; w < kWarps; ++w) mm = fmaxf(mm, sm.red[par][w]);
       if (b == p / kBlock) mm += MSA_LOCAL_BIAS;
       P.bs[out] = mm;
     }
