@@ -21,6 +21,10 @@ What it computes, and where each step is stated (page titles as cited):
 * same page, review comment on --kv-unified: blocks are anchored to absolute
   slots (the flat slot index is pooled every 128 slots); the local block is
   position/128.
+* same page, issue thread on unified KV caches: with streams interleaved in
+  one buffer, scoring and gathering must map a stream's logical position to
+  the physical slot holding it through a page indirection
+  (``logical_cache``, ``paged_append``);
 * "mtmd: Add Vision Support for Minimax-M3" commit message (squash of the MSA
   branch): indexer scores are accumulated in F32 (the oracle uses FP64, which
   is at least that exact) and the KV length is a multiple of 128.
@@ -212,6 +216,49 @@ def sparse_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
                 w = torch.exp(logits - logits.max())
                 w = w / w.sum()
                 out[i, h] = w @ V
+    return out
+
+
+# ---------------------------------------------------------------------------
+# paged caches: a sequence-relative page indirection
+# ---------------------------------------------------------------------------
+def logical_cache(pool: torch.Tensor, block_table: torch.Tensor, block: int) -> torch.Tensor:
+    """The per-stream cache that a page pool holds: slot j of stream s (group
+    g) is slot j % block of page block_table[s][j // block].
+
+    "Add MiniMax-M3 ..." pull request, issue thread on --kv-unified: block
+    scoring and gathering index absolute slots of one flat buffer, which is
+    only right while each stream owns a fixed range; a unified cache needs a
+    map from a stream's logical position to the physical slot holding it,
+    consulted by the scoring and gather steps (the page index of the
+    reference MSA kernel).  pool is [n_pages][G][block][row]; block_table is
+    [S][n_blocks].  Blocks whose entry names no page are NaN, so reading one
+    poisons the result.
+    """
+    S, n_blocks = block_table.shape
+    n_pages, G, B, row = pool.shape
+    if B != block:
+        raise ValueError("a page holds one block")
+    out = torch.full((S, G, n_blocks * block, row), float("nan"), dtype=pool.dtype)
+    for s in range(S):
+        for b in range(n_blocks):
+            page = int(block_table[s, b])
+            if 0 <= page < n_pages:
+                out[s, :, b * block:(b + 1) * block, :] = pool[page]
+    return out
+
+
+def paged_append(pool: torch.Tensor, new_rows: torch.Tensor, tok_stream: torch.Tensor,
+                 tok_pos: torch.Tensor, block_table: torch.Tensor, block: int) -> torch.Tensor:
+    """Return a copy of the pool with row new_rows[t] (every group) written at
+    slot tok_pos[t] % block of the page that holds block tok_pos[t] // block
+    of stream tok_stream[t]: the append of ``indexer_append`` through the
+    page indirection of ``logical_cache``."""
+    out = pool.clone()
+    for t in range(tok_stream.numel()):
+        s, p = int(tok_stream[t]), int(tok_pos[t])
+        page = int(block_table[s, p // block])
+        out[page, :, p % block, :] = new_rows[t].to(pool.dtype)
     return out
 
 

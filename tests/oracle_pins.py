@@ -326,9 +326,72 @@ def pin_append_random(o, seed=8):
                 assert torch.equal(out[s, :, p], cache[s, :, p])
 
 
+def _pool_from_contiguous(cache, block):
+    """Closed form of the identity paging: page s * n_blocks + b holds block b
+    of stream s, i.e. the [S][G][cap][row] cache with its block axis moved in
+    front of the group axis."""
+    S, G, cap, row = cache.shape
+    nb = cap // block
+    return cache.reshape(S, G, nb, block, row).permute(0, 2, 1, 3, 4).reshape(S * nb, G, block, row)
+
+
+def pin_paged_identity_layout(o, seed=9):
+    """Identity block table over a reshaped contiguous cache: the logical view
+    must return the cache exactly (a transposed table, a slot reordered inside
+    a page or a wrong page index all break it)."""
+    g = torch.Generator().manual_seed(seed)
+    cache = torch.randn((3, 2, 12, 5), generator=g, dtype=torch.float64)
+    pool = _pool_from_contiguous(cache, 4)
+    table = torch.arange(9, dtype=torch.int32).view(3, 3)
+    assert torch.equal(o.logical_cache(pool, table, 4), cache)
+
+
+def pin_paged_permutation_and_sharing(o, seed=10):
+    """Moving pages to other pool slots (spare pages holding garbage) and
+    renaming the table entries the same way leaves the logical view unchanged;
+    a block mapped to another stream's page shows that page's rows; a block
+    with no page reads as NaN."""
+    g = torch.Generator().manual_seed(seed)
+    cache = torch.randn((3, 2, 12, 5), generator=g, dtype=torch.float64)
+    pool = _pool_from_contiguous(cache, 4)
+    table = torch.arange(9, dtype=torch.int32).view(3, 3)
+    perm = torch.randperm(11, generator=g)              # old page i -> new slot perm[i]
+    moved = torch.full((11, 2, 4, 5), 1.0e6, dtype=torch.float64)
+    moved[perm[:9]] = pool
+    table2 = perm[table.long()].to(torch.int32)
+    assert torch.equal(o.logical_cache(moved, table2, 4), cache)
+    table3 = table2.clone()
+    table3[2, 0] = table2[0, 0]                          # stream 2 shares stream 0's first page
+    table3[1, 2] = -1                                    # stream 1's last block unmapped
+    view = o.logical_cache(moved, table3, 4)
+    assert torch.equal(view[2, :, :4], cache[0, :, :4]) and torch.equal(view[2, :, 4:], cache[2, :, 4:])
+    assert bool(torch.isnan(view[1, :, 8:]).all()) and torch.equal(view[1, :, :8], cache[1, :, :8])
+
+
+def pin_paged_append_commutes(o, seed=11):
+    """Appending through the page table and then taking the logical view equals
+    taking the view and appending to it (the contiguous append is pinned by
+    pin_append_random); pages no token maps to are left untouched."""
+    g = torch.Generator().manual_seed(seed)
+    cache = torch.randn((3, 2, 12, 5), generator=g, dtype=torch.float64)
+    pool = torch.cat([_pool_from_contiguous(cache, 4), torch.randn((2, 2, 4, 5), generator=g, dtype=torch.float64)])
+    perm = torch.randperm(11, generator=g)
+    moved = torch.empty_like(pool)
+    moved[perm] = pool
+    table = perm[torch.arange(9).view(3, 3)].to(torch.int32)
+    new = torch.randn((6, 2, 5), generator=g, dtype=torch.float64)
+    ts = torch.tensor([2, 0, 2, 1, 0, 1], dtype=torch.int32)
+    tp = torch.tensor([11, 0, 3, 5, 6, 8], dtype=torch.int32)
+    after = o.paged_append(moved, new, ts, tp, table, 4)
+    assert torch.equal(o.logical_cache(after, table, 4), o.indexer_append(cache, new, ts, tp))
+    spare = perm[9:]
+    assert torch.equal(after[spare], moved[spare])
+
+
 ALL_PINS = [pin_golden, pin_basis_query_pooling, pin_scores_bilinear, pin_selection_bruteforce,
             pin_selection_invariants, pin_local_forced, pin_dense_equivalence,
-            pin_block_mask_equivalence, pin_attention_closed_forms, pin_append_random]
+            pin_block_mask_equivalence, pin_attention_closed_forms, pin_append_random,
+            pin_paged_identity_layout, pin_paged_permutation_and_sharing, pin_paged_append_commutes]
 
 
 def run_all(o):

@@ -153,10 +153,41 @@ def _mut_append_swapped(o):
     o.indexer_append = indexer_append
 
 
+def _mut_paged_table_transposed(o):
+    def logical_cache(pool, table, block):
+        S, nb = table.shape
+        out = torch.full((S, pool.shape[1], nb * block, pool.shape[3]), float("nan"), dtype=pool.dtype)
+        for s in range(S):
+            for b in range(nb):
+                page = int(table[b % S, s % nb])
+                out[s, :, b * block:(b + 1) * block] = pool[page]
+        return out
+    o.logical_cache = logical_cache
+
+
+def _mut_paged_slots_reversed(o):
+    orig = o.logical_cache
+
+    def logical_cache(pool, table, block):
+        return orig(pool.flip(2), table, block)
+    o.logical_cache = logical_cache
+
+
+def _mut_paged_append_next_slot(o):
+    def paged_append(pool, new, ts, tp, table, block):
+        out = pool.clone()
+        for t in range(ts.numel()):
+            s, p = int(ts[t]), int(tp[t])
+            out[int(table[s, p // block]), :, (p + 1) % block] = new[t]
+        return out
+    o.paged_append = paged_append
+
+
 MUTATIONS = [_mut_causal_off_by_one, _mut_no_causal_mask, _mut_tie_higher_index, _mut_no_bias,
              _mut_gqa_modulo, _mut_no_scale, _mut_nvis_off_by_one, _mut_transposed_scores,
              _mut_dropped_term, _mut_future_rows, _mut_sign, _mut_k_minus_one,
-             _mut_unsorted_ids, _mut_lowest_scores, _mut_append_swapped]
+             _mut_unsorted_ids, _mut_lowest_scores, _mut_append_swapped, _mut_paged_table_transposed,
+             _mut_paged_slots_reversed, _mut_paged_append_next_slot]
 
 
 @pytest.mark.parametrize("mut", MUTATIONS, ids=lambda f: f.__name__[5:])
