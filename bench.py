@@ -51,6 +51,12 @@ SCORES_TRAFFIC = {"source_sha": "7065233549d01316",
                   "bytes_per_launch": {"f32": 4 * (536_908_544 + 3_283_712), "f16": 4 * (268_472_832 + 3_113_984)}}
 
 
+def variant_metric(metric: str, args) -> str:
+    """The metric name, marked with the cache variant a run uses."""
+    tags = (["F16 indexer cache"] if args.idx_f16 else []) + (["paged caches"] if args.paged else [])
+    return metric.replace("x32 streams", "x32 streams, " + ", ".join(tags)) if tags else metric
+
+
 def scores_source_sha() -> str:
     p = os.path.join(ROOT, "block_sparse_attention_maxpool_b200", "csrc", "msa_scores_gemv.cuh")
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
@@ -182,6 +188,14 @@ def run_ours(args, rank, world, dev):
     d = {n: getattr(inp, n).to(dev) for n in ("idx_k_cache", "k_cache", "v_cache", "tok_stream",
                                                "tok_pos", "idx_k_new", "k_new", "v_new",
                                                "q_stream", "q_pos", "idx_q", "q")}
+    pages = None
+    if args.paged:
+        # the same caches as shuffled page pools behind a block table
+        lay = W.page_layout(inp, seed=rank)
+        d["idx_k_cache"], d["k_cache"], d["v_cache"] = (lay.idx_pool.to(dev), lay.k_pool.to(dev),
+                                                      lay.v_pool.to(dev))
+        pages = msa.Pages(lay.block_table.to(dev), lay.n_pages)
+        del lay
     del inp
     if args.idx_f16:
         d["idx_k_cache"] = d["idx_k_cache"].half()         # F16 indexer-key cache variant
@@ -206,19 +220,19 @@ def run_ours(args, rank, world, dev):
 
     def part_append(st):
         append = msa.msa_indexer_append_f16 if args.idx_f16 else msa.msa_indexer_append
-        append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st)
+        append(shape, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st, pages)
         msa.msa_kv_append(shape, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
-                          d["tok_pos"], st)
+                          d["tok_pos"], st, pages)
 
     def part_scores(st):
         msa.msa_block_scores(shape, d["idx_q"], d["idx_k_cache"], d["q_stream"], d["q_pos"],
-                             bufs["block_scores"], st, bufs["workspace"])
+                             bufs["block_scores"], st, bufs["workspace"], pages)
 
     def part_attend(st):
         msa.msa_select_topk(shape, bufs["block_scores"], d["q_pos"], bufs["sel"], bufs["n_sel"], st)
         attn = msa.msa_sparse_attn_prefill if prefill else msa.msa_sparse_attn_decode
         attn(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"], d["q_pos"], scale,
-             bufs["out"], bufs["workspace"], st)
+             bufs["out"], bufs["workspace"], st, pages)
 
     def step(ev=None):
         part_append(stream)
@@ -319,11 +333,11 @@ def run_ours(args, rank, world, dev):
     sbytes = scores_bytes(w, key_bytes)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     traffic = None
-    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD:
+    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD and not args.paged:
         traffic = SCORES_TRAFFIC["bytes_per_launch"]["f16" if args.idx_f16 else "f32"]   # this workload only
     step_gbs = step_bytes(w, key_bytes) / (ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC if not args.idx_f16 else METRIC.replace("x32 streams", "x32 streams, F16 indexer cache"),
+        "metric": variant_metric(METRIC, args),
         "value": job_tokens_per_s(w.n_streams, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -337,6 +351,7 @@ def run_ours(args, rank, world, dev):
         "data": "synthetic (seeded N(0,1) K/V/Q bf16, indexer N(0,1)/sqrt(128) f32)",
         "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "context": w.l_total,
                    "launch": "cuda graphs" if graphs is not None else "direct",
+                   "caches": "paged (shuffled pages + block table)" if args.paged else "contiguous",
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                    "block": w.block, "top_k": w.top_k, "parallelism": f"replicas{world}",
                    "l2": f"inputs {2 * w.n_streams * w.capacity * w.n_kv_heads * 512 / 1e9:.1f} GB per GPU > 126 MB L2, no flush"},
@@ -380,6 +395,7 @@ def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches
         "vs_baseline": None, "dtype": "f32 indexer / bf16 attention (f32 accumulate)", "data": "synthetic",
         "config": {"workload": w.name, "streams_per_gpu": w.n_streams, "new_tokens": w.n_new,
                    "context": w.l_total, "parallelism": f"replicas{world}",
+                   "caches": "paged (shuffled pages + block table)" if args.paged else "contiguous",
                    "launch": "cuda graphs" if graphs is not None else "direct"},
         "step_tensor": {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
                         "frac": tf / peaks["bf16_tflops"], "indexer_flops": ind, "attention_flops": att},
@@ -460,6 +476,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--idx-f16", action="store_true",
                     help="decode with the F16 indexer-key cache variant instead of the F32 cache")
+    ap.add_argument("--paged", action="store_true",
+                    help="run the paged calls on the same caches laid out as shuffled page pools")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from Python in the timed loop instead of replaying CUDA graphs")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD.name,
@@ -488,7 +506,8 @@ def main():
     try:
         line = run_ours(args, rank, world, local)
         if line is not None:
-            if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name and not args.idx_f16:
+            if (world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name and not args.idx_f16
+                    and not args.paged):
                 line["cpu_baseline"] = cpu_baseline()
             print(json.dumps(line), flush=True)
     finally:

@@ -21,7 +21,10 @@ __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_bloc
            "msa_indexer_append_f16",
            "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
            "msa_workspace_bytes", "msa_get_device_error", "msa_sparse_attn_decode_noalloc", "msa_version", "library", "LIB_PATH",
-           "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step"]
+           "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step",
+           "Pages", "msa_indexer_append_paged", "msa_indexer_append_f16_paged", "msa_kv_append_paged",
+           "msa_block_scores_paged", "msa_block_scores_f16_paged", "msa_sparse_attn_decode_paged",
+           "msa_sparse_attn_prefill_paged"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
 MODE_DECODE = 0
@@ -30,7 +33,7 @@ LOCAL_BIAS = 2.0 ** 100
 
 STATUS = {0: "MSA_OK", -1: "MSA_ERR_NULL", -2: "MSA_ERR_ALIGN", -3: "MSA_ERR_SHAPE",
           -4: "MSA_ERR_RANGE", -5: "MSA_ERR_WORKSPACE", -6: "MSA_ERR_CUDA"}
-DEVERR = {0x1: "QUERY_RANGE", 0x2: "TOKEN_RANGE", 0x4: "SEL_RANGE", 0x8: "TIMEOUT"}
+DEVERR = {0x1: "QUERY_RANGE", 0x2: "TOKEN_RANGE", 0x4: "SEL_RANGE", 0x8: "TIMEOUT", 0x10: "PAGE_RANGE"}
 
 
 class MsaError(RuntimeError):
@@ -67,6 +70,23 @@ class Shape:
                       self.head_dim, self.idx_dim, self.block, self.top_k)
 
 
+class CPages(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("n_pages", ctypes.c_int32)]
+
+
+@dataclass(frozen=True)
+class Pages:
+    """Block table of paged caches (msa_pages): ``block_table`` is an int32
+    device tensor [n_streams][capacity / 128] naming the pool page that holds
+    each logical block; pools are [n_pages][G][128][row]."""
+    block_table: torch.Tensor
+    n_pages: int
+
+    def c(self, shape: "Shape") -> CPages:
+        t = _ptr(self.block_table, torch.int32, (shape.n_streams, shape.n_blocks), "block_table")
+        return CPages(t, int(self.n_pages))
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -90,6 +110,20 @@ _SIGS = {
     "msa_get_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "msa_version": (ctypes.c_int, []),
 }
+_PG = ctypes.POINTER(CPages)
+_SIGS.update({
+    "msa_indexer_append_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P]),
+    "msa_indexer_append_f16_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P]),
+    "msa_kv_append_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "msa_block_scores_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P, _P,
+                                              ctypes.c_size_t, _P]),
+    "msa_block_scores_f16_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P, _P,
+                                                  ctypes.c_size_t, _P]),
+    "msa_sparse_attn_decode_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
+                                                    ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_sparse_attn_prefill_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
+                                                     ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+})
 
 
 def library() -> ctypes.CDLL:
@@ -140,27 +174,41 @@ def _n(t: torch.Tensor, name: str) -> int:
     return t.shape[0]
 
 
-def msa_indexer_append(shape: Shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, stream=None):
-    n = _n(tok_stream, "tok_stream")
+def _cache_shape(shape: Shape, pages: Pages | None, row: int) -> tuple:
+    """[S][G][capacity][row] for a contiguous cache, [n_pages][G][128][row] for a pool."""
+    if pages is None:
+        return (shape.n_streams, shape.n_kv_heads, shape.capacity, row)
+    return (pages.n_pages, shape.n_kv_heads, shape.block, row)
+
+
+def _call(fn: str, shape: Shape, pages: Pages | None, *args) -> None:
+    """Call fn (or fn + '_paged' with the page table after the shape)."""
     s = shape.c()
-    _check("msa_indexer_append", library().msa_indexer_append(
-        ctypes.byref(s),
-        _ptr(idx_k_cache, torch.float32, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
-        _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
-        _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
-        n, _stream(stream)))
+    if pages is None:
+        _check(fn, getattr(library(), fn)(ctypes.byref(s), *args))
+    else:
+        pg = pages.c(shape)
+        _check(fn + "_paged", getattr(library(), fn + "_paged")(ctypes.byref(s), ctypes.byref(pg), *args))
 
 
-def msa_kv_append(shape: Shape, k_cache, v_cache, k_new, v_new, tok_stream, tok_pos, stream=None):
+def msa_indexer_append(shape: Shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, stream=None, pages=None):
     n = _n(tok_stream, "tok_stream")
-    cs = (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.head_dim)
+    _call("msa_indexer_append", shape, pages,
+          _ptr(idx_k_cache, torch.float32, _cache_shape(shape, pages, shape.idx_dim), "idx_k_cache"),
+          _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
+          _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+          n, _stream(stream))
+
+
+def msa_kv_append(shape: Shape, k_cache, v_cache, k_new, v_new, tok_stream, tok_pos, stream=None, pages=None):
+    n = _n(tok_stream, "tok_stream")
+    cs = _cache_shape(shape, pages, shape.head_dim)
     ns = (n, shape.n_kv_heads, shape.head_dim)
-    s = shape.c()
-    _check("msa_kv_append", library().msa_kv_append(
-        ctypes.byref(s), _ptr(k_cache, torch.bfloat16, cs, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, cs, "v_cache"), _ptr(k_new, torch.bfloat16, ns, "k_new"),
-        _ptr(v_new, torch.bfloat16, ns, "v_new"), _ptr(tok_stream, torch.int32, (n,), "tok_stream"),
-        _ptr(tok_pos, torch.int32, (n,), "tok_pos"), n, _stream(stream)))
+    _call("msa_kv_append", shape, pages,
+          _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+          _ptr(k_new, torch.bfloat16, ns, "k_new"), _ptr(v_new, torch.bfloat16, ns, "v_new"),
+          _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+          n, _stream(stream))
 
 
 def _workspace(shape: Shape, n: int, mode: int, workspace, device):
@@ -173,21 +221,20 @@ def _workspace(shape: Shape, n: int, mode: int, workspace, device):
     return _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), workspace
 
 
-def msa_indexer_append_f16(shape: Shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, stream=None):
+def msa_indexer_append_f16(shape: Shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, stream=None,
+                           pages=None):
     """F16 indexer-key cache variant of msa_indexer_append (float16 cache;
     the new F32 keys are rounded to fp16 as they are written)."""
     n = _n(tok_stream, "tok_stream")
-    s = shape.c()
-    _check("msa_indexer_append_f16", library().msa_indexer_append_f16(
-        ctypes.byref(s),
-        _ptr(idx_k_cache, torch.float16, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
-        _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
-        _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
-        n, _stream(stream)))
+    _call("msa_indexer_append_f16", shape, pages,
+          _ptr(idx_k_cache, torch.float16, _cache_shape(shape, pages, shape.idx_dim), "idx_k_cache"),
+          _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
+          _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+          n, _stream(stream))
 
 
 def msa_block_scores(shape: Shape, idx_q, idx_k_cache, q_stream, q_pos, block_scores=None, stream=None,
-                     workspace=None):
+                     workspace=None, pages=None):
     """Block scores over the F32 indexer-key cache, or over the F16 cache
     variant when idx_k_cache is a float16 tensor."""
     n = _n(q_pos, "q_pos")
@@ -199,13 +246,11 @@ def msa_block_scores(shape: Shape, idx_q, idx_k_cache, q_stream, q_pos, block_sc
         block_scores = torch.empty((n, shape.n_kv_heads, shape.n_blocks), dtype=torch.float32,
                                    device=idx_q.device)
     ws_ptr, ws_bytes, _keep = _workspace(shape, n, MODE_DECODE, workspace, idx_q.device)
-    s = shape.c()
-    _check(fn, getattr(library(), fn)(
-        ctypes.byref(s), _ptr(idx_q, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_q"),
-        _ptr(idx_k_cache, kdt, (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.idx_dim), "idx_k_cache"),
-        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
-        _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
-        ws_ptr, ws_bytes, _stream(stream)))
+    _call(fn, shape, pages, _ptr(idx_q, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_q"),
+          _ptr(idx_k_cache, kdt, _cache_shape(shape, pages, shape.idx_dim), "idx_k_cache"),
+          _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+          _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
+          ws_ptr, ws_bytes, _stream(stream))
     return block_scores
 
 
@@ -235,35 +280,74 @@ def msa_workspace_bytes(shape: Shape, n_q: int, mode: int) -> int:
 
 
 def _attn(fn_name: str, mode: int, shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos,
-          softmax_scale=None, out=None, workspace=None, stream=None):
+          softmax_scale=None, out=None, workspace=None, stream=None, pages=None):
     n = _n(q_pos, "q_pos")
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(shape.head_dim)
     if out is None:
         out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=q.device)
     ws_ptr, ws_bytes, _keep = _workspace(shape, n, mode, workspace, q.device)
-    cs = (shape.n_streams, shape.n_kv_heads, shape.capacity, shape.head_dim)
-    s = shape.c()
-    _check(fn_name, getattr(library(), fn_name)(
-        ctypes.byref(s), _ptr(q, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
-        _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
-        _ptr(sel, torch.int32, (n, shape.n_kv_heads, shape.top_k), "sel"),
-        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
-        float(softmax_scale), _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"),
-        ws_ptr, ws_bytes, _stream(stream)))
+    cs = _cache_shape(shape, pages, shape.head_dim)
+    _call(fn_name, shape, pages, _ptr(q, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
+          _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+          _ptr(sel, torch.int32, (n, shape.n_kv_heads, shape.top_k), "sel"),
+          _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+          float(softmax_scale), _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"),
+          ws_ptr, ws_bytes, _stream(stream))
     return out
 
 
 def msa_sparse_attn_decode(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos, softmax_scale=None,
-                           out=None, workspace=None, stream=None):
+                           out=None, workspace=None, stream=None, pages=None):
     return _attn("msa_sparse_attn_decode", MODE_DECODE, shape, q, k_cache, v_cache, sel, q_stream,
-                 q_pos, softmax_scale, out, workspace, stream)
+                 q_pos, softmax_scale, out, workspace, stream, pages)
 
 
 def msa_sparse_attn_prefill(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos, softmax_scale=None,
-                            out=None, workspace=None, stream=None):
+                            out=None, workspace=None, stream=None, pages=None):
     return _attn("msa_sparse_attn_prefill", MODE_PREFILL, shape, q, k_cache, v_cache, sel, q_stream,
-                 q_pos, softmax_scale, out, workspace, stream)
+                 q_pos, softmax_scale, out, workspace, stream, pages)
+
+
+# ---- paged caches: the C ABI's *_paged calls --------------------------------
+def msa_indexer_append_paged(shape: Shape, pages: Pages, idx_k_pool, idx_k_new, tok_stream, tok_pos,
+                             stream=None):
+    msa_indexer_append(shape, idx_k_pool, idx_k_new, tok_stream, tok_pos, stream, pages)
+
+
+def msa_indexer_append_f16_paged(shape: Shape, pages: Pages, idx_k_pool, idx_k_new, tok_stream, tok_pos,
+                                 stream=None):
+    msa_indexer_append_f16(shape, idx_k_pool, idx_k_new, tok_stream, tok_pos, stream, pages)
+
+
+def msa_kv_append_paged(shape: Shape, pages: Pages, k_pool, v_pool, k_new, v_new, tok_stream, tok_pos,
+                        stream=None):
+    msa_kv_append(shape, k_pool, v_pool, k_new, v_new, tok_stream, tok_pos, stream, pages)
+
+
+def msa_block_scores_paged(shape: Shape, pages: Pages, idx_q, idx_k_pool, q_stream, q_pos, block_scores=None,
+                           stream=None, workspace=None):
+    """Paged block scores; a float16 pool selects msa_block_scores_f16_paged."""
+    return msa_block_scores(shape, idx_q, idx_k_pool, q_stream, q_pos, block_scores, stream, workspace, pages)
+
+
+def msa_block_scores_f16_paged(shape: Shape, pages: Pages, idx_q, idx_k_pool, q_stream, q_pos,
+                               block_scores=None, stream=None, workspace=None):
+    if idx_k_pool.dtype != torch.float16:
+        raise ValueError("idx_k_pool must be float16")
+    return msa_block_scores(shape, idx_q, idx_k_pool, q_stream, q_pos, block_scores, stream, workspace, pages)
+
+
+def msa_sparse_attn_decode_paged(shape: Shape, pages: Pages, q, k_pool, v_pool, sel, q_stream, q_pos,
+                                 softmax_scale=None, out=None, workspace=None, stream=None):
+    return msa_sparse_attn_decode(shape, q, k_pool, v_pool, sel, q_stream, q_pos, softmax_scale, out,
+                                  workspace, stream, pages)
+
+
+def msa_sparse_attn_prefill_paged(shape: Shape, pages: Pages, q, k_pool, v_pool, sel, q_stream, q_pos,
+                                  softmax_scale=None, out=None, workspace=None, stream=None):
+    return msa_sparse_attn_prefill(shape, q, k_pool, v_pool, sel, q_stream, q_pos, softmax_scale, out,
+                                   workspace, stream, pages)
 
 
 NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
@@ -305,30 +389,31 @@ def msa_version() -> int:
 
 
 def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None, stream=None,
-                prefill: bool = False):
+                prefill: bool = False, pages: Pages | None = None):
     """One MSA step through the C ABI: append the new tokens' indexer keys
     and K/V rows, score blocks, select the top-k and attend.
 
     caches: idx_k_cache (float32, or float16 for the F16 cache variant),
     k_cache, v_cache (device); new: tok_stream, tok_pos,
     idx_k_new, k_new, v_new, q_stream, q_pos, idx_q, q (device).  ``bufs`` may
-    hold preallocated block_scores / sel / n_sel / out / workspace.
+    hold preallocated block_scores / sel / n_sel / out / workspace.  With
+    ``pages`` the caches are page pools addressed through its block table.
     Returns (out, sel, n_sel, block_scores).
     """
     b = bufs or {}
     append = msa_indexer_append_f16 if caches["idx_k_cache"].dtype == torch.float16 else msa_indexer_append
-    append(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"], new["tok_pos"], stream)
+    append(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"], new["tok_pos"], stream, pages)
     msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
-                  new["tok_stream"], new["tok_pos"], stream)
+                  new["tok_stream"], new["tok_pos"], stream, pages)
     n = new["q_pos"].shape[0]
     mode = MODE_PREFILL if prefill else MODE_DECODE
     if b.get("workspace") is None and msa_workspace_bytes(shape, n, mode) > 0:
         b = dict(b, workspace=torch.empty((msa_workspace_bytes(shape, n, mode),), dtype=torch.uint8,
                                           device=new["q"].device))
     bs = msa_block_scores(shape, new["idx_q"], caches["idx_k_cache"], new["q_stream"], new["q_pos"],
-                          b.get("block_scores"), stream, b.get("workspace"))
+                          b.get("block_scores"), stream, b.get("workspace"), pages)
     sel, n_sel = msa_select_topk(shape, bs, new["q_pos"], b.get("sel"), b.get("n_sel"), stream)
     attn = msa_sparse_attn_prefill if prefill else msa_sparse_attn_decode
     out = attn(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
-               new["q_pos"], None, b.get("out"), b.get("workspace"), stream)
+               new["q_pos"], None, b.get("out"), b.get("workspace"), stream, pages)
     return out, sel, n_sel, bs

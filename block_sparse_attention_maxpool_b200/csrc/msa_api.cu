@@ -38,6 +38,24 @@ int check_shape(const msa_shape* sh) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
+// Device view of a page table (null: contiguous caches) and the number of
+// rows of the cache (or page pool) viewed as 2-D [rows][128].  Every row
+// index must fit a signed 32-bit TMA coordinate.
+int pages_of(const msa_shape* sh, const msa_pages* pg, msa::KvPages* out, int64_t* rows) {
+  out->table = nullptr;
+  out->n_pages = 0;
+  *rows = static_cast<int64_t>(sh->n_streams) * sh->n_kv_heads * sh->capacity;
+  if (pg == nullptr) return MSA_OK;
+  if (pg->block_table == nullptr) return MSA_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(pg->block_table) & 3u) != 0) return MSA_ERR_ALIGN;
+  if (pg->n_pages <= 0) return MSA_ERR_RANGE;
+  *rows = static_cast<int64_t>(pg->n_pages) * sh->n_kv_heads * 128;
+  if (*rows >= (int64_t{1} << 31)) return MSA_ERR_SHAPE;
+  out->table = pg->block_table;
+  out->n_pages = pg->n_pages;
+  return MSA_OK;
+}
+
 int current_device_sms(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MSA_ERR_CUDA;
@@ -123,7 +141,7 @@ size_t attn_workspace(int64_t n_pairs, int mode) {
 int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache, const msa_bf16* v_cache,
                 const int32_t* sel, const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
                 float softmax_scale, msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream,
-                int mode) {
+                int mode, const msa_pages* pages) {
   int st = check_shape(sh);
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
@@ -140,7 +158,9 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     if (workspace == nullptr || workspace_bytes < need) return MSA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MSA_ERR_ALIGN;
   }
-  const int64_t rows = static_cast<int64_t>(sh->n_streams) * G * sh->capacity;
+  msa::KvPages pg;
+  int64_t rows = 0;
+  if ((st = pages_of(sh, pages, &pg, &rows)) != MSA_OK) return st;
   CUtensorMap tm_k, tm_v;
   if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
   if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
@@ -167,6 +187,7 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     Q.n_streams = sh->n_streams;
     Q.capacity = sh->capacity;
     Q.scale_log2 = softmax_scale * 1.4426950408889634f;
+    Q.pages = pg;
     const int64_t grid = std::min<int64_t>(sms, n_pairs);
     msa::pattn::sparse_attn_prefill_tc_kernel<<<static_cast<unsigned>(grid), msa::pattn::kThreads,
                                                 msa::pattn::Layout::kBytes, s>>>(tm_q, tm_k, tm_v, Q);
@@ -192,6 +213,7 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   P.n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), P.n_units,
                                                 static_cast<int64_t>(msa::dattn::kMaxCtas)}));
   P.scale_log2 = softmax_scale * 1.4426950408889634f;
+  P.pages = pg;
   msa::dattn::sparse_attn_decode_sk_kernel<<<static_cast<unsigned>(P.n_cta), msa::dattn::kThreads,
                                              msa::dattn::Layout::kBytes, s>>>(tm_k, tm_v, P);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
@@ -202,7 +224,7 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
 
 int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache1, const void* src1,
                 const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, int row_bytes,
-                void* stream) {
+                void* stream, const msa_pages* pages) {
   int st = check_shape(sh);
   if (st != MSA_OK) return st;
   if (n_tok < 0) return MSA_ERR_RANGE;
@@ -210,20 +232,23 @@ int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache
   if (!cache0 || !src0 || !tok_stream || !tok_pos) return MSA_ERR_NULL;
   if (!aligned16(cache0) || !aligned16(src0) || (cache1 && !aligned16(cache1)) || (src1 && !aligned16(src1)))
     return MSA_ERR_ALIGN;
+  msa::KvPages pg;
+  int64_t rows = 0;
+  if ((st = pages_of(sh, pages, &pg, &rows)) != MSA_OK) return st;
   const int64_t warps = static_cast<int64_t>(n_tok) * sh->n_kv_heads;
   if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
   const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
   msa::append_rows_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint8_t*>(cache0), static_cast<const uint8_t*>(src0), static_cast<uint8_t*>(cache1),
       static_cast<const uint8_t*>(src1), tok_stream, tok_pos, n_tok, sh->n_streams, sh->n_kv_heads,
-      sh->capacity, row_bytes);
+      sh->capacity, row_bytes, pg);
   return cuda_status(cudaGetLastError());
 }
 
 template <typename KeyT>
 int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* idx_k_cache,
                       const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
-                      void* workspace, size_t workspace_bytes, void* stream) {
+                      void* workspace, size_t workspace_bytes, void* stream, const msa_pages* pages) {
   constexpr bool kF16 = std::is_same<KeyT, __half>::value;
   using Cfg = msa::gemv::Config<KeyT>;
   int st = check_shape(shape);
@@ -232,6 +257,9 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
   if (n_q == 0) return MSA_OK;
   if (!idx_q || !idx_k_cache || !q_stream || !q_pos || !block_scores) return MSA_ERR_NULL;
   if (!aligned16(idx_q) || !aligned16(idx_k_cache) || !aligned16(block_scores)) return MSA_ERR_ALIGN;
+  msa::KvPages pg;
+  int64_t key_rows_all = 0;
+  if ((st = pages_of(shape, pages, &pg, &key_rows_all)) != MSA_OK) return st;
   const bool tiles = scores_use_tiles(shape, n_q);
   const size_t need = scores_workspace(shape, n_q);
   if (need > 0) {
@@ -260,6 +288,7 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
   P.n_tasks = static_cast<long long>(n_q) * G * P.nblk;
   P.q_list = nullptr;
   P.q_count = nullptr;
+  P.pages = pg;
   const size_t smem = sizeof(Smem<KeyT, Cfg::kStages, Cfg::kWarps>);
   const auto kernel = block_scores_gemv_kernel<KeyT, Cfg::kStages, Cfg::kWarps, Cfg::kCtasPerSm>;
   constexpr int kThreads = (Cfg::kWarps + 1) * 32;
@@ -295,6 +324,7 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
     Q.kscale = reinterpret_cast<float*>(ws + L.kscale);
     Q.khi = reinterpret_cast<__half*>(ws + L.khi);
     Q.klo = reinterpret_cast<__half*>(ws + L.klo);
+    Q.pages = pg;
     const int64_t key_rows = static_cast<int64_t>(S) * G * cap;
     const int64_t q_rows = static_cast<int64_t>(G) * L.n_q_pad;
     CUtensorMap m_qhi, m_qlo, m_khi, m_klo;
@@ -325,6 +355,27 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
   return cuda_status(cudaGetLastError());
 }
 
+int append_idx_f16(const msa_shape* shape, msa_f16* idx_k_cache, const float* idx_k_new,
+                   const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream,
+                   const msa_pages* pages) {
+  int st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_tok < 0) return MSA_ERR_RANGE;
+  if (n_tok == 0) return MSA_OK;
+  if (!idx_k_cache || !idx_k_new || !tok_stream || !tok_pos) return MSA_ERR_NULL;
+  if (!aligned16(idx_k_cache) || !aligned16(idx_k_new)) return MSA_ERR_ALIGN;
+  msa::KvPages pg;
+  int64_t rows = 0;
+  if ((st = pages_of(shape, pages, &pg, &rows)) != MSA_OK) return st;
+  const int64_t warps = static_cast<int64_t>(n_tok) * shape->n_kv_heads;
+  if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
+  msa::append_idx_f16_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<__half*>(idx_k_cache), idx_k_new, tok_stream, tok_pos, n_tok, shape->n_streams,
+      shape->n_kv_heads, shape->capacity, pg);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -332,7 +383,7 @@ extern "C" {
 int msa_indexer_append(const msa_shape* shape, float* idx_k_cache, const float* idx_k_new,
                        const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
   return append_rows(shape, idx_k_cache, idx_k_new, nullptr, nullptr, tok_stream, tok_pos, n_tok,
-                     128 * static_cast<int>(sizeof(float)), stream);
+                     128 * static_cast<int>(sizeof(float)), stream, nullptr);
 }
 
 int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, const msa_bf16* k_new,
@@ -340,38 +391,26 @@ int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, 
                   void* stream) {
   if (n_tok > 0 && (!v_cache || !v_new)) return MSA_ERR_NULL;
   return append_rows(shape, k_cache, k_new, v_cache, v_new, tok_stream, tok_pos, n_tok,
-                     128 * static_cast<int>(sizeof(msa_bf16)), stream);
+                     128 * static_cast<int>(sizeof(msa_bf16)), stream, nullptr);
 }
 
 int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,
                      const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
                      void* workspace, size_t workspace_bytes, void* stream) {
   return block_scores_impl<float>(shape, idx_q, idx_k_cache, q_stream, q_pos, n_q, block_scores, workspace,
-                                  workspace_bytes, stream);
+                                  workspace_bytes, stream, nullptr);
 }
 
 int msa_block_scores_f16(const msa_shape* shape, const float* idx_q, const msa_f16* idx_k_cache,
                          const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
                          void* workspace, size_t workspace_bytes, void* stream) {
   return block_scores_impl<__half>(shape, idx_q, reinterpret_cast<const __half*>(idx_k_cache), q_stream, q_pos,
-                                   n_q, block_scores, workspace, workspace_bytes, stream);
+                                   n_q, block_scores, workspace, workspace_bytes, stream, nullptr);
 }
 
 int msa_indexer_append_f16(const msa_shape* shape, msa_f16* idx_k_cache, const float* idx_k_new,
                            const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
-  int st = check_shape(shape);
-  if (st != MSA_OK) return st;
-  if (n_tok < 0) return MSA_ERR_RANGE;
-  if (n_tok == 0) return MSA_OK;
-  if (!idx_k_cache || !idx_k_new || !tok_stream || !tok_pos) return MSA_ERR_NULL;
-  if (!aligned16(idx_k_cache) || !aligned16(idx_k_new)) return MSA_ERR_ALIGN;
-  const int64_t warps = static_cast<int64_t>(n_tok) * shape->n_kv_heads;
-  if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
-  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
-  msa::append_idx_f16_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<__half*>(idx_k_cache), idx_k_new, tok_stream, tok_pos, n_tok, shape->n_streams,
-      shape->n_kv_heads, shape->capacity);
-  return cuda_status(cudaGetLastError());
+  return append_idx_f16(shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, n_tok, stream, nullptr);
 }
 
 int msa_select_topk(const msa_shape* shape, const float* block_scores, const int32_t* q_pos, int32_t n_q,
@@ -406,7 +445,7 @@ int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, const msa_
                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
                            void* workspace, size_t workspace_bytes, void* stream) {
   return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
-                     workspace_bytes, stream, MSA_MODE_DECODE);
+                     workspace_bytes, stream, MSA_MODE_DECODE, nullptr);
 }
 
 int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
@@ -414,7 +453,7 @@ int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, const msa
                             const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
                             void* workspace, size_t workspace_bytes, void* stream) {
   return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
-                     workspace_bytes, stream, MSA_MODE_PREFILL);
+                     workspace_bytes, stream, MSA_MODE_PREFILL, nullptr);
 }
 
 // ---- attention without a caller workspace ----------------------------------
@@ -467,7 +506,68 @@ int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf16* q, co
     if (s2 != MSA_OK) return s2;
   }
   return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, scratch,
-                     MSA_NOALLOC_SCRATCH_BYTES, stream, MSA_MODE_DECODE);
+                     MSA_NOALLOC_SCRATCH_BYTES, stream, MSA_MODE_DECODE, nullptr);
+}
+
+// ---- paged caches ----------------------------------------------------------
+int msa_indexer_append_paged(const msa_shape* shape, const msa_pages* pages, float* idx_k_pool,
+                             const float* idx_k_new, const int32_t* tok_stream, const int32_t* tok_pos,
+                             int32_t n_tok, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return append_rows(shape, idx_k_pool, idx_k_new, nullptr, nullptr, tok_stream, tok_pos, n_tok,
+                     128 * static_cast<int>(sizeof(float)), stream, pages);
+}
+
+int msa_indexer_append_f16_paged(const msa_shape* shape, const msa_pages* pages, msa_f16* idx_k_pool,
+                                 const float* idx_k_new, const int32_t* tok_stream, const int32_t* tok_pos,
+                                 int32_t n_tok, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return append_idx_f16(shape, idx_k_pool, idx_k_new, tok_stream, tok_pos, n_tok, stream, pages);
+}
+
+int msa_kv_append_paged(const msa_shape* shape, const msa_pages* pages, msa_bf16* k_pool, msa_bf16* v_pool,
+                        const msa_bf16* k_new, const msa_bf16* v_new, const int32_t* tok_stream,
+                        const int32_t* tok_pos, int32_t n_tok, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  if (n_tok > 0 && (!v_pool || !v_new)) return MSA_ERR_NULL;
+  return append_rows(shape, k_pool, k_new, v_pool, v_new, tok_stream, tok_pos, n_tok,
+                     128 * static_cast<int>(sizeof(msa_bf16)), stream, pages);
+}
+
+int msa_block_scores_paged(const msa_shape* shape, const msa_pages* pages, const float* idx_q,
+                           const float* idx_k_pool, const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                           float* block_scores, void* workspace, size_t workspace_bytes, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return block_scores_impl<float>(shape, idx_q, idx_k_pool, q_stream, q_pos, n_q, block_scores, workspace,
+                                  workspace_bytes, stream, pages);
+}
+
+int msa_block_scores_f16_paged(const msa_shape* shape, const msa_pages* pages, const float* idx_q,
+                               const msa_f16* idx_k_pool, const int32_t* q_stream, const int32_t* q_pos,
+                               int32_t n_q, float* block_scores, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return block_scores_impl<__half>(shape, idx_q, reinterpret_cast<const __half*>(idx_k_pool), q_stream, q_pos,
+                                   n_q, block_scores, workspace, workspace_bytes, stream, pages);
+}
+
+int msa_sparse_attn_decode_paged(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
+                                 const msa_bf16* k_pool, const msa_bf16* v_pool, const int32_t* sel,
+                                 const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float softmax_scale,
+                                 msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return sparse_attn(shape, q, k_pool, v_pool, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_DECODE, pages);
+}
+
+int msa_sparse_attn_prefill_paged(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
+                                  const msa_bf16* k_pool, const msa_bf16* v_pool, const int32_t* sel,
+                                  const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                                  float softmax_scale, msa_bf16* out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return sparse_attn(shape, q, k_pool, v_pool, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_PREFILL, pages);
 }
 
 size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {

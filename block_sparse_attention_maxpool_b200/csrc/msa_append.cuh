@@ -1,7 +1,8 @@
-// Cache append: copies new tokens' rows into a [S][G][cap][row] cache.
-// Used for the F32 indexer-key cache (row = 128 floats = 512 B) and the
-// bf16 K/V caches (row = 128 bf16 = 256 B).  Pure data movement: one warp
-// per (token, group) row, 16-byte vector loads and stores.
+// Cache append: copies new tokens' rows into a [S][G][cap][row] cache, or
+// into the page its block table names for a paged cache.  Used for the F32
+// indexer-key cache (row = 128 floats = 512 B) and the bf16 K/V caches
+// (row = 128 bf16 = 256 B).  Pure data movement: one warp per (token, group)
+// row, 16-byte vector loads and stores.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -17,7 +18,7 @@ __global__ void __launch_bounds__(256) append_rows_kernel(
     uint8_t* __restrict__ cache0, const uint8_t* __restrict__ src0, uint8_t* __restrict__ cache1,
     const uint8_t* __restrict__ src1, const int32_t* __restrict__ tok_stream,
     const int32_t* __restrict__ tok_pos, int n_tok, int n_streams, int n_groups, int capacity,
-    int row_bytes) {
+    int row_bytes, const KvPages pages) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok * n_groups) return;
@@ -29,7 +30,12 @@ __global__ void __launch_bounds__(256) append_rows_kernel(
     if (g == 0 && lane == 0) raise_error(MSA_DEVERR_TOKEN_RANGE);
     return;
   }
-  const size_t dst_row = (static_cast<size_t>(s) * n_groups + g) * capacity + p;
+  const long long blk = kv_block_row(pages, s, g, p / 128, n_groups, capacity);
+  if (blk < 0) {
+    if (lane == 0) raise_error(MSA_DEVERR_PAGE_RANGE);
+    return;
+  }
+  const size_t dst_row = static_cast<size_t>(blk) + (p & 127);
   const size_t src_row = static_cast<size_t>(t) * n_groups + g;
   const int vecs = row_bytes >> 4;
   if (lane < vecs) {
@@ -51,7 +57,8 @@ __global__ void __launch_bounds__(256) append_idx_f16_kernel(__half* __restrict_
                                                              const float* __restrict__ src,
                                                              const int32_t* __restrict__ tok_stream,
                                                              const int32_t* __restrict__ tok_pos, int n_tok,
-                                                             int n_streams, int n_groups, int capacity) {
+                                                             int n_streams, int n_groups, int capacity,
+                                                             const KvPages pages) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok * n_groups) return;
@@ -63,13 +70,18 @@ __global__ void __launch_bounds__(256) append_idx_f16_kernel(__half* __restrict_
     if (g == 0 && lane == 0) raise_error(MSA_DEVERR_TOKEN_RANGE);
     return;
   }
+  const long long blk = kv_block_row(pages, s, g, p / 128, n_groups, capacity);
+  if (blk < 0) {
+    if (lane == 0) raise_error(MSA_DEVERR_PAGE_RANGE);
+    return;
+  }
   const float4 x = __ldg(reinterpret_cast<const float4*>(src + (static_cast<size_t>(t) * n_groups + g) * 128) + lane);
   const __half2 a = __floats2half2_rn(x.x, x.y);
   const __half2 b = __floats2half2_rn(x.z, x.w);
   uint2 out;
   out.x = *reinterpret_cast<const uint32_t*>(&a);
   out.y = *reinterpret_cast<const uint32_t*>(&b);
-  *(reinterpret_cast<uint2*>(cache + ((static_cast<size_t>(s) * n_groups + g) * capacity + p) * 128) + lane) = out;
+  *(reinterpret_cast<uint2*>(cache + (static_cast<size_t>(blk) + (p & 127)) * 128) + lane) = out;
 }
 
 }  // namespace msa

@@ -58,6 +58,7 @@ struct Params {
   int n_q, G, n_streams, capacity, n_cta;
   long long n_units;          // n_q * G * 16
   float scale_log2;
+  KvPages pages;              // block table of paged K/V caches (table null: contiguous)
 };
 
 __host__ __device__ inline long long unit_begin(long long U, int C, int c) { return U * c / C; }
@@ -71,8 +72,9 @@ __device__ inline int cta_of(long long U, int C, long long u) {
 }
 
 // Cache row of unit u's block, or -1 when the unit has nothing to attend
-// (padding, an invalid selection or an invalid query).  p: query position.
-__device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, bool report) {
+// (padding, an invalid selection, an invalid query or a block with no valid
+// page).  p: query position; slot0: first slot of the block in its stream.
+__device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, int& slot0, bool report) {
   const long long pair = u / kTopK;
   const int j = static_cast<int>(u - pair * kTopK);
   const int qi = static_cast<int>(pair / P.G);
@@ -89,7 +91,13 @@ __device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, bo
     if (report) raise_error(MSA_DEVERR_SEL_RANGE);
     return -1;
   }
-  return (s * P.G + g) * P.capacity + b * kBlock;
+  const long long row = kv_block_row(P.pages, s, g, b, P.G, P.capacity);
+  if (row < 0) {
+    if (report) raise_error(MSA_DEVERR_PAGE_RANGE);
+    return -1;
+  }
+  slot0 = b * kBlock;
+  return static_cast<int>(row);   // the host checks that every row fits 31 bits
 }
 
 // Merge the eight warps' states of one pair and write the output rows (or
@@ -190,8 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k = 0;
     bool ok = true;
     for (long long u = u0; u < u1 && ok; ++u) {
-      int p;
-      const int row = unit_row(P, u, p, false);
+      int p, slot0;
+      const int row = unit_row(P, u, p, slot0, false);
       if (row < 0) continue;
       const int st = k % kStages;
       const int use = k / kStages;
@@ -242,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         qa[ks][3] = __ldg(r1 + c + 4);
       }
     }
-    int p;
-    const int row = unit_row(P, u, p, warp == 0 && lane == 0);
+    int p, slot0;
+    const int row = unit_row(P, u, p, slot0, warp == 0 && lane == 0);
     if (row < 0) continue;
     const int st = k % kStages;
     if (ok) ok = mbar_wait(&full[st], (k / kStages) & 1);
@@ -265,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_bf16_16816(sacc[1], qa[ks], b[2], b[3]);
       }
       // causal mask inside the block, base-2 scaling, online softmax
-      const int jb = (row % P.capacity) + wr;    // absolute slot of this warp's first key
+      const int jb = slot0 + wr;    // slot (in the stream) of this warp's first key
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {

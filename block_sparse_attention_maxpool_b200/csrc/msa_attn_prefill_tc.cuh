@@ -68,11 +68,13 @@ struct Params {
   __nv_bfloat16* out;        // [n_q][Hq][D]
   int n_q, G, n_streams, capacity;
   float scale_log2;
+  KvPages pages;             // block table of paged K/V caches (table null: contiguous)
 };
 
 struct PairInfo {
-  int qi, g, p, nb, row0;
-  int blocks[kTopK];
+  int qi, g, p, nb;
+  int blocks[kTopK];         // selected visible blocks, ascending
+  int rows[kTopK];           // first cache row of each
 };
 
 // Pair t -> (group, query); the selected blocks that are visible.
@@ -82,12 +84,10 @@ __device__ __forceinline__ void pair_info(const Params& P, int t, PairInfo& I, b
   const int s = P.q_stream[I.qi];
   I.p = P.q_pos[I.qi];
   I.nb = 0;
-  I.row0 = 0;
   if (s < 0 || s >= P.n_streams || I.p < 0 || I.p >= P.capacity) {
     if (report && I.g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
     return;
   }
-  I.row0 = (s * P.G + I.g) * P.capacity;
   const int nvis = I.p / kBlock + 1;
   const int32_t* sl = P.sel + (static_cast<size_t>(I.qi) * P.G + I.g) * kTopK;
 #pragma unroll
@@ -98,6 +98,12 @@ __device__ __forceinline__ void pair_info(const Params& P, int t, PairInfo& I, b
       if (report) raise_error(MSA_DEVERR_SEL_RANGE);
       continue;
     }
+    const long long row = kv_block_row(P.pages, s, I.g, b, P.G, P.capacity);
+    if (row < 0) {
+      if (report) raise_error(MSA_DEVERR_PAGE_RANGE);
+      continue;
+    }
+    I.rows[I.nb] = static_cast<int>(row);   // the host checks that every row fits 31 bits
     I.blocks[I.nb++] = b;
   }
 }
@@ -202,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0) ok = mbar_wait(&rempty[st], (use - 1) & 1);
           if (!ok) break;
           uint8_t* dst = rbase + st * kTile;
-          const int row = I.row0 + I.blocks[j] * kBlock;
+          const int row = I.rows[j];
           mbar_arrive_expect_tx(&rfull[st], kTile);
           tma_load_2d(dst, map, 0, row, &rfull[st]);
           tma_load_2d(dst + kHalf, map, 64, row, &rfull[st]);

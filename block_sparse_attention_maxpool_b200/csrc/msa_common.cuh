@@ -19,6 +19,27 @@ __device__ unsigned int g_dev_error = 0;
 
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_dev_error, bit); }
 
+// Where a cache keeps the 128 slots of logical block b of (stream s, group g).
+// Contiguous caches are [S][G][capacity][row]; paged caches are pools of
+// pages [n_pages][G][128][row] with a block table [S][capacity / 128] that
+// names the page holding each logical block (MSA pull request, issue thread
+// on unified KV caches: block selection and gathering must go through a
+// sequence-relative page indirection, as the reference MSA kernel's page
+// index does, instead of absolute slots of one flat buffer).
+struct KvPages {
+  const int32_t* table;   // null: contiguous cache
+  int n_pages;
+};
+
+// First row of the block in the cache viewed as 2-D [rows][row]; -1 when a
+// paged cache maps the block to no valid page.
+__device__ __forceinline__ long long kv_block_row(const KvPages& pg, int s, int g, int b, int G, int capacity) {
+  if (pg.table == nullptr) return (static_cast<long long>(s) * G + g) * capacity + static_cast<long long>(b) * 128;
+  const int page = __ldg(pg.table + static_cast<size_t>(s) * (capacity / 128) + b);
+  if (page < 0 || page >= pg.n_pages) return -1;
+  return (static_cast<long long>(page) * G + g) * 128;
+}
+
 // A wait on an mbarrier gives up after this many SM clock cycles (about half
 // a second at the B200's boost clock), records MSA_DEVERR_TIMEOUT and lets
 // the kernel return instead of hanging the GPU.

@@ -69,7 +69,7 @@ struct Smem {
 template <typename KeyT>
 struct Params {
   const float* idx_q;    // [n_q][G][Di]
-  const KeyT* idx_k;     // [S][G][cap][Di]
+  const KeyT* idx_k;     // [S][G][cap][Di], or pages [n_pages][G][128][Di]
   const int32_t* q_stream;
   const int32_t* q_pos;
   float* bs;             // [n_q][G][nblk]
@@ -77,6 +77,7 @@ struct Params {
   long long n_tasks;     // n_q * G * nblk (ignored in list mode)
   const int32_t* q_list;   // list mode: score only these query indices ...
   const int32_t* q_count;  // ... of which there are *q_count (device memory)
+  KvPages pages;           // block table of a paged cache (table null: contiguous)
 };
 
 // Walks the task space (query slot, group, block) in order, block fastest,
@@ -196,9 +197,10 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv
     for (long long t = t_begin; t < t_end && ok; ++t) {
       if (t > t_begin) cur.next(P);
       if (cur.b >= cur.nvis) continue;
+      const long long row = kv_block_row(P.pages, cur.s, cur.g, cur.b, P.G, P.capacity);
+      if (row < 0) continue;
       const int n_chunks = min(cur.p - cur.b * kBlock, kBlock - 1) / R::kPerStage + 1;
-      const KeyT* src = P.idx_k + ((static_cast<size_t>(cur.s) * P.G + cur.g) * P.capacity +
-                                   static_cast<size_t>(cur.b) * kBlock) * kDi;
+      const KeyT* src = P.idx_k + static_cast<size_t>(row) * kDi;
       for (int c = 0; c < n_chunks; ++c, ++k) {
         const int st = k % kStages;
         const uint32_t use = static_cast<uint32_t>(k / kStages);
@@ -236,6 +238,13 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv
       if (warp == 0 && lane == 0) {
         P.bs[out] = -INFINITY;
         if (cur.nvis == 0 && b == 0 && cur.g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
+      }
+      continue;
+    }
+    if (P.pages.table != nullptr && kv_block_row(P.pages, cur.s, cur.g, b, P.G, P.capacity) < 0) {
+      if (warp == 0 && lane == 0) {   // the producer skipped this block too
+        P.bs[out] = -INFINITY;
+        raise_error(MSA_DEVERR_PAGE_RANGE);
       }
       continue;
     }

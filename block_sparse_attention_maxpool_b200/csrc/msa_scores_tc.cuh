@@ -84,8 +84,8 @@ __host__ inline Workspace workspace_layout(int n_q, int G, int S, int cap) {
 
 struct Params {
   const float* idx_q;       // [n_q][G][Di]
-  const float* idx_k;       // [S][G][cap][Di] F32 cache (null when idx_k16 is used)
-  const __half* idx_k16;    // [S][G][cap][Di] F16 cache variant (null for the F32 cache)
+  const float* idx_k;       // [S][G][cap][Di] F32 cache, or its pages (null when idx_k16 is used)
+  const __half* idx_k16;    // the same for the F16 cache variant (null for the F32 cache)
   const int32_t* q_stream;
   const int32_t* q_pos;
   float* bs;                // [n_q][G][nblk]
@@ -100,6 +100,7 @@ struct Params {
   float* kscale;            // [S][G][cap]   2^-e_k
   __half* khi;              // [S][G][cap][Di]
   __half* klo;
+  KvPages pages;            // block table of a paged key cache (table null: contiguous)
 };
 
 __device__ __forceinline__ bool query_ok(const Params& P, int q, int& s, int& p) {
@@ -213,23 +214,43 @@ __global__ void __launch_bounds__(256) tc_split_queries_kernel(const Params P) {
   if (!ok && lane == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
 }
 
-// One warp per key row (stream, group, slot) that some tile will read.
+// One warp per key row (stream, group, slot) that some tile will read.  The
+// split rows are laid out by logical slot whatever the cache layout, so the
+// tile kernel never sees the page table.  A row of a paged block with no
+// valid page gets scale NaN: its scores drop out of the max-pool (the block
+// scores -inf) and MSA_DEVERR_PAGE_RANGE is set.
 __global__ void __launch_bounds__(256) tc_split_keys_kernel(const Params P) {
   const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(P.n_streams) * P.G * P.capacity;
   if (w >= rows) return;
   const int j = static_cast<int>(w % P.capacity);
-  const int s = static_cast<int>(w / (static_cast<long long>(P.G) * P.capacity));
+  const long long sg = w / P.capacity;
+  const int s = static_cast<int>(sg / P.G);
   if (j >= P.counters[1 + s] * kBlock) return;
+  long long src = w;
+  if (P.pages.table != nullptr) {
+    const int g = static_cast<int>(sg - static_cast<long long>(s) * P.G);
+    const long long blk = kv_block_row(P.pages, s, g, j / kBlock, P.G, P.capacity);
+    if (blk < 0) {
+      *reinterpret_cast<uint2*>(P.khi + w * kDi + lane * 4) = make_uint2(0u, 0u);
+      *reinterpret_cast<uint2*>(P.klo + w * kDi + lane * 4) = make_uint2(0u, 0u);
+      if (lane == 0) {
+        P.kscale[w] = __int_as_float(0x7fc00000);
+        if ((j & (kBlock - 1)) == 0) raise_error(MSA_DEVERR_PAGE_RANGE);
+      }
+      return;
+    }
+    src = blk + (j & (kBlock - 1));
+  }
   float4 x;
   if (P.idx_k16 != nullptr) {
-    const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(P.idx_k16 + w * kDi) + lane);
+    const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(P.idx_k16 + src * kDi) + lane);
     const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
     const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
     x = make_float4(a.x, a.y, b.x, b.y);
   } else {
-    x = __ldcs(reinterpret_cast<const float4*>(P.idx_k + w * kDi) + lane);
+    x = __ldcs(reinterpret_cast<const float4*>(P.idx_k + src * kDi) + lane);
   }
   __half2 hi[2], lo[2];
   const int e = split_row4(x, hi, lo);

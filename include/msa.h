@@ -72,6 +72,7 @@ extern "C" {
 #define MSA_DEVERR_TOKEN_RANGE 0x2u /* tok_stream/tok_pos outside the cache: token skipped   */
 #define MSA_DEVERR_SEL_RANGE   0x4u /* sel id not a visible block: that block skipped       */
 #define MSA_DEVERR_TIMEOUT     0x8u /* a bounded wait on a copy gave up: output incomplete  */
+#define MSA_DEVERR_PAGE_RANGE  0x10u /* paged cache: a touched block has no valid page: skipped */
 
 /* The local-force bias added to the score of each query's own block
  * ("a large positive bias on each query's local block", MSA pull request,
@@ -229,6 +230,65 @@ MSA_API int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf1
                                            const int32_t* sel, const int32_t* q_stream,
                                            const int32_t* q_pos, int32_t n_q, float softmax_scale,
                                            msa_bf16* out, void* stream);
+
+/* ---- paged caches --------------------------------------------------------
+ * The calls above address a cache as one region per stream, so logical slot
+ * j of stream s is physical slot j of region s.  The MSA pull request's
+ * issue thread on unified KV caches finds that block scoring and gathering
+ * by absolute slot breaks once streams share one buffer, and that a fix
+ * needs a sequence-relative page indirection consulted by the scoring and
+ * gather steps (what the reference MSA kernel's page index provides).  These
+ * calls are that indirection.
+ *
+ * A page holds the 128 slots of one key block for every group.  Pools:
+ *   idx_k_pool [n_pages][G][128][Di] f32 (or fp16 for the _f16 calls),
+ *   k_pool, v_pool [n_pages][G][128][D] bf16.
+ * block_table [n_streams][capacity / 128] int32 (device memory, 4-byte
+ * aligned) names the page that holds logical block b of stream s; capacity
+ * is the logical length of a stream.  Several streams may name the same
+ * page (a shared prefix) for reading; writing a shared page is the caller's
+ * race.  Each paged call computes exactly what its contiguous counterpart
+ * computes on the logical cache cache[s][g][j] = pool[block_table[s][j/128]]
+ * [g][j % 128]: same arguments otherwise, same layouts of every other array,
+ * same workspace (msa_workspace_bytes).  Only blocks a call touches are
+ * looked up (a token's block for the appends, blocks b <= q_pos/128 for
+ * scores, selected blocks for attention).  A touched block whose entry is
+ * negative or >= n_pages is skipped and sets MSA_DEVERR_PAGE_RANGE: the
+ * token is not written, the block scores -inf, attention leaves the block
+ * out.  Host-side errors: pages or block_table NULL (MSA_ERR_NULL),
+ * n_pages < 1 (MSA_ERR_RANGE), n_pages * G * 128 >= 2^31 (MSA_ERR_SHAPE). */
+typedef struct msa_pages {
+  const int32_t* block_table;  /* [n_streams][capacity / block], page ids      */
+  int32_t n_pages;             /* pages in each pool                           */
+} msa_pages;
+
+MSA_API int msa_indexer_append_paged(const msa_shape* shape, const msa_pages* pages, float* idx_k_pool,
+                                     const float* idx_k_new, const int32_t* tok_stream, const int32_t* tok_pos,
+                                     int32_t n_tok, void* stream);
+MSA_API int msa_indexer_append_f16_paged(const msa_shape* shape, const msa_pages* pages, msa_f16* idx_k_pool,
+                                         const float* idx_k_new, const int32_t* tok_stream,
+                                         const int32_t* tok_pos, int32_t n_tok, void* stream);
+MSA_API int msa_kv_append_paged(const msa_shape* shape, const msa_pages* pages, msa_bf16* k_pool,
+                                msa_bf16* v_pool, const msa_bf16* k_new, const msa_bf16* v_new,
+                                const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream);
+MSA_API int msa_block_scores_paged(const msa_shape* shape, const msa_pages* pages, const float* idx_q,
+                                   const float* idx_k_pool, const int32_t* q_stream, const int32_t* q_pos,
+                                   int32_t n_q, float* block_scores, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+MSA_API int msa_block_scores_f16_paged(const msa_shape* shape, const msa_pages* pages, const float* idx_q,
+                                       const msa_f16* idx_k_pool, const int32_t* q_stream, const int32_t* q_pos,
+                                       int32_t n_q, float* block_scores, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+MSA_API int msa_sparse_attn_decode_paged(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
+                                         const msa_bf16* k_pool, const msa_bf16* v_pool, const int32_t* sel,
+                                         const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                                         float softmax_scale, msa_bf16* out, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+MSA_API int msa_sparse_attn_prefill_paged(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
+                                          const msa_bf16* k_pool, const msa_bf16* v_pool, const int32_t* sel,
+                                          const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                                          float softmax_scale, msa_bf16* out, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace that msa_block_scores and the attention call of `mode`
  * need for n_q queries (the larger of the two; one buffer serves both calls

@@ -21,12 +21,14 @@ Comparison rules
 """
 from __future__ import annotations
 
+import dataclasses
 import math
 
 import torch
 
 import block_sparse_attention_maxpool_b200 as msa
 import oracle
+import workloads as W
 from tests.oracle_pins import near_tie_excused
 
 U32 = 2.0 ** -24
@@ -49,9 +51,9 @@ def to_dev(inp, dev="cuda", idx_f16=False):
     return d
 
 
-def run_step(shape, d, prefill=False):
+def run_step(shape, d, prefill=False, pages=None):
     caches = {k: d[k] for k in ("idx_k_cache", "k_cache", "v_cache")}
-    out, sel, n_sel, bs = msa.decode_step(shape, caches, d, prefill=prefill)
+    out, sel, n_sel, bs = msa.decode_step(shape, caches, d, prefill=prefill, pages=pages)
     err = msa.msa_get_device_error()
     return out, sel, n_sel, bs, err
 
@@ -138,17 +140,43 @@ def check_attention(out_gpu, out_orc, rows=None):
     return float((g - w).abs().max()), mean
 
 
-def full_parity(inp, queries=None, prefill=False, dev="cuda", idx_f16=False):
+def full_parity(inp, queries=None, prefill=False, dev="cuda", idx_f16=False, paged=None):
     """Run one step on the GPU and compare every part with the oracle on the
-    query indices ``queries`` (all when None).  Returns a small report."""
+    query indices ``queries`` (all when None).  With ``paged`` (keyword
+    arguments of workloads.page_layout) the GPU runs the paged calls on
+    shuffled page pools and the oracle reads the same pools through its own
+    logical view.  Returns a small report."""
     w = inp.w
     shape = shape_of(w)
     d = to_dev(inp, dev, idx_f16)
-    out, sel, n_sel, bs, err = run_step(shape, d, prefill)
+    pages = None
+    if paged is not None:
+        lay = W.page_layout(inp, **paged)
+        d["idx_k_cache"] = lay.idx_pool.to(dev)
+        if idx_f16:
+            d["idx_k_cache"] = d["idx_k_cache"].half()
+        d["k_cache"], d["v_cache"] = lay.k_pool.to(dev), lay.v_pool.to(dev)
+        pages = msa.Pages(lay.block_table.to(dev), lay.n_pages)
+        # the oracle's inputs: the pools seen through its logical view
+        inp = dataclasses.replace(
+            inp, idx_k_cache=oracle.logical_cache(lay.idx_pool, lay.block_table, w.block),
+            k_cache=oracle.logical_cache(lay.k_pool, lay.block_table, w.block),
+            v_cache=oracle.logical_cache(lay.v_pool, lay.block_table, w.block))
+    out, sel, n_sel, bs, err = run_step(shape, d, prefill, pages)
     assert err == 0, f"device error word {err:#x}"
     idx_o, k_o, v_o = oracle_caches(inp, idx_f16)
-    assert torch.equal(d["idx_k_cache"].cpu(), idx_o), "indexer cache after append"
-    assert torch.equal(d["k_cache"].cpu(), k_o) and torch.equal(d["v_cache"].cpu(), v_o), "K/V append"
+    if paged is None:
+        assert torch.equal(d["idx_k_cache"].cpu(), idx_o), "indexer cache after append"
+        assert torch.equal(d["k_cache"].cpu(), k_o) and torch.equal(d["v_cache"].cpu(), v_o), "K/V append"
+    else:
+        bt = lay.block_table
+        ipool = lay.idx_pool.half() if idx_f16 else lay.idx_pool
+        new_idx = inp.idx_k_new.half() if idx_f16 else inp.idx_k_new
+        want_i = oracle.paged_append(ipool, new_idx, inp.tok_stream, inp.tok_pos, bt, w.block)
+        want_k = oracle.paged_append(lay.k_pool, inp.k_new, inp.tok_stream, inp.tok_pos, bt, w.block)
+        want_v = oracle.paged_append(lay.v_pool, inp.v_new, inp.tok_stream, inp.tok_pos, bt, w.block)
+        assert torch.equal(d["idx_k_cache"].cpu(), want_i), "indexer pool after append"
+        assert torch.equal(d["k_cache"].cpu(), want_k) and torch.equal(d["v_cache"].cpu(), want_v), "K/V pools"
     n_q = inp.q_pos.numel()
     qsub = torch.arange(n_q) if queries is None else torch.as_tensor(queries, dtype=torch.long)
     qs, qp = inp.q_stream[qsub], inp.q_pos[qsub]

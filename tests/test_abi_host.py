@@ -145,3 +145,29 @@ def test_binding_rejects_cpu_tensors():
         msa.msa_select_topk(sh, torch.zeros((1, 4, 1)), torch.zeros(1, dtype=torch.int32),
                             sel=torch.zeros((1, 4, 16), dtype=torch.int32),
                             n_sel=torch.zeros((1, 4), dtype=torch.int32), stream=0)
+
+
+def test_paged_calls_validate_the_page_table(lib):
+    s = GOOD.c()
+    fake = FAKE
+
+    def pages(table, n):
+        return ctypes.byref(msa.CPages(table, n))
+
+    # a NULL msa_pages is rejected by every paged call
+    assert lib.msa_indexer_append_paged(ctypes.byref(s), None, fake, fake, fake, fake, 2, None) == -1
+    assert lib.msa_kv_append_paged(ctypes.byref(s), None, fake, fake, fake, fake, fake, fake, 2, None) == -1
+    assert lib.msa_block_scores_paged(ctypes.byref(s), None, fake, fake, fake, fake, 2, fake, 0, 0, None) == -1
+    assert lib.msa_sparse_attn_decode_paged(ctypes.byref(s), None, fake, fake, fake, fake, fake, fake, 2,
+                                            ctypes.c_float(0.088), fake, fake, 1 << 24, None) == -1
+    # the table itself: NULL, misaligned, no pages, a pool too large for 31-bit rows
+    args = (fake, fake, fake, fake, 2, None)
+    assert lib.msa_indexer_append_paged(ctypes.byref(s), pages(None, 4), *args) == -1
+    assert lib.msa_indexer_append_paged(ctypes.byref(s), pages(fake + 2, 4), *args) == -2
+    assert lib.msa_indexer_append_paged(ctypes.byref(s), pages(fake, 0), *args) == -4
+    assert lib.msa_indexer_append_f16_paged(ctypes.byref(s), pages(fake, (1 << 31) // (4 * 128)), *args) == -3
+    assert lib.msa_indexer_append_paged(ctypes.byref(s), pages(fake, 4), fake, fake, fake, fake, 0, None) == 0
+    assert lib.msa_block_scores_f16_paged(ctypes.byref(s), pages(fake, 0), fake, fake, fake, fake, 2, fake,
+                                          0, 0, None) == -4
+    assert lib.msa_sparse_attn_prefill_paged(ctypes.byref(s), pages(None, 4), fake, fake, fake, fake, fake, fake,
+                                             2, ctypes.c_float(0.088), fake, 0, 0, None) == -1

@@ -205,3 +205,57 @@ def make_custom(n_streams: int, capacity: int, lengths, q_positions, *, seed: in
     idx_q = _idx_draw(g, (n_q, G, idx_dim), idx_dim, quantize_idx)
     q = torch.randn((n_q, n_q_heads, head_dim), generator=g).to(kv_dtype)
     return idx, k, v, q_stream, q_pos, idx_q, q
+
+
+# ---------------------------------------------------------------------------
+# paged layout of a step's caches
+# ---------------------------------------------------------------------------
+POISON = 64.0   # value of every row in a page no stream maps (reading one shows)
+
+
+@dataclass
+class PagedCaches:
+    """The step's caches laid out as page pools [n_pages][G][block][row] plus
+    the block table [S][capacity / block] (int32) naming each logical block's
+    page.  Spare pages and the pages of unmapped blocks hold POISON."""
+    block_table: torch.Tensor
+    n_pages: int
+    idx_pool: torch.Tensor
+    k_pool: torch.Tensor
+    v_pool: torch.Tensor
+
+
+def page_layout(inp: Inputs, seed: int = 0, spare_pages: int = 3, shared_prefix_blocks: int = 0,
+                unmapped_from: int | None = None) -> PagedCaches:
+    """Scatter the contiguous caches of ``inp`` into shuffled pages.
+
+    Every (stream, block) gets its own page at a random pool slot, except
+    that streams 1.. map their first ``shared_prefix_blocks`` blocks to
+    stream 0's pages (a shared prefix: their logical rows there become stream
+    0's rows; keep those blocks below the existing length so no step appends
+    into a shared page).  Blocks from ``unmapped_from`` on get table entry -1.
+    """
+    S, G, cap, Di = inp.idx_k_cache.shape
+    D = inp.k_cache.shape[3]
+    B = inp.w.block
+    nb = cap // B
+    last = nb if unmapped_from is None else min(nb, unmapped_from)
+    own = [(s, b) for s in range(S) for b in range(last) if s == 0 or b >= shared_prefix_blocks]
+    n_pages = len(own) + spare_pages
+    g = torch.Generator().manual_seed(seed * 7919 + 101)
+    slot = torch.randperm(n_pages, generator=g)
+    table = torch.full((S, nb), -1, dtype=torch.int32)
+    for i, (s, b) in enumerate(own):
+        table[s, b] = int(slot[i])
+    for s in range(1, S):
+        for b in range(min(shared_prefix_blocks, last)):
+            table[s, b] = table[0, b]
+    idx_pool = torch.full((n_pages, G, B, Di), POISON, dtype=inp.idx_k_cache.dtype)
+    k_pool = torch.full((n_pages, G, B, D), POISON, dtype=inp.k_cache.dtype)
+    v_pool = torch.full((n_pages, G, B, D), POISON, dtype=inp.v_cache.dtype)
+    for s, b in own:
+        pg = int(table[s, b])
+        idx_pool[pg] = inp.idx_k_cache[s, :, b * B:(b + 1) * B]
+        k_pool[pg] = inp.k_cache[s, :, b * B:(b + 1) * B]
+        v_pool[pg] = inp.v_cache[s, :, b * B:(b + 1) * B]
+    return PagedCaches(table, n_pages, idx_pool, k_pool, v_pool)
