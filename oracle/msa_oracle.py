@@ -29,6 +29,11 @@ What it computes, and where each step is stated (page titles as cited):
   branch): indexer scores are accumulated in F32 (the oracle uses FP64, which
   is at least that exact) and the KV length is a multiple of 128.
 
+* "deepseek2 : GLM-DSA sparse attention (lightning indexer)" (ik_llama.cpp
+  pull request), section "What this does" and its review thread: the
+  token-level variant (``dsa_*`` functions): per-head indexer products times
+  per-head weights, summed over the indexer heads, top-k tokens kept.
+
 Readings where the pages are silent (each also listed in the design notes):
 * the local-force bias is the constant LOCAL_BIAS = 2**100 (any bias larger
   than twice the largest |score| gives the same selection);
@@ -269,3 +274,102 @@ def msa_step(inp_idx_k_cache, k_cache, v_cache, idx_q, q, q_stream, q_pos, block
     sel, n_sel = select_blocks(bs, q_pos, block, top_k)
     out = sparse_attention(q, k_cache, v_cache, sel, q_stream, q_pos, block, scale, queries)
     return bs, sel, n_sel, out
+
+
+# ---------------------------------------------------------------------------
+# token-level variant: the lightning indexer (DSA)
+# ---------------------------------------------------------------------------
+# "deepseek2 : GLM-DSA sparse attention (lightning indexer)" (ik_llama.cpp
+# pull request), section "What this does": the indexer scores each query
+# against the indexer keys, keeps the top-k highest-scoring keys per query
+# (tokens, not blocks; GLM-5.2's indexer top_k is 2048) and masks the rest out
+# of attention.  The indexer-key cache holds one F16 key per token
+# ([head_size, kv_size]).  The review thread describes the score as the
+# per-indexer-head products q_h . k "element-wise multiplied with another
+# matrix" (per-head weights) and then reduced over the indexer heads.  The
+# keys' Hadamard rotation is applied by the caller before the keys reach the
+# cache (an orthogonal rotation of both sides leaves q . k unchanged).
+# Readings where the page is silent: each head's product passes through a
+# ReLU when ``relu`` is true (the published lightning-indexer definition the
+# page names; the page itself does not print the formula); equal scores keep
+# the lower token index; with at most top_k visible tokens every visible token
+# is kept (the page's "no-op-exact" check: the sparse mask then equals the
+# causal mask).
+def dsa_token_scores(q_idx: torch.Tensor, weights: torch.Tensor, k_idx_cache: torch.Tensor,
+                     q_stream: torch.Tensor, q_pos: torch.Tensor, relu: bool = True) -> torch.Tensor:
+    """I[t][s] = sum_h weights[t][h] * act(q_idx[t][h] . k_idx_cache[stream][s])
+    for the visible tokens s <= q_pos[t], -inf for s > q_pos[t].
+
+    q_idx [n_q][H][Di], weights [n_q][H], k_idx_cache [S][cap][Di]."""
+    n_q, H, Di = q_idx.shape
+    cap = k_idx_cache.shape[1]
+    out = torch.full((n_q, cap), NEG_INF, dtype=F64)
+    for t in range(n_q):
+        s, p = int(q_stream[t]), int(q_pos[t])
+        keys = _cpu64(k_idx_cache[s, :p + 1])                  # [p+1][Di]
+        per_head = keys @ _cpu64(q_idx[t]).T                   # [p+1][H]
+        if relu:
+            per_head = per_head.clamp_min(0.0)
+        out[t, :p + 1] = per_head @ _cpu64(weights[t])
+    return out
+
+
+def dsa_ranked_tokens(scores_row: torch.Tensor, pos: int) -> list[int]:
+    """Visible tokens ordered by (score descending, index ascending)."""
+    return sorted(range(pos + 1), key=lambda s: (-float(scores_row[s]), s))
+
+
+def dsa_select_one(scores_row: torch.Tensor, pos: int, top_k: int) -> list[int]:
+    """Kept tokens of one query, ascending: every visible token when there
+    are at most top_k of them, else the first top_k of the ranking."""
+    if pos + 1 <= top_k:
+        return list(range(pos + 1))
+    return sorted(dsa_ranked_tokens(scores_row, pos)[:top_k])
+
+
+def dsa_select_tokens(scores: torch.Tensor, q_pos: torch.Tensor, top_k: int, width: int):
+    """sel [n_q][width] int32 (ascending token ids, -1 padded) and n_sel [n_q]."""
+    n_q = scores.shape[0]
+    sel = torch.full((n_q, width), -1, dtype=torch.int32)
+    n_sel = torch.zeros((n_q,), dtype=torch.int32)
+    for t in range(n_q):
+        ids = dsa_select_one(scores[t], int(q_pos[t]), top_k)
+        sel[t, :len(ids)] = torch.tensor(ids, dtype=torch.int32)
+        n_sel[t] = len(ids)
+    return sel, n_sel
+
+
+def dsa_boundary_scores(scores_row: torch.Tensor, pos: int, top_k: int):
+    """(score of rank top_k, score of rank top_k + 1), or None when every
+    visible token is kept."""
+    if pos + 1 <= top_k:
+        return None
+    ranked = dsa_ranked_tokens(scores_row, pos)
+    return float(scores_row[ranked[top_k - 1]]), float(scores_row[ranked[top_k]])
+
+
+def dsa_sparse_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                         sel_tok: torch.Tensor, q_stream: torch.Tensor, q_pos: torch.Tensor,
+                         scale: float | None = None) -> torch.Tensor:
+    """out[n_q][Hq][D] float64: every head h (group g = h // (Hq/G)) attends to
+    the kept tokens of its query (one token set shared by all groups) in its
+    group's K/V rows: softmax(scale * q_h . K_rows^T) . V_rows."""
+    n_q, Hq, D = q.shape
+    G = k_cache.shape[1]
+    heads_per_group = Hq // G
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = torch.zeros((n_q, Hq, D), dtype=F64)
+    for t in range(n_q):
+        s, p = int(q_stream[t]), int(q_pos[t])
+        rows = [int(j) for j in sel_tok[t].tolist() if 0 <= int(j) <= p]
+        if not rows:
+            continue
+        for g in range(G):
+            K = _cpu64(k_cache[s, g, rows])
+            V = _cpu64(v_cache[s, g, rows])
+            for h in range(g * heads_per_group, (g + 1) * heads_per_group):
+                logits = (K @ _cpu64(q[t, h])) * scale
+                w = torch.exp(logits - logits.max())
+                out[t, h] = (w / w.sum()) @ V
+    return out

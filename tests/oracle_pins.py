@@ -388,10 +388,128 @@ def pin_paged_append_commutes(o, seed=11):
     assert torch.equal(after[spare], moved[spare])
 
 
+def _dsa_case(seed, S=2, cap=12, H=3, Di=4, n_q=3):
+    g = torch.Generator().manual_seed(seed)
+    keys = torch.randn((S, cap, Di), generator=g, dtype=F64)
+    q = torch.randn((n_q, H, Di), generator=g, dtype=F64)
+    w = torch.randn((n_q, H), generator=g, dtype=F64)
+    qs = torch.tensor([i % S for i in range(n_q)], dtype=torch.int32)
+    qp = torch.tensor([cap - 1 - 3 * i for i in range(n_q)], dtype=torch.int32)
+    return keys, q, w, qs, qp
+
+
+def pin_dsa_scores_identities(o, seed=12):
+    """Lightning-indexer score identities: a basis query on one head with unit
+    weight reads one key coordinate (through the ReLU when enabled); the score
+    is linear in the weights; relu(x) - relu(-x) = x turns the ReLU scores of
+    q and -q into the plain weighted dot products; tokens past the query are
+    -inf."""
+    keys, q, w, qs, qp = _dsa_case(seed)
+    n_q, H, Di = q.shape
+    # basis query: head 1 = e_2, weight e_1 -> score[s] = act(key[s][2])
+    qb = torch.zeros_like(q)
+    qb[:, 1, 2] = 1.0
+    wb = torch.zeros_like(w)
+    wb[:, 1] = 1.0
+    for relu in (False, True):
+        sc = o.dsa_token_scores(qb, wb, keys, qs, qp, relu=relu)
+        for t in range(n_q):
+            p = int(qp[t])
+            col = keys[int(qs[t]), :p + 1, 2]
+            want = col.clamp_min(0.0) if relu else col
+            assert torch.equal(sc[t, :p + 1], want)
+            assert bool(torch.isneginf(sc[t, p + 1:]).all())
+    # linear in the weights
+    w2 = torch.randn(w.shape, generator=torch.Generator().manual_seed(seed + 1), dtype=F64)
+    for relu in (False, True):
+        a = o.dsa_token_scores(q, w + 2.0 * w2, keys, qs, qp, relu)
+        b = o.dsa_token_scores(q, w, keys, qs, qp, relu) + 2.0 * o.dsa_token_scores(q, w2, keys, qs, qp, relu)
+        fin = torch.isfinite(a)
+        assert torch.equal(fin, torch.isfinite(b))
+        assert torch.allclose(a[fin], b[fin], rtol=0, atol=1e-12)
+    # relu(x) - relu(-x) = x
+    plus = o.dsa_token_scores(q, w, keys, qs, qp, True)
+    minus = o.dsa_token_scores(-q, w, keys, qs, qp, True)
+    plain = o.dsa_token_scores(q, w, keys, qs, qp, False)
+    fin = torch.isfinite(plain)
+    assert torch.allclose((plus - minus)[fin], plain[fin], rtol=0, atol=1e-12)
+    # a ReLU score with nonnegative weights is nonnegative
+    assert bool((o.dsa_token_scores(q, w.abs(), keys, qs, qp, True)[fin] >= 0).all())
+
+
+def _bruteforce_tokens(row, pos, top_k):
+    """The k-subset of visible tokens whose (score, -index) pairs, sorted
+    descending, are lexicographically largest."""
+    nvis = pos + 1
+    k = min(top_k, nvis)
+    best, best_ids = None, None
+    for comb in itertools.combinations(range(nvis), k):
+        key = sorted(((float(row[s]), -s) for s in comb), reverse=True)
+        if best is None or key > best:
+            best, best_ids = key, sorted(comb)
+    return best_ids
+
+
+def pin_dsa_selection_bruteforce(o, seed=13):
+    """Token top-k against brute force over every subset, on small integer
+    scores with many ties, for every visible length and several k."""
+    g = torch.Generator().manual_seed(seed)
+    for trial in range(40):
+        n = 9
+        row = torch.randint(-2, 3, (n,), generator=g).to(F64)
+        pos = int(torch.randint(0, n, (1,), generator=g))
+        for top_k in (1, 2, 3, 5, 9):
+            assert o.dsa_select_one(row, pos, top_k) == _bruteforce_tokens(row, pos, top_k), (row, pos, top_k)
+    sel, n_sel = o.dsa_select_tokens(torch.tensor([[3.0, 1.0, 3.0, 2.0, float("-inf")]], dtype=F64),
+                                     torch.tensor([3], dtype=torch.int32), 2, 4)
+    assert sel.tolist() == [[0, 2, -1, -1]] and n_sel.tolist() == [2]
+    assert o.dsa_boundary_scores(torch.tensor([3.0, 1.0, 3.0, 2.0], dtype=F64), 3, 2) == (3.0, 2.0)
+    assert o.dsa_boundary_scores(torch.tensor([3.0, 1.0], dtype=F64), 1, 2) is None
+
+
+def _dsa_attn_case(seed, cap=12, G=2, Hq=4, D=6):
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn((2, G, cap, D), generator=g, dtype=F64)
+    v = torch.randn((2, G, cap, D), generator=g, dtype=F64)
+    q = torch.randn((3, Hq, D), generator=g, dtype=F64)
+    qs = torch.tensor([0, 1, 1], dtype=torch.int32)
+    qp = torch.tensor([11, 7, 4], dtype=torch.int32)
+    return k, v, q, qs, qp
+
+
+def pin_dsa_noop_exact(o, seed=14):
+    """With at most top_k visible tokens every token is kept and the attention
+    is dense causal attention (the DSA page's "no-op-exact" check), against
+    scaled_dot_product_attention in float64."""
+    k, v, q, qs, qp = _dsa_attn_case(seed)
+    scores = torch.randn((3, 12), generator=torch.Generator().manual_seed(seed), dtype=F64)
+    sel, n_sel = o.dsa_select_tokens(scores, qp, 16, 16)
+    assert n_sel.tolist() == [12, 8, 5]
+    got = o.dsa_sparse_attention(q, k, v, sel, qs, qp)
+    want = _sdpa_reference(q, k, v, qs, qp, lambda i, g, p: list(range(p + 1)))
+    assert torch.allclose(got, want, rtol=0, atol=1e-12), (got - want).abs().max()
+
+
+def pin_dsa_mask_equivalence(o, seed=15):
+    """With more visible tokens than top_k the attention equals
+    scaled_dot_product_attention under a boolean mask of the kept tokens, the
+    same set for every group."""
+    k, v, q, qs, qp = _dsa_attn_case(seed)
+    scores = torch.randn((3, 12), generator=torch.Generator().manual_seed(seed), dtype=F64)
+    top_k = 3
+    sel, n_sel = o.dsa_select_tokens(scores, qp, top_k, 4)
+    assert n_sel.tolist() == [3, 3, 3]
+    kept = [_bruteforce_tokens(scores[i], int(qp[i]), top_k) for i in range(3)]
+    got = o.dsa_sparse_attention(q, k, v, sel, qs, qp)
+    want = _sdpa_reference(q, k, v, qs, qp, lambda i, g, p: kept[i])
+    assert torch.allclose(got, want, rtol=0, atol=1e-12), (got - want).abs().max()
+
+
 ALL_PINS = [pin_golden, pin_basis_query_pooling, pin_scores_bilinear, pin_selection_bruteforce,
             pin_selection_invariants, pin_local_forced, pin_dense_equivalence,
             pin_block_mask_equivalence, pin_attention_closed_forms, pin_append_random,
-            pin_paged_identity_layout, pin_paged_permutation_and_sharing, pin_paged_append_commutes]
+            pin_paged_identity_layout, pin_paged_permutation_and_sharing, pin_paged_append_commutes,
+            pin_dsa_scores_identities, pin_dsa_selection_bruteforce, pin_dsa_noop_exact, pin_dsa_mask_equivalence]
 
 
 def run_all(o):

@@ -183,11 +183,58 @@ def _mut_paged_append_next_slot(o):
     o.paged_append = paged_append
 
 
+def _mut_dsa_no_relu(o):
+    orig = o.dsa_token_scores
+
+    def dsa_token_scores(q, w, k, qs, qp, relu=True):
+        return orig(q, w, k, qs, qp, False)
+    o.dsa_token_scores = dsa_token_scores
+
+
+def _mut_dsa_unweighted(o):
+    orig = o.dsa_token_scores
+
+    def dsa_token_scores(q, w, k, qs, qp, relu=True):
+        return orig(q, torch.ones_like(w), k, qs, qp, relu)
+    o.dsa_token_scores = dsa_token_scores
+
+
+def _mut_dsa_future_tokens(o):
+    orig = o.dsa_token_scores
+
+    def dsa_token_scores(q, w, k, qs, qp, relu=True):
+        full = torch.full_like(qp, k.shape[1] - 1)
+        return orig(q, w, k, qs, full, relu)
+    o.dsa_token_scores = dsa_token_scores
+
+
+def _mut_dsa_tie_higher_index(o):
+    def dsa_ranked_tokens(row, pos):
+        return sorted(range(pos + 1), key=lambda s: (-float(row[s]), -s))
+    o.dsa_ranked_tokens = dsa_ranked_tokens
+
+
+def _mut_dsa_k_minus_one(o):
+    orig = o.dsa_select_one
+
+    def dsa_select_one(row, pos, top_k):
+        return orig(row, pos, top_k)[:max(1, top_k - 1)] if pos + 1 > top_k else orig(row, pos, top_k)
+    o.dsa_select_one = dsa_select_one
+
+
+def _mut_dsa_group_zero(o):
+    def dsa_sparse_attention(q, k, v, sel, qs, qp, scale=None):
+        return orig(q, k[:, :1].expand_as(k), v[:, :1].expand_as(v), sel, qs, qp, scale)
+    orig = o.dsa_sparse_attention
+    o.dsa_sparse_attention = dsa_sparse_attention
+
+
 MUTATIONS = [_mut_causal_off_by_one, _mut_no_causal_mask, _mut_tie_higher_index, _mut_no_bias,
              _mut_gqa_modulo, _mut_no_scale, _mut_nvis_off_by_one, _mut_transposed_scores,
              _mut_dropped_term, _mut_future_rows, _mut_sign, _mut_k_minus_one,
              _mut_unsorted_ids, _mut_lowest_scores, _mut_append_swapped, _mut_paged_table_transposed,
-             _mut_paged_slots_reversed, _mut_paged_append_next_slot]
+             _mut_paged_slots_reversed, _mut_paged_append_next_slot, _mut_dsa_no_relu, _mut_dsa_unweighted,
+             _mut_dsa_future_tokens, _mut_dsa_tie_higher_index, _mut_dsa_k_minus_one, _mut_dsa_group_zero]
 
 
 @pytest.mark.parametrize("mut", MUTATIONS, ids=lambda f: f.__name__[5:])
