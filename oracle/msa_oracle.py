@@ -315,8 +315,12 @@ def dsa_token_scores(q_idx: torch.Tensor, weights: torch.Tensor, k_idx_cache: to
 
 
 def dsa_ranked_tokens(scores_row: torch.Tensor, pos: int) -> list[int]:
-    """Visible tokens ordered by (score descending, index ascending)."""
-    return sorted(range(pos + 1), key=lambda s: (-float(scores_row[s]), s))
+    """Visible tokens ordered by (score descending, index ascending); a NaN
+    score ranks as -inf (the variant's stated rule)."""
+    def rank_key(s):
+        v = float(scores_row[s])
+        return (math.inf if v != v else -v, s)
+    return sorted(range(pos + 1), key=rank_key)
 
 
 def dsa_select_one(scores_row: torch.Tensor, pos: int, top_k: int) -> list[int]:

@@ -465,6 +465,9 @@ def pin_dsa_selection_bruteforce(o, seed=13):
     assert sel.tolist() == [[0, 2, -1, -1]] and n_sel.tolist() == [2]
     assert o.dsa_boundary_scores(torch.tensor([3.0, 1.0, 3.0, 2.0], dtype=F64), 3, 2) == (3.0, 2.0)
     assert o.dsa_boundary_scores(torch.tensor([3.0, 1.0], dtype=F64), 1, 2) is None
+    # a NaN score ranks as -inf: below every finite score, ties with -inf by index
+    nan_row = torch.tensor([float("nan"), 0.5, float("-inf"), -3.0, float("nan")], dtype=F64)
+    assert o.dsa_ranked_tokens(nan_row, 4) == [1, 3, 0, 2, 4]
 
 
 def _dsa_attn_case(seed, cap=12, G=2, Hq=4, D=6):
