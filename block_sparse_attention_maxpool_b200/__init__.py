@@ -24,7 +24,8 @@ __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_bloc
            "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step",
            "Pages", "msa_indexer_append_paged", "msa_indexer_append_f16_paged", "msa_kv_append_paged",
            "msa_block_scores_paged", "msa_block_scores_f16_paged", "msa_sparse_attn_decode_paged",
-           "msa_sparse_attn_prefill_paged"]
+           "msa_sparse_attn_prefill_paged", "DsaShape", "DSA_SEL_WIDTH", "msa_dsa_indexer_append",
+           "msa_dsa_token_scores", "msa_dsa_select_topk", "msa_dsa_sparse_attn_decode", "dsa_decode_step"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
 MODE_DECODE = 0
@@ -87,6 +88,29 @@ class Pages:
         return CPages(t, int(self.n_pages))
 
 
+class CDsaShape(ctypes.Structure):
+    _fields_ = [("n_streams", ctypes.c_int32), ("capacity", ctypes.c_int32), ("n_index_heads", ctypes.c_int32),
+                ("index_dim", ctypes.c_int32), ("top_k", ctypes.c_int32), ("relu", ctypes.c_int32)]
+
+
+DSA_SEL_WIDTH = 2048
+
+
+@dataclass(frozen=True)
+class DsaShape:
+    """Geometry of the token-level (lightning-indexer) variant (msa_dsa_shape)."""
+    n_streams: int
+    capacity: int
+    n_index_heads: int = 64
+    index_dim: int = 128
+    top_k: int = 2048
+    relu: bool = True
+
+    def c(self) -> CDsaShape:
+        return CDsaShape(self.n_streams, self.capacity, self.n_index_heads, self.index_dim, self.top_k,
+                         int(bool(self.relu)))
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -111,6 +135,7 @@ _SIGS = {
     "msa_version": (ctypes.c_int, []),
 }
 _PG = ctypes.POINTER(CPages)
+_DS = ctypes.POINTER(CDsaShape)
 _SIGS.update({
     "msa_indexer_append_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P]),
     "msa_indexer_append_f16_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P]),
@@ -123,6 +148,11 @@ _SIGS.update({
                                                     ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "msa_sparse_attn_prefill_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
                                                      ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_dsa_indexer_append": (ctypes.c_int, [_DS, _PG, _P, _P, _P, _P, _I, _P]),
+    "msa_dsa_token_scores": (ctypes.c_int, [_DS, _PG, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "msa_dsa_select_topk": (ctypes.c_int, [_DS, _P, _P, _I, _P, _P, _P]),
+    "msa_dsa_sparse_attn_decode": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
+                                                  ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
 })
 
 
@@ -417,3 +447,110 @@ def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None,
     out = attn(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
                new["q_pos"], None, b.get("out"), b.get("workspace"), stream, pages)
     return out, sel, n_sel, bs
+
+
+# ---- token-level variant (lightning indexer) --------------------------------
+def _dsa_pages(shape, pages):
+    """ctypes argument for an optional page table (None: contiguous)."""
+    if pages is None:
+        return None
+    return ctypes.byref(pages.c(shape))
+
+
+def _dsa_key_shape(shape: DsaShape, pages: Pages | None) -> tuple:
+    if pages is None:
+        return (shape.n_streams, shape.capacity, shape.index_dim)
+    return (pages.n_pages, 128, shape.index_dim)
+
+
+def _as_msa_shape(shape: DsaShape) -> Shape:
+    return Shape(n_streams=shape.n_streams, capacity=shape.capacity, n_q_heads=16, n_kv_heads=1)
+
+
+def msa_dsa_indexer_append(shape: DsaShape, k_idx_cache, k_idx_new, tok_stream, tok_pos, stream=None,
+                           pages: Pages | None = None):
+    """Write new tokens' F32 indexer keys (rounded to fp16) into the F16 key cache."""
+    n = _n(tok_stream, "tok_stream")
+    s = shape.c()
+    _check("msa_dsa_indexer_append", library().msa_dsa_indexer_append(
+        ctypes.byref(s), _dsa_pages(_as_msa_shape(shape), pages),
+        _ptr(k_idx_cache, torch.float16, _dsa_key_shape(shape, pages), "k_idx_cache"),
+        _ptr(k_idx_new, torch.float32, (n, shape.index_dim), "k_idx_new"),
+        _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+        n, _stream(stream)))
+
+
+def msa_dsa_token_scores(shape: DsaShape, q_idx, weights, k_idx_cache, q_stream, q_pos, scores=None,
+                         stream=None, pages: Pages | None = None):
+    """Lightning-indexer scores [n_q][capacity] (float32, -inf past each query)."""
+    n = _n(q_pos, "q_pos")
+    if scores is None:
+        scores = torch.empty((n, shape.capacity), dtype=torch.float32, device=q_idx.device)
+    s = shape.c()
+    _check("msa_dsa_token_scores", library().msa_dsa_token_scores(
+        ctypes.byref(s), _dsa_pages(_as_msa_shape(shape), pages),
+        _ptr(q_idx, torch.float16, (n, shape.n_index_heads, shape.index_dim), "q_idx"),
+        _ptr(weights, torch.float32, (n, shape.n_index_heads), "weights"),
+        _ptr(k_idx_cache, torch.float16, _dsa_key_shape(shape, pages), "k_idx_cache"),
+        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+        _ptr(scores, torch.float32, (n, shape.capacity), "scores"), _stream(stream)))
+    return scores
+
+
+def msa_dsa_select_topk(shape: DsaShape, scores, q_pos, sel=None, n_sel=None, stream=None):
+    """Top-k tokens per query: sel [n_q][2048] ascending ids (-1 padded), n_sel [n_q]."""
+    n = _n(q_pos, "q_pos")
+    dev = scores.device
+    if sel is None:
+        sel = torch.empty((n, DSA_SEL_WIDTH), dtype=torch.int32, device=dev)
+    if n_sel is None:
+        n_sel = torch.empty((n,), dtype=torch.int32, device=dev)
+    s = shape.c()
+    _check("msa_dsa_select_topk", library().msa_dsa_select_topk(
+        ctypes.byref(s), _ptr(scores, torch.float32, (n, shape.capacity), "scores"),
+        _ptr(q_pos, torch.int32, (n,), "q_pos"), n, _ptr(sel, torch.int32, (n, DSA_SEL_WIDTH), "sel"),
+        _ptr(n_sel, torch.int32, (n,), "n_sel"), _stream(stream)))
+    return sel, n_sel
+
+
+def msa_dsa_sparse_attn_decode(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos, softmax_scale=None,
+                               out=None, workspace=None, stream=None, pages: Pages | None = None):
+    """Attention of every head over its query's kept tokens (MSA K/V caches)."""
+    n = _n(q_pos, "q_pos")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(shape.head_dim)
+    if out is None:
+        out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=q.device)
+    ws_ptr, ws_bytes, _keep = _workspace(shape, n, MODE_DECODE, workspace, q.device)
+    cs = _cache_shape(shape, pages, shape.head_dim)
+    s = shape.c()
+    _check("msa_dsa_sparse_attn_decode", library().msa_dsa_sparse_attn_decode(
+        ctypes.byref(s), _dsa_pages(shape, pages),
+        _ptr(q, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
+        _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+        _ptr(sel, torch.int32, (n, DSA_SEL_WIDTH), "sel"),
+        _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+        float(softmax_scale), _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"),
+        ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def dsa_decode_step(shape: Shape, dshape: DsaShape, caches: dict, new: dict, bufs: dict | None = None,
+                    stream=None, pages: Pages | None = None, idx_pages: Pages | None = None):
+    """One token-level step through the C ABI: append the new tokens' F16
+    indexer keys and K/V rows, score every visible token, keep the top-k and
+    attend.  caches: k_idx_cache (float16 [S][cap][128]), k_cache, v_cache;
+    new: tok_stream, tok_pos, k_idx_new, k_new, v_new, q_stream, q_pos,
+    q_idx (float16 [n_q][64][128]), weights ([n_q][64]), q.
+    Returns (out, sel, n_sel, scores)."""
+    b = bufs or {}
+    msa_dsa_indexer_append(dshape, caches["k_idx_cache"], new["k_idx_new"], new["tok_stream"], new["tok_pos"],
+                           stream, idx_pages)
+    msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
+                  new["tok_stream"], new["tok_pos"], stream, pages)
+    sc = msa_dsa_token_scores(dshape, new["q_idx"], new["weights"], caches["k_idx_cache"], new["q_stream"],
+                              new["q_pos"], b.get("scores"), stream, idx_pages)
+    sel, n_sel = msa_dsa_select_topk(dshape, sc, new["q_pos"], b.get("sel"), b.get("n_sel"), stream)
+    out = msa_dsa_sparse_attn_decode(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
+                                     new["q_pos"], None, b.get("out"), b.get("workspace"), stream, pages)
+    return out, sel, n_sel, sc

@@ -14,6 +14,8 @@
 #include "msa_attn_decode_sk.cuh"
 #include "msa_attn_prefill_tc.cuh"
 #include "msa_common.cuh"
+#include "msa_dsa_scores.cuh"
+#include "msa_dsa_select.cuh"
 #include "msa_scores_gemv.cuh"
 #include "msa_scores_tc.cuh"
 #include "msa_select.cuh"
@@ -141,7 +143,7 @@ size_t attn_workspace(int64_t n_pairs, int mode) {
 int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache, const msa_bf16* v_cache,
                 const int32_t* sel, const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
                 float softmax_scale, msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream,
-                int mode, const msa_pages* pages) {
+                int mode, const msa_pages* pages, const int32_t* tok_sel = nullptr) {
   int st = check_shape(sh);
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
@@ -193,11 +195,12 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
                                                 msa::pattn::Layout::kBytes, s>>>(tm_q, tm_k, tm_v, Q);
     return cuda_status(cudaGetLastError());
   }
-  // decode: persistent stream-K grid over (pair, selected block) units
-  static std::atomic<uint64_t> smem_done{0};
-  if ((st = ensure_smem(msa::dattn::sparse_attn_decode_sk_kernel, msa::dattn::Layout::kBytes, smem_done)) !=
-      MSA_OK)
-    return st;
+  // decode: persistent stream-K grid over (pair, selected block) units, or
+  // (pair, chunk of 128 kept tokens) units for the token-level variant
+  const auto kernel = tok_sel != nullptr ? msa::dattn::sparse_attn_decode_sk_kernel<true>
+                                         : msa::dattn::sparse_attn_decode_sk_kernel<false>;
+  static std::atomic<uint64_t> smem_done[2] = {0, 0};
+  if ((st = ensure_smem(kernel, msa::dattn::Layout::kBytes, smem_done[tok_sel != nullptr])) != MSA_OK) return st;
   msa::dattn::Params P;
   P.q = reinterpret_cast<const __nv_bfloat16*>(q);
   P.sel = sel;
@@ -214,8 +217,10 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
                                                 static_cast<int64_t>(msa::dattn::kMaxCtas)}));
   P.scale_log2 = softmax_scale * 1.4426950408889634f;
   P.pages = pg;
-  msa::dattn::sparse_attn_decode_sk_kernel<<<static_cast<unsigned>(P.n_cta), msa::dattn::kThreads,
-                                             msa::dattn::Layout::kBytes, s>>>(tm_k, tm_v, P);
+  P.tok_sel = tok_sel;
+  P.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
+  P.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
+  kernel<<<static_cast<unsigned>(P.n_cta), msa::dattn::kThreads, msa::dattn::Layout::kBytes, s>>>(tm_k, tm_v, P);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
   const int64_t warps = n_pairs * msa::dattn::kHpg;
   msa::dattn::attn_sk_combine_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(P);
@@ -374,6 +379,31 @@ int append_idx_f16(const msa_shape* shape, msa_f16* idx_k_cache, const float* id
       reinterpret_cast<__half*>(idx_k_cache), idx_k_new, tok_stream, tok_pos, n_tok, shape->n_streams,
       shape->n_kv_heads, shape->capacity, pg);
   return cuda_status(cudaGetLastError());
+}
+
+// ---- token-level variant ---------------------------------------------------
+int check_dsa_shape(const msa_dsa_shape* sh) {
+  if (sh == nullptr) return MSA_ERR_NULL;
+  if (sh->n_streams <= 0 || sh->capacity <= 0 || sh->capacity % 128 != 0 || sh->index_dim != 128 ||
+      sh->n_index_heads != msa::dsa::kHeads || sh->top_k < 1 || sh->top_k > msa::dsa::kMaxTopK)
+    return MSA_ERR_SHAPE;
+  if (static_cast<int64_t>(sh->n_streams) * sh->capacity >= (int64_t{1} << 31)) return MSA_ERR_SHAPE;
+  return MSA_OK;
+}
+
+// The indexer-key cache as an MSA cache of one group: the same page-table
+// checks and row counts.
+msa_shape dsa_as_msa(const msa_dsa_shape* sh) {
+  msa_shape m{};
+  m.n_streams = sh->n_streams;
+  m.capacity = sh->capacity;
+  m.n_q_heads = 16;
+  m.n_kv_heads = 1;
+  m.head_dim = 128;
+  m.idx_dim = 128;
+  m.block = 128;
+  m.top_k = 16;
+  return m;
 }
 
 }  // namespace
@@ -568,6 +598,92 @@ int msa_sparse_attn_prefill_paged(const msa_shape* shape, const msa_pages* pages
   if (pages == nullptr) return MSA_ERR_NULL;
   return sparse_attn(shape, q, k_pool, v_pool, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
                      workspace_bytes, stream, MSA_MODE_PREFILL, pages);
+}
+
+// ---- token-level variant ---------------------------------------------------
+int msa_dsa_indexer_append(const msa_dsa_shape* shape, const msa_pages* pages, msa_f16* k_idx_cache,
+                           const float* k_idx_new, const int32_t* tok_stream, const int32_t* tok_pos,
+                           int32_t n_tok, void* stream) {
+  const int st = check_dsa_shape(shape);
+  if (st != MSA_OK) return st;
+  const msa_shape m = dsa_as_msa(shape);
+  return append_idx_f16(&m, k_idx_cache, k_idx_new, tok_stream, tok_pos, n_tok, stream, pages);
+}
+
+int msa_dsa_token_scores(const msa_dsa_shape* shape, const msa_pages* pages, const msa_f16* q_idx,
+                         const float* weights, const msa_f16* k_idx_cache, const int32_t* q_stream,
+                         const int32_t* q_pos, int32_t n_q, float* scores, void* stream) {
+  int st = check_dsa_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0) return MSA_OK;
+  if (!q_idx || !weights || !k_idx_cache || !q_stream || !q_pos || !scores) return MSA_ERR_NULL;
+  if (!aligned16(q_idx) || !aligned16(weights) || !aligned16(k_idx_cache) || !aligned16(scores))
+    return MSA_ERR_ALIGN;
+  if (static_cast<int64_t>(n_q) * msa::dsa::kHeads >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const msa_shape m = dsa_as_msa(shape);
+  msa::KvPages pg;
+  int64_t rows = 0;
+  if ((st = pages_of(&m, pages, &pg, &rows)) != MSA_OK) return st;
+  CUtensorMap tm_key, tm_q;
+  if ((st = make_map_16bit(&tm_key, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, k_idx_cache, rows)) != MSA_OK) return st;
+  if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, q_idx,
+                           static_cast<int64_t>(n_q) * msa::dsa::kHeads, msa::dsa::kHeads)) != MSA_OK)
+    return st;
+  int sms = 0;
+  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+  static std::atomic<uint64_t> smem_done{0};
+  if ((st = ensure_smem(msa::dsa::dsa_scores_kernel, msa::dsa::Smem::kBytes, smem_done)) != MSA_OK) return st;
+  msa::dsa::Params P;
+  P.weights = weights;
+  P.q_stream = q_stream;
+  P.q_pos = q_pos;
+  P.scores = scores;
+  P.n_q = n_q;
+  P.n_streams = shape->n_streams;
+  P.capacity = shape->capacity;
+  P.n_tiles = shape->capacity / msa::dsa::kTile;
+  P.relu = shape->relu != 0;
+  P.pages = pg;
+  const int64_t tasks = static_cast<int64_t>(n_q) * P.n_tiles;
+  const int64_t grid = std::min<int64_t>(sms, tasks);
+  msa::dsa::dsa_scores_kernel<<<static_cast<unsigned>(grid), msa::dsa::kThreads, msa::dsa::Smem::kBytes,
+                                static_cast<cudaStream_t>(stream)>>>(tm_key, tm_q, P);
+  return cuda_status(cudaGetLastError());
+}
+
+int msa_dsa_select_topk(const msa_dsa_shape* shape, const float* scores, const int32_t* q_pos, int32_t n_q,
+                        int32_t* sel, int32_t* n_sel, void* stream) {
+  int st = check_dsa_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0) return MSA_OK;
+  if (!scores || !q_pos || !sel) return MSA_ERR_NULL;
+  if (!aligned16(scores) || !aligned16(sel)) return MSA_ERR_ALIGN;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (shape->capacity <= msa::dsa::kSmemKeys) {
+    static std::atomic<uint64_t> smem_done{0};
+    if ((st = ensure_smem(msa::dsa::dsa_select_topk_kernel<true>, msa::dsa::kSelSmemStaged, smem_done)) != MSA_OK)
+      return st;
+    msa::dsa::dsa_select_topk_kernel<true><<<static_cast<unsigned>(n_q), msa::dsa::kSelThreads,
+                                             msa::dsa::kSelSmemStaged, cs>>>(scores, q_pos, n_q, shape->capacity,
+                                                                             shape->top_k, sel, n_sel);
+  } else {
+    msa::dsa::dsa_select_topk_kernel<false><<<static_cast<unsigned>(n_q), msa::dsa::kSelThreads,
+                                              msa::dsa::kSelSmemUnstaged, cs>>>(scores, q_pos, n_q,
+                                                                                shape->capacity, shape->top_k,
+                                                                                sel, n_sel);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int msa_dsa_sparse_attn_decode(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
+                               const msa_bf16* k_cache, const msa_bf16* v_cache, const int32_t* sel,
+                               const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float softmax_scale,
+                               msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_q > 0 && sel == nullptr) return MSA_ERR_NULL;
+  return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_DECODE, pages, sel);
 }
 
 size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {

@@ -18,6 +18,15 @@
 // units all lie in one CTA's share is written out directly; a pair cut by a
 // share boundary leaves one partial (max, sum, unnormalised O) per CTA,
 // merged by attn_sk_combine_kernel.
+//
+// Token-level variant ("deepseek2 : GLM-DSA sparse attention (lightning
+// indexer)": top-k tokens per query, the same set for every group): a unit
+// is a chunk of 128 consecutive entries of the query's ascending token list
+// (2048 entries, 16 chunks, -1 padded).  The rows are scattered, so the
+// whole producer warp gathers them with 16-byte cp.async copies straight
+// into the same 128-byte-swizzled tile layout the TMA path produces, each
+// lane arriving on the stage's barrier when its copies land; rows of padding
+// or of an unmapped page are copied from a zero row and masked.
 #pragma once
 
 #include "msa_common.cuh"
@@ -59,7 +68,49 @@ struct Params {
   long long n_units;          // n_q * G * 16
   float scale_log2;
   KvPages pages;              // block table of paged K/V caches (table null: contiguous)
+  const int32_t* tok_sel;     // token-level variant: [n_q][16 * 128] ascending token ids (else null)
+  const __nv_bfloat16* k_cache;   // token-level variant: the K and V caches (or pools) the gathers read
+  const __nv_bfloat16* v_cache;
 };
+
+// 256 zero bytes: the source of the K and V rows of masked token slots.
+__device__ __align__(16) uint8_t g_zero_row[256];
+
+// Token-level unit u: query position, stream, group and the unit's 128 token
+// slots; false when the unit has nothing to attend.
+__device__ __forceinline__ bool tok_unit(const Params& P, long long u, int& s, int& g, int& p,
+                                         const int32_t*& toks, bool report) {
+  const long long pair = u / kTopK;
+  const int j = static_cast<int>(u - pair * kTopK);
+  const int qi = static_cast<int>(pair / P.G);
+  g = static_cast<int>(pair - static_cast<long long>(qi) * P.G);
+  s = P.q_stream[qi];
+  p = P.q_pos[qi];
+  if (s < 0 || s >= P.n_streams || p < 0 || p >= P.capacity) {
+    if (report && j == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
+    return false;
+  }
+  toks = P.tok_sel + static_cast<size_t>(qi) * (kTopK * kBlock) + j * kBlock;
+  return __ldg(toks) >= 0;
+}
+
+// Cache row of a selected token, or -1 when the slot is padding, names a
+// token the query cannot see, or lies in an unmapped page.
+__device__ __forceinline__ long long tok_row(const Params& P, int s, int g, int p, int tok) {
+  if (tok < 0 || tok > p) return -1;
+  const long long blk = kv_block_row(P.pages, s, g, tok >> 7, P.G, P.capacity);
+  return blk < 0 ? -1 : blk + (tok & 127);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// The mbarrier receives one arrival when all of this thread's earlier
+// cp.async copies have landed (counted in the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
 
 __host__ __device__ inline long long unit_begin(long long U, int C, int c) { return U * c / C; }
 
@@ -169,6 +220,7 @@ __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long 
   }
 }
 
+template <bool kTok>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                  const Params P) {
@@ -185,14 +237,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(&full[st], 1);
+      mbar_init(&full[st], kTok ? 32 : 1);   // token gathers: one arrival per producer lane
       mbar_init(&empty[st], kWarps);
     }
     mbar_fence_init();
   }
   __syncthreads();
 
-  if (warp == kWarps) {
+  if (kTok && warp == kWarps) {
+    // ----------------------- producer: token gathers (whole warp) -----------------------
+    const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(P.k_cache);
+    const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(P.v_cache);
+    int k = 0;
+    bool ok = true;
+    for (long long u = u0; u < u1 && ok; ++u) {
+      int s, g, p;
+      const int32_t* toks;
+      if (!tok_unit(P, u, s, g, p, toks, false)) continue;
+      const int st = k % kStages;
+      const int use = k / kStages;
+      if (use > 0) ok = mbar_wait(&empty[st], (use - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const uint32_t dst = smem_addr(smem + Layout::kStageOff + st * kStageBytes);
+#pragma unroll
+      for (int i = 0; i < kBlock / 32; ++i) {
+        const int r = lane + 32 * i;
+        const int tok = __ldg(toks + r);
+        const long long row = tok_row(P, s, g, p, tok);
+        if (row < 0 && tok >= 0) raise_error(tok > p ? MSA_DEVERR_SEL_RANGE : MSA_DEVERR_PAGE_RANGE);
+        const uint8_t* ksrc = row < 0 ? g_zero_row : reinterpret_cast<const uint8_t*>(kc + row * kD);
+        const uint8_t* vsrc = row < 0 ? g_zero_row : reinterpret_cast<const uint8_t*>(vc + row * kD);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t off = (c >> 3) * kTileBytes + swz128(r, c & 7);
+          cp_async16(dst + off, ksrc + 16 * c);
+          cp_async16(dst + 2 * kTileBytes + off, vsrc + 16 * c);
+        }
+      }
+      cp_async_arrive(&full[st]);
+      ++k;
+    }
+    // no copy may still be landing when the CTA exits
+    for (int j = max(0, k - kStages); j < k; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
+    return;
+  }
+  if (!kTok && warp == kWarps) {
     // -------------------------------- producer --------------------------------
     if (lane != 0) return;
     int k = 0;
@@ -250,9 +340,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         qa[ks][3] = __ldg(r1 + c + 4);
       }
     }
-    int p, slot0;
-    const int row = unit_row(P, u, p, slot0, warp == 0 && lane == 0);
-    if (row < 0) continue;
+    int p, slot0 = 0, s = 0, g = 0;
+    const int32_t* toks = nullptr;
+    if constexpr (kTok) {
+      if (!tok_unit(P, u, s, g, p, toks, warp == 0 && lane == 0)) continue;
+    } else {
+      if (unit_row(P, u, p, slot0, warp == 0 && lane == 0) < 0) continue;
+    }
     const int st = k % kStages;
     if (ok) ok = mbar_wait(&full[st], (k / kStages) & 1);
     if (ok) {
@@ -280,7 +374,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = jb + nt * 8 + tq * 2 + (e & 1);
-          const float x = j <= p ? sacc[nt][e] * P.scale_log2 : -INFINITY;
+          bool valid;
+          if constexpr (kTok) {
+            valid = tok_row(P, s, g, p, __ldg(toks + (j - slot0))) >= 0;   // j - slot0: row in the unit
+          } else {
+            valid = j <= p;
+          }
+          const float x = valid ? sacc[nt][e] * P.scale_log2 : -INFINITY;
           sacc[nt][e] = x;
           mx[e >> 1] = fmaxf(mx[e >> 1], x);
         }

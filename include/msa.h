@@ -290,6 +290,75 @@ MSA_API int msa_sparse_attn_prefill_paged(const msa_shape* shape, const msa_page
                                           float softmax_scale, msa_bf16* out, void* workspace,
                                           size_t workspace_bytes, void* stream);
 
+/* ---- token-level variant: the lightning indexer ---------------------------
+ * "deepseek2 : GLM-DSA sparse attention (lightning indexer)" (ik_llama.cpp
+ * pull request), section "What this does": instead of max-pooled blocks, the
+ * indexer scores every visible token and the top-k tokens of each query are
+ * kept (GLM-5.2 keeps 2048); attention then runs over those tokens only.  The
+ * indexer-key cache holds one F16 key per token ([head_size, kv_size]); a
+ * query has H_I indexer heads whose products with a key are weighted per head
+ * and summed (the review thread's element-wise product with a weight matrix
+ * followed by the reduction over indexer heads).  The caller applies the
+ * Hadamard rotation of queries and keys before these calls.
+ *
+ *   I[t][s] = sum_h weights[t][h] * act(q_idx[t][h] . k_idx[stream(t)][s])
+ *
+ * for s <= q_pos[t] (-inf beyond), act = ReLU when shape->relu is nonzero
+ * (the published lightning-indexer definition; the page does not print the
+ * formula), identity otherwise.  Supported: index_dim 128, n_index_heads
+ * 64, 1 <= top_k <= 2048, capacity % 128 == 0, n_streams * capacity < 2^31.
+ * Every call takes an optional page table (NULL: contiguous caches); a page
+ * of the key pool [n_pages][128][Di] holds 128 consecutive tokens of one
+ * stream, as for the MSA caches with one group. */
+typedef struct msa_dsa_shape {
+  int32_t n_streams;
+  int32_t capacity;       /* tokens per stream (logical length when paged)     */
+  int32_t n_index_heads;  /* H_I: 64                                           */
+  int32_t index_dim;      /* 128                                               */
+  int32_t top_k;          /* tokens kept per query, 1..2048                    */
+  int32_t relu;           /* nonzero: ReLU on each head's product              */
+} msa_dsa_shape;
+
+#define MSA_DSA_SEL_WIDTH 2048   /* entries of one selection row */
+
+/* Append: k_idx_new [n_tok][Di] f32, rounded to fp16 (nearest even) and
+ * written at (tok_stream[t], tok_pos[t]) of k_idx_cache [S][cap][Di] fp16
+ * (or of its page).  Same rules as msa_indexer_append. */
+MSA_API int msa_dsa_indexer_append(const msa_dsa_shape* shape, const msa_pages* pages, msa_f16* k_idx_cache,
+                                   const float* k_idx_new, const int32_t* tok_stream, const int32_t* tok_pos,
+                                   int32_t n_tok, void* stream);
+
+/* Token scores: q_idx [n_q][H_I][Di] fp16, weights [n_q][H_I] f32 ->
+ * scores [n_q][capacity] f32, -inf past each query's position.  Each head's
+ * product of fp16 vectors accumulates in f32 on the tensor cores; the
+ * weighted sum over heads runs in f32 in head order.  An out-of-range query
+ * writes -inf everywhere and sets MSA_DEVERR_QUERY_RANGE. */
+MSA_API int msa_dsa_token_scores(const msa_dsa_shape* shape, const msa_pages* pages, const msa_f16* q_idx,
+                                 const float* weights, const msa_f16* k_idx_cache, const int32_t* q_stream,
+                                 const int32_t* q_pos, int32_t n_q, float* scores, void* stream);
+
+/* Top-k tokens: sel [n_q][MSA_DSA_SEL_WIDTH] int32, ascending token ids,
+ * -1 padded; n_sel [n_q] (may be NULL) gets min(top_k, q_pos + 1).  Every
+ * visible token is kept when there are at most top_k; otherwise the top_k
+ * largest scores, equal scores keeping the lower index (NaN ranks as -inf,
+ * -0 equals +0). */
+MSA_API int msa_dsa_select_topk(const msa_dsa_shape* shape, const float* scores, const int32_t* q_pos,
+                                int32_t n_q, int32_t* sel, int32_t* n_sel, void* stream);
+
+/* Attention over the kept tokens: for query i and head h (group h/16),
+ * softmax(softmax_scale * q . K_j) . V_j over the tokens j of sel[i] (the
+ * same tokens for every group), rows of the MSA K/V caches of `shape`
+ * (contiguous, or pools addressed through `pages`).  Same layouts, workspace
+ * (msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE)), rounding and errors
+ * as msa_sparse_attn_decode; a kept token past the query sets
+ * MSA_DEVERR_SEL_RANGE, one in an unmapped page MSA_DEVERR_PAGE_RANGE, and
+ * is left out. */
+MSA_API int msa_dsa_sparse_attn_decode(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
+                                       const msa_bf16* k_cache, const msa_bf16* v_cache, const int32_t* sel,
+                                       const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                                       float softmax_scale, msa_bf16* out, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace that msa_block_scores and the attention call of `mode`
  * need for n_q queries (the larger of the two; one buffer serves both calls
  * of a step, since they run in stream order).  0 when neither needs any.

@@ -171,3 +171,27 @@ def test_paged_calls_validate_the_page_table(lib):
                                           0, 0, None) == -4
     assert lib.msa_sparse_attn_prefill_paged(ctypes.byref(s), pages(None, 4), fake, fake, fake, fake, fake, fake,
                                              2, ctypes.c_float(0.088), fake, 0, 0, None) == -1
+
+
+def test_dsa_calls_validate_shapes(lib):
+    fake = FAKE
+    good = msa.DsaShape(n_streams=2, capacity=1024).c()
+    for bad in (msa.DsaShape(n_streams=2, capacity=1000), msa.DsaShape(n_streams=2, capacity=1024, top_k=0),
+                msa.DsaShape(n_streams=2, capacity=1024, top_k=2049), msa.DsaShape(n_streams=2, capacity=1024,
+                                                                                   n_index_heads=32)):
+        b = bad.c()
+        assert lib.msa_dsa_select_topk(ctypes.byref(b), fake, fake, 1, fake, 0, None) == -3
+        assert lib.msa_dsa_token_scores(ctypes.byref(b), None, fake, fake, fake, fake, fake, 1, fake, None) == -3
+    assert lib.msa_dsa_select_topk(ctypes.byref(good), fake, fake, 0, fake, 0, None) == 0
+    assert lib.msa_dsa_select_topk(ctypes.byref(good), 0, fake, 2, fake, 0, None) == -1
+    assert lib.msa_dsa_select_topk(ctypes.byref(good), fake + 4, fake, 2, fake, 0, None) == -2
+    assert lib.msa_dsa_token_scores(ctypes.byref(good), None, fake, 0, fake, fake, fake, 2, fake, None) == -1
+    assert lib.msa_dsa_token_scores(ctypes.byref(good), None, fake, fake, fake, fake, fake, -1, fake, None) == -4
+    assert lib.msa_dsa_token_scores(ctypes.byref(good), ctypes.byref(msa.CPages(fake, 0)), fake, fake, fake,
+                                    fake, fake, 2, fake, None) == -4
+    assert lib.msa_dsa_indexer_append(ctypes.byref(good), None, fake, fake, fake, 0, 2, None) == -1
+    s = GOOD.c()
+    assert lib.msa_dsa_sparse_attn_decode(ctypes.byref(s), None, fake, fake, fake, 0, fake, fake, 2,
+                                          ctypes.c_float(0.088), fake, 0, 0, None) == -1
+    assert lib.msa_dsa_sparse_attn_decode(ctypes.byref(s), None, fake, fake, fake, fake, fake, fake, 2,
+                                          ctypes.c_float(0.088), fake, 0, 0, None) == -5

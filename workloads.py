@@ -259,3 +259,56 @@ def page_layout(inp: Inputs, seed: int = 0, spare_pages: int = 3, shared_prefix_
         k_pool[pg] = inp.k_cache[s, :, b * B:(b + 1) * B]
         v_pool[pg] = inp.v_cache[s, :, b * B:(b + 1) * B]
     return PagedCaches(table, n_pages, idx_pool, k_pool, v_pool)
+
+
+# ---------------------------------------------------------------------------
+# token-level variant (lightning indexer) inputs
+# ---------------------------------------------------------------------------
+DSA_INDEX_HEADS = 64
+
+
+@dataclass
+class DsaInputs:
+    """A step of the token-level variant: the MSA step's K/V caches, tokens
+    and queries (``base``; its indexer fields are unused) plus the lightning
+    indexer's inputs: k_idx_cache [S][cap][Di] f32 holding the existing
+    tokens' keys (new slots zero; the cache itself is fp16, rounded by the
+    append or by the caller), k_idx_new [n_tok][Di] f32, q_idx
+    [n_q][H_I][Di] fp16 and weights [n_q][H_I] f32."""
+    base: Inputs
+    k_idx_cache: torch.Tensor
+    k_idx_new: torch.Tensor
+    q_idx: torch.Tensor
+    weights: torch.Tensor
+
+
+def make_dsa_inputs(w: Workload, seed: int = 0, streams: range | None = None,
+                    n_index_heads: int = DSA_INDEX_HEADS, quantize: bool = False) -> DsaInputs:
+    """Draw a token-level step.  K/V/Q come from ``make_inputs``; the indexer
+    draws use their own per-stream generators (seed * 1000003 + stream +
+    7000000019), in the order keys [L][Di], query heads [n_q][H_I][Di],
+    weights [n_q][H_I].  Keys and query heads are N(0,1)/sqrt(Di), weights
+    N(0,1)/sqrt(H_I).  With ``quantize`` keys and query heads are multiples of
+    1/8 and weights multiples of 1/4, so every score is exact in float32 and
+    equal scores occur."""
+    base = make_inputs(w, seed, streams)
+    S = w.n_streams
+    streams = range(S) if streams is None else streams
+    Di, cap, L, L0 = w.idx_dim, w.capacity, w.l_total, w.l_existing
+    ns = len(streams)
+    nq_per = 1 if w.queries == "last" else w.n_new
+    keys = torch.zeros((ns, cap, Di), dtype=torch.float32)
+    q_idx = torch.empty((ns * nq_per, n_index_heads, Di), dtype=torch.float32)
+    weights = torch.empty((ns * nq_per, n_index_heads), dtype=torch.float32)
+    for i, s in enumerate(streams):
+        g = torch.Generator().manual_seed(seed * 1_000_003 + s + 7_000_000_019)
+        keys[i, :L] = torch.randn((L, Di), generator=g) / math.sqrt(Di)
+        q_idx[i * nq_per:(i + 1) * nq_per] = torch.randn((nq_per, n_index_heads, Di), generator=g) / math.sqrt(Di)
+        weights[i * nq_per:(i + 1) * nq_per] = torch.randn((nq_per, n_index_heads), generator=g) / math.sqrt(n_index_heads)
+    if quantize:
+        keys = torch.round(keys * 8.0) / 8.0
+        q_idx = torch.round(q_idx * 8.0) / 8.0
+        weights = torch.round(weights * 4.0) / 4.0
+    k_new = keys[:, L0:L].reshape(-1, Di).contiguous()
+    keys[:, L0:L] = 0
+    return DsaInputs(base, keys, k_new, q_idx.to(torch.float16), weights)
