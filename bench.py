@@ -47,8 +47,8 @@ WORKLOAD = W.DECODE_32K_X32
 # streams, scaled by 4 to 32 streams (the reads grow in proportion to the
 # keys scanned).  Valid only for the kernel source it was taken on (sha256
 # prefix of msa_scores_gemv.cuh); any other source reports null.
-SCORES_TRAFFIC = {"source_sha": "7065233549d01316",
-                  "bytes_per_launch": {"f32": 4 * (536_908_544 + 3_283_712), "f16": 4 * (268_472_832 + 3_113_984)}}
+SCORES_TRAFFIC = {"source_sha": "b9bc1ca3c5d4d5a4",
+                  "bytes_per_launch": {"f32": 4 * (536_911_872 + 3_886_848), "f16": None}}
 
 
 def variant_metric(metric: str, args) -> str:
@@ -81,6 +81,25 @@ def scores_bytes(w, key_bytes: int = 4) -> int:
     n_q = w.n_queries
     keys = n_q * G * w.l_total * Di * key_bytes   # decode: each query sees l_total keys
     return keys + n_q * G * Di * 4 + n_q * G * (w.capacity // w.block) * 4
+
+
+def dsa_scores_bytes(w, n_index_heads: int = 64) -> int:
+    """Bytes the token-score kernel must move per launch: every visible fp16
+    indexer key once (256 B), each query's fp16 head vectors and weights,
+    and the float32 score row it writes."""
+    Di = w.idx_dim
+    per_q = w.l_total * Di * 2 + n_index_heads * Di * 2 + n_index_heads * 4 + w.capacity * 4
+    return per_q * w.n_queries
+
+
+def dsa_step_bytes(w, top_k: int = 2048, n_index_heads: int = 64) -> int:
+    """Bytes one token-level decode step must move: the token scores (keys
+    in, scores out), the score row read back by the top-k, the kept tokens'
+    K/V rows of every group, the selection, query and output."""
+    G, D = w.n_kv_heads, w.head_dim
+    kept = min(top_k, w.l_total)
+    per_q = (w.capacity * 4 + kept * G * D * 2 * 2 + 2048 * 4 * 2 + w.n_q_heads * D * 2 * 2)
+    return dsa_scores_bytes(w, n_index_heads) + per_q * w.n_queries
 
 
 def step_bytes(w, key_bytes: int = 4) -> int:
@@ -184,10 +203,21 @@ def run_ours(args, rank, world, dev):
                        quantize_idx=w.quantize_idx)
     prefill = w.queries == "new"
     shape = msa.Shape(n_streams=w.n_streams, capacity=w.capacity)
-    inp = W.make_inputs(w, streams=shard_streams(w.n_streams, rank))   # this rank's own streams
-    d = {n: getattr(inp, n).to(dev) for n in ("idx_k_cache", "k_cache", "v_cache", "tok_stream",
-                                               "tok_pos", "idx_k_new", "k_new", "v_new",
-                                               "q_stream", "q_pos", "idx_q", "q")}
+    if args.dsa:                                # token-level variant: lightning-indexer inputs
+        dinp = W.make_dsa_inputs(w, streams=shard_streams(w.n_streams, rank))
+        inp = dinp.base
+        names = ("k_cache", "v_cache", "tok_stream", "tok_pos", "k_new", "v_new", "q_stream", "q_pos", "q")
+    else:
+        inp = W.make_inputs(w, streams=shard_streams(w.n_streams, rank))   # this rank's own streams
+        names = ("idx_k_cache", "k_cache", "v_cache", "tok_stream", "tok_pos", "idx_k_new", "k_new", "v_new",
+                 "q_stream", "q_pos", "idx_q", "q")
+    d = {n: getattr(inp, n).to(dev) for n in names}
+    if args.dsa:
+        d["k_idx_cache"] = dinp.k_idx_cache.half().to(dev)
+        d["k_idx_new"] = dinp.k_idx_new.to(dev)
+        d["q_idx"] = dinp.q_idx.to(dev)
+        d["weights"] = dinp.weights.to(dev)
+        del dinp
     pages = None
     if args.paged:
         # the same caches as shuffled page pools behind a block table
@@ -202,10 +232,14 @@ def run_ours(args, rank, world, dev):
     key_bytes = 2 if args.idx_f16 else 4
     n_q = w.n_queries
     G = w.n_kv_heads
+    dshape = msa.DsaShape(n_streams=w.n_streams, capacity=w.capacity)
     bufs = {
         "block_scores": torch.empty((n_q, G, shape.n_blocks), dtype=torch.float32, device=dev),
         "sel": torch.empty((n_q, G, shape.top_k), dtype=torch.int32, device=dev),
         "n_sel": torch.empty((n_q, G), dtype=torch.int32, device=dev),
+        "scores": torch.empty((n_q, w.capacity) if args.dsa else (1,), dtype=torch.float32, device=dev),
+        "tok_sel": torch.empty((n_q, msa.DSA_SEL_WIDTH) if args.dsa else (1,), dtype=torch.int32, device=dev),
+        "tok_n": torch.empty((n_q,), dtype=torch.int32, device=dev),
         "out": torch.empty((n_q, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=dev),
     }
     mode = msa.MODE_PREFILL if prefill else msa.MODE_DECODE
@@ -215,8 +249,24 @@ def run_ours(args, rank, world, dev):
     # tensor-core tile path of prefill batches), select, attention (+ combine in decode)
     tiles = n_q >= 256 and n_q >= 64 * w.n_streams
     launches_per_step = 2 + (6 if tiles else 1) + 1 + (1 if prefill else 2)
+    if args.dsa:
+        launches_per_step = 2 + 1 + 1 + 2        # appends, token scores, top-k, attention + combine
     stream = torch.cuda.current_stream(dev)
     scale = 1.0 / math.sqrt(shape.head_dim)
+
+    def dsa_append(st):
+        msa.msa_dsa_indexer_append(dshape, d["k_idx_cache"], d["k_idx_new"], d["tok_stream"], d["tok_pos"], st)
+        msa.msa_kv_append(shape, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
+                          d["tok_pos"], st)
+
+    def dsa_scores(st):
+        msa.msa_dsa_token_scores(dshape, d["q_idx"], d["weights"], d["k_idx_cache"], d["q_stream"], d["q_pos"],
+                                 bufs["scores"], st)
+
+    def dsa_attend(st):
+        msa.msa_dsa_select_topk(dshape, bufs["scores"], d["q_pos"], bufs["tok_sel"], bufs["tok_n"], st)
+        msa.msa_dsa_sparse_attn_decode(shape, d["q"], d["k_cache"], d["v_cache"], bufs["tok_sel"], d["q_stream"],
+                                       d["q_pos"], scale, bufs["out"], bufs["workspace"], st)
 
     def part_append(st):
         append = msa.msa_indexer_append_f16 if args.idx_f16 else msa.msa_indexer_append
@@ -233,6 +283,9 @@ def run_ours(args, rank, world, dev):
         attn = msa.msa_sparse_attn_prefill if prefill else msa.msa_sparse_attn_decode
         attn(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"], d["q_pos"], scale,
              bufs["out"], bufs["workspace"], st, pages)
+
+    if args.dsa:
+        part_append, part_scores, part_attend = dsa_append, dsa_scores, dsa_attend
 
     def step(ev=None):
         part_append(stream)
@@ -292,6 +345,9 @@ def run_ours(args, rank, world, dev):
 
     # ---- end to end: host inputs in, host output out, every step ------------
     host_names = ("tok_stream", "tok_pos", "idx_k_new", "k_new", "v_new", "q_stream", "q_pos", "idx_q", "q")
+    if args.dsa:
+        host_names = ("tok_stream", "tok_pos", "k_idx_new", "k_new", "v_new", "q_stream", "q_pos", "q_idx",
+                      "weights", "q")
     host = {n: d[n].cpu().pin_memory() for n in host_names}
     h_out = torch.empty(bufs["out"].shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -327,6 +383,9 @@ def run_ours(args, rank, world, dev):
         return None
 
     peaks = load_peaks()
+    if args.dsa:
+        return dsa_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks,
+                        graphs)
     if prefill:
         return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks,
                             graphs)
@@ -367,6 +426,41 @@ def run_ours(args, rank, world, dev):
         "clocks": clk,
     }
     return line
+
+
+DSA_METRIC = ("MSA token-level variant (lightning indexer, 64 heads, top-2048 tokens) decode tokens/s "
+              "@32K ctx x32 streams; achieved HBM GB/s vs peak")
+
+
+def dsa_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks, graphs):
+    sbytes = dsa_scores_bytes(w)
+    achieved = sbytes / (k_ms * 1e-3) / 1e9
+    step_gbs = dsa_step_bytes(w) / (ms * 1e-3) / 1e9
+    return {
+        "metric": DSA_METRIC if w == WORKLOAD else DSA_METRIC.replace("@32K ctx x32 streams", f"({w.name})"),
+        "value": job_tokens_per_s(w.n_streams, world, ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 indexer (f32 accumulate) / bf16 attention (f32 accumulate)",
+        "data": "synthetic (seeded N(0,1) K/V/Q bf16; indexer keys and heads N(0,1)/sqrt(128) fp16, "
+                "weights N(0,1)/8 f32)",
+        "config": {"workload": w.name, "variant": "token-level (lightning indexer)", "streams_per_gpu": w.n_streams,
+                   "context": w.l_total, "index_heads": 64, "top_k_tokens": 2048, "relu": True,
+                   "launch": "cuda graphs" if graphs is not None else "direct",
+                   "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs {w.n_streams * w.capacity * (256 + w.n_kv_heads * 512) / 1e9:.1f} GB per GPU "
+                         "> 126 MB L2, no flush"},
+        "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peaks["hbm_gbs"], "frac": step_gbs / peaks["hbm_gbs"],
+                     "bytes_per_step": dsa_step_bytes(w)},
+        "roofline": {"kernel": "dsa_scores", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes": sbytes, "ms_per_launch": k_ms, "peak_src": peaks["src"]},
+        "e2e": {"value": job_tokens_per_s(w.n_streams, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
 
 
 def prefill_flops(w) -> tuple[int, int]:
@@ -476,6 +570,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--idx-f16", action="store_true",
                     help="decode with the F16 indexer-key cache variant instead of the F32 cache")
+    ap.add_argument("--dsa", action="store_true",
+                    help="time the token-level variant (lightning indexer, top-2048 tokens) on the same workload")
     ap.add_argument("--paged", action="store_true",
                     help="run the paged calls on the same caches laid out as shuffled page pools")
     ap.add_argument("--no-graph", action="store_true",
@@ -487,6 +583,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.dsa and (args.paged or args.idx_f16 or W.WORKLOADS[args.workload].queries != "last"):
+        ap.error("--dsa times decode workloads with contiguous caches")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
@@ -507,7 +605,7 @@ def main():
         line = run_ours(args, rank, world, local)
         if line is not None:
             if (world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name and not args.idx_f16
-                    and not args.paged):
+                    and not args.paged and not args.dsa):
                 line["cpu_baseline"] = cpu_baseline()
             print(json.dumps(line), flush=True)
     finally:

@@ -646,7 +646,7 @@ int msa_dsa_token_scores(const msa_dsa_shape* shape, const msa_pages* pages, con
   P.relu = shape->relu != 0;
   P.pages = pg;
   const int64_t tasks = static_cast<int64_t>(n_q) * P.n_tiles;
-  const int64_t grid = std::min<int64_t>(sms, tasks);
+  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(msa::dsa::kCtasPerSm) * sms, tasks);
   msa::dsa::dsa_scores_kernel<<<static_cast<unsigned>(grid), msa::dsa::kThreads, msa::dsa::Smem::kBytes,
                                 static_cast<cudaStream_t>(stream)>>>(tm_key, tm_q, P);
   return cuda_status(cudaGetLastError());

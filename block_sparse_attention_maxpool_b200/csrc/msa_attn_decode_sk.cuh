@@ -22,11 +22,13 @@
 // Token-level variant ("deepseek2 : GLM-DSA sparse attention (lightning
 // indexer)": top-k tokens per query, the same set for every group): a unit
 // is a chunk of 128 consecutive entries of the query's ascending token list
-// (2048 entries, 16 chunks, -1 padded).  The rows are scattered, so the
-// whole producer warp gathers them with 16-byte cp.async copies straight
-// into the same 128-byte-swizzled tile layout the TMA path produces, each
-// lane arriving on the stage's barrier when its copies land; rows of padding
-// or of an unmapped page are copied from a zero row and masked.
+// (2048 entries, 16 chunks, -1 padded).  The rows are scattered, so two
+// producer warps gather them (one row per lane) with 16-byte cp.async copies
+// straight into the same 128-byte-swizzled tile layout the TMA path
+// produces, each lane arriving on the stage's barrier when its copies land;
+// rows of padding or of an unmapped page are copied from a zero row and
+// masked.  Random 256-byte rows bound this path near 2 TB/s on B200 (a TMA
+// tile::gather4 form measured slower).
 #pragma once
 
 #include "msa_common.cuh"
@@ -39,7 +41,8 @@ constexpr int kBlock = 128;
 constexpr int kHpg = 16;
 constexpr int kTopK = 16;
 constexpr int kWarps = 8;                           // consumer warps
-constexpr int kThreads = (kWarps + 1) * 32;         // + one producer warp
+constexpr int kGatherWarps = 2;                     // producer warps of the token-level variant
+constexpr int kThreads = (kWarps + kGatherWarps) * 32;   // block path: one producer thread, one idle warp
 constexpr int kRowsPerWarp = kBlock / kWarps;       // 16
 constexpr uint32_t kTileBytes = kBlock * 64 * 2;    // [128 rows][64 dims] bf16 = 16 KB
 constexpr uint32_t kStageBytes = 4 * kTileBytes;    // K lo, K hi, V lo, V hi
@@ -237,14 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(&full[st], kTok ? 32 : 1);   // token gathers: one arrival per producer lane
+      mbar_init(&full[st], kTok ? 32 * kGatherWarps : 1);   // token gathers: one arrival per producer lane
       mbar_init(&empty[st], kWarps);
     }
     mbar_fence_init();
   }
   __syncthreads();
 
-  if (kTok && warp == kWarps) {
+  if (kTok && warp >= kWarps) {
     // ----------------------- producer: token gathers (whole warp) -----------------------
     const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(P.k_cache);
     const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(P.v_cache);
@@ -260,9 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const uint32_t dst = smem_addr(smem + Layout::kStageOff + st * kStageBytes);
+      // one row per lane (two producer warps: 64 rows each), all 16 chunks of
+      // K and V; measured faster than spreading a row over 16 lanes
 #pragma unroll
-      for (int i = 0; i < kBlock / 32; ++i) {
-        const int r = lane + 32 * i;
+      for (int i = 0; i < 2; ++i) {
+        const int r = (warp - kWarps) * 64 + lane + 32 * i;
         const int tok = __ldg(toks + r);
         const long long row = tok_row(P, s, g, p, tok);
         if (row < 0 && tok >= 0) raise_error(tok > p ? MSA_DEVERR_SEL_RANGE : MSA_DEVERR_PAGE_RANGE);
@@ -282,9 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = max(0, k - kStages); j < k; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
     return;
   }
-  if (!kTok && warp == kWarps) {
+  if (!kTok && warp >= kWarps) {
     // -------------------------------- producer --------------------------------
-    if (lane != 0) return;
+    if (warp != kWarps || lane != 0) return;
     int k = 0;
     bool ok = true;
     for (long long u = u0; u < u1 && ok; ++u) {

@@ -9,12 +9,20 @@
 // One CTA of 1024 threads per query.  Each visible score becomes an
 // order-preserving 32-bit key, staged in shared memory (contexts up to 48K
 // tokens; longer ones are re-read from global memory, where they stay in
-// L2).  A most-significant-digit-first radix select (4 passes of 8 bits,
-// warp-aggregated shared-memory histograms) finds the k-th largest key T and
-// how many keys equal to T are still needed.  A final pass walks the tokens
-// in index order, one contiguous range per warp, and writes every token with
-// key > T plus the first needed tokens with key == T, so the output is
+// L2).  The k-th largest key T comes from a sample-select: the keys of 2048
+// evenly spaced tokens bracket the rank k/n quantile (two exact radix
+// selects on the sample), one ballot-compacted pass keeps the few thousand
+// keys inside the bracket and counts those above it, and an exact radix
+// select among the kept keys gives T and how many keys equal to T are still
+// needed.  If the bracket misses (rare), the radix select runs over all
+// keys, so the result is always exact.  A final pass walks the tokens in
+// index order, one contiguous range per warp, and writes every token with
+// key > T plus the first needed tokens with key == T: the output is
 // ascending with no sort.
+//
+// The radix select is most-significant-digit first, 8 bits per pass, with
+// shared-memory atomic histograms; the filter and emit passes take four
+// keys per lane per step and place them with warp scans.
 #pragma once
 
 #include "msa_common.cuh"
@@ -26,6 +34,9 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kMaxTopK = 2048;                 // width of a selection row
 constexpr int kSmemKeys = 48 * 1024;           // scores staged in shared memory up to this context
+constexpr int kSamples = 2048;                 // sample of the sample-select
+constexpr int kMaxCands = 4096;                // keys kept inside the sample bracket
+constexpr int kSampleMin = 8192;               // shorter contexts take the plain radix select
 
 struct SelSmem {
   unsigned int hist[256];
@@ -33,10 +44,15 @@ struct SelSmem {
   int warp_eq[kSelWarps];
   uint32_t prefix;
   int need;
+  int n_above;                 // sample-select: keys above the bracket
+  int n_cand;                  // sample-select: keys kept inside it
+  uint32_t samples[kSamples];
+  uint32_t cands[kMaxCands];
   uint32_t keys[kSmemKeys];    // last: the unstaged kernel is launched without it
 };
 constexpr size_t kSelSmemStaged = sizeof(SelSmem);
 constexpr size_t kSelSmemUnstaged = sizeof(SelSmem) - sizeof(uint32_t) * kSmemKeys;
+static_assert(kSelSmemStaged <= 232448, "shared memory budget");
 
 // Order-preserving key of a score: larger score, larger key.  NaN maps to
 // the key of -inf and -0 to the key of +0.
@@ -47,63 +63,45 @@ __device__ __forceinline__ uint32_t score_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <bool kStaged>
-__device__ __forceinline__ uint32_t key_at(const SelSmem& sm, const float* row, int i) {
-  if constexpr (kStaged) return sm.keys[i];
-  return score_key(__ldg(row + i));
-}
+// Keys read from a shared-memory array (16-byte aligned).  get4(i): keys
+// i .. i+3 for i a multiple of 4, in one vector load; callers ignore keys at
+// or past n, and every array is long enough for the whole vector.
+struct SmemKeys {
+  const uint32_t* a;
+  __device__ __forceinline__ uint32_t operator()(int i) const { return a[i]; }
+  __device__ __forceinline__ uint4 get4(int i) const { return *reinterpret_cast<const uint4*>(a + i); }
+};
+// Keys computed from a score row in global memory (rows are whole multiples
+// of 128 floats, 16-byte aligned).
+struct RowKeys {
+  const float* row;
+  __device__ __forceinline__ uint32_t operator()(int i) const { return score_key(__ldg(row + i)); }
+  __device__ __forceinline__ uint4 get4(int i) const {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(row + i));
+    return make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+  }
+};
 
-template <bool kStaged>
-__global__ void __launch_bounds__(kSelThreads, 1)
-    dsa_select_topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int n_q,
-                           int capacity, int top_k, int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
-  const int t = blockIdx.x;
+// The k-th largest (1 <= k <= n) of the n keys get(0..n-1): *T receives it
+// and *need how many keys equal to it rank within the first k.  Called by
+// the whole CTA; ends with a barrier.
+template <typename Get>
+__device__ void radix_kth(SelSmem& sm, Get get, int n, int k, uint32_t* T, int* need_out) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  if (t >= n_q) return;
-  const int p = q_pos[t];
-  int32_t* out = sel + static_cast<size_t>(t) * kMaxTopK;
-  if (p < 0 || p >= capacity) {
-    for (int i = tid; i < kMaxTopK; i += kSelThreads) out[i] = -1;
-    if (tid == 0) {
-      if (n_sel != nullptr) n_sel[t] = 0;
-      raise_error(MSA_DEVERR_QUERY_RANGE);
-    }
-    return;
-  }
-  const int n = p + 1;
-  if (n <= top_k) {                                   // every visible token is kept
-    for (int i = tid; i < kMaxTopK; i += kSelThreads) out[i] = i < n ? i : -1;
-    if (tid == 0 && n_sel != nullptr) n_sel[t] = n;
-    return;
-  }
-  const float* row = scores + static_cast<size_t>(t) * capacity;
-  if constexpr (kStaged) {
-    for (int i = tid; i < n; i += kSelThreads) sm.keys[i] = score_key(__ldg(row + i));
-  }
   if (tid == 0) {
     sm.prefix = 0;
-    sm.need = top_k;
+    sm.need = k;
   }
-  __syncthreads();
-
-  // ---- radix select: the top_k-th largest key, 8 bits per pass ------------
   uint32_t mask = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = tid; b < 256; b += kSelThreads) sm.hist[b] = 0;
     __syncthreads();
     const uint32_t prefix = sm.prefix;
-    for (int base = 0; base < n; base += kSelThreads) {
-      const int i = base + tid;
-      const bool in = i < n;
-      const uint32_t key = in ? key_at<kStaged>(sm, row, i) : 0u;
-      const bool cand = in && (key & mask) == prefix;
-      const unsigned int digit = cand ? (key >> shift) & 255u : 256u + lane;   // unique dummy digit
-      const unsigned int peers = __match_any_sync(0xffffffffu, digit);
-      if (cand && (__ffs(peers) - 1) == lane) atomicAdd(&sm.hist[digit], __popc(peers));
+    for (int i = tid; i < n; i += kSelThreads) {
+      const uint32_t key = get(i);
+      if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
     if (warp == 0) {
@@ -124,8 +122,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         if (lane >= o) incl += v;
       }
       const unsigned int excl = incl - local;
-      const bool here = excl < static_cast<unsigned int>(need) && incl >= static_cast<unsigned int>(need);
-      if (here) {
+      if (excl < static_cast<unsigned int>(need) && incl >= static_cast<unsigned int>(need)) {
         unsigned int cum = excl;
         int bin = 255 - 8 * lane;
 #pragma unroll
@@ -143,19 +140,112 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     mask |= 255u << shift;
     __syncthreads();
   }
-  const uint32_t T = sm.prefix;
-  const int need_eq = sm.need;                        // keys equal to T still to keep (>= 1)
+  *T = sm.prefix;
+  *need_out = sm.need;
+  __syncthreads();
+}
 
-  // ---- emit in index order: one contiguous range of tokens per warp --------
-  const int per_warp = (n + kSelWarps - 1) / kSelWarps;
+// Sample-select of the k-th largest of the n keys get(0..n-1) (n >= 4 *
+// kSamples): false when the sample bracket misses the k-th key or keeps too
+// many keys, in which case nothing is returned.  Called by the whole CTA.
+template <typename Get>
+__device__ bool sample_kth(SelSmem& sm, Get get, int n, int k, uint32_t* T, int* need) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  for (int j = tid; j < kSamples; j += kSelThreads)
+    sm.samples[j] = get(static_cast<int>(static_cast<long long>(j) * n / kSamples));
+  if (tid == 0) {
+    sm.n_above = 0;
+    sm.n_cand = 0;
+  }
+  __syncthreads();
+  // the k-th key's expected rank in the sample, +- three binomial standard deviations
+  const float r = static_cast<float>(k) * kSamples / n;
+  const int delta = static_cast<int>(3.f * sqrtf(r) + 8.f);
+  const int r_hi = static_cast<int>(r) - delta;                  // 1-based ranks
+  const int r_lo = min(kSamples, static_cast<int>(r) + delta + 1);
+  const bool has_hi = r_hi >= 1;
+  uint32_t t_hi = 0xffffffffu, t_lo = 0u;
+  int unused;
+  if (has_hi) radix_kth(sm, SmemKeys{sm.samples}, kSamples, r_hi, &t_hi, &unused);
+  radix_kth(sm, SmemKeys{sm.samples}, kSamples, r_lo, &t_lo, &unused);
+
+  // one pass: count the keys above the bracket, keep the keys inside it
+  // (four keys per lane per iteration; order inside the kept list is free)
+  int above = 0;
+  for (int base0 = 0; base0 < n; base0 += 4 * kSelThreads) {      // same trip count in every lane
+    const int base = base0 + 4 * tid;
+    const uint4 kv = base < n ? get.get4(base) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t key[4] = {kv.x, kv.y, kv.z, kv.w};
+    int keep_n = 0;
+    bool keep[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool in = base + j < n;
+      const bool up = in && has_hi && key[j] > t_hi;
+      keep[j] = in && !up && key[j] >= t_lo;
+      above += up ? 1 : 0;
+      keep_n += keep[j] ? 1 : 0;
+    }
+    int incl = keep_n;                                   // warp inclusive scan of the kept counts
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int slot0 = 0;
+    if (lane == 31 && total > 0) slot0 = atomicAdd(&sm.n_cand, total);
+    int slot = __shfl_sync(0xffffffffu, slot0, 31) + incl - keep_n;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (keep[j]) {
+        if (slot < kMaxCands) sm.cands[slot] = key[j];
+        ++slot;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+  if (lane == 0 && above != 0) atomicAdd(&sm.n_above, above);
+  __syncthreads();
+  const int n_above = sm.n_above;
+  const int n_cand = sm.n_cand;
+  __syncthreads();
+  if (n_cand > kMaxCands || n_above >= k || n_above + n_cand < k) return false;
+  radix_kth(sm, SmemKeys{sm.cands}, n_cand, k - n_above, T, need);
+  return true;
+}
+
+// Write, in index order, every token with key > T and the first need_eq
+// tokens with key == T (k tokens in all).  Each warp owns a contiguous range
+// and walks it 128 keys at a time, four consecutive keys per lane: a count
+// pass, one block-wide exchange of the warps' counts, then an emit pass
+// whose positions come from one warp scan per 128 keys.
+template <typename Get>
+__device__ void emit_topk(SelSmem& sm, Get get, int n, uint32_t T, int need_eq, int32_t* out) {
+  constexpr int kSpan = 4 * 32;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int per_warp = (n + kSelWarps * kSpan - 1) / (kSelWarps * kSpan) * kSpan;
   const int w0 = min(n, warp * per_warp);
   const int w1 = min(n, w0 + per_warp);
   int gt = 0, eq = 0;
-  for (int base = w0; base < w1; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < w1 ? key_at<kStaged>(sm, row, i) : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, i < w1 && key > T));
-    eq += __popc(__ballot_sync(0xffffffffu, i < w1 && key == T));
+  for (int b0 = w0; b0 < w1; b0 += kSpan) {
+    const int i0 = b0 + 4 * lane;
+    const uint4 kv = i0 < w1 ? get.get4(i0) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t key[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      gt += (i0 + j < w1 && key[j] > T) ? 1 : 0;
+      eq += (i0 + j < w1 && key[j] == T) ? 1 : 0;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
   }
   if (lane == 0) {
     sm.warp_gt[warp] = gt;
@@ -167,19 +257,84 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     gt_before += sm.warp_gt[w];
     eq_before += sm.warp_eq[w];
   }
-  const unsigned int lt_mask = (1u << lane) - 1u;
-  for (int base = w0; base < w1; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < w1 ? key_at<kStaged>(sm, row, i) : 0u;
-    const bool is_gt = i < w1 && key > T;
-    const bool is_eq = i < w1 && key == T;
-    const unsigned int bgt = __ballot_sync(0xffffffffu, is_gt);
-    const unsigned int beq = __ballot_sync(0xffffffffu, is_eq);
-    const int my_eq = eq_before + __popc(beq & lt_mask);          // equal keys before token i
-    const int my_gt = gt_before + __popc(bgt & lt_mask);
-    if (is_gt || (is_eq && my_eq < need_eq)) out[my_gt + min(my_eq, need_eq)] = i;
-    gt_before += __popc(bgt);
-    eq_before += __popc(beq);
+  for (int b0 = w0; b0 < w1; b0 += kSpan) {
+    bool is_gt[4], is_eq[4];
+    int packed = 0;                                   // gt count | eq count << 16
+    const int i0 = b0 + 4 * lane;
+    const uint4 kv = i0 < w1 ? get.get4(i0) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t key[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = i0 + j;
+      is_gt[j] = i < w1 && key[j] > T;
+      is_eq[j] = i < w1 && key[j] == T;
+      packed += (is_gt[j] ? 1 : 0) + (is_eq[j] ? 1 << 16 : 0);
+    }
+    int incl = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - packed;
+    int g = gt_before + (excl & 0xffff);
+    int e = eq_before + (excl >> 16);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = b0 + 4 * lane + j;
+      if (is_gt[j]) {
+        out[g + min(e, need_eq)] = i;
+        ++g;
+      } else if (is_eq[j]) {
+        if (e < need_eq) out[g + e] = i;
+        ++e;
+      }
+    }
+    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+    gt_before += tot & 0xffff;
+    eq_before += tot >> 16;
+  }
+}
+
+template <bool kStaged>
+__global__ void __launch_bounds__(kSelThreads, 1)
+    dsa_select_topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int n_q,
+                           int capacity, int top_k, int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  if (t >= n_q) return;
+  const int p = q_pos[t];
+  int32_t* out = sel + static_cast<size_t>(t) * kMaxTopK;
+  if (p < 0 || p >= capacity) {
+    for (int i = tid; i < kMaxTopK; i += kSelThreads) out[i] = -1;
+    if (tid == 0) {
+      if (n_sel != nullptr) n_sel[t] = 0;
+      raise_error(MSA_DEVERR_QUERY_RANGE);
+    }
+    return;
+  }
+  const int n = p + 1;
+  if (n <= top_k) {                                   // every visible token is kept
+    for (int i = tid; i < kMaxTopK; i += kSelThreads) out[i] = i < n ? i : -1;
+    if (tid == 0 && n_sel != nullptr) n_sel[t] = n;
+    return;
+  }
+  const float* row = scores + static_cast<size_t>(t) * capacity;
+  uint32_t T;
+  int need;
+  if constexpr (kStaged) {
+#pragma unroll 8
+    for (int i = tid; i < n; i += kSelThreads) sm.keys[i] = score_key(__ldg(row + i));   // loads in flight
+    __syncthreads();
+    const SmemKeys get{sm.keys};
+    if (n < kSampleMin || !sample_kth(sm, get, n, top_k, &T, &need)) radix_kth(sm, get, n, top_k, &T, &need);
+    emit_topk(sm, get, n, T, need, out);
+  } else {
+    const RowKeys get{row};
+    if (!sample_kth(sm, get, n, top_k, &T, &need)) radix_kth(sm, get, n, top_k, &T, &need);
+    emit_topk(sm, get, n, T, need, out);
   }
   for (int i = top_k + tid; i < kMaxTopK; i += kSelThreads) out[i] = -1;
   if (tid == 0 && n_sel != nullptr) n_sel[t] = top_k;

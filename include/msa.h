@@ -331,7 +331,7 @@ MSA_API int msa_dsa_indexer_append(const msa_dsa_shape* shape, const msa_pages* 
 /* Token scores: q_idx [n_q][H_I][Di] fp16, weights [n_q][H_I] f32 ->
  * scores [n_q][capacity] f32, -inf past each query's position.  Each head's
  * product of fp16 vectors accumulates in f32 on the tensor cores; the
- * weighted sum over heads runs in f32 in head order.  An out-of-range query
+ * weighted sum over heads runs in f32 in a fixed order (deterministic).  An out-of-range query
  * writes -inf everywhere and sets MSA_DEVERR_QUERY_RANGE. */
 MSA_API int msa_dsa_token_scores(const msa_dsa_shape* shape, const msa_pages* pages, const msa_f16* q_idx,
                                  const float* weights, const msa_f16* k_idx_cache, const int32_t* q_stream,

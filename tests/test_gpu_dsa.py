@@ -36,7 +36,8 @@ def _scores_with_ties(n_q, cap, seed):
     return sc
 
 
-@pytest.mark.parametrize("cap,top_k", [(4096, 2048), (4096, 7), (4096, 1), (9984, 100), (65536, 2048)])
+@pytest.mark.parametrize("cap,top_k", [(4096, 2048), (4096, 7), (4096, 1), (9984, 100), (32768, 2048),
+                                       (32768, 100), (65536, 2048), (131072, 2048)])
 def test_select_bitexact_from_identical_scores(cap, top_k):
     n_q = 12
     sc = _scores_with_ties(n_q, cap, seed=cap + top_k)
@@ -51,6 +52,22 @@ def test_select_bitexact_from_identical_scores(cap, top_k):
     sel_o, nsel_o = oracle.dsa_select_tokens(sc.double(), q_pos, top_k, msa.DSA_SEL_WIDTH)
     assert torch.equal(n_sel.cpu(), nsel_o)
     assert torch.equal(sel.cpu(), sel_o)
+
+
+def test_select_constant_and_two_valued_rows():
+    """Rows where the sample bracket keeps too many keys (all equal) or where
+    the k-th key sits in a huge tie run: the exact fallback must agree."""
+    cap = 32768
+    sc = torch.zeros((3, cap))
+    sc[1, ::2] = 1.0
+    sc[2] = torch.randn(cap, generator=torch.Generator().manual_seed(3))
+    sc[2, 5000:30000] = 0.25
+    q_pos = torch.full((3,), cap - 1, dtype=torch.int32)
+    ds = msa.DsaShape(n_streams=1, capacity=cap, top_k=2048)
+    sel, n_sel = msa.msa_dsa_select_topk(ds, sc.cuda(), q_pos.cuda())
+    assert msa.msa_get_device_error() == 0
+    sel_o, nsel_o = oracle.dsa_select_tokens(sc.double(), q_pos, 2048, msa.DSA_SEL_WIDTH)
+    assert torch.equal(sel.cpu(), sel_o) and torch.equal(n_sel.cpu(), nsel_o)
 
 
 def test_select_invalid_query_flags():
