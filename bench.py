@@ -48,7 +48,12 @@ WORKLOAD = W.DECODE_32K_X32
 # keys scanned).  Valid only for the kernel source it was taken on (sha256
 # prefix of msa_scores_gemv.cuh); any other source reports null.
 SCORES_TRAFFIC = {"source_sha": "b9bc1ca3c5d4d5a4",
-                  "bytes_per_launch": {"f32": 4 * (536_911_872 + 3_886_848), "f16": None}}
+                  "bytes_per_launch": {"f32": 4 * (536_911_872 + 3_886_848), "f16": 4 * (268_474_112 + 2_967_040)}}
+
+# The same for the token-score kernel of the token-level variant, from the
+# 16-stream capture summarised in profiles/dsa_token_scores_decode_16x32k.md,
+# scaled by 2 to 32 streams (sha256 prefix of msa_dsa_scores.cuh).
+DSA_SCORES_TRAFFIC = {"source_sha": "6c6fa9e892144930", "bytes_per_launch": 2 * (134_557_696 + 5_160_960)}
 
 
 def variant_metric(metric: str, args) -> str:
@@ -57,8 +62,8 @@ def variant_metric(metric: str, args) -> str:
     return metric.replace("x32 streams", "x32 streams, " + ", ".join(tags)) if tags else metric
 
 
-def scores_source_sha() -> str:
-    p = os.path.join(ROOT, "block_sparse_attention_maxpool_b200", "csrc", "msa_scores_gemv.cuh")
+def scores_source_sha(name: str = "msa_scores_gemv.cuh") -> str:
+    p = os.path.join(ROOT, "block_sparse_attention_maxpool_b200", "csrc", name)
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
@@ -434,6 +439,9 @@ DSA_METRIC = ("MSA token-level variant (lightning indexer, 64 heads, top-2048 to
 
 def dsa_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks, graphs):
     sbytes = dsa_scores_bytes(w)
+    traffic = None
+    if DSA_SCORES_TRAFFIC["source_sha"] == scores_source_sha("msa_dsa_scores.cuh") and w == WORKLOAD:
+        traffic = DSA_SCORES_TRAFFIC["bytes_per_launch"]
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     step_gbs = dsa_step_bytes(w) / (ms * 1e-3) / 1e9
     return {
@@ -454,7 +462,7 @@ def dsa_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per
         "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peaks["hbm_gbs"], "frac": step_gbs / peaks["hbm_gbs"],
                      "bytes_per_step": dsa_step_bytes(w)},
         "roofline": {"kernel": "dsa_scores", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes": sbytes, "ms_per_launch": k_ms, "peak_src": peaks["src"]},
         "e2e": {"value": job_tokens_per_s(w.n_streams, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
