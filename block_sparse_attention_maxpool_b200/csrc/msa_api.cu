@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "msa.h"
 #include "msa_append.cuh"
@@ -56,6 +57,27 @@ int pages_of(const msa_shape* sh, const msa_pages* pg, msa::KvPages* out, int64_
   out->table = pg->block_table;
   out->n_pages = pg->n_pages;
   return MSA_OK;
+}
+
+// Every kernel is launched with programmatic stream serialization: its grid
+// may begin launching while the previous kernel in the stream finishes (so
+// launch latency and the prologue overlap it); the kernel waits in
+// pdl_wait() before it touches global memory, so results are the same as
+// with plain stream order.
+template <typename... Params, typename... Args>
+cudaError_t launch(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 int current_device_sms(int* sms) {
@@ -191,8 +213,7 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     Q.scale_log2 = softmax_scale * 1.4426950408889634f;
     Q.pages = pg;
     const int64_t grid = std::min<int64_t>(sms, n_pairs);
-    msa::pattn::sparse_attn_prefill_tc_kernel<<<static_cast<unsigned>(grid), msa::pattn::kThreads,
-                                                msa::pattn::Layout::kBytes, s>>>(tm_q, tm_k, tm_v, Q);
+    launch(msa::pattn::sparse_attn_prefill_tc_kernel, dim3(static_cast<unsigned>(grid)), dim3(msa::pattn::kThreads), msa::pattn::Layout::kBytes, s, tm_q, tm_k, tm_v, Q);
     return cuda_status(cudaGetLastError());
   }
   // decode: persistent stream-K grid over (pair, selected block) units, or
@@ -220,10 +241,10 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   P.tok_sel = tok_sel;
   P.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
   P.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
-  kernel<<<static_cast<unsigned>(P.n_cta), msa::dattn::kThreads, msa::dattn::Layout::kBytes, s>>>(tm_k, tm_v, P);
+  launch(kernel, dim3(static_cast<unsigned>(P.n_cta)), dim3(msa::dattn::kThreads), msa::dattn::Layout::kBytes, s, tm_k, tm_v, P);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
   const int64_t warps = n_pairs * msa::dattn::kHpg;
-  msa::dattn::attn_sk_combine_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(P);
+  launch(msa::dattn::attn_sk_combine_kernel, dim3(static_cast<unsigned>((warps * 32 + 255) / 256)), dim3(256), 0, s, P);
   return cuda_status(cudaGetLastError());
 }
 
@@ -243,7 +264,7 @@ int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache
   const int64_t warps = static_cast<int64_t>(n_tok) * sh->n_kv_heads;
   if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
   const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
-  msa::append_rows_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch(msa::append_rows_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), 
       static_cast<uint8_t*>(cache0), static_cast<const uint8_t*>(src0), static_cast<uint8_t*>(cache1),
       static_cast<const uint8_t*>(src1), tok_stream, tok_pos, n_tok, sh->n_streams, sh->n_kv_heads,
       sh->capacity, row_bytes, pg);
@@ -340,23 +361,22 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
     static std::atomic<uint64_t> tc_smem_done{0};
     if ((st = ensure_smem(T::block_scores_tc_kernel, T::SmemLayout::kBytes, tc_smem_done)) != MSA_OK) return st;
 
-    T::tc_init_kernel<<<1, 256, 0, cs>>>(Q.counters, 1 + S);
-    T::tc_tile_info_kernel<<<(L.n_tiles * 32 + 255) / 256, 256, 0, cs>>>(Q);
-    T::tc_split_queries_kernel<<<static_cast<unsigned>((q_rows * 32 + 255) / 256), 256, 0, cs>>>(Q);
-    T::tc_split_keys_kernel<<<static_cast<unsigned>((key_rows * 32 + 255) / 256), 256, 0, cs>>>(Q);
+    launch(T::tc_init_kernel, dim3(1), dim3(256), 0, cs, Q.counters, 1 + S);
+    launch(T::tc_tile_info_kernel, dim3((L.n_tiles * 32 + 255) / 256), dim3(256), 0, cs, Q);
+    launch(T::tc_split_queries_kernel, dim3(static_cast<unsigned>((q_rows * 32 + 255) / 256)), dim3(256), 0, cs, Q);
+    launch(T::tc_split_keys_kernel, dim3(static_cast<unsigned>((key_rows * 32 + 255) / 256)), dim3(256), 0, cs, Q);
     const int n_tasks = G * Q.n_chunks * Q.n_tiles;
-    T::block_scores_tc_kernel<<<static_cast<unsigned>(std::min(sms, n_tasks)), T::kThreads,
-                                T::SmemLayout::kBytes, cs>>>(m_qhi, m_qlo, m_khi, m_klo, Q);
+    launch(T::block_scores_tc_kernel, dim3(static_cast<unsigned>(std::min(sms, n_tasks))), dim3(T::kThreads), T::SmemLayout::kBytes, cs, m_qhi, m_qlo, m_khi, m_klo, Q);
     if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
     // queries of mixed-stream tiles: streaming kernel over the leftover list
     P.q_list = Q.leftover;
     P.q_count = Q.counters;
-    kernel<<<static_cast<unsigned>(Cfg::kCtasPerSm * sms), kThreads, smem, cs>>>(P);
+    launch(kernel, dim3(static_cast<unsigned>(Cfg::kCtasPerSm * sms)), dim3(kThreads), smem, cs, P);
     return cuda_status(cudaGetLastError());
   }
 
   const long long grid = std::min<long long>(static_cast<long long>(Cfg::kCtasPerSm) * sms, P.n_tasks);
-  kernel<<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(P);
+  launch(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, cs, P);
   return cuda_status(cudaGetLastError());
 }
 
@@ -375,7 +395,7 @@ int append_idx_f16(const msa_shape* shape, msa_f16* idx_k_cache, const float* id
   const int64_t warps = static_cast<int64_t>(n_tok) * shape->n_kv_heads;
   if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
   const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
-  msa::append_idx_f16_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch(msa::append_idx_f16_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), 
       reinterpret_cast<__half*>(idx_k_cache), idx_k_new, tok_stream, tok_pos, n_tok, shape->n_streams,
       shape->n_kv_heads, shape->capacity, pg);
   return cuda_status(cudaGetLastError());
@@ -458,13 +478,13 @@ int msa_select_topk(const msa_shape* shape, const float* block_scores, const int
   const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (nblk <= 32 * 8) {
-    msa::sel::select_topk_kernel<8><<<grid, 256, 0, s>>>(block_scores, q_pos, n_q, G, nblk, shape->capacity,
+    launch(msa::sel::select_topk_kernel<8>, dim3(grid), dim3(256), 0, s, block_scores, q_pos, n_q, G, nblk, shape->capacity,
                                                           sel, n_sel);
   } else if (nblk <= 32 * 32) {
-    msa::sel::select_topk_kernel<32><<<grid, 256, 0, s>>>(block_scores, q_pos, n_q, G, nblk, shape->capacity,
+    launch(msa::sel::select_topk_kernel<32>, dim3(grid), dim3(256), 0, s, block_scores, q_pos, n_q, G, nblk, shape->capacity,
                                                            sel, n_sel);
   } else {
-    msa::sel::select_topk_kernel<0><<<grid, 256, 0, s>>>(block_scores, q_pos, n_q, G, nblk, shape->capacity,
+    launch(msa::sel::select_topk_kernel<0>, dim3(grid), dim3(256), 0, s, block_scores, q_pos, n_q, G, nblk, shape->capacity,
                                                           sel, n_sel);
   }
   return cuda_status(cudaGetLastError());
@@ -647,8 +667,7 @@ int msa_dsa_token_scores(const msa_dsa_shape* shape, const msa_pages* pages, con
   P.pages = pg;
   const int64_t tasks = static_cast<int64_t>(n_q) * P.n_tiles;
   const int64_t grid = std::min<int64_t>(static_cast<int64_t>(msa::dsa::kCtasPerSm) * sms, tasks);
-  msa::dsa::dsa_scores_kernel<<<static_cast<unsigned>(grid), msa::dsa::kThreads, msa::dsa::Smem::kBytes,
-                                static_cast<cudaStream_t>(stream)>>>(tm_key, tm_q, P);
+  launch(msa::dsa::dsa_scores_kernel, dim3(static_cast<unsigned>(grid)), dim3(msa::dsa::kThreads), msa::dsa::Smem::kBytes, static_cast<cudaStream_t>(stream), tm_key, tm_q, P);
   return cuda_status(cudaGetLastError());
 }
 
@@ -665,12 +684,10 @@ int msa_dsa_select_topk(const msa_dsa_shape* shape, const float* scores, const i
     static std::atomic<uint64_t> smem_done{0};
     if ((st = ensure_smem(msa::dsa::dsa_select_topk_kernel<true>, msa::dsa::kSelSmemStaged, smem_done)) != MSA_OK)
       return st;
-    msa::dsa::dsa_select_topk_kernel<true><<<static_cast<unsigned>(n_q), msa::dsa::kSelThreads,
-                                             msa::dsa::kSelSmemStaged, cs>>>(scores, q_pos, n_q, shape->capacity,
+    launch(msa::dsa::dsa_select_topk_kernel<true>, dim3(static_cast<unsigned>(n_q)), dim3(msa::dsa::kSelThreads), msa::dsa::kSelSmemStaged, cs, scores, q_pos, n_q, shape->capacity,
                                                                              shape->top_k, sel, n_sel);
   } else {
-    msa::dsa::dsa_select_topk_kernel<false><<<static_cast<unsigned>(n_q), msa::dsa::kSelThreads,
-                                              msa::dsa::kSelSmemUnstaged, cs>>>(scores, q_pos, n_q,
+    launch(msa::dsa::dsa_select_topk_kernel<false>, dim3(static_cast<unsigned>(n_q)), dim3(msa::dsa::kSelThreads), msa::dsa::kSelSmemUnstaged, cs, scores, q_pos, n_q,
                                                                                 shape->capacity, shape->top_k,
                                                                                 sel, n_sel);
   }

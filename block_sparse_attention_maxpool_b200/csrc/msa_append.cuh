@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(256) append_rows_kernel(
     const uint8_t* __restrict__ src1, const int32_t* __restrict__ tok_stream,
     const int32_t* __restrict__ tok_pos, int n_tok, int n_streams, int n_groups, int capacity,
     int row_bytes, const KvPages pages) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok * n_groups) return;
@@ -59,6 +61,8 @@ __global__ void __launch_bounds__(256) append_idx_f16_kernel(__half* __restrict_
                                                              const int32_t* __restrict__ tok_pos, int n_tok,
                                                              int n_streams, int n_groups, int capacity,
                                                              const KvPages pages) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok * n_groups) return;

@@ -246,6 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();
 
   if (kTok && warp >= kWarps) {
     // ----------------------- producer: token gathers (whole warp) -----------------------
@@ -449,6 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Pairs cut by a share boundary: merge the partials of every CTA whose share
 // touches the pair.  One warp per (pair, head), four dims per lane.
 __global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
+  pdl_trigger();
+  pdl_wait();
   const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long n_pairs = P.n_units / kTopK;

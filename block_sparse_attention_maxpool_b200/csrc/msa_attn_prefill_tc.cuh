@@ -178,6 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t v_base = smem_addr(smem + Layout::kVOff);
   const uint32_t q_base = smem_addr(smem + Layout::kQOff);
   const uint32_t p_base = smem_addr(smem + Layout::kPOff);
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0 || warp == 2) {
     // --------------------- TMA loaders: warp 0 Q and K, warp 2 V --------------------

@@ -19,6 +19,17 @@ __device__ unsigned int g_dev_error = 0;
 
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_dev_error, bit); }
 
+// Programmatic dependent launch.  Every kernel is launched with programmatic
+// stream serialization, so its grid may start while the previous kernel in
+// the stream is still running.  pdl_wait() blocks until every prerequisite
+// grid has completed and its memory writes are visible: each kernel calls it
+// before its first global-memory access (reads and writes alike), after any
+// prologue that touches only shared or tensor memory.  pdl_trigger() lets
+// the next grid in the stream begin launching at once; it still waits in its
+// own pdl_wait().  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Where a cache keeps the 128 slots of logical block b of (stream s, group g).
 // Contiguous caches are [S][G][capacity][row]; paged caches are pools of
 // pages [n_pages][G][128][row] with a block table [S][capacity / 128] that

@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   volatile int* abort_v = abort_flag;
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------

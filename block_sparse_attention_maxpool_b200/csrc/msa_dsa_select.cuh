@@ -304,6 +304,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   if (t >= n_q) return;
   const int p = q_pos[t];
   int32_t* out = sel + static_cast<size_t>(t) * kMaxTopK;

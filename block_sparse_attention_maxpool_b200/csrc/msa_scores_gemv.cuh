@@ -171,6 +171,8 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv
   Smem<KeyT, kStages, kWarps>& sm = *reinterpret_cast<Smem<KeyT, kStages, kWarps>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
   const long long T = P.q_list != nullptr ? static_cast<long long>(*P.q_count) * P.G * P.nblk : P.n_tasks;
   const long long t_begin = T * blockIdx.x / gridDim.x;
   const long long t_end = T * (blockIdx.x + 1) / gridDim.x;

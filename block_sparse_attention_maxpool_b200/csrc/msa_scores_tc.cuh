@@ -110,6 +110,8 @@ __device__ __forceinline__ bool query_ok(const Params& P, int q, int& s, int& p)
 }
 
 __global__ void tc_init_kernel(int* counters, int n) {
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0;
 }
 
@@ -118,6 +120,8 @@ __global__ void tc_init_kernel(int* counters, int n) {
 // among that stream's queries in the tile.  Valid queries of any other
 // stream are appended to the leftover list (scored by the streaming kernel).
 __global__ void __launch_bounds__(256) tc_tile_info_kernel(const Params P) {
+  pdl_trigger();
+  pdl_wait();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= P.n_tiles) return;
@@ -189,6 +193,8 @@ __device__ __forceinline__ int split_row4(float4 x, __half2* hi, __half2* lo) {
 // One warp per (padded query, group) row.  Also writes -inf for the blocks
 // past the query's position and flags invalid queries.
 __global__ void __launch_bounds__(256) tc_split_queries_kernel(const Params P) {
+  pdl_trigger();
+  pdl_wait();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= P.n_q_pad * P.G) return;
@@ -220,6 +226,8 @@ __global__ void __launch_bounds__(256) tc_split_queries_kernel(const Params P) {
 // valid page gets scale NaN: its scores drop out of the max-pool (the block
 // scores -inf) and MSA_DEVERR_PAGE_RANGE is set.
 __global__ void __launch_bounds__(256) tc_split_keys_kernel(const Params P) {
+  pdl_trigger();
+  pdl_wait();
   const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(P.n_streams) * P.G * P.capacity;
@@ -318,6 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   volatile int* abort_v = abort_flag;
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------

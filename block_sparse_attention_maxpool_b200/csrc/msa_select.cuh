@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restric
                                                           int n_q, int G, int nblk, int capacity,
                                                           int32_t* __restrict__ sel,
                                                           int32_t* __restrict__ n_sel) {
+  pdl_trigger();
+  pdl_wait();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= n_q * G) return;
