@@ -58,7 +58,8 @@ DSA_SCORES_TRAFFIC = {"source_sha": "6c6fa9e892144930", "bytes_per_launch": 2 * 
 
 def variant_metric(metric: str, args) -> str:
     """The metric name, marked with the cache variant a run uses."""
-    tags = (["F16 indexer cache"] if args.idx_f16 else []) + (["paged caches"] if args.paged else [])
+    tags = ((["F16 indexer cache"] if args.idx_f16 else []) + (["paged caches"] if args.paged else [])
+            + (["one fused kernel"] if getattr(args, "fused", False) else []))
     return metric.replace("x32 streams", "x32 streams, " + ", ".join(tags)) if tags else metric
 
 
@@ -291,6 +292,19 @@ def run_ours(args, rank, world, dev):
 
     if args.dsa:
         part_append, part_scores, part_attend = dsa_append, dsa_scores, dsa_attend
+    if args.fused:                                   # the whole step as one persistent kernel
+        bufs["workspace_fused"] = torch.empty((msa.msa_decode_step_fused_workspace_bytes(shape, n_q),),
+                                              dtype=torch.uint8, device=dev)
+        launches_per_step = 1
+
+        def part_append(st):                         # noqa: F811
+            pass
+
+        def part_scores(st):                         # noqa: F811
+            msa.decode_step_fused(shape, {k: d[k] for k in ("idx_k_cache", "k_cache", "v_cache")}, d, bufs, st)
+
+        def part_attend(st):                         # noqa: F811
+            pass
 
     def step(ev=None):
         part_append(stream)
@@ -313,19 +327,24 @@ def run_ours(args, rank, world, dev):
         # the same buffers, without per-launch host work.  Three graphs, so
         # events between them still time the block-score kernel on its own.
         graphs = [torch.cuda.CUDAGraph() for _ in range(3)]
-        for g, part in zip(graphs, (part_append, part_scores, part_attend)):
+        for i, (g, part) in enumerate(zip(graphs, (part_append, part_scores, part_attend))):
+            if args.fused and i != 1:                        # the fused step is one kernel: one graph
+                graphs[i] = None
+                continue
             with torch.cuda.graph(g):
                 part(None)
         torch.cuda.synchronize(dev)
 
         def step(ev=None):                                   # noqa: F811  (graph replay)
-            graphs[0].replay()
+            if graphs[0] is not None:
+                graphs[0].replay()
             if ev is not None:
                 ev[0].record(stream)
             graphs[1].replay()
             if ev is not None:
                 ev[1].record(stream)
-            graphs[2].replay()
+            if graphs[2] is not None:
+                graphs[2].replay()
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize(dev)
@@ -394,10 +413,10 @@ def run_ours(args, rank, world, dev):
     if prefill:
         return prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per_step, clk, peaks,
                             graphs)
-    sbytes = scores_bytes(w, key_bytes)
+    sbytes = scores_bytes(w, key_bytes) if not args.fused else step_bytes(w, key_bytes)
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     traffic = None
-    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD and not args.paged:
+    if SCORES_TRAFFIC["source_sha"] == scores_source_sha() and w == WORKLOAD and not args.paged and not args.fused:
         traffic = SCORES_TRAFFIC["bytes_per_launch"]["f16" if args.idx_f16 else "f32"]   # this workload only
     step_gbs = step_bytes(w, key_bytes) / (ms * 1e-3) / 1e9
     line = {
@@ -421,7 +440,8 @@ def run_ours(args, rank, world, dev):
                    "l2": f"inputs {2 * w.n_streams * w.capacity * w.n_kv_heads * 512 / 1e9:.1f} GB per GPU > 126 MB L2, no flush"},
         "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peaks["hbm_gbs"],
                      "frac": step_gbs / peaks["hbm_gbs"], "bytes_per_step": step_bytes(w, key_bytes)},
-        "roofline": {"kernel": "block_scores_gemv", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": "decode_step_fused" if args.fused else "block_scores_gemv", "bound": "hbm",
+                     "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "algorithmic_bytes": sbytes, "ms_per_launch": k_ms,
                      "peak_src": peaks["src"]},
@@ -580,6 +600,8 @@ def main():
                     help="decode with the F16 indexer-key cache variant instead of the F32 cache")
     ap.add_argument("--dsa", action="store_true",
                     help="time the token-level variant (lightning indexer, top-2048 tokens) on the same workload")
+    ap.add_argument("--fused", action="store_true",
+                    help="run the whole decode step as one persistent kernel (msa_decode_step_fused)")
     ap.add_argument("--paged", action="store_true",
                     help="run the paged calls on the same caches laid out as shuffled page pools")
     ap.add_argument("--no-graph", action="store_true",
@@ -593,6 +615,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.dsa and (args.paged or args.idx_f16 or W.WORKLOADS[args.workload].queries != "last"):
         ap.error("--dsa times decode workloads with contiguous caches")
+    if args.fused and (args.paged or args.idx_f16 or args.dsa or W.WORKLOADS[args.workload].queries != "last"):
+        ap.error("--fused times decode workloads with contiguous F32 caches")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
@@ -613,7 +637,7 @@ def main():
         line = run_ours(args, rank, world, local)
         if line is not None:
             if (world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD.name and not args.idx_f16
-                    and not args.paged and not args.dsa):
+                    and not args.paged and not args.dsa and not args.fused):
                 line["cpu_baseline"] = cpu_baseline()
             print(json.dumps(line), flush=True)
     finally:

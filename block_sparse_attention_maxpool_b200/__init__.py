@@ -25,7 +25,8 @@ __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_bloc
            "Pages", "msa_indexer_append_paged", "msa_indexer_append_f16_paged", "msa_kv_append_paged",
            "msa_block_scores_paged", "msa_block_scores_f16_paged", "msa_sparse_attn_decode_paged",
            "msa_sparse_attn_prefill_paged", "DsaShape", "DSA_SEL_WIDTH", "msa_dsa_indexer_append",
-           "msa_dsa_token_scores", "msa_dsa_select_topk", "msa_dsa_sparse_attn_decode", "dsa_decode_step"]
+           "msa_dsa_token_scores", "msa_dsa_select_topk", "msa_dsa_sparse_attn_decode", "dsa_decode_step",
+           "msa_decode_step_fused", "msa_decode_step_fused_workspace_bytes", "decode_step_fused"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
 MODE_DECODE = 0
@@ -153,6 +154,9 @@ _SIGS.update({
     "msa_dsa_select_topk": (ctypes.c_int, [_DS, _P, _P, _I, _P, _P, _P]),
     "msa_dsa_sparse_attn_decode": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
                                                   ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_decode_step_fused": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                                             _P, _P, _I, ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "msa_decode_step_fused_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(CShape), _I]),
 })
 
 
@@ -554,3 +558,65 @@ def dsa_decode_step(shape: Shape, dshape: DsaShape, caches: dict, new: dict, buf
     out = msa_dsa_sparse_attn_decode(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
                                      new["q_pos"], None, b.get("out"), b.get("workspace"), stream, pages)
     return out, sel, n_sel, sc
+
+
+# ---- the whole decode step in one kernel ---------------------------------------
+def msa_decode_step_fused_workspace_bytes(shape: Shape, n_q: int) -> int:
+    s = shape.c()
+    v = library().msa_decode_step_fused_workspace_bytes(ctypes.byref(s), n_q)
+    if v == ctypes.c_size_t(-1).value:
+        raise MsaError("msa_decode_step_fused_workspace_bytes", -3)
+    return v
+
+
+def msa_decode_step_fused(shape: Shape, caches: dict, new: dict, bufs: dict | None = None, stream=None,
+                          softmax_scale=None):
+    """One decode step (appends, block scores, top-16, attention) as a single
+    persistent kernel; same inputs and results as ``decode_step`` (F32
+    indexer cache, decode-shaped batches).  Returns (out, sel, n_sel,
+    block_scores)."""
+    b = bufs or {}
+    n = _n(new["q_pos"], "q_pos")
+    nt = _n(new["tok_stream"], "tok_stream")
+    dev = new["q"].device
+    G = shape.n_kv_heads
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(shape.head_dim)
+    bs = b.get("block_scores")
+    if bs is None:
+        bs = torch.empty((n, G, shape.n_blocks), dtype=torch.float32, device=dev)
+    sel = b.get("sel")
+    if sel is None:
+        sel = torch.empty((n, G, shape.top_k), dtype=torch.int32, device=dev)
+    n_sel = b.get("n_sel")
+    if n_sel is None:
+        n_sel = torch.empty((n, G), dtype=torch.int32, device=dev)
+    out = b.get("out")
+    if out is None:
+        out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=dev)
+    ws = b.get("workspace_fused")
+    need = msa_decode_step_fused_workspace_bytes(shape, n) if n > 0 else 0
+    if ws is None and need > 0:
+        ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    cs = (shape.n_streams, G, shape.capacity)
+    s = shape.c()
+    _check("msa_decode_step_fused", library().msa_decode_step_fused(
+        ctypes.byref(s), _ptr(caches["idx_k_cache"], torch.float32, cs + (shape.idx_dim,), "idx_k_cache"),
+        _ptr(caches["k_cache"], torch.bfloat16, cs + (shape.head_dim,), "k_cache"),
+        _ptr(caches["v_cache"], torch.bfloat16, cs + (shape.head_dim,), "v_cache"),
+        _ptr(new["idx_k_new"], torch.float32, (nt, G, shape.idx_dim), "idx_k_new"),
+        _ptr(new["k_new"], torch.bfloat16, (nt, G, shape.head_dim), "k_new"),
+        _ptr(new["v_new"], torch.bfloat16, (nt, G, shape.head_dim), "v_new"),
+        _ptr(new["tok_stream"], torch.int32, (nt,), "tok_stream"), _ptr(new["tok_pos"], torch.int32, (nt,), "tok_pos"),
+        nt, _ptr(new["idx_q"], torch.float32, (n, G, shape.idx_dim), "idx_q"),
+        _ptr(new["q"], torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
+        _ptr(new["q_stream"], torch.int32, (n,), "q_stream"), _ptr(new["q_pos"], torch.int32, (n,), "q_pos"), n,
+        float(softmax_scale), _ptr(bs, torch.float32, (n, G, shape.n_blocks), "block_scores"),
+        _ptr(sel, torch.int32, (n, G, shape.top_k), "sel"), _ptr(n_sel, torch.int32, (n, G), "n_sel"),
+        _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"),
+        _ptr(ws, torch.uint8, None, "workspace") if ws is not None else 0, ws.numel() if ws is not None else 0,
+        _stream(stream)))
+    return out, sel, n_sel, bs
+
+
+decode_step_fused = msa_decode_step_fused

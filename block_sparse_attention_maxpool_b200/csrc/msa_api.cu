@@ -15,6 +15,7 @@
 #include "msa_attn_decode_sk.cuh"
 #include "msa_attn_prefill_tc.cuh"
 #include "msa_common.cuh"
+#include "msa_decode_fused.cuh"
 #include "msa_dsa_scores.cuh"
 #include "msa_dsa_select.cuh"
 #include "msa_scores_gemv.cuh"
@@ -701,6 +702,125 @@ int msa_dsa_sparse_attn_decode(const msa_shape* shape, const msa_pages* pages, c
   if (n_q > 0 && sel == nullptr) return MSA_ERR_NULL;
   return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
                      workspace_bytes, stream, MSA_MODE_DECODE, pages, sel);
+}
+
+// ---- the whole decode step in one kernel ---------------------------------------
+size_t msa_decode_step_fused_workspace_bytes(const msa_shape* shape, int32_t n_q) {
+  if (check_shape(shape) != MSA_OK || n_q < 1 || scores_use_tiles(shape, n_q)) return static_cast<size_t>(-1);
+  const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
+  return msa::tc::align256(attn_workspace(n_pairs, MSA_MODE_DECODE)) + 256;   // partials, then barrier words
+}
+
+int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* k_cache, msa_bf16* v_cache,
+                          const float* idx_k_new, const msa_bf16* k_new, const msa_bf16* v_new,
+                          const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, const float* idx_q,
+                          const msa_bf16* q, const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
+                          float softmax_scale, float* block_scores, int32_t* sel, int32_t* n_sel, msa_bf16* out,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (n_tok < 0 || n_q < 0) return MSA_ERR_RANGE;
+  if (n_q == 0 && n_tok == 0) return MSA_OK;
+  if (n_q == 0) {                                            // nothing to score: the appends alone
+    if ((st = msa_indexer_append(shape, idx_k_cache, idx_k_new, tok_stream, tok_pos, n_tok, stream)) != MSA_OK)
+      return st;
+    return msa_kv_append(shape, k_cache, v_cache, k_new, v_new, tok_stream, tok_pos, n_tok, stream);
+  }
+  if (!idx_k_cache || !k_cache || !v_cache || !idx_q || !q || !q_stream || !q_pos || !block_scores || !sel || !out)
+    return MSA_ERR_NULL;
+  if (n_tok > 0 && (!idx_k_new || !k_new || !v_new || !tok_stream || !tok_pos)) return MSA_ERR_NULL;
+  if (!aligned16(idx_k_cache) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx_q) || !aligned16(q) ||
+      !aligned16(block_scores) || !aligned16(sel) || !aligned16(out) || (n_tok > 0 && (!aligned16(idx_k_new) ||
+      !aligned16(k_new) || !aligned16(v_new))))
+    return MSA_ERR_ALIGN;
+  if (!std::isfinite(softmax_scale)) return MSA_ERR_RANGE;
+  if (scores_use_tiles(shape, n_q)) return MSA_ERR_SHAPE;       // prefill-shaped: use the separate calls
+  const int G = shape->n_kv_heads;
+  const int64_t n_pairs = static_cast<int64_t>(n_q) * G;
+  if (static_cast<int64_t>(n_tok) * G >= (int64_t{1} << 31) || n_pairs * msa::dattn::kHpg >= (int64_t{1} << 31))
+    return MSA_ERR_RANGE;
+  const size_t need = msa_decode_step_fused_workspace_bytes(shape, n_q);
+  if (workspace == nullptr || workspace_bytes < need) return MSA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MSA_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+  const auto kernel = msa::fused::decode_step_fused_kernel;
+  static std::atomic<uint64_t> smem_done{0};
+  if ((st = ensure_smem(kernel, msa::fused::kSmemBytes, smem_done)) != MSA_OK) return st;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, msa::fused::kThreads, msa::fused::kSmemBytes) !=
+          cudaSuccess || per_sm < 1)
+    return MSA_ERR_CUDA;
+  const int grid = sms;                                      // one resident CTA per SM, as the separate kernels use
+  const int64_t rows = static_cast<int64_t>(shape->n_streams) * G * shape->capacity;
+  CUtensorMap tm_k, tm_v;
+  if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
+  if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
+
+  msa::fused::Params F;
+  F.idx_k_cache = idx_k_cache;
+  F.idx_k_new = idx_k_new;
+  F.k_cache = reinterpret_cast<uint8_t*>(k_cache);
+  F.v_cache = reinterpret_cast<uint8_t*>(v_cache);
+  F.k_new = reinterpret_cast<const uint8_t*>(k_new);
+  F.v_new = reinterpret_cast<const uint8_t*>(v_new);
+  F.tok_stream = tok_stream;
+  F.tok_pos = tok_pos;
+  F.n_tok = n_tok;
+  msa::gemv::Params<float>& S = F.scores;
+  S.idx_q = idx_q;
+  S.idx_k = idx_k_cache;
+  S.q_stream = q_stream;
+  S.q_pos = q_pos;
+  S.bs = block_scores;
+  S.n_q = n_q;
+  S.G = G;
+  S.n_streams = shape->n_streams;
+  S.capacity = shape->capacity;
+  S.nblk = shape->capacity / 128;
+  S.n_tasks = static_cast<long long>(n_q) * G * S.nblk;
+  S.q_list = nullptr;
+  S.q_count = nullptr;
+  S.pages = msa::KvPages{nullptr, 0};
+  F.sel = sel;
+  F.n_sel = n_sel;
+  msa::dattn::Params& A = F.attn;
+  A.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  A.sel = sel;
+  A.q_stream = q_stream;
+  A.q_pos = q_pos;
+  A.out = reinterpret_cast<__nv_bfloat16*>(out);
+  A.ws = static_cast<float*>(workspace);
+  A.n_q = n_q;
+  A.G = G;
+  A.n_streams = shape->n_streams;
+  A.capacity = shape->capacity;
+  A.n_units = n_pairs * msa::dattn::kTopK;
+  A.n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(grid), A.n_units,
+                                                static_cast<int64_t>(msa::dattn::kMaxCtas)}));
+  A.scale_log2 = softmax_scale * 1.4426950408889634f;
+  A.pages = msa::KvPages{nullptr, 0};
+  A.tok_sel = nullptr;
+  A.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
+  A.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
+  unsigned int* bar = reinterpret_cast<unsigned int*>(
+      static_cast<uint8_t*>(workspace) + msa::tc::align256(attn_workspace(n_pairs, MSA_MODE_DECODE)));
+  F.bar_count = bar;
+  F.bar_gen = bar + 1;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), cs) != cudaSuccess) return MSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(msa::fused::kThreads);
+  cfg.dynamicSmemBytes = msa::fused::kSmemBytes;
+  cfg.stream = cs;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, F) != cudaSuccess) return MSA_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {

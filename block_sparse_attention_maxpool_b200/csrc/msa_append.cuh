@@ -11,19 +11,14 @@
 
 namespace msa {
 
-// rows_bytes: bytes of one row (a multiple of 16, at most 512).
-// Up to two caches (K and V) are written by the same launch; cache1/src1
-// may be null.
-__global__ void __launch_bounds__(256) append_rows_kernel(
-    uint8_t* __restrict__ cache0, const uint8_t* __restrict__ src0, uint8_t* __restrict__ cache1,
-    const uint8_t* __restrict__ src1, const int32_t* __restrict__ tok_stream,
-    const int32_t* __restrict__ tok_pos, int n_tok, int n_streams, int n_groups, int capacity,
-    int row_bytes, const KvPages pages) {
-  pdl_trigger();
-  pdl_wait();
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= n_tok * n_groups) return;
+// One (token, group) row: warp `warp` of the n_tok * n_groups rows.
+// rows_bytes: bytes of one row (a multiple of 16, at most 512).  Up to two
+// caches (K and V) are written at once; cache1/src1 may be null.
+__device__ __forceinline__ void append_row(uint8_t* __restrict__ cache0, const uint8_t* __restrict__ src0,
+                                           uint8_t* __restrict__ cache1, const uint8_t* __restrict__ src1,
+                                           const int32_t* __restrict__ tok_stream,
+                                           const int32_t* __restrict__ tok_pos, int n_streams, int n_groups,
+                                           int capacity, int row_bytes, const KvPages& pages, int warp, int lane) {
   const int t = warp / n_groups;
   const int g = warp - t * n_groups;
   const int s = tok_stream[t];
@@ -50,6 +45,19 @@ __global__ void __launch_bounds__(256) append_rows_kernel(
       *d = __ldg(c);
     }
   }
+}
+
+__global__ void __launch_bounds__(256) append_rows_kernel(
+    uint8_t* __restrict__ cache0, const uint8_t* __restrict__ src0, uint8_t* __restrict__ cache1,
+    const uint8_t* __restrict__ src1, const int32_t* __restrict__ tok_stream,
+    const int32_t* __restrict__ tok_pos, int n_tok, int n_streams, int n_groups, int capacity,
+    int row_bytes, const KvPages pages) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= n_tok * n_groups) return;
+  append_row(cache0, src0, cache1, src1, tok_stream, tok_pos, n_streams, n_groups, capacity, row_bytes, pages,
+             warp, threadIdx.x & 31);
 }
 
 // F16 indexer-key cache variant: each F32 key of 128 values is rounded to

@@ -139,7 +139,7 @@ __device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, in
     if (report && j == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
     return -1;
   }
-  const int b = P.sel[pair * kTopK + j];
+  const int b = __ldcg(P.sel + pair * kTopK + j);   // L2 only: may come from other CTAs of this grid
   if (b < 0) return -1;
   if (b > p / kBlock) {
     if (report) raise_error(MSA_DEVERR_SEL_RANGE);
@@ -223,20 +223,20 @@ __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long 
   }
 }
 
+// The kernel body for CTA `cta` of the P.n_cta sharing the units.  tm_k, tm_v:
+// tensor maps of the K and V caches (block path); smem: Layout::kBytes,
+// 1024-byte aligned; the CTA has kThreads threads.
 template <bool kTok>
-__global__ void __launch_bounds__(kThreads, 1)
-    sparse_attn_decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                                 const Params P) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                                           const Params& P, uint8_t* smem, int cta) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Layout::kBarOff);
   uint64_t* empty = full + kStages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long U = P.n_units;
-  const long long u0 = unit_begin(U, P.n_cta, blockIdx.x);
-  const long long u1 = unit_begin(U, P.n_cta, blockIdx.x + 1);
+  const long long u0 = unit_begin(U, P.n_cta, cta);
+  const long long u1 = unit_begin(U, P.n_cta, cta + 1);
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
@@ -246,8 +246,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
-  pdl_trigger();
-  pdl_wait();
 
   if (kTok && warp >= kWarps) {
     // ----------------------- producer: token gathers (whole warp) -----------------------
@@ -304,10 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       uint8_t* dst = smem + Layout::kStageOff + st * kStageBytes;
       mbar_arrive_expect_tx(&full[st], kStageBytes);
-      tma_load_2d(dst, &tm_k, 0, row, &full[st]);
-      tma_load_2d(dst + kTileBytes, &tm_k, 64, row, &full[st]);
-      tma_load_2d(dst + 2 * kTileBytes, &tm_v, 0, row, &full[st]);
-      tma_load_2d(dst + 3 * kTileBytes, &tm_v, 64, row, &full[st]);
+      tma_load_2d(dst, tm_k, 0, row, &full[st]);
+      tma_load_2d(dst + kTileBytes, tm_k, 64, row, &full[st]);
+      tma_load_2d(dst + 2 * kTileBytes, tm_v, 0, row, &full[st]);
+      tma_load_2d(dst + 3 * kTileBytes, tm_v, 64, row, &full[st]);
       ++k;
     }
     // no copy may still be landing when the CTA exits
@@ -328,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (long long u = u0; u < u1; ++u) {
     const long long pair = u / kTopK;
     if (pair != cur) {
-      if (cur >= 0) flush_pair(P, smem, cur, u0, u1, blockIdx.x, o, m_run, l_run, warp, lane);
+      if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane);
       cur = pair;
 #pragma unroll
       for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -445,18 +443,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(&empty[st]);
     ++k;
   }
-  if (cur >= 0) flush_pair(P, smem, cur, u0, u1, blockIdx.x, o, m_run, l_run, warp, lane);
+  if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane);
+}
+
+template <bool kTok>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                                 const Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  pdl_trigger();
+  pdl_wait();
+  sparse_attn_decode_sk_body<kTok>(&tm_k, &tm_v, P, smem, blockIdx.x);
 }
 
 // Pairs cut by a share boundary: merge the partials of every CTA whose share
 // touches the pair.  One warp per (pair, head), four dims per lane.
-__global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
-  pdl_trigger();
-  pdl_wait();
-  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const long long n_pairs = P.n_units / kTopK;
-  if (w >= n_pairs * kHpg) return;
+__device__ __forceinline__ void combine_pair_head(const Params& P, long long w, int lane) {
   const long long pair = w / kHpg;
   const int head = static_cast<int>(w - pair * kHpg);
   const long long U = P.n_units;
@@ -466,7 +469,7 @@ __global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
   float M = -INFINITY;
   for (int c = c_lo; c <= c_hi; ++c) {
     const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
-    M = fmaxf(M, P.ws[(static_cast<size_t>(c) * 2 + slot) * kPartial + kHpg * kD + head]);
+    M = fmaxf(M, __ldcg(P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial + kHpg * kD + head));
   }
   const float Mu = M == -INFINITY ? 0.f : M;
   float L = 0.f;
@@ -474,9 +477,9 @@ __global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
   for (int c = c_lo; c <= c_hi; ++c) {
     const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
     const float* part = P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial;
-    const float sc = exp2f(part[kHpg * kD + head] - Mu);
-    L += part[kHpg * kD + kHpg + head] * sc;
-    const float4 v = *reinterpret_cast<const float4*>(part + head * kD + lane * 4);
+    const float sc = exp2f(__ldcg(part + kHpg * kD + head) - Mu);
+    L += __ldcg(part + kHpg * kD + kHpg + head) * sc;
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(part + head * kD + lane * 4));
     acc.x += v.x * sc;
     acc.y += v.y * sc;
     acc.z += v.z * sc;
@@ -485,6 +488,14 @@ __global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
   const float inv = L > 0.f ? 1.f / L : 0.f;
   __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + lane * 4;
   *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+}
+
+__global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
+  pdl_trigger();
+  pdl_wait();
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (w >= P.n_units / kTopK * kHpg) return;
+  combine_pair_head(P, w, threadIdx.x & 31);
 }
 
 }  // namespace dattn

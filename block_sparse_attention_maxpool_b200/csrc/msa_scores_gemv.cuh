@@ -162,20 +162,21 @@ __device__ __forceinline__ float dot8_f16(const uint4 raw, const float4 qa, cons
   return fmaf(qb.w, d.y, acc);
 }
 
-template <typename KeyT, int kStages, int kWarps, int kMinCtas>
-__global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv_kernel(const Params<KeyT> P) {
+// The kernel body: CTA `cta` of `n_cta` takes its contiguous share of the
+// tasks.  smem_raw: at least sizeof(Smem<...>) bytes, 128-byte aligned.
+// Warps past the producer warp (when a caller's CTA has more) only join the
+// initial barrier.
+template <typename KeyT, int kStages, int kWarps>
+__device__ __forceinline__ void block_scores_gemv_body(const Params<KeyT>& P, uint8_t* smem_raw, int cta, int n_cta) {
   constexpr bool kF16 = sizeof(KeyT) == 2;
   using R = Rows<KeyT, kWarps>;
   constexpr int kStageElems = R::kPerStage * kDi;
-  extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem<KeyT, kStages, kWarps>& sm = *reinterpret_cast<Smem<KeyT, kStages, kWarps>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  pdl_trigger();
-  pdl_wait();
   const long long T = P.q_list != nullptr ? static_cast<long long>(*P.q_count) * P.G * P.nblk : P.n_tasks;
-  const long long t_begin = T * blockIdx.x / gridDim.x;
-  const long long t_end = T * (blockIdx.x + 1) / gridDim.x;
+  const long long t_begin = T * cta / n_cta;
+  const long long t_end = T * (cta + 1) / n_cta;
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv
     mbar_fence_init();
   }
   __syncthreads();
+  if (warp > kWarps) return;
 
   Cursor<KeyT> cur;
   cur.start(P, t_begin, t_end);
@@ -299,6 +301,26 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv
       P.bs[out] = mm;
     }
     par ^= 1;
+  }
+}
+
+template <typename KeyT, int kStages, int kWarps, int kMinCtas>
+__global__ void __launch_bounds__((kWarps + 1) * 32, kMinCtas) block_scores_gemv_kernel(const Params<KeyT> P) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  pdl_trigger();
+  pdl_wait();
+  block_scores_gemv_body<KeyT, kStages, kWarps>(P, smem_raw, blockIdx.x, gridDim.x);
+}
+
+// Invalidate the body's mbarriers (one thread, after every thread of the CTA
+// is past its last use) so that the shared memory can be used for other data.
+template <typename KeyT, int kStages, int kWarps>
+__device__ __forceinline__ void block_scores_gemv_release(uint8_t* smem_raw) {
+  Smem<KeyT, kStages, kWarps>& sm = *reinterpret_cast<Smem<KeyT, kStages, kWarps>*>(smem_raw);
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) {
+    mbar_inval(&sm.full[s]);
+    mbar_inval(&sm.empty[s]);
   }
 }
 

@@ -46,16 +46,9 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t x) {
 // kPerLane > 0: the visible scores (at most 32 * kPerLane) are held in
 // registers; kPerLane == 0: any count, re-read from global memory each round.
 template <int kPerLane>
-__global__ void __launch_bounds__(256) select_topk_kernel(const float* __restrict__ bs,
-                                                          const int32_t* __restrict__ q_pos,
-                                                          int n_q, int G, int nblk, int capacity,
-                                                          int32_t* __restrict__ sel,
-                                                          int32_t* __restrict__ n_sel) {
-  pdl_trigger();
-  pdl_wait();
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= n_q * G) return;
+__device__ __forceinline__ void select_pair(const float* __restrict__ bs, const int32_t* __restrict__ q_pos,
+                                            int G, int nblk, int capacity, int32_t* __restrict__ sel,
+                                            int32_t* __restrict__ n_sel, int wid, int lane) {
   const int qi = wid / G;
   const int p = q_pos[qi];
   int32_t* out = sel + static_cast<size_t>(wid) * kTopK;
@@ -76,7 +69,7 @@ __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restric
 #pragma unroll
     for (int j = 0; j < kPerLane; ++j) {
       const int b = lane + 32 * j;
-      keys[j] = b < nvis ? block_key(__ldg(row + b), b) : 0ull;
+      keys[j] = b < nvis ? block_key(__ldcg(row + b), b) : 0ull;
     }
   }
 
@@ -92,7 +85,7 @@ __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restric
       }
     } else {
       for (int b = lane; b < nvis; b += 32) {
-        const uint64_t x = block_key(__ldg(row + b), b);
+        const uint64_t x = block_key(__ldcg(row + b), b);
         if (x < prev && x > best) best = x;
       }
     }
@@ -113,6 +106,33 @@ __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restric
     out[lane] = -1;
   }
   if (lane == 0 && n_sel != nullptr) n_sel[wid] = k;
+}
+
+
+// One warp per (query, group).
+template <int kPerLane>
+__global__ void __launch_bounds__(256) select_topk_kernel(const float* __restrict__ bs,
+                                                          const int32_t* __restrict__ q_pos,
+                                                          int n_q, int G, int nblk, int capacity,
+                                                          int32_t* __restrict__ sel,
+                                                          int32_t* __restrict__ n_sel) {
+  pdl_trigger();
+  pdl_wait();
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (wid >= n_q * G) return;
+  select_pair<kPerLane>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, threadIdx.x & 31);
+}
+
+// The same for any block count, choosing the register-held variant.
+__device__ __forceinline__ void select_pair_any(const float* bs, const int32_t* q_pos, int G, int nblk,
+                                                int capacity, int32_t* sel, int32_t* n_sel, int wid, int lane) {
+  if (nblk <= 32 * 8) {
+    select_pair<8>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, lane);
+  } else if (nblk <= 32 * 32) {
+    select_pair<32>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, lane);
+  } else {
+    select_pair<0>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, lane);
+  }
 }
 
 }  // namespace sel

@@ -359,6 +359,33 @@ MSA_API int msa_dsa_sparse_attn_decode(const msa_shape* shape, const msa_pages* 
                                        float softmax_scale, msa_bf16* out, void* workspace,
                                        size_t workspace_bytes, void* stream);
 
+/* msa_decode_step_fused - one whole decode step in a single persistent
+ * kernel: append the new tokens (msa_indexer_append + msa_kv_append), block
+ * scores (msa_block_scores), top-16 (msa_select_topk) and block-sparse
+ * attention (msa_sparse_attn_decode), with the same arguments, layouts,
+ * rounding and errors as those calls and bit-identical results.  The MSA
+ * pull request runs the step as separate graph nodes per layer; here the
+ * phases are separated by grid-wide barriers of one cooperative launch (one
+ * CTA per SM), so a small decode batch pays one launch instead of six.  F32
+ * indexer cache, contiguous caches and decode-shaped batches only (fewer
+ * than 256 queries, or fewer than 64 per stream on average; otherwise
+ * MSA_ERR_SHAPE).  n_sel may be NULL.  workspace: at least
+ * msa_decode_step_fused_workspace_bytes(shape, n_q) bytes, 256-byte aligned
+ * (partials of pairs cut between CTAs, and the barrier words, which the call
+ * zeroes on `stream` before the launch).  A barrier wait that gives up sets
+ * MSA_DEVERR_TIMEOUT and leaves the outputs incomplete.  n_q == 0 only
+ * appends. */
+MSA_API int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* k_cache, msa_bf16* v_cache,
+                                  const float* idx_k_new, const msa_bf16* k_new, const msa_bf16* v_new,
+                                  const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok,
+                                  const float* idx_q, const msa_bf16* q, const int32_t* q_stream,
+                                  const int32_t* q_pos, int32_t n_q, float softmax_scale, float* block_scores,
+                                  int32_t* sel, int32_t* n_sel, msa_bf16* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+/* Workspace bytes of msa_decode_step_fused, or (size_t)-1 for an
+ * unsupported shape or batch. */
+MSA_API size_t msa_decode_step_fused_workspace_bytes(const msa_shape* shape, int32_t n_q);
+
 /* Bytes of workspace that msa_block_scores and the attention call of `mode`
  * need for n_q queries (the larger of the two; one buffer serves both calls
  * of a step, since they run in stream order).  0 when neither needs any.

@@ -195,3 +195,25 @@ def test_dsa_calls_validate_shapes(lib):
                                           ctypes.c_float(0.088), fake, 0, 0, None) == -1
     assert lib.msa_dsa_sparse_attn_decode(ctypes.byref(s), None, fake, fake, fake, fake, fake, fake, 2,
                                           ctypes.c_float(0.088), fake, 0, 0, None) == -5
+
+
+def test_fused_step_validation(lib):
+    s = GOOD.c()
+    fake = FAKE
+    ws = lib.msa_decode_step_fused_workspace_bytes(ctypes.byref(s), 2)
+    assert 0 < ws < (1 << 24)
+    assert lib.msa_decode_step_fused_workspace_bytes(ctypes.byref(s), 0) == ctypes.c_size_t(-1).value
+    assert lib.msa_decode_step_fused_workspace_bytes(ctypes.byref(s), 4096) == ctypes.c_size_t(-1).value  # prefill-shaped
+    f = lib.msa_decode_step_fused
+
+    def call(n_tok=1, n_q=2, null_at=None, ws_ptr=fake, ws_bytes=1 << 24):
+        args = [fake] * 8 + [n_tok] + [fake] * 4 + [n_q, ctypes.c_float(0.088)] + [fake] * 4 + [ws_ptr, ws_bytes, None]
+        if null_at is not None:
+            args[null_at] = 0
+        return f(ctypes.byref(s), *args)
+    assert call(n_q=-1) == -4
+    assert call(null_at=0) == -1                      # idx_k_cache
+    assert call(null_at=9) == -1                      # idx_q
+    assert call(n_q=4096) == -3                       # prefill-shaped batch
+    assert call(ws_ptr=0, ws_bytes=0) == -5
+    assert call(ws_ptr=fake + 16) == -2               # workspace not 256-byte aligned
