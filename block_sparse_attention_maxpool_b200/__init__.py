@@ -26,7 +26,7 @@ __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_bloc
            "msa_block_scores_paged", "msa_block_scores_f16_paged", "msa_sparse_attn_decode_paged",
            "msa_sparse_attn_prefill_paged", "DsaShape", "DSA_SEL_WIDTH", "msa_dsa_indexer_append",
            "msa_dsa_token_scores", "msa_dsa_select_topk", "msa_dsa_sparse_attn_decode", "dsa_decode_step",
-           "msa_decode_step_fused", "msa_decode_step_fused_workspace_bytes", "decode_step_fused"]
+           "msa_decode_step_fused", "msa_decode_step_fused_workspace_bytes", "decode_step_fused", "DecodeGraph"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
 MODE_DECODE = 0
@@ -620,3 +620,83 @@ def msa_decode_step_fused(shape: Shape, caches: dict, new: dict, bufs: dict | No
 
 
 decode_step_fused = msa_decode_step_fused
+
+
+# ---- replaying a captured step ----------------------------------------------
+STEP_INPUTS = ("tok_stream", "tok_pos", "idx_k_new", "k_new", "v_new", "q_stream", "q_pos", "idx_q", "q")
+
+
+class DecodeGraph:
+    """One MSA step (``decode_step``: appends, block scores, top-k, attention)
+    captured once as a CUDA graph on fixed device buffers and replayed.
+
+    The step's inputs (tok_stream, tok_pos, idx_k_new, k_new, v_new,
+    q_stream, q_pos, idx_q, q) live in one device staging buffer; ``inputs``
+    holds views of it, and every replay reads whatever they hold.  A caller
+    either writes the views directly, or packs a step's host tensors into
+    one pinned buffer (``host_buffer`` + ``pack``) and calls
+    ``replay_from(buffer)``, which moves all of them in a single
+    host-to-device copy before the replay.  ``out`` holds the result.  The
+    graph's kernels are the library's own; shapes are fixed at capture;
+    ``caches`` are updated in place by every replay."""
+
+    def __init__(self, shape: Shape, caches: dict, inputs: dict, bufs: dict | None = None, prefill: bool = False,
+                 pages: Pages | None = None):
+        self.shape, self.caches, self.prefill, self.pages = shape, caches, prefill, pages
+        dev = inputs["q"].device
+        self._layout = []
+        off = 0
+        for name in STEP_INPUTS:
+            t = inputs[name]
+            off = (off + 255) // 256 * 256
+            self._layout.append((name, off, t.numel() * t.element_size(), t.dtype, tuple(t.shape)))
+            off += t.numel() * t.element_size()
+        self.staging = torch.empty((max(off, 16),), dtype=torch.uint8, device=dev)
+        self.inputs = {name: self.staging[o:o + nb].view(dt).view(shp) for name, o, nb, dt, shp in self._layout}
+        for name in STEP_INPUTS:
+            self.inputs[name].copy_(inputs[name])
+        n = inputs["q_pos"].shape[0]
+        G = shape.n_kv_heads
+        b = dict(bufs or {})
+        b.setdefault("block_scores", torch.empty((n, G, shape.n_blocks), dtype=torch.float32, device=dev))
+        b.setdefault("sel", torch.empty((n, G, shape.top_k), dtype=torch.int32, device=dev))
+        b.setdefault("n_sel", torch.empty((n, G), dtype=torch.int32, device=dev))
+        b.setdefault("out", torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=dev))
+        mode = MODE_PREFILL if prefill else MODE_DECODE
+        b.setdefault("workspace", torch.empty((max(16, msa_workspace_bytes(shape, n, mode)),), dtype=torch.uint8,
+                                              device=dev))
+        self.bufs = b
+        self.out, self.sel, self.n_sel, self.block_scores = b["out"], b["sel"], b["n_sel"], b["block_scores"]
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):                # first run outside the capture (one-time set-up)
+            decode_step(shape, caches, self.inputs, b, side, prefill, pages)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            decode_step(shape, caches, self.inputs, b, None, prefill, pages)
+
+    def host_buffer(self) -> torch.Tensor:
+        """A pinned host buffer with the staging buffer's layout."""
+        return torch.empty(self.staging.shape, dtype=torch.uint8).pin_memory()
+
+    def pack(self, host_inputs: dict, buffer: torch.Tensor) -> torch.Tensor:
+        """Copy a step's host tensors (same names, dtypes and shapes as the
+        captured inputs) into ``buffer`` (a ``host_buffer()``)."""
+        for name, o, nb, dt, shp in self._layout:
+            t = host_inputs[name]
+            if t.dtype != dt or tuple(t.shape) != shp:
+                raise ValueError(f"{name} must be {dt} {shp}")
+            buffer[o:o + nb].view(dt).view(shp).copy_(t)
+        return buffer
+
+    def replay(self):
+        """Run the captured step on the current stream."""
+        self.graph.replay()
+        return self.out
+
+    def replay_from(self, buffer: torch.Tensor):
+        """One host-to-device copy of a packed step, then the replay."""
+        self.staging.copy_(buffer, non_blocking=True)
+        return self.replay()

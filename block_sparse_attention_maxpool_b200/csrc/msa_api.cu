@@ -198,9 +198,10 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q,
                              static_cast<int64_t>(n_q) * sh->n_q_heads, 16)) != MSA_OK)
       return st;
-    static std::atomic<uint64_t> tc_smem_done{0};
-    if ((st = ensure_smem(msa::pattn::sparse_attn_prefill_tc_kernel, msa::pattn::Layout::kBytes, tc_smem_done)) !=
-        MSA_OK)
+    const auto pkernel = pg.table != nullptr ? msa::pattn::sparse_attn_prefill_tc_kernel<true>
+                                             : msa::pattn::sparse_attn_prefill_tc_kernel<false>;
+    static std::atomic<uint64_t> tc_smem_done[2] = {0, 0};
+    if ((st = ensure_smem(pkernel, msa::pattn::Layout::kBytes, tc_smem_done[pg.table != nullptr])) != MSA_OK)
       return st;
     msa::pattn::Params Q;
     Q.sel = sel;
@@ -214,7 +215,8 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     Q.scale_log2 = softmax_scale * 1.4426950408889634f;
     Q.pages = pg;
     const int64_t grid = std::min<int64_t>(sms, n_pairs);
-    launch(msa::pattn::sparse_attn_prefill_tc_kernel, dim3(static_cast<unsigned>(grid)), dim3(msa::pattn::kThreads), msa::pattn::Layout::kBytes, s, tm_q, tm_k, tm_v, Q);
+    launch(pkernel, dim3(static_cast<unsigned>(grid)), dim3(msa::pattn::kThreads), msa::pattn::Layout::kBytes, s, tm_q,
+           tm_k, tm_v, Q);
     return cuda_status(cudaGetLastError());
   }
   // decode: persistent stream-K grid over (pair, selected block) units, or

@@ -72,16 +72,18 @@ struct Params {
 };
 
 struct PairInfo {
-  int qi, g, p, nb;
-  int blocks[kTopK];         // selected visible blocks, ascending
-  int rows[kTopK];           // first cache row of each
+  int qi, g, p, s, nb;
+  int blocks[kTopK];         // selected visible blocks (with a page, when paged), ascending
 };
 
-// Pair t -> (group, query); the selected blocks that are visible.
+// Pair t -> (group, query); the selected blocks that are visible (and, for
+// a paged cache, mapped to a page).
+template <bool kPaged>
 __device__ __forceinline__ void pair_info(const Params& P, int t, PairInfo& I, bool report) {
   I.g = t / P.n_q;
   I.qi = t - I.g * P.n_q;
   const int s = P.q_stream[I.qi];
+  I.s = s;
   I.p = P.q_pos[I.qi];
   I.nb = 0;
   if (s < 0 || s >= P.n_streams || I.p < 0 || I.p >= P.capacity) {
@@ -98,27 +100,29 @@ __device__ __forceinline__ void pair_info(const Params& P, int t, PairInfo& I, b
       if (report) raise_error(MSA_DEVERR_SEL_RANGE);
       continue;
     }
-    const long long row = kv_block_row(P.pages, s, I.g, b, P.G, P.capacity);
-    if (row < 0) {
+    if (kPaged && kv_block_row(P.pages, s, I.g, b, P.G, P.capacity) < 0) {
       if (report) raise_error(MSA_DEVERR_PAGE_RANGE);
       continue;
     }
-    I.rows[I.nb] = static_cast<int>(row);   // the host checks that every row fits 31 bits
     I.blocks[I.nb++] = b;
   }
 }
 
 // Next pair (from *t on, stride gridDim.x) that has at least one block to
 // attend; false at the end of this CTA's pairs.
+template <bool kPaged>
 __device__ __forceinline__ bool next_pair(const Params& P, int n_pairs, int& t, PairInfo& I) {
   while (t < n_pairs) {
-    pair_info(P, t, I, false);
+    pair_info<kPaged>(P, t, I, false);
     t += gridDim.x;
     if (I.nb > 0) return true;
   }
   return false;
 }
 
+// kPaged: K/V are page pools addressed through P.pages (a separate
+// instantiation, so the contiguous path carries no page-table code).
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                                   const __grid_constant__ CUtensorMap tm_v, const Params P) {
@@ -193,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t = blockIdx.x, u = 0, ring = 0;
       bool ok = true;
       PairInfo I;
-      while (ok && next_pair(P, n_pairs, t, I)) {
+      while (ok && next_pair<kPaged>(P, n_pairs, t, I)) {
         if (is_k) {
           const int slot = u & 1;
           if (u >= 2) ok = mbar_wait(&q_empty[slot], ((u >> 1) - 1) & 1);
@@ -210,7 +214,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0) ok = mbar_wait(&rempty[st], (use - 1) & 1);
           if (!ok) break;
           uint8_t* dst = rbase + st * kTile;
-          const int row = I.rows[j];
+          // the host checks that every row fits 31 bits
+          const int row = kPaged ? static_cast<int>(kv_block_row(P.pages, I.s, I.g, I.blocks[j], P.G, P.capacity))
+                                 : (I.s * P.G + I.g) * P.capacity + I.blocks[j] * kBlock;
           mbar_arrive_expect_tx(&rfull[st], kTile);
           tma_load_2d(dst, map, 0, row, &rfull[st]);
           tma_load_2d(dst + kHalf, map, 64, row, &rfull[st]);
@@ -229,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t = blockIdx.x, u = 0, ring = 0;
       bool ok = true;
       PairInfo I;
-      while (ok && next_pair(P, n_pairs, t, I)) {
+      while (ok && next_pair<kPaged>(P, n_pairs, t, I)) {
         const int slot = u & 1;
         if (u >= 2) ok = mbar_wait(&slot_free[slot], ((u >> 1) - 1) & 1);
         if (ok) ok = mbar_wait(&q_full[slot], (u >> 1) & 1);
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pcnt[2] = {0, 0};
       bool ok = true;
       PairInfo I;
-      while (ok && next_pair(P, n_pairs, t, I)) {
+      while (ok && next_pair<kPaged>(P, n_pairs, t, I)) {
         const int sl = u & 1;
         const uint32_t d = tmem_base + static_cast<uint32_t>(sl * 256);
         for (int j = 0; j < I.nb && ok; ++j) {
@@ -304,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     PairInfo I;
     for (int t = blockIdx.x; t < n_pairs; t += gridDim.x) {
-      pair_info(P, t, I, q4 == 0 && lane == 0);
+      pair_info<kPaged>(P, t, I, q4 == 0 && lane == 0);
       __nv_bfloat16* out = P.out + (static_cast<size_t>(I.qi) * P.G * kHpg + I.g * kHpg) * kD + row;
       if (I.nb == 0) {
 #pragma unroll
