@@ -14,6 +14,7 @@
 #include "msa_append.cuh"
 #include "msa_attn_decode_sk.cuh"
 #include "msa_attn_prefill_tc.cuh"
+#include "msa_attn_prefill_union.cuh"
 #include "msa_common.cuh"
 #include "msa_decode_fused.cuh"
 #include "msa_dsa_scores.cuh"
@@ -198,6 +199,29 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q,
                              static_cast<int64_t>(n_q) * sh->n_q_heads, 16)) != MSA_OK)
       return st;
+    if (pg.table == nullptr) {
+      // contiguous caches: tiles of 8 queries over the union of their blocks
+      static std::atomic<uint64_t> u_smem_done{0};
+      if ((st = ensure_smem(msa::uattn::sparse_attn_prefill_union_kernel, msa::uattn::Layout::kBytes,
+                            u_smem_done)) != MSA_OK)
+        return st;
+      msa::uattn::Params U;
+      U.sel = sel;
+      U.q_stream = q_stream;
+      U.q_pos = q_pos;
+      U.out = reinterpret_cast<__nv_bfloat16*>(out);
+      U.n_q = n_q;
+      U.G = G;
+      U.n_streams = sh->n_streams;
+      U.capacity = sh->capacity;
+      U.n_tiles = (n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ;
+      U.scale_log2 = softmax_scale * 1.4426950408889634f;
+      const int64_t tasks = static_cast<int64_t>(G) * U.n_tiles;
+      const int64_t ugrid = std::min<int64_t>(sms, tasks);
+      launch(msa::uattn::sparse_attn_prefill_union_kernel, dim3(static_cast<unsigned>(ugrid)),
+             dim3(msa::uattn::kThreads), msa::uattn::Layout::kBytes, s, tm_q, tm_k, tm_v, U);
+      return cuda_status(cudaGetLastError());
+    }
     const auto pkernel = pg.table != nullptr ? msa::pattn::sparse_attn_prefill_tc_kernel<true>
                                              : msa::pattn::sparse_attn_prefill_tc_kernel<false>;
     static std::atomic<uint64_t> tc_smem_done[2] = {0, 0};

@@ -1,0 +1,562 @@
+// Block-sparse GQA attention for prefill batches: query tiles over the union
+// of their selected blocks (tcgen05, flash-style).
+//
+// MSA pull request "Add MiniMax-M3 (MSA) support", section "Overview": each
+// query attends to the rows of its selected blocks only, shared by the 16
+// heads of its GQA group; the token-level causal mask applies inside the
+// local block.
+//
+// A tile is 8 consecutive queries of one group: 8 x 16 = 128 query-head
+// rows, the M dimension of every MMA.  A planner warp merges the 8 queries'
+// sorted selections into the tile's union of blocks, each with an 8-bit mask
+// of the queries that selected it (queries of different streams form
+// separate segments of the union).  For every block b of the union:
+//   S = Q . K_b^T          M=128 rows, N=128 keys, K=128 dims (TMEM, f32)
+//   P = exp2(S - m)        masked: a row keeps only keys of blocks its query
+//                          selected and j <= its position; one thread per
+//                          row; bf16, written back over S in tensor memory
+//   O += P . V_b           M=128 rows, N=128 dims, K=128 keys: A (P) from
+//                          tensor memory, B (V) from shared memory
+// with an online softmax per row whose reference max m is raised (and O
+// rescaled in tensor memory) only when a block's max exceeds it by more than
+// 2^8, so P stays below 256 and the rescale is rare.  Each K and V block is
+// read once per tile instead of once per (query, group).
+//
+// Pipelining: two S buffers in tensor memory, so the softmax of block b+1
+// runs while the tensor cores do P . V of block b; a warp whose two queries
+// did not select block b writes zeros without computing exponentials.  The Q
+// tile is released after the tile's last S MMA, so the next tile's Q loads
+// while the last blocks' softmax runs.
+//
+// Warp roles: 0 K loader (and the Q tile), 1 MMA issuer, 2 V loader,
+// 3 planner (one tile ahead), 4-7 softmax and output (one TMEM lane quarter
+// each).  Shared memory: Q 32 KB, K ring 3 x 32 KB, V ring 2 x 32 KB, two
+// plans.  Tensor memory: two S/P buffers and O (384 of 512 columns).
+#pragma once
+
+#include "msa_common.cuh"
+
+namespace msa {
+namespace uattn {
+
+constexpr int kD = 128;
+constexpr int kBlock = 128;
+constexpr int kHpg = 16;
+constexpr int kTopK = 16;
+constexpr int kTileQ = 8;                           // queries per tile
+constexpr int kRows = kTileQ * kHpg;                // 128 MMA rows
+constexpr int kMaxUnion = kTileQ * kTopK;           // 128 blocks at most
+constexpr uint32_t kHalf = 128 * 128;               // [128 rows][64 bf16] = 16 KB
+constexpr uint32_t kTile = 2 * kHalf;               // 32 KB
+constexpr int kKRing = 3;
+constexpr int kVRing = 2;
+constexpr int kSBufs = 2;                           // S/P buffers in tensor memory
+constexpr int kThreads = 8 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCol = 0;                       // S/P buffer i: columns 128 i .. 128 i + 127
+constexpr uint32_t kOCol = 128 * kSBufs;            // O: 128 columns after the S buffers
+constexpr uint32_t kIdescS = umma_idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescPV = umma_idesc_bf16_f32(128, 128, false, true);
+constexpr float kRescale = 8.f;                     // raise the reference max past this (log2 units)
+static_assert(kOCol + 128 <= kTmemCols, "tensor memory budget");
+
+struct Plan {
+  int n;                          // blocks in the union
+  int pos[kTileQ];                // query positions (-1: no query / invalid)
+  int seg_stream[kTileQ];         // stream of the segment whose id is this query index
+  uint8_t seg_rows[kTileQ];       // queries of that segment
+  int blocks[kMaxUnion];          // ascending within each segment
+  uint8_t masks[kMaxUnion];       // queries that selected the block
+  uint8_t segs[kMaxUnion];        // segment id (index of its first query)
+};
+
+struct Layout {
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKOff = kQOff + kTile;
+  static constexpr uint32_t kVOff = kKOff + kKRing * kTile;
+  static constexpr uint32_t kPlanOff = kVOff + kVRing * kTile;
+  static constexpr uint32_t kPlanBytes = (sizeof(Plan) + 127) / 128 * 128;
+  static constexpr uint32_t kKeysOff = kPlanOff + 2 * kPlanBytes;     // planner scratch: 128 keys
+  static constexpr uint32_t kBarOff = kKeysOff + kMaxUnion * 4;
+  static constexpr uint32_t kEnd = kBarOff + 40 * 8;
+  static constexpr size_t kBytes = kEnd + 1024;
+};
+static_assert(Layout::kBytes <= 232448, "shared memory budget");
+
+struct Params {
+  const int32_t* sel;        // [n_q][G][16]
+  const int32_t* q_stream;
+  const int32_t* q_pos;
+  __nv_bfloat16* out;        // [n_q][Hq][D]
+  int n_q, G, n_streams, capacity, n_tiles;
+  float scale_log2;
+};
+
+// Barrier slots (uint64 each, from Layout::kBarOff).
+struct Bars {
+  uint64_t *plan_full, *plan_empty, *q_full, *q_empty, *kfull, *kempty, *vfull, *vempty;
+  uint64_t *s_full, *p_full, *pv_done, *o_empty, *mma_done;
+  uint32_t* tmem_slot;
+  __device__ explicit Bars(uint8_t* smem) {
+    uint64_t* b = reinterpret_cast<uint64_t*>(smem + Layout::kBarOff);
+    plan_full = b;                 // [2]
+    plan_empty = plan_full + 2;    // [2]
+    q_full = plan_empty + 2;
+    q_empty = q_full + 1;
+    kfull = q_empty + 1;           // [kKRing]
+    kempty = kfull + kKRing;
+    vfull = kempty + kKRing;       // [kVRing]
+    vempty = vfull + kVRing;
+    s_full = vempty + kVRing;      // [kSBufs]: S of the buffer's block is in tensor memory
+    p_full = s_full + kSBufs;      // [kSBufs]: its P is written (4 softmax warps)
+    pv_done = p_full + kSBufs;     // [kSBufs]: its P . V finished (buffer free, O updated)
+    o_empty = pv_done + kSBufs;
+    mma_done = o_empty + 1;
+    tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  }
+};
+static_assert(6 + 2 * kKRing + 2 * kVRing + 3 * kSBufs + 2 + 1 <= 40, "barrier slots");
+
+// exp2 on the special-function unit (ex2.approx.ftz: ~2 ulp; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ Plan& plan_at(uint8_t* smem, int slot) {
+  return *reinterpret_cast<Plan*>(smem + Layout::kPlanOff + slot * Layout::kPlanBytes);
+}
+
+// Tile t -> (group, first query).  Group-major, so the CTAs running at the
+// same time work on nearby queries of one group and share its blocks in L2.
+__device__ __forceinline__ void tile_coords(const Params& P, int t, int& g, int& q0) {
+  g = t / P.n_tiles;
+  q0 = (t - g * P.n_tiles) * kTileQ;
+}
+
+// The planner warp: union of the tile's selections, by segment, into `pl`.
+__device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, uint32_t* keys, int lane) {
+  int g, q0;
+  tile_coords(P, t, g, q0);
+  // per query: position (or -1) and stream
+  int pos = -1, stream = -1;
+  if (lane < kTileQ) {
+    const int qi = q0 + lane;
+    if (qi < P.n_q) {
+      const int s = P.q_stream[qi];
+      const int p = P.q_pos[qi];
+      if (s >= 0 && s < P.n_streams && p >= 0 && p < P.capacity) {
+        pos = p;
+        stream = s;
+      } else if (g == 0) {
+        raise_error(MSA_DEVERR_QUERY_RANGE);
+      }
+    }
+  }
+  // segment id: the first query of the tile with the same stream
+  int seg = -1;
+#pragma unroll
+  for (int q = 0; q < kTileQ; ++q) {
+    const int sq = __shfl_sync(0xffffffffu, stream, q);
+    if (seg < 0 && stream >= 0 && sq == stream) seg = q;
+  }
+  if (lane < kTileQ) {
+    pl.pos[lane] = pos;
+    pl.seg_stream[lane] = stream;
+  }
+  uint32_t rows = 0;
+#pragma unroll
+  for (int q = 0; q < kTileQ; ++q) {
+    const int sq = __shfl_sync(0xffffffffu, seg, q);
+    if (sq == lane) rows |= 1u << q;
+  }
+  if (lane < kTileQ) pl.seg_rows[lane] = static_cast<uint8_t>(rows);
+  // the 128 selection entries as sortable keys (segment << 24 | block); past-the-end: ~0
+#pragma unroll
+  for (int m = 0; m < kMaxUnion / 32; ++m) {
+    const int e = lane + 32 * m;
+    const int q = e / kTopK;
+    const int qpos = __shfl_sync(0xffffffffu, pos, q);
+    const int qseg = __shfl_sync(0xffffffffu, seg, q);
+    uint32_t key = 0xffffffffu;
+    if (qpos >= 0) {
+      const int b = __ldg(P.sel + (static_cast<size_t>(q0 + q) * P.G + g) * kTopK + (e % kTopK));
+      if (b >= 0 && b <= qpos / kBlock) {
+        key = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
+      } else if (b > qpos / kBlock) {
+        raise_error(MSA_DEVERR_SEL_RANGE);
+      }
+    }
+    keys[e] = key;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    // 8-way merge of the per-query lists (each ascending, ~0 entries last)
+    int head[kTileQ];
+#pragma unroll
+    for (int q = 0; q < kTileQ; ++q) head[q] = 0;
+    int n = 0;
+    uint32_t last = 0xffffffffu;
+    for (int step = 0; step < kMaxUnion; ++step) {
+      uint32_t best = 0xffffffffu;
+      int bq = -1;
+#pragma unroll
+      for (int q = 0; q < kTileQ; ++q) {
+        const uint32_t k = head[q] < kTopK ? keys[q * kTopK + head[q]] : 0xffffffffu;
+        if (k < best) {
+          best = k;
+          bq = q;
+        }
+      }
+      if (bq < 0) break;
+      ++head[bq];
+      if (best != last) {
+        pl.blocks[n] = static_cast<int>(best & 0xffffffu);
+        pl.segs[n] = static_cast<uint8_t>(best >> 24);
+        pl.masks[n] = static_cast<uint8_t>(1u << bq);
+        ++n;
+        last = best;
+      } else {
+        pl.masks[n - 1] |= static_cast<uint8_t>(1u << bq);
+      }
+    }
+    pl.n = n;
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_prefill_union_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                                     const __grid_constant__ CUtensorMap tm_v, const Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Bars B(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tasks = P.G * P.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.plan_full[i], 1);
+      mbar_init(&B.plan_empty[i], 7);       // K loader, V loader, MMA, 4 softmax warps
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&B.s_full[i], 1);
+      mbar_init(&B.p_full[i], 4);
+      mbar_init(&B.pv_done[i], 1);
+    }
+    mbar_init(B.q_full, 1);
+    mbar_init(B.q_empty, 1);
+    for (int i = 0; i < kKRing; ++i) {
+      mbar_init(&B.kfull[i], 1);
+      mbar_init(&B.kempty[i], 1);
+    }
+    for (int i = 0; i < kVRing; ++i) {
+      mbar_init(&B.vfull[i], 1);
+      mbar_init(&B.vempty[i], 1);
+    }
+    mbar_init(B.o_empty, 4);
+    mbar_init(B.mma_done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(B.tmem_slot, kTmemCols);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *B.tmem_slot;
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 3) {
+    // ------------------------------ planner ------------------------------------
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + Layout::kKeysOff);
+    int tc = 0;
+    for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++tc) {
+      const int slot = tc & 1;
+      bool ok = true;
+      if (tc >= 2) ok = mbar_wait(&B.plan_empty[slot], ((tc >> 1) - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      build_plan(P, t, plan_at(smem, slot), keys, lane);
+      if (lane == 0) mbar_arrive(&B.plan_full[slot]);
+    }
+  } else if (warp == 0 || warp == 2) {
+    // ---------------- loaders: warp 0 the Q tile and K blocks, warp 2 V blocks ----
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      uint64_t* rfull = is_k ? B.kfull : B.vfull;
+      uint64_t* rempty = is_k ? B.kempty : B.vempty;
+      uint8_t* rbase = smem + (is_k ? Layout::kKOff : Layout::kVOff);
+      const int ring_n = is_k ? kKRing : kVRing;
+      int tc = 0, ring = 0, q_use = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+        const int slot = tc & 1;
+        ok = mbar_wait(&B.plan_full[slot], (tc >> 1) & 1);
+        if (!ok) break;
+        const Plan& pl = plan_at(smem, slot);
+        int g, q0;
+        tile_coords(P, t, g, q0);
+        if (is_k && pl.n > 0) {
+          // the previous tile's S MMAs have finished with the Q tile
+          if (q_use > 0) ok = mbar_wait(B.q_empty, (q_use - 1) & 1);
+          if (!ok) break;
+          int nq = 0;
+          for (int q = 0; q < kTileQ; ++q) nq += q0 + q < P.n_q ? 1 : 0;
+          mbar_arrive_expect_tx(B.q_full, static_cast<uint32_t>(nq) * 2 * (kHpg * 128));
+          for (int q = 0; q < nq; ++q) {
+            const int row = (q0 + q) * (P.G * kHpg) + g * kHpg;      // q viewed as [n_q * Hq][128]
+            uint8_t* dst = smem + Layout::kQOff + q * (kHpg * 128);
+            tma_load_2d(dst, &tm_q, 0, row, B.q_full);
+            tma_load_2d(dst + kHalf, &tm_q, 64, row, B.q_full);
+          }
+          ++q_use;
+        }
+        for (int j = 0; j < pl.n && ok; ++j, ++ring) {
+          const int st = ring % ring_n;
+          const int use = ring / ring_n;
+          if (use > 0) ok = mbar_wait(&rempty[st], (use - 1) & 1);
+          if (!ok) break;
+          const int s = pl.seg_stream[pl.segs[j]];
+          const int row = (s * P.G + g) * P.capacity + pl.blocks[j] * kBlock;
+          uint8_t* dst = rbase + st * kTile;
+          mbar_arrive_expect_tx(&rfull[st], kTile);
+          tma_load_2d(dst, map, 0, row, &rfull[st]);
+          tma_load_2d(dst + kHalf, map, 64, row, &rfull[st]);
+        }
+        mbar_arrive(&B.plan_empty[slot]);
+      }
+      // no copy may still be landing when the CTA exits
+      for (int j = max(0, ring - ring_n); j < ring; ++j) mbar_wait(&rfull[j % ring_n], (j / ring_n) & 1);
+      if (is_k && q_use > 0) mbar_wait(B.q_full, (q_use - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer -----------------------------------
+    if (lane == 0) {
+      const uint32_t q_base = smem_addr(smem + Layout::kQOff);
+      const uint32_t k_base = smem_addr(smem + Layout::kKOff);
+      const uint32_t v_base = smem_addr(smem + Layout::kVOff);
+      int tc = 0, kr = 0, vr = 0, blk = 0, segs_done = 0, q_use = 0;
+      bool ok = true;
+      // O (+)= P . V for global block `b` (union position j of the current plan)
+      auto pv = [&](const Plan& pl, int j, int b) {
+        const bool seg_first = j == 0 || pl.segs[j] != pl.segs[j - 1];
+        const int sb = b % kSBufs;
+        if (ok) ok = mbar_wait(&B.p_full[sb], (b / kSBufs) & 1);
+        if (ok && seg_first && segs_done > 0) ok = mbar_wait(B.o_empty, (segs_done - 1) & 1);
+        const int st = vr % kVRing;
+        if (ok) ok = mbar_wait(&B.vfull[st], (vr / kVRing) & 1);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t vb = v_base + st * kTile;
+        const uint32_t pa = tmem_base + kSCol + sb * 128;      // P: 64 columns of bf16 pairs
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ts(tmem_base + kOCol, pa + kk * 8, umma_desc_sw128_mn(vb + kk * 2048, kHalf), kIdescPV,
+                      (seg_first && kk == 0) ? 0u : 1u);
+        umma_commit(&B.vempty[st]);
+        umma_commit(&B.pv_done[sb]);
+        ++vr;
+        if (seg_first) ++segs_done;
+      };
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+        const int slot = tc & 1;
+        ok = mbar_wait(&B.plan_full[slot], (tc >> 1) & 1);
+        if (!ok) break;
+        const Plan& pl = plan_at(smem, slot);
+        if (pl.n > 0) {
+          ok = mbar_wait(B.q_full, q_use & 1);
+          ++q_use;
+          tc_fence_after();
+          for (int j = 0; j < pl.n && ok; ++j) {
+            const int b = blk + j;
+            const int kst = kr % kKRing;
+            const int sb = b % kSBufs;
+            ok = mbar_wait(&B.kfull[kst], (kr / kKRing) & 1);
+            // the buffer's previous block has finished its P . V
+            if (ok && b >= kSBufs) ok = mbar_wait(&B.pv_done[sb], ((b / kSBufs) - 1) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t kb = k_base + kst * kTile;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+              umma_f16_ss(tmem_base + kSCol + sb * 128, umma_desc_sw128(q_base + off), umma_desc_sw128(kb + off),
+                          kIdescS, kk != 0);
+            }
+            umma_commit(&B.kempty[kst]);
+            umma_commit(&B.s_full[sb]);
+            if (j == pl.n - 1) umma_commit(B.q_empty);         // the tile's last use of Q
+            ++kr;
+            if (j > 0) pv(pl, j - 1, b - 1);
+          }
+          if (ok) pv(pl, pl.n - 1, blk + pl.n - 1);
+          blk += pl.n;
+        }
+        mbar_arrive(&B.plan_empty[slot]);
+      }
+      umma_commit(B.mma_done);
+      mbar_wait(B.mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    // ---------------- softmax and output: one thread per (query, head) row --------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;             // TMEM lane = MMA row
+    const int q = r / kHpg;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    int tc = 0, blk = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++tc) {
+      const int slot = tc & 1;
+      if (ok) ok = mbar_wait(&B.plan_full[slot], (tc >> 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const Plan& pl = plan_at(smem, slot);
+      int g, q0;
+      tile_coords(P, t, g, q0);
+      const int qi = q0 + q;
+      const int pq = pl.pos[q];
+      bool wrote = false;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < pl.n && ok; ++j) {
+        const int b = blk + j;
+        const int seg = pl.segs[j];
+        const bool seg_first = j == 0 || pl.segs[j - 1] != seg;
+        const bool seg_last = j == pl.n - 1 || pl.segs[j + 1] != seg;
+        if (seg_first) {
+          m_ref = -INFINITY;
+          l = 0.f;
+        }
+        const int sb = b % kSBufs;
+        const uint32_t sbuf = tmem_base + lane_addr + kSCol + sb * 128;
+        ok = mbar_wait(&B.s_full[sb], (b / kSBufs) & 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        float s[kBlock];
+        {
+          float v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(sbuf, v0);
+          tmem_ld32(sbuf + 32, v1);
+          tmem_ld32(sbuf + 64, v2);
+          tmem_ld32(sbuf + 96, v3);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            s[i] = v0[i];
+            s[32 + i] = v1[i];
+            s[64 + i] = v2[i];
+            s[96 + i] = v3[i];
+          }
+        }
+        // mask: the row's query selected this block, and keys j <= its position
+        const bool mine = ((pl.masks[j] >> q) & 1) != 0 && pq >= 0;
+        const int jmax = mine ? pq - pl.blocks[j] * kBlock : -1;       // last visible key in the block
+        float mb = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBlock; ++c) {
+          s[c] = c <= jmax ? s[c] * P.scale_log2 : -INFINITY;
+          mb = fmaxf(mb, s[c]);
+        }
+        const bool raise = mb > m_ref + kRescale;
+        const bool rescale = raise && !seg_first && m_ref != -INFINITY;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O of the rows that raise their max is rescaled once the previous
+          // block's P . V (in the other buffer) has finished
+          const int pb = b - 1;
+          ok = mbar_wait(&B.pv_done[pb % kSBufs], (pb / kSBufs) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const float f = rescale ? ex2_approx(m_ref - mb) : 1.f;
+          l *= f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tmem_ld32(tmem_base + lane_addr + kOCol + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= f;
+            tmem_st32(tmem_base + lane_addr + kOCol + c * 32, v);
+          }
+        }
+        if (raise) m_ref = mb;
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+        // P = exp2(s - m_ref) as bf16 pairs over the first 64 columns of the buffer
+        if (__any_sync(0xffffffffu, mine)) {
+          float rs = 0.f;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float a = ex2_approx(s[h * 64 + 2 * i] - mr);
+              const float c2 = ex2_approx(s[h * 64 + 2 * i + 1] - mr);
+              rs += a + c2;
+              pk[i] = __uint_as_float(pack_bf16(a, c2));
+            }
+            tmem_st32(sbuf + h * 32, pk);
+          }
+          l += rs;
+        } else {
+          float z[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) z[i] = 0.f;
+          tmem_st32(sbuf, z);
+          tmem_st32(sbuf + 32, z);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.p_full[sb]);
+        if (seg_last) {
+          // O of the segment is complete once this block's P . V has finished
+          ok = mbar_wait(&B.pv_done[sb], (b / kSBufs) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const bool row_here = ((pl.seg_rows[seg] >> q) & 1) != 0 && pq >= 0;
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          __nv_bfloat16* dst = P.out + (static_cast<size_t>(qi) * (P.G * kHpg) + g * kHpg + (r % kHpg)) * kD;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tmem_ld32(tmem_base + lane_addr + kOCol + c * 32, v);
+            tmem_ld_wait();
+            if (row_here) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                *reinterpret_cast<uint4*>(dst + c * 32 + i) =
+                    make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv), pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
+                               pack_bf16(v[i + 4] * inv, v[i + 5] * inv), pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
+              }
+            }
+          }
+          if (row_here) wrote = true;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B.o_empty);
+        }
+      }
+      if (!ok) break;
+      blk += pl.n;
+      // queries with nothing to attend (invalid, or no visible selected block): zeros
+      if (!wrote && qi < P.n_q) {
+        __nv_bfloat16* dst = P.out + (static_cast<size_t>(qi) * (P.G * kHpg) + g * kHpg + (r % kHpg)) * kD;
+#pragma unroll
+        for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(dst + i) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.plan_empty[slot]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace uattn
+}  // namespace msa

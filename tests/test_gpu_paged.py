@@ -68,10 +68,17 @@ def _contiguous_vs_paged(w, seed, prefill):
     pages = msa.Pages(lay.block_table.cuda(), lay.n_pages)
     out_p, sel_p, nsel_p, bs_p, err_p = PT.run_step(shape, dp, prefill, pages)
     assert err_c == 0 and err_p == 0
-    # same arithmetic on the same rows: bit-identical results
+    # same arithmetic on the same rows: bit-identical scores and selection;
+    # decode attention runs the same kernel on both layouts (bit-identical),
+    # contiguous prefill runs the union-tile kernel and paged prefill the
+    # per-pair kernel, whose accumulation orders differ (both are checked
+    # against the oracle elsewhere): compare within the attention tolerance
     assert torch.equal(bs_c, bs_p)
     assert torch.equal(sel_c, sel_p) and torch.equal(nsel_c, nsel_p)
-    assert torch.equal(out_c, out_p)
+    if prefill:
+        PT.check_attention(out_p.cpu(), out_c.cpu().double())
+    else:
+        assert torch.equal(out_c, out_p)
 
 
 def test_paged_equals_contiguous_bitwise_decode():
