@@ -22,16 +22,17 @@
 // 2^8, so P stays below 256 and the rescale is rare.  Each K and V block is
 // read once per tile instead of once per (query, group).
 //
-// Pipelining: two S buffers in tensor memory, so the softmax of block b+1
-// runs while the tensor cores do P . V of block b; a warp whose two queries
-// did not select block b writes zeros without computing exponentials.  The Q
+// Pipelining: three S/P buffers in tensor memory and S MMAs issued two
+// blocks ahead of P . V, so the softmax warps run up to two blocks apart
+// and overlap P . V; a warp whose two queries did not select a block writes
+// zeros without computing exponentials.  The Q
 // tile is released after the tile's last S MMA, so the next tile's Q loads
 // while the last blocks' softmax runs.
 //
 // Warp roles: 0 K loader (and the Q tile), 1 MMA issuer, 2 V loader,
 // 3 planner (one tile ahead), 4-7 softmax and output (one TMEM lane quarter
 // each).  Shared memory: Q 32 KB, K ring 3 x 32 KB, V ring 2 x 32 KB, two
-// plans.  Tensor memory: two S/P buffers and O (384 of 512 columns).
+// plans.  Tensor memory: three S/P buffers and O (all 512 columns).
 #pragma once
 
 #include "msa_common.cuh"
@@ -50,7 +51,8 @@ constexpr uint32_t kHalf = 128 * 128;               // [128 rows][64 bf16] = 16 
 constexpr uint32_t kTile = 2 * kHalf;               // 32 KB
 constexpr int kKRing = 3;
 constexpr int kVRing = 2;
-constexpr int kSBufs = 2;                           // S/P buffers in tensor memory
+constexpr int kSBufs = 3;                           // S/P buffers in tensor memory
+constexpr int kLag = kSBufs - 1;                    // S MMAs run this many blocks ahead of P . V
 constexpr int kThreads = 8 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 0;                       // S/P buffer i: columns 128 i .. 128 i + 127
@@ -389,9 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(&B.s_full[sb]);
             if (j == pl.n - 1) umma_commit(B.q_empty);         // the tile's last use of Q
             ++kr;
-            if (j > 0) pv(pl, j - 1, b - 1);
+            if (j >= kLag) pv(pl, j - kLag, b - kLag);
           }
-          if (ok) pv(pl, pl.n - 1, blk + pl.n - 1);
+          for (int j = max(0, pl.n - kLag); j < pl.n && ok; ++j) pv(pl, j, blk + j);
           blk += pl.n;
         }
         mbar_arrive(&B.plan_empty[slot]);
@@ -450,15 +452,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             s[96 + i] = v3[i];
           }
         }
-        // mask: the row's query selected this block, and keys j <= its position
+        // mask: the row's query selected this block (else its P row is
+        // exp2(-inf) = 0), and keys j <= its position (only its local block
+        // is cut)
         const bool mine = ((pl.masks[j] >> q) & 1) != 0 && pq >= 0;
         const int jmax = mine ? pq - pl.blocks[j] * kBlock : -1;       // last visible key in the block
+        if (__any_sync(0xffffffffu, mine && jmax < kBlock - 1)) {
+#pragma unroll
+          for (int c = 0; c < kBlock; ++c) s[c] = c <= jmax ? s[c] : -INFINITY;
+        }
         float mb = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kBlock; ++c) {
-          s[c] = c <= jmax ? s[c] * P.scale_log2 : -INFINITY;
-          mb = fmaxf(mb, s[c]);
-        }
+        for (int c = 0; c < kBlock; ++c) mb = fmaxf(mb, s[c]);
+        mb = mine ? mb * P.scale_log2 : -INFINITY;                       // max of the scaled scores
         const bool raise = mb > m_ref + kRescale;
         const bool rescale = raise && !seg_first && m_ref != -INFINITY;
         if (__any_sync(0xffffffffu, rescale)) {
@@ -482,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (raise) m_ref = mb;
-        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+        const float neg_m = mine ? -m_ref : -INFINITY;
         // P = exp2(s - m_ref) as bf16 pairs over the first 64 columns of the buffer
         if (__any_sync(0xffffffffu, mine)) {
           float rs = 0.f;
@@ -491,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float a = ex2_approx(s[h * 64 + 2 * i] - mr);
-              const float c2 = ex2_approx(s[h * 64 + 2 * i + 1] - mr);
+              const float a = ex2_approx(fmaf(s[h * 64 + 2 * i], P.scale_log2, neg_m));
+              const float c2 = ex2_approx(fmaf(s[h * 64 + 2 * i + 1], P.scale_log2, neg_m));
               rs += a + c2;
               pk[i] = __uint_as_float(pack_bf16(a, c2));
             }
