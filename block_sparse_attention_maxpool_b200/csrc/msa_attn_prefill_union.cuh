@@ -25,7 +25,7 @@
 // Pipelining: three S/P buffers in tensor memory and S MMAs issued two
 // blocks ahead of P . V, so the softmax warps run up to two blocks apart
 // and overlap P . V; a warp whose two queries did not select a block writes
-// zeros without computing exponentials.  The Q
+// zeros without reading S or computing exponentials.  The Q
 // tile is released after the tile's last S MMA, so the next tile's Q loads
 // while the last blocks' softmax runs.
 //
@@ -436,8 +436,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
+        // mask: the row's query selected this block (else its P row is
+        // exp2(-inf) = 0), and keys j <= its position (only its local block
+        // is cut)
+        const bool mine = ((pl.masks[j] >> q) & 1) != 0 && pq >= 0;
+        const int jmax = mine ? pq - pl.blocks[j] * kBlock : -1;       // last visible key in the block
+        const bool active = __any_sync(0xffffffffu, mine);
         float s[kBlock];
-        {
+        if (active) {
           float v0[32], v1[32], v2[32], v3[32];
           tmem_ld32(sbuf, v0);
           tmem_ld32(sbuf + 32, v1);
@@ -452,19 +458,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             s[96 + i] = v3[i];
           }
         }
-        // mask: the row's query selected this block (else its P row is
-        // exp2(-inf) = 0), and keys j <= its position (only its local block
-        // is cut)
-        const bool mine = ((pl.masks[j] >> q) & 1) != 0 && pq >= 0;
-        const int jmax = mine ? pq - pl.blocks[j] * kBlock : -1;       // last visible key in the block
-        if (__any_sync(0xffffffffu, mine && jmax < kBlock - 1)) {
-#pragma unroll
-          for (int c = 0; c < kBlock; ++c) s[c] = c <= jmax ? s[c] : -INFINITY;
-        }
         float mb = -INFINITY;
+        if (active) {
+          if (__any_sync(0xffffffffu, mine && jmax < kBlock - 1)) {
 #pragma unroll
-        for (int c = 0; c < kBlock; ++c) mb = fmaxf(mb, s[c]);
-        mb = mine ? mb * P.scale_log2 : -INFINITY;                       // max of the scaled scores
+            for (int c = 0; c < kBlock; ++c) s[c] = c <= jmax ? s[c] : -INFINITY;
+          }
+#pragma unroll
+          for (int c = 0; c < kBlock; ++c) mb = fmaxf(mb, s[c]);
+          mb = mine ? mb * P.scale_log2 : -INFINITY;                     // max of the scaled scores
+        }
         const bool raise = mb > m_ref + kRescale;
         const bool rescale = raise && !seg_first && m_ref != -INFINITY;
         if (__any_sync(0xffffffffu, rescale)) {
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (raise) m_ref = mb;
         const float neg_m = mine ? -m_ref : -INFINITY;
         // P = exp2(s - m_ref) as bf16 pairs over the first 64 columns of the buffer
-        if (__any_sync(0xffffffffu, mine)) {
+        if (active) {
           float rs = 0.f;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
