@@ -157,6 +157,10 @@ size_t scores_workspace(const msa_shape* sh, int32_t n_q) {
 // Decode attention workspace: two partial results per CTA of the persistent
 // grid (at most kMaxCtas CTAs, at most one per unit).  Depends only on the
 // pair count, so the workspace query and the launch always agree.
+// Prefill attention takes the union-tile kernel up to this cache capacity
+// (tokens per stream) and the per-pair kernel beyond it.
+constexpr int kUnionMaxContext = 32768;
+
 size_t attn_workspace(int64_t n_pairs, int mode) {
   if (mode == MSA_MODE_PREFILL || n_pairs == 0) return 0;
   const int64_t units = n_pairs * msa::dattn::kTopK;
@@ -199,11 +203,17 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
     if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q,
                              static_cast<int64_t>(n_q) * sh->n_q_heads, 16)) != MSA_OK)
       return st;
-    if (pg.table == nullptr) {
-      // contiguous caches: tiles of 8 queries over the union of their blocks
-      static std::atomic<uint64_t> u_smem_done{0};
-      if ((st = ensure_smem(msa::uattn::sparse_attn_prefill_union_kernel, msa::uattn::Layout::kBytes,
-                            u_smem_done)) != MSA_OK)
+    // Short contexts: tiles of 8 queries over the union of their blocks.  A
+    // union block costs ~1.1 us of a CTA and a per-pair (query, group) ~14 us,
+    // so the union wins while 8 queries' selections overlap enough: with
+    // selections spread over V visible blocks the union holds about
+    // V (1 - (1 - 16/V)^8) blocks, below the per-pair cost of 8 pairs up to
+    // V ~ 256.  The cache capacity bounds V.
+    if (sh->capacity <= kUnionMaxContext) {
+      const auto ukernel = pg.table != nullptr ? msa::uattn::sparse_attn_prefill_union_kernel<true>
+                                               : msa::uattn::sparse_attn_prefill_union_kernel<false>;
+      static std::atomic<uint64_t> u_smem_done[2] = {0, 0};
+      if ((st = ensure_smem(ukernel, msa::uattn::Layout::kBytes, u_smem_done[pg.table != nullptr])) != MSA_OK)
         return st;
       msa::uattn::Params U;
       U.sel = sel;
@@ -216,12 +226,14 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
       U.capacity = sh->capacity;
       U.n_tiles = (n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ;
       U.scale_log2 = softmax_scale * 1.4426950408889634f;
+      U.pages = pg;
       const int64_t tasks = static_cast<int64_t>(G) * U.n_tiles;
       const int64_t ugrid = std::min<int64_t>(sms, tasks);
-      launch(msa::uattn::sparse_attn_prefill_union_kernel, dim3(static_cast<unsigned>(ugrid)),
-             dim3(msa::uattn::kThreads), msa::uattn::Layout::kBytes, s, tm_q, tm_k, tm_v, U);
+      launch(ukernel, dim3(static_cast<unsigned>(ugrid)), dim3(msa::uattn::kThreads), msa::uattn::Layout::kBytes, s, tm_q,
+             tm_k, tm_v, U);
       return cuda_status(cudaGetLastError());
     }
+    // long contexts: one (query, group) pair at a time, its 16 blocks only
     const auto pkernel = pg.table != nullptr ? msa::pattn::sparse_attn_prefill_tc_kernel<true>
                                              : msa::pattn::sparse_attn_prefill_tc_kernel<false>;
     static std::atomic<uint64_t> tc_smem_done[2] = {0, 0};

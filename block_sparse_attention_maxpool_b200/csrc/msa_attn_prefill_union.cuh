@@ -92,6 +92,7 @@ struct Params {
   __nv_bfloat16* out;        // [n_q][Hq][D]
   int n_q, G, n_streams, capacity, n_tiles;
   float scale_log2;
+  KvPages pages;             // kPaged: K/V are page pools addressed through the block table
 };
 
 // Barrier slots (uint64 each, from Layout::kBarOff).
@@ -138,6 +139,9 @@ __device__ __forceinline__ void tile_coords(const Params& P, int t, int& g, int&
 }
 
 // The planner warp: union of the tile's selections, by segment, into `pl`.
+// With paged caches a selected block whose page is missing is left out (and
+// MSA_DEVERR_PAGE_RANGE set), as if the query had not selected it.
+template <bool kPaged>
 __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, uint32_t* keys, int lane) {
   int g, q0;
   tile_coords(P, t, g, q0);
@@ -181,11 +185,15 @@ __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, uin
     const int q = e / kTopK;
     const int qpos = __shfl_sync(0xffffffffu, pos, q);
     const int qseg = __shfl_sync(0xffffffffu, seg, q);
+    const int qstream = __shfl_sync(0xffffffffu, stream, q);
     uint32_t key = 0xffffffffu;
     if (qpos >= 0) {
       const int b = __ldg(P.sel + (static_cast<size_t>(q0 + q) * P.G + g) * kTopK + (e % kTopK));
       if (b >= 0 && b <= qpos / kBlock) {
-        key = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
+        if (kPaged && kv_block_row(P.pages, qstream, g, b, P.G, P.capacity) < 0)
+          raise_error(MSA_DEVERR_PAGE_RANGE);
+        else
+          key = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
       } else if (b > qpos / kBlock) {
         raise_error(MSA_DEVERR_SEL_RANGE);
       }
@@ -228,6 +236,7 @@ __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, uin
   __syncwarp();
 }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_prefill_union_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                                      const __grid_constant__ CUtensorMap tm_v, const Params P) {
@@ -279,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tc >= 2) ok = mbar_wait(&B.plan_empty[slot], ((tc >> 1) - 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      build_plan(P, t, plan_at(smem, slot), keys, lane);
+      build_plan<kPaged>(P, t, plan_at(smem, slot), keys, lane);
       if (lane == 0) mbar_arrive(&B.plan_full[slot]);
     }
   } else if (warp == 0 || warp == 2) {
@@ -321,7 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0) ok = mbar_wait(&rempty[st], (use - 1) & 1);
           if (!ok) break;
           const int s = pl.seg_stream[pl.segs[j]];
-          const int row = (s * P.G + g) * P.capacity + pl.blocks[j] * kBlock;
+          const int row = kPaged ? static_cast<int>(kv_block_row(P.pages, s, g, pl.blocks[j], P.G, P.capacity))
+                                 : (s * P.G + g) * P.capacity + pl.blocks[j] * kBlock;
           uint8_t* dst = rbase + st * kTile;
           mbar_arrive_expect_tx(&rfull[st], kTile);
           tma_load_2d(dst, map, 0, row, &rfull[st]);

@@ -140,6 +140,23 @@ def test_attention_given_selection(n_q, mode):
     report(f"attention n_q={n_q} {mode}", PT.check_attention(out.cpu(), want))
 
 
+def test_prefill_attention_long_context_per_pair_path():
+    """Caches above 32K tokens per stream take the per-pair prefill kernel
+    (shorter ones the union-tile kernel): the same oracle check there."""
+    g = torch.Generator().manual_seed(91)
+    S, cap, G = 2, 128 * 300, 4
+    lengths = [cap, 20000]
+    qpos = [(i % S, int(torch.randint(0, lengths[i % S], (1,), generator=g))) for i in range(37)]
+    qpos[0] = (0, cap - 1)
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, lengths, qpos, seed=91)
+    sel = _random_selection(g, qp, G)
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    out = msa.msa_sparse_attn_prefill(sh, q.cuda(), k.cuda(), v.cuda(), sel.cuda(), qs.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() == 0
+    want = oracle.sparse_attention(q, k, v, sel, qs, qp, 128, 1 / math.sqrt(128))
+    report("prefill attention, 38400-token caches", PT.check_attention(out.cpu(), want))
+
+
 def test_attention_empty_and_invalid_selection():
     S, cap = 1, 512
     idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, [512], [(0, 300), (0, 100)], seed=5)
