@@ -269,8 +269,10 @@ def run_ours(args, rank, world, dev):
         msa.msa_dsa_token_scores(dshape, d["q_idx"], d["weights"], d["k_idx_cache"], d["q_stream"], d["q_pos"],
                                  bufs["scores"], st)
 
-    def dsa_attend(st):
+    def dsa_select(st):
         msa.msa_dsa_select_topk(dshape, bufs["scores"], d["q_pos"], bufs["tok_sel"], bufs["tok_n"], st)
+
+    def dsa_attend(st):
         msa.msa_dsa_sparse_attn_decode(shape, d["q"], d["k_cache"], d["v_cache"], bufs["tok_sel"], d["q_stream"],
                                        d["q_pos"], scale, bufs["out"], bufs["workspace"], st)
 
@@ -284,14 +286,16 @@ def run_ours(args, rank, world, dev):
         msa.msa_block_scores(shape, d["idx_q"], d["idx_k_cache"], d["q_stream"], d["q_pos"],
                              bufs["block_scores"], st, bufs["workspace"], pages)
 
-    def part_attend(st):
+    def part_select(st):
         msa.msa_select_topk(shape, bufs["block_scores"], d["q_pos"], bufs["sel"], bufs["n_sel"], st)
+
+    def part_attend(st):
         attn = msa.msa_sparse_attn_prefill if prefill else msa.msa_sparse_attn_decode
         attn(shape, d["q"], d["k_cache"], d["v_cache"], bufs["sel"], d["q_stream"], d["q_pos"], scale,
              bufs["out"], bufs["workspace"], st, pages)
 
     if args.dsa:
-        part_append, part_scores, part_attend = dsa_append, dsa_scores, dsa_attend
+        part_append, part_scores, part_select, part_attend = dsa_append, dsa_scores, dsa_select, dsa_attend
     if args.fused:                                   # the whole step as one persistent kernel
         bufs["workspace_fused"] = torch.empty((msa.msa_decode_step_fused_workspace_bytes(shape, n_q),),
                                               dtype=torch.uint8, device=dev)
@@ -303,17 +307,24 @@ def run_ours(args, rank, world, dev):
         def part_scores(st):                         # noqa: F811
             msa.decode_step_fused(shape, {k: d[k] for k in ("idx_k_cache", "k_cache", "v_cache")}, d, bufs, st)
 
+        def part_select(st):                         # noqa: F811
+            pass
+
         def part_attend(st):                         # noqa: F811
             pass
 
+    # the kernel the roofline line describes: attention in prefill batches
+    # (most of the step), the score kernel otherwise
+    parts = [part_append, part_scores, part_select, part_attend]
+    timed = 3 if (prefill and not args.dsa and not args.fused) else 1
+
     def step(ev=None):
-        part_append(stream)
-        if ev is not None:
-            ev[0].record(stream)
-        part_scores(stream)
-        if ev is not None:
-            ev[1].record(stream)
-        part_attend(stream)
+        for i, part in enumerate(parts):
+            if ev is not None and i == timed:
+                ev[0].record(stream)
+            part(stream)
+            if ev is not None and i == timed:
+                ev[1].record(stream)
 
     clocks = ClockSampler(dev) if rank == 0 else None
     for _ in range(args.warmup):
@@ -324,10 +335,10 @@ def run_ours(args, rank, world, dev):
     graphs = None
     if not args.no_graph:
         # The step's launches captured once and replayed: the same kernels on
-        # the same buffers, without per-launch host work.  Three graphs, so
-        # events between them still time the block-score kernel on its own.
-        graphs = [torch.cuda.CUDAGraph() for _ in range(3)]
-        for i, (g, part) in enumerate(zip(graphs, (part_append, part_scores, part_attend))):
+        # the same buffers, without per-launch host work.  One graph per part,
+        # so events between them still time the roofline kernel on its own.
+        graphs = [torch.cuda.CUDAGraph() for _ in range(4)]
+        for i, (g, part) in enumerate(zip(graphs, parts)):
             if args.fused and i != 1:                        # the fused step is one kernel: one graph
                 graphs[i] = None
                 continue
@@ -336,15 +347,13 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize(dev)
 
         def step(ev=None):                                   # noqa: F811  (graph replay)
-            if graphs[0] is not None:
-                graphs[0].replay()
-            if ev is not None:
-                ev[0].record(stream)
-            graphs[1].replay()
-            if ev is not None:
-                ev[1].record(stream)
-            if graphs[2] is not None:
-                graphs[2].replay()
+            for i, g in enumerate(graphs):
+                if ev is not None and i == timed:
+                    ev[0].record(stream)
+                if g is not None:
+                    g.replay()
+                if ev is not None and i == timed:
+                    ev[1].record(stream)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize(dev)
@@ -379,9 +388,8 @@ def run_ours(args, rank, world, dev):
     e2e_steps = max(3, min(args.steps, 200 if not prefill else 20))
 
     def api_step():
-        part_append(stream)
-        part_scores(stream)
-        part_attend(stream)
+        for part in parts:
+            part(stream)
 
     e2e_launch = "direct"
     if not args.no_graph:
@@ -399,9 +407,8 @@ def run_ours(args, rank, world, dev):
         else:
             g_api = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_api):
-                part_append(None)
-                part_scores(None)
-                part_attend(None)
+                for part in parts:
+                    part(None)
             api_step = g_api.replay                             # noqa: F811
         e2e_launch = "cuda graph"
 
@@ -515,6 +522,11 @@ def dsa_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per
     }
 
 
+# Prefill attention runs the union-tile kernel up to this cache capacity
+# (tokens per stream) and the per-pair kernel beyond it.
+UNION_MAX_CONTEXT = 32768
+
+
 def prefill_flops(w) -> tuple[int, int]:
     """Algorithmic FLOPs of one prefill step: the indexer contraction over
     each query's visible keys (2 * Di per key per group) and the attention
@@ -533,7 +545,8 @@ def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches
     ind, att = prefill_flops(w)
     tokens = w.n_queries * world
     tf = (ind + att) / (ms * 1e-3) / 1e12
-    ktf = ind / (k_ms * 1e-3) / 1e12
+    ktf = att / (k_ms * 1e-3) / 1e12                 # the attention kernel: its algorithmic FLOPs
+    kernel = "sparse_attn_prefill_union" if w.capacity <= UNION_MAX_CONTEXT else "sparse_attn_prefill_tc"
     return {
         "metric": f"MSA prefill tokens/s ({w.name}); achieved TFLOP/s vs bf16 peak",
         "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -545,7 +558,7 @@ def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches
                    "launch": "cuda graphs" if graphs is not None else "direct"},
         "step_tensor": {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
                         "frac": tf / peaks["bf16_tflops"], "indexer_flops": ind, "attention_flops": att},
-        "roofline": {"kernel": "block_scores", "bound": "tensor", "achieved": ktf, "peak": peaks["bf16_tflops"],
+        "roofline": {"kernel": kernel, "bound": "tensor", "achieved": ktf, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": ktf / peaks["bf16_tflops"], "traffic": None,
                      "ms_per_launch": k_ms, "peak_src": peaks["src"]},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
