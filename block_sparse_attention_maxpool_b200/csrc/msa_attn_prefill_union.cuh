@@ -7,8 +7,8 @@
 // local block.
 //
 // A tile is 8 consecutive queries of one group: 8 x 16 = 128 query-head
-// rows, the M dimension of every MMA.  A planner warp merges the 8 queries'
-// sorted selections into the tile's union of blocks, each with an 8-bit mask
+// rows, the M dimension of every MMA.  A planner warp builds the tile's
+// union of the 8 queries' selected blocks, each with an 8-bit mask
 // of the queries that selected it (queries of different streams form
 // separate segments of the union).  For every block b of the union:
 //   S = Q . K_b^T          M=128 rows, N=128 keys, K=128 dims (TMEM, f32)
@@ -78,8 +78,7 @@ struct Layout {
   static constexpr uint32_t kVOff = kKOff + kKRing * kTile;
   static constexpr uint32_t kPlanOff = kVOff + kVRing * kTile;
   static constexpr uint32_t kPlanBytes = (sizeof(Plan) + 127) / 128 * 128;
-  static constexpr uint32_t kKeysOff = kPlanOff + 2 * kPlanBytes;     // planner scratch: 128 keys
-  static constexpr uint32_t kBarOff = kKeysOff + kMaxUnion * 4;
+  static constexpr uint32_t kBarOff = kPlanOff + 2 * kPlanBytes;
   static constexpr uint32_t kEnd = kBarOff + 40 * 8;
   static constexpr size_t kBytes = kEnd + 1024;
 };
@@ -139,10 +138,16 @@ __device__ __forceinline__ void tile_coords(const Params& P, int t, int& g, int&
 }
 
 // The planner warp: union of the tile's selections, by segment, into `pl`.
-// With paged caches a selected block whose page is missing is left out (and
-// MSA_DEVERR_PAGE_RANGE set), as if the query had not selected it.
+// Every lane holds 4 of the 128 (query, slot) entries as sortable keys
+// (segment << 24 | block); an entry leads its key if no earlier entry has
+// it, the key's mask ORs the queries of all its entries, and a leader's
+// place in the union is the number of smaller leading keys.  So the union
+// comes out ascending within each segment whatever the order of a query's
+// list, and a -1 or out-of-range entry anywhere in it is simply left out.
+// With paged caches a selected block whose page is missing is left out too
+// (and MSA_DEVERR_PAGE_RANGE set), as if the query had not selected it.
 template <bool kPaged>
-__device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, uint32_t* keys, int lane) {
+__device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, int lane) {
   int g, q0;
   tile_coords(P, t, g, q0);
   // per query: position (or -1) and stream
@@ -178,61 +183,70 @@ __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, uin
     if (sq == lane) rows |= 1u << q;
   }
   if (lane < kTileQ) pl.seg_rows[lane] = static_cast<uint8_t>(rows);
-  // the 128 selection entries as sortable keys (segment << 24 | block); past-the-end: ~0
+  // entries e = lane + 32 m belong to query e / 16
+  uint32_t key[4];
 #pragma unroll
-  for (int m = 0; m < kMaxUnion / 32; ++m) {
+  for (int m = 0; m < 4; ++m) {
     const int e = lane + 32 * m;
     const int q = e / kTopK;
     const int qpos = __shfl_sync(0xffffffffu, pos, q);
     const int qseg = __shfl_sync(0xffffffffu, seg, q);
     const int qstream = __shfl_sync(0xffffffffu, stream, q);
-    uint32_t key = 0xffffffffu;
+    key[m] = 0xffffffffu;
     if (qpos >= 0) {
       const int b = __ldg(P.sel + (static_cast<size_t>(q0 + q) * P.G + g) * kTopK + (e % kTopK));
       if (b >= 0 && b <= qpos / kBlock) {
         if (kPaged && kv_block_row(P.pages, qstream, g, b, P.G, P.capacity) < 0)
           raise_error(MSA_DEVERR_PAGE_RANGE);
         else
-          key = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
+          key[m] = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
       } else if (b > qpos / kBlock) {
         raise_error(MSA_DEVERR_SEL_RANGE);
       }
     }
-    keys[e] = key;
   }
-  __syncwarp();
-  if (lane == 0) {
-    // 8-way merge of the per-query lists (each ascending, ~0 entries last)
-    int head[kTileQ];
+  // leaders and query masks
+  bool lead[4] = {true, true, true, true};
+  uint32_t qmask[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int q = 0; q < kTileQ; ++q) head[q] = 0;
-    int n = 0;
-    uint32_t last = 0xffffffffu;
-    for (int step = 0; step < kMaxUnion; ++step) {
-      uint32_t best = 0xffffffffu;
-      int bq = -1;
+  for (int m2 = 0; m2 < 4; ++m2) {
+    for (int src = 0; src < 32; ++src) {
+      const uint32_t k2 = __shfl_sync(0xffffffffu, key[m2], src);
+      const int e2 = src + 32 * m2;
 #pragma unroll
-      for (int q = 0; q < kTileQ; ++q) {
-        const uint32_t k = head[q] < kTopK ? keys[q * kTopK + head[q]] : 0xffffffffu;
-        if (k < best) {
-          best = k;
-          bq = q;
+      for (int m = 0; m < 4; ++m) {
+        if (k2 == key[m]) {
+          qmask[m] |= 1u << (e2 / kTopK);
+          if (e2 < lane + 32 * m) lead[m] = false;
         }
       }
-      if (bq < 0) break;
-      ++head[bq];
-      if (best != last) {
-        pl.blocks[n] = static_cast<int>(best & 0xffffffu);
-        pl.segs[n] = static_cast<uint8_t>(best >> 24);
-        pl.masks[n] = static_cast<uint8_t>(1u << bq);
-        ++n;
-        last = best;
-      } else {
-        pl.masks[n - 1] |= static_cast<uint8_t>(1u << bq);
-      }
     }
-    pl.n = n;
   }
+  // place of each leader: leading keys smaller than its own
+  int rank[4] = {0, 0, 0, 0};
+  int n = 0;
+#pragma unroll
+  for (int m2 = 0; m2 < 4; ++m2) {
+    const bool l2 = lead[m2] && key[m2] != 0xffffffffu;
+    uint32_t ballot = __ballot_sync(0xffffffffu, l2);
+    n += __popc(ballot);
+    while (ballot != 0u) {
+      const int src = __ffs(ballot) - 1;
+      ballot &= ballot - 1u;
+      const uint32_t k2 = __shfl_sync(0xffffffffu, key[m2], src);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) rank[m] += k2 < key[m] ? 1 : 0;
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    if (lead[m] && key[m] != 0xffffffffu) {
+      pl.blocks[rank[m]] = static_cast<int>(key[m] & 0xffffffu);
+      pl.segs[rank[m]] = static_cast<uint8_t>(key[m] >> 24);
+      pl.masks[rank[m]] = static_cast<uint8_t>(qmask[m]);
+    }
+  }
+  if (lane == 0) pl.n = n;
   __syncwarp();
 }
 
@@ -280,7 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 3) {
     // ------------------------------ planner ------------------------------------
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + Layout::kKeysOff);
     int tc = 0;
     for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++tc) {
       const int slot = tc & 1;
@@ -288,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tc >= 2) ok = mbar_wait(&B.plan_empty[slot], ((tc >> 1) - 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      build_plan<kPaged>(P, t, plan_at(smem, slot), keys, lane);
+      build_plan<kPaged>(P, t, plan_at(smem, slot), lane);
       if (lane == 0) mbar_arrive(&B.plan_full[slot]);
     }
   } else if (warp == 0 || warp == 2) {

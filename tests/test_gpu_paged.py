@@ -143,6 +143,42 @@ def test_unmapped_page_is_skipped_and_flagged():
     PT.check_attention(out.cpu(), o)
 
 
+@pytest.mark.parametrize("cap_blocks", [24, 260], ids=["union_path", "per_pair_path"])
+def test_unmapped_page_is_skipped_in_prefill(cap_blocks):
+    """Prefill attention with a selected block on an unmapped page: the block
+    drops out of that query's attention (bit-identical to dropping it from the
+    selection) and MSA_DEVERR_PAGE_RANGE is set."""
+    n_new = 40
+    L = cap_blocks * 128
+    w = W.Workload(f"unmapped_prefill_{cap_blocks}", 2, L - n_new, L, "new")
+    inp = W.make_inputs(w, seed=51)
+    shape = PT.shape_of(w)
+    lay = W.page_layout(inp, seed=8, spare_pages=2)
+    dev = "cuda"
+    k_pool, v_pool = lay.k_pool.to(dev), lay.v_pool.to(dev)
+    qs, qp, q = inp.q_stream.to(dev), inp.q_pos.to(dev), inp.q.to(dev)
+    good = msa.Pages(lay.block_table.to(dev), lay.n_pages)
+    g = torch.Generator().manual_seed(cap_blocks)
+    from tests.test_gpu_parity import _random_selection
+    sel = _random_selection(g, inp.q_pos, w.n_kv_heads).to(dev)
+    # unmap a block that query 5 (stream 1) selects, other than its local block
+    s_bad = int(inp.q_stream[5])
+    b_bad = int([b for b in sel[5, 0].tolist() if 0 <= b < int(inp.q_pos[5]) // 128][0])
+    table = lay.block_table.clone()
+    table[s_bad, b_bad] = -1
+    bad = msa.Pages(table.to(dev), lay.n_pages)
+    out = msa.msa_sparse_attn_prefill_paged(shape, bad, q, k_pool, v_pool, sel, qs, qp)
+    assert msa.msa_get_device_error() & 0x10
+    sel_drop = sel.clone()
+    for i in range(sel.shape[0]):
+        if int(inp.q_stream[i]) == s_bad:
+            row = sel_drop[i]
+            row[row == b_bad] = -1
+    out_ref = msa.msa_sparse_attn_prefill_paged(shape, good, q, k_pool, v_pool, sel_drop, qs, qp)
+    assert msa.msa_get_device_error() == 0
+    assert torch.equal(out, out_ref)
+
+
 def test_paged_append_flags_unmapped_token():
     w = W.Workload("append_unmapped_2x600", 2, 500, 600, "last", n_q_heads=16, n_kv_heads=1)
     inp = W.make_inputs(w, seed=48)

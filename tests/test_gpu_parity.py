@@ -157,6 +157,43 @@ def test_prefill_attention_long_context_per_pair_path():
     report("prefill attention, 38400-token caches", PT.check_attention(out.cpu(), want))
 
 
+@pytest.mark.parametrize("cap", [1024, 128 * 260], ids=["union_path", "per_pair_path"])
+def test_prefill_attention_edge_queries(cap):
+    """Prefill attention on a ragged batch (21 queries: two 8-query tiles and
+    a tail of 5) whose tiles mix streams, with shuffled selection lists (-1
+    in the middle), an invalid selected block, an empty selection, a
+    position past the cache and a bad stream id: the invalid block is skipped
+    (SEL_RANGE), the bad queries give zeros (QUERY_RANGE), everything else
+    matches the oracle."""
+    g = torch.Generator().manual_seed(cap)
+    S, G = 2, 4
+    lengths = [cap, cap // 2]
+    qpos = [(int(torch.randint(0, S, (1,), generator=g)), 0) for _ in range(21)]
+    qpos = [(st, int(torch.randint(0, lengths[st], (1,), generator=g))) for st, _ in qpos]
+    qpos[0] = (0, 700)
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, lengths, qpos, seed=cap)
+    sel = _random_selection(g, qp, G)
+    # a selection is a set of blocks: lists in any order, -1 anywhere
+    for i in range(4, 21, 3):
+        for gg in range(G):
+            sel[i, gg] = sel[i, gg][torch.randperm(16, generator=g)]
+    sel[0, 2, 15] = 6                 # block 6 starts past position 700: invalid, skipped
+    sel[1] = -1                       # empty selection: zeros
+    qp_dev = qp.clone()
+    qs_dev = qs.clone()
+    qp_dev[2] = cap                   # past the capacity: zeros, QUERY_RANGE
+    qs_dev[3] = -1                    # no such stream: zeros, QUERY_RANGE
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    out = msa.msa_sparse_attn_prefill(sh, q.cuda(), k.cuda(), v.cuda(), sel.cuda(), qs_dev.cuda(), qp_dev.cuda())
+    err = msa.msa_get_device_error()
+    assert err & 0x1 and err & 0x4 and not err & ~0x5, err
+    sel_clean = sel.clone()
+    sel_clean[0, 2, 15] = -1
+    want = oracle.sparse_attention(q, k, v, sel_clean, qs, qp, 128, 1 / math.sqrt(128))
+    want[1:4] = 0.0
+    report(f"prefill attention edge queries, cap {cap}", PT.check_attention(out.cpu(), want))
+
+
 def test_attention_empty_and_invalid_selection():
     S, cap = 1, 512
     idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, [512], [(0, 300), (0, 100)], seed=5)
