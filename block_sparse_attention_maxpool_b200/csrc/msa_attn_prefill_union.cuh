@@ -45,7 +45,6 @@ constexpr int kBlock = 128;
 constexpr int kHpg = 16;
 constexpr int kTopK = 16;
 constexpr int kTileQ = 8;                           // queries per tile
-constexpr int kRows = kTileQ * kHpg;                // 128 MMA rows
 constexpr int kMaxUnion = kTileQ * kTopK;           // 128 blocks at most
 constexpr uint32_t kHalf = 128 * 128;               // [128 rows][64 bf16] = 16 KB
 constexpr uint32_t kTile = 2 * kHalf;               // 32 KB
