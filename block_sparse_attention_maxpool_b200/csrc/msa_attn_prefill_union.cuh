@@ -29,6 +29,17 @@
 // tile is released after the tile's last S MMA, so the next tile's Q loads
 // while the last blocks' softmax runs.
 //
+// What bounds it on B200: the tensor pipe drains whenever consecutive MMAs
+// change operand source or major-ness (S: both operands from shared memory,
+// K-major; P . V: A from tensor memory, B MN-major), about 300 cycles each,
+// twice per block, and every hand-off between the issuer and the softmax
+// warps (a commit or an mbarrier arrive and its waiter) costs ~230 cycles,
+// which three S buffers hide only in part.
+//
+// Paged caches (kPaged): the loaders address blocks through the block table;
+// the planner leaves out a selected block whose page is missing (and sets
+// MSA_DEVERR_PAGE_RANGE), as if the query had not selected it.
+//
 // Warp roles: 0 K loader (and the Q tile), 1 MMA issuer, 2 V loader,
 // 3 planner (one tile ahead), 4-7 softmax and output (one TMEM lane quarter
 // each).  Shared memory: Q 32 KB, K ring 3 x 32 KB, V ring 2 x 32 KB, two
