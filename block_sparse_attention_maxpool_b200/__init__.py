@@ -26,7 +26,8 @@ __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_bloc
            "msa_block_scores_paged", "msa_block_scores_f16_paged", "msa_sparse_attn_decode_paged",
            "msa_sparse_attn_prefill_paged", "DsaShape", "DSA_SEL_WIDTH", "msa_dsa_indexer_append",
            "msa_dsa_token_scores", "msa_dsa_select_topk", "msa_dsa_sparse_attn_decode", "dsa_decode_step",
-           "msa_decode_step_fused", "msa_decode_step_fused_workspace_bytes", "decode_step_fused", "DecodeGraph"]
+           "msa_decode_step_fused", "msa_decode_step_fused_workspace_bytes", "decode_step_fused", "DecodeGraph",
+           "StepPipeline"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
 MODE_DECODE = 0
@@ -700,3 +701,70 @@ class DecodeGraph:
         """One host-to-device copy of a packed step, then the replay."""
         self.staging.copy_(buffer, non_blocking=True)
         return self.replay()
+
+
+class StepPipeline:
+    """Back-to-back steps with their host transfers overlapped.
+
+    Two ``DecodeGraph`` captures on the same caches alternate (each with its
+    own staging buffer and result buffers).  ``step(buffer)`` queues, for the
+    next step, the host-to-device copy of its packed inputs on one copy
+    stream, the replay on the current stream, and the device-to-host copy of
+    its output on a second copy stream; events order them, so step i+1's
+    inputs and step i-1's output move while step i runs, and the steps
+    still run one after another on the caches.  It returns the pinned host
+    tensor that will hold the output and an event recorded when it has
+    landed; that tensor is reused two steps later, so read it (after
+    ``event.synchronize()``) before then.  Building the pipeline runs the
+    first inputs twice (one step per capture, as ``DecodeGraph`` does)."""
+
+    def __init__(self, shape: Shape, caches: dict, inputs: dict, prefill: bool = False,
+                 pages: Pages | None = None):
+        dev = inputs["q"].device
+        self.graphs = [DecodeGraph(shape, caches, inputs, None, prefill, pages) for _ in range(2)]
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        self.host_out = [torch.empty(g.out.shape, dtype=g.out.dtype).pin_memory() for g in self.graphs]
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of the slot's step are on the device
+        self.ev_done = [torch.cuda.Event() for _ in range(2)]    # the slot's replay has finished
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]     # the slot's output is on the host
+        self.used = [False, False]
+        self.n = 0
+
+    def host_buffer(self) -> torch.Tensor:
+        """A pinned host buffer with the staging layout (both captures share it)."""
+        return self.graphs[0].host_buffer()
+
+    def pack(self, host_inputs: dict, buffer: torch.Tensor) -> torch.Tensor:
+        return self.graphs[0].pack(host_inputs, buffer)
+
+    def step(self, buffer: torch.Tensor):
+        """Queue one step whose packed inputs are in ``buffer`` (pinned; not
+        to be rewritten before the returned event).  Returns (host output,
+        event)."""
+        i = self.n % 2
+        g = self.graphs[i]
+        cur = torch.cuda.current_stream(g.out.device)
+        if self.used[i]:
+            self.h2d.wait_event(self.ev_done[i])      # the slot's staging buffer is free again
+            cur.wait_event(self.ev_out[i])            # and its output has been read
+        with torch.cuda.stream(self.h2d):
+            g.staging.copy_(buffer, non_blocking=True)
+            self.ev_in[i].record(self.h2d)
+        cur.wait_event(self.ev_in[i])
+        g.graph.replay()
+        self.ev_done[i].record(cur)
+        self.d2h.wait_event(self.ev_done[i])
+        with torch.cuda.stream(self.d2h):
+            self.host_out[i].copy_(g.out, non_blocking=True)
+            self.ev_out[i].record(self.d2h)
+        self.used[i] = True
+        self.n += 1
+        return self.host_out[i], self.ev_out[i]
+
+    def wait_all(self):
+        """Make the current stream wait until every queued output has landed."""
+        cur = torch.cuda.current_stream(self.graphs[0].out.device)
+        for i in range(2):
+            if self.used[i]:
+                cur.wait_event(self.ev_out[i])

@@ -50,3 +50,41 @@ def test_replay_with_new_inputs_matches_direct_calls(prefill):
         assert torch.equal(caches_g[k], caches_d[k]), k
     assert torch.equal(out_g, out_d)
     assert torch.equal(graph.sel, sel_d) and torch.equal(graph.block_scores, bs_d)
+
+
+@pytest.mark.parametrize("prefill", [False, True])
+def test_step_pipeline_matches_direct_calls(prefill):
+    """Four steps through StepPipeline (overlapped host transfers, two
+    alternating captures) give the outputs and caches of four direct steps."""
+    if prefill:
+        ws = [W.Workload("pipe_prefill_2x200", 2, 200 * i, 200 * (i + 1), "new") for i in range(1, 5)]
+    else:
+        ws = [W.Workload("pipe_decode_5x2000", 5, 1995 + i, 1996 + i, "last") for i in range(4)]
+    steps = [W.make_inputs(w, seed=90 + i) for i, w in enumerate(ws)]
+    shape = PT.shape_of(ws[-1])                  # every step's positions fit the last one's capacity
+    base = steps[0]
+    cache_src = W.make_inputs(ws[-1], seed=89)
+
+    # the same starting caches twice (pipeline / direct)
+    def fresh():
+        return {k: getattr(cache_src, k).clone().cuda() for k in ("idx_k_cache", "k_cache", "v_cache")}
+    cache_p, cache_d = fresh(), fresh()
+    first = {n: getattr(base, n).cuda() for n in NAMES}
+    pipe = msa.StepPipeline(shape, cache_p, first, prefill=prefill)
+    host_bufs = [pipe.host_buffer() for _ in steps]
+    outs = []
+    for st, hb in zip(steps, host_bufs):
+        h, ev = pipe.step(pipe.pack({n: getattr(st, n).contiguous() for n in NAMES}, hb))
+        ev.synchronize()
+        outs.append(h.clone())
+    torch.cuda.synchronize()
+    # direct: the two set-up runs of the first inputs, then the four steps
+    first_d = {n: getattr(base, n).cuda() for n in NAMES}
+    msa.decode_step(shape, cache_d, first_d, prefill=prefill)
+    msa.decode_step(shape, cache_d, first_d, prefill=prefill)
+    for st, got in zip(steps, outs):
+        out, _, _, _ = msa.decode_step(shape, cache_d, {n: getattr(st, n).cuda() for n in NAMES}, prefill=prefill)
+        assert torch.equal(got, out.cpu())
+    assert msa.msa_get_device_error() == 0
+    for k in ("idx_k_cache", "k_cache", "v_cache"):
+        assert torch.equal(cache_p[k], cache_d[k]), k
