@@ -194,6 +194,22 @@ def test_prefill_attention_edge_queries(cap):
     report(f"prefill attention edge queries, cap {cap}", PT.check_attention(out.cpu(), want))
 
 
+def test_prefill_attention_every_tile_spans_eight_streams():
+    """Prefill queries interleaved over 8 streams, so each 8-query tile of the
+    union kernel holds 8 segments (one per stream, each with its own blocks)."""
+    g = torch.Generator().manual_seed(77)
+    S, cap, G = 8, 128 * 12, 4
+    lengths = [cap - 97 * s for s in range(S)]
+    qpos = [(i % S, int(torch.randint(0, lengths[i % S], (1,), generator=g))) for i in range(83)]
+    idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, lengths, qpos, seed=77)
+    sel = _random_selection(g, qp, G)
+    sh = msa.Shape(n_streams=S, capacity=cap)
+    out = msa.msa_sparse_attn_prefill(sh, q.cuda(), k.cuda(), v.cuda(), sel.cuda(), qs.cuda(), qp.cuda())
+    assert msa.msa_get_device_error() == 0
+    want = oracle.sparse_attention(q, k, v, sel, qs, qp, 128, 1 / math.sqrt(128))
+    report("prefill attention, 8 streams per tile", PT.check_attention(out.cpu(), want))
+
+
 def test_attention_empty_and_invalid_selection():
     S, cap = 1, 512
     idx, k, v, qs, qp, iq, q = W.make_custom(S, cap, [512], [(0, 300), (0, 100)], seed=5)
