@@ -161,9 +161,18 @@ size_t scores_workspace(const msa_shape* sh, int32_t n_q) {
 // (tokens per stream) and the per-pair kernel beyond it.
 constexpr int kUnionMaxContext = 32768;
 
-size_t attn_workspace(int64_t n_pairs, int mode) {
-  if (mode == MSA_MODE_PREFILL || n_pairs == 0) return 0;
-  const int64_t units = n_pairs * msa::dattn::kTopK;
+// Prefill attention on short contexts: the plan of every 8-query tile.
+int64_t union_tasks(const msa_shape* sh, int32_t n_q) {
+  return static_cast<int64_t>(sh->n_kv_heads) * ((n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ);
+}
+
+size_t attn_workspace(const msa_shape* sh, int32_t n_q, int mode) {
+  if (n_q == 0) return 0;
+  if (mode == MSA_MODE_PREFILL) {
+    if (sh->capacity > kUnionMaxContext) return 0;
+    return static_cast<size_t>(union_tasks(sh, n_q)) * sizeof(msa::uattn::Plan);
+  }
+  const int64_t units = static_cast<int64_t>(n_q) * sh->n_kv_heads * msa::dattn::kTopK;
   const int64_t ctas = std::min<int64_t>(units, msa::dattn::kMaxCtas);
   return static_cast<size_t>(ctas) * 2 * msa::dattn::kPartial * sizeof(float);
 }
@@ -183,14 +192,14 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   const int G = sh->n_kv_heads;
   const int64_t n_pairs = static_cast<int64_t>(n_q) * G;
   if (n_pairs * msa::dattn::kTopK >= (int64_t{1} << 40)) return MSA_ERR_RANGE;
-  const size_t need = attn_workspace(n_pairs, mode);
+  msa::KvPages pg;
+  int64_t rows = 0;
+  if ((st = pages_of(sh, pages, &pg, &rows)) != MSA_OK) return st;
+  const size_t need = attn_workspace(sh, n_q, mode);
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need) return MSA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MSA_ERR_ALIGN;
   }
-  msa::KvPages pg;
-  int64_t rows = 0;
-  if ((st = pages_of(sh, pages, &pg, &rows)) != MSA_OK) return st;
   CUtensorMap tm_k, tm_v;
   if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
   if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
@@ -227,8 +236,12 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
       U.n_tiles = (n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ;
       U.scale_log2 = softmax_scale * 1.4426950408889634f;
       U.pages = pg;
+      U.plans = static_cast<msa::uattn::Plan*>(workspace);
       const int64_t tasks = static_cast<int64_t>(G) * U.n_tiles;
       const int64_t ugrid = std::min<int64_t>(sms, tasks);
+      const auto pkernel_plan = pg.table != nullptr ? msa::uattn::plan_tiles_kernel<true>
+                                                    : msa::uattn::plan_tiles_kernel<false>;
+      launch(pkernel_plan, dim3(static_cast<unsigned>((tasks + 7) / 8)), dim3(256), 0, s, U);
       launch(ukernel, dim3(static_cast<unsigned>(ugrid)), dim3(msa::uattn::kThreads), msa::uattn::Layout::kBytes, s, tm_q,
              tm_k, tm_v, U);
       return cuda_status(cudaGetLastError());
@@ -586,8 +599,7 @@ int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf16* q, co
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(sel) || !aligned16(out))
     return MSA_ERR_ALIGN;
   if (!std::isfinite(softmax_scale)) return MSA_ERR_RANGE;
-  const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
-  const size_t need = attn_workspace(n_pairs, MSA_MODE_DECODE);
+  const size_t need = attn_workspace(shape, n_q, MSA_MODE_DECODE);
   if (need > MSA_NOALLOC_SCRATCH_BYTES) return MSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (need > 0) {
@@ -745,8 +757,7 @@ int msa_dsa_sparse_attn_decode(const msa_shape* shape, const msa_pages* pages, c
 // ---- the whole decode step in one kernel ---------------------------------------
 size_t msa_decode_step_fused_workspace_bytes(const msa_shape* shape, int32_t n_q) {
   if (check_shape(shape) != MSA_OK || n_q < 1 || scores_use_tiles(shape, n_q)) return static_cast<size_t>(-1);
-  const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
-  return msa::tc::align256(attn_workspace(n_pairs, MSA_MODE_DECODE)) + 256;   // partials, then barrier words
+  return msa::tc::align256(attn_workspace(shape, n_q, MSA_MODE_DECODE)) + 256;   // partials, then barrier words
 }
 
 int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* k_cache, msa_bf16* v_cache,
@@ -842,7 +853,7 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   A.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
   A.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
   unsigned int* bar = reinterpret_cast<unsigned int*>(
-      static_cast<uint8_t*>(workspace) + msa::tc::align256(attn_workspace(n_pairs, MSA_MODE_DECODE)));
+      static_cast<uint8_t*>(workspace) + msa::tc::align256(attn_workspace(shape, n_q, MSA_MODE_DECODE)));
   F.bar_count = bar;
   F.bar_gen = bar + 1;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -864,8 +875,7 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
 size_t msa_workspace_bytes(const msa_shape* shape, int32_t n_q, int32_t mode) {
   if (check_shape(shape) != MSA_OK || n_q < 0 || (mode != MSA_MODE_DECODE && mode != MSA_MODE_PREFILL))
     return static_cast<size_t>(-1);
-  const int64_t n_pairs = static_cast<int64_t>(n_q) * shape->n_kv_heads;
-  return std::max(scores_workspace(shape, n_q), attn_workspace(n_pairs, mode));
+  return std::max(scores_workspace(shape, n_q), attn_workspace(shape, n_q, mode));
 }
 
 const char* msa_status_string(int status) {

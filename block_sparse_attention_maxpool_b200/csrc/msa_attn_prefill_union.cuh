@@ -22,28 +22,30 @@
 // 2^8, so P stays below 256 and the rescale is rare.  Each K and V block is
 // read once per tile instead of once per (query, group).
 //
-// Pipelining: three S/P buffers in tensor memory and S MMAs issued two
-// blocks ahead of P . V, so the softmax warps run up to two blocks apart
-// and overlap P . V; a warp whose two queries did not select a block writes
-// zeros without reading S or computing exponentials.  The Q
-// tile is released after the tile's last S MMA, so the next tile's Q loads
-// while the last blocks' softmax runs.
+// Pipelining: three S/P buffers in tensor memory; S of block b needs only
+// the P . V of block b - 3 done, so the S MMAs run up to two blocks ahead of
+// P . V and the softmax warps can drift two blocks apart.  A warp whose two
+// queries did not select a block writes zeros without reading S or
+// computing exponentials.  The Q tile is released after the tile's last S
+// MMA, so the next tile's Q loads while the last blocks' softmax runs.
 //
-// What bounds it on B200: the tensor pipe drains whenever consecutive MMAs
-// change operand source or major-ness (S: both operands from shared memory,
-// K-major; P . V: A from tensor memory, B MN-major), about 300 cycles each,
-// twice per block, and every hand-off between the issuer and the softmax
-// warps (a commit or an mbarrier arrive and its waiter) costs ~230 cycles,
-// which three S buffers hide only in part.
+// S and P . V are issued by two threads (warps 1 and 3).  On B200 the
+// tensor pipe drains, ~300 cycles, whenever one issuing thread changes
+// operand configuration (S: both operands from shared memory, K-major;
+// P . V: A from tensor memory, B MN-major), but streams of two threads
+// interleave at full rate.  What remains is the hand-off latency: a commit
+// or an mbarrier arrive reaches its waiter after ~230 cycles, and three S
+// buffers hide it only in part.
 //
 // Paged caches (kPaged): the loaders address blocks through the block table;
 // the planner leaves out a selected block whose page is missing (and sets
 // MSA_DEVERR_PAGE_RANGE), as if the query had not selected it.
 //
-// Warp roles: 0 K loader (and the Q tile), 1 MMA issuer, 2 V loader,
-// 3 planner (one tile ahead), 4-7 softmax and output (one TMEM lane quarter
-// each).  Shared memory: Q 32 KB, K ring 3 x 32 KB, V ring 2 x 32 KB, two
-// plans.  Tensor memory: three S/P buffers and O (all 512 columns).
+// Warp roles: 0 loads the Q tile and the K blocks, 1 issues S, 2 loads the
+// V blocks, 3 issues P . V, 4-7 run the softmax and write the output (one
+// TMEM lane quarter each), 8 plans the tiles one tile ahead.  Shared
+// memory: Q 32 KB, K ring 3 x 32 KB, V ring 2 x 32 KB, two plans.  Tensor
+// memory: three S/P buffers and O (all 512 columns).
 #pragma once
 
 #include "msa_common.cuh"
@@ -62,7 +64,6 @@ constexpr uint32_t kTile = 2 * kHalf;               // 32 KB
 constexpr int kKRing = 3;
 constexpr int kVRing = 2;
 constexpr int kSBufs = 3;                           // S/P buffers in tensor memory
-constexpr int kLag = kSBufs - 1;                    // S MMAs run this many blocks ahead of P . V
 constexpr int kThreads = 8 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 0;                       // S/P buffer i: columns 128 i .. 128 i + 127
@@ -86,9 +87,7 @@ struct Layout {
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = kQOff + kTile;
   static constexpr uint32_t kVOff = kKOff + kKRing * kTile;
-  static constexpr uint32_t kPlanOff = kVOff + kVRing * kTile;
-  static constexpr uint32_t kPlanBytes = (sizeof(Plan) + 127) / 128 * 128;
-  static constexpr uint32_t kBarOff = kPlanOff + 2 * kPlanBytes;
+  static constexpr uint32_t kBarOff = kVOff + kVRing * kTile;
   static constexpr uint32_t kEnd = kBarOff + 40 * 8;
   static constexpr size_t kBytes = kEnd + 1024;
 };
@@ -102,18 +101,17 @@ struct Params {
   int n_q, G, n_streams, capacity, n_tiles;
   float scale_log2;
   KvPages pages;             // kPaged: K/V are page pools addressed through the block table
+  Plan* plans;               // [G * n_tiles]: written by plan_tiles_kernel, read by the attention kernel
 };
 
 // Barrier slots (uint64 each, from Layout::kBarOff).
 struct Bars {
-  uint64_t *plan_full, *plan_empty, *q_full, *q_empty, *kfull, *kempty, *vfull, *vempty;
+  uint64_t *q_full, *q_empty, *kfull, *kempty, *vfull, *vempty;
   uint64_t *s_full, *p_full, *pv_done, *o_empty, *mma_done;
   uint32_t* tmem_slot;
   __device__ explicit Bars(uint8_t* smem) {
     uint64_t* b = reinterpret_cast<uint64_t*>(smem + Layout::kBarOff);
-    plan_full = b;                 // [2]
-    plan_empty = plan_full + 2;    // [2]
-    q_full = plan_empty + 2;
+    q_full = b;
     q_empty = q_full + 1;
     kfull = q_empty + 1;           // [kKRing]
     kempty = kfull + kKRing;
@@ -123,21 +121,17 @@ struct Bars {
     p_full = s_full + kSBufs;      // [kSBufs]: its P is written (4 softmax warps)
     pv_done = p_full + kSBufs;     // [kSBufs]: its P . V finished (buffer free, O updated)
     o_empty = pv_done + kSBufs;
-    mma_done = o_empty + 1;
-    tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    mma_done = o_empty + 1;        // [2]: the S issuer's and the P . V issuer's last MMAs
+    tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
   }
 };
-static_assert(6 + 2 * kKRing + 2 * kVRing + 3 * kSBufs + 2 + 1 <= 40, "barrier slots");
+static_assert(2 + 2 * kKRing + 2 * kVRing + 3 * kSBufs + 3 + 1 <= 40, "barrier slots");
 
 // exp2 on the special-function unit (ex2.approx.ftz: ~2 ulp; 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-__device__ __forceinline__ Plan& plan_at(uint8_t* smem, int slot) {
-  return *reinterpret_cast<Plan*>(smem + Layout::kPlanOff + slot * Layout::kPlanBytes);
 }
 
 // Tile t -> (group, first query).  Group-major, so the CTAs running at the
@@ -148,16 +142,21 @@ __device__ __forceinline__ void tile_coords(const Params& P, int t, int& g, int&
 }
 
 // The planner warp: union of the tile's selections, by segment, into `pl`.
-// Every lane holds 4 of the 128 (query, slot) entries as sortable keys
-// (segment << 24 | block); an entry leads its key if no earlier entry has
-// it, the key's mask ORs the queries of all its entries, and a leader's
-// place in the union is the number of smaller leading keys.  So the union
-// comes out ascending within each segment whatever the order of a query's
-// list, and a -1 or out-of-range entry anywhere in it is simply left out.
-// With paged caches a selected block whose page is missing is left out too
-// (and MSA_DEVERR_PAGE_RANGE set), as if the query had not selected it.
+// The 128 (query, slot) entries become sortable keys (segment << 24 |
+// block; ~0 for an empty or invalid entry), each carrying its query's bit;
+// lane l holds entries 4l .. 4l+3.  A bitonic sort of the 128 keys (28
+// compare-exchange steps, shuffles across lanes) puts equal keys side by
+// side, a segmented OR over each run of equal keys gives the run's query
+// mask, and a prefix count of run heads gives each distinct key its place
+// in the union.  So the union comes out ascending within each segment
+// whatever the order of a query's list, and a -1 or out-of-range entry
+// anywhere in it is simply left out.  With paged caches a selected block
+// whose page is missing is left out too (and MSA_DEVERR_PAGE_RANGE set), as
+// if the query had not selected it.
 template <bool kPaged>
 __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, int lane) {
+  constexpr uint32_t kFull = 0xffffffffu;
+  constexpr uint32_t kNone = 0xffffffffu;
   int g, q0;
   tile_coords(P, t, g, q0);
   // per query: position (or -1) and stream
@@ -179,7 +178,7 @@ __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, int
   int seg = -1;
 #pragma unroll
   for (int q = 0; q < kTileQ; ++q) {
-    const int sq = __shfl_sync(0xffffffffu, stream, q);
+    const int sq = __shfl_sync(kFull, stream, q);
     if (seg < 0 && stream >= 0 && sq == stream) seg = q;
   }
   if (lane < kTileQ) {
@@ -189,75 +188,139 @@ __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, int
   uint32_t rows = 0;
 #pragma unroll
   for (int q = 0; q < kTileQ; ++q) {
-    const int sq = __shfl_sync(0xffffffffu, seg, q);
+    const int sq = __shfl_sync(kFull, seg, q);
     if (sq == lane) rows |= 1u << q;
   }
   if (lane < kTileQ) pl.seg_rows[lane] = static_cast<uint8_t>(rows);
-  // entries e = lane + 32 m belong to query e / 16
-  uint32_t key[4];
+  // entries 4 lane + i: query lane / 4, slots 4 (lane % 4) + i
+  const int q = lane >> 2;
+  const int qpos = __shfl_sync(kFull, pos, q);
+  const int qseg = __shfl_sync(kFull, seg, q);
+  const int qstream = __shfl_sync(kFull, stream, q);
+  uint32_t key[4], val[4];
+  {
+    int4 sel4 = make_int4(-1, -1, -1, -1);
+    if (qpos >= 0)
+      sel4 = __ldg(reinterpret_cast<const int4*>(P.sel + (static_cast<size_t>(q0 + q) * P.G + g) * kTopK) + (lane & 3));
+    const int b4[4] = {sel4.x, sel4.y, sel4.z, sel4.w};
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int e = lane + 32 * m;
-    const int q = e / kTopK;
-    const int qpos = __shfl_sync(0xffffffffu, pos, q);
-    const int qseg = __shfl_sync(0xffffffffu, seg, q);
-    const int qstream = __shfl_sync(0xffffffffu, stream, q);
-    key[m] = 0xffffffffu;
-    if (qpos >= 0) {
-      const int b = __ldg(P.sel + (static_cast<size_t>(q0 + q) * P.G + g) * kTopK + (e % kTopK));
-      if (b >= 0 && b <= qpos / kBlock) {
-        if (kPaged && kv_block_row(P.pages, qstream, g, b, P.G, P.capacity) < 0)
-          raise_error(MSA_DEVERR_PAGE_RANGE);
-        else
-          key[m] = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
-      } else if (b > qpos / kBlock) {
-        raise_error(MSA_DEVERR_SEL_RANGE);
-      }
-    }
-  }
-  // leaders and query masks
-  bool lead[4] = {true, true, true, true};
-  uint32_t qmask[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int m2 = 0; m2 < 4; ++m2) {
-    for (int src = 0; src < 32; ++src) {
-      const uint32_t k2 = __shfl_sync(0xffffffffu, key[m2], src);
-      const int e2 = src + 32 * m2;
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        if (k2 == key[m]) {
-          qmask[m] |= 1u << (e2 / kTopK);
-          if (e2 < lane + 32 * m) lead[m] = false;
+    for (int i = 0; i < 4; ++i) {
+      const int b = b4[i];
+      key[i] = kNone;
+      val[i] = 1u << q;
+      if (qpos >= 0) {
+        if (b >= 0 && b <= qpos / kBlock) {
+          if (kPaged && kv_block_row(P.pages, qstream, g, b, P.G, P.capacity) < 0)
+            raise_error(MSA_DEVERR_PAGE_RANGE);
+          else
+            key[i] = (static_cast<uint32_t>(qseg) << 24) | static_cast<uint32_t>(b);
+        } else if (b > qpos / kBlock) {
+          raise_error(MSA_DEVERR_SEL_RANGE);
         }
       }
     }
   }
-  // place of each leader: leading keys smaller than its own
-  int rank[4] = {0, 0, 0, 0};
-  int n = 0;
+  // bitonic sort, ascending by key (element e = 4 lane + i)
 #pragma unroll
-  for (int m2 = 0; m2 < 4; ++m2) {
-    const bool l2 = lead[m2] && key[m2] != 0xffffffffu;
-    uint32_t ballot = __ballot_sync(0xffffffffu, l2);
-    n += __popc(ballot);
-    while (ballot != 0u) {
-      const int src = __ffs(ballot) - 1;
-      ballot &= ballot - 1u;
-      const uint32_t k2 = __shfl_sync(0xffffffffu, key[m2], src);
+  for (int k = 2; k <= 128; k <<= 1) {
 #pragma unroll
-      for (int m = 0; m < 4; ++m) rank[m] += k2 < key[m] ? 1 : 0;
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = 4 * lane + i;
+          const uint32_t ok2 = __shfl_xor_sync(kFull, key[i], j >> 2);
+          const uint32_t ov2 = __shfl_xor_sync(kFull, val[i], j >> 2);
+          const bool up = (e & k) == 0;
+          const bool lower = (e & j) == 0;
+          if (lower == up ? ok2 < key[i] : ok2 > key[i]) {
+            key[i] = ok2;
+            val[i] = ov2;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if ((i & j) != 0) continue;
+          const int i2 = i | j;
+          const bool up = ((4 * lane + i) & k) == 0;
+          if ((key[i] > key[i2]) == up && key[i] != key[i2]) {
+            const uint32_t tk = key[i], tv = val[i];
+            key[i] = key[i2];
+            val[i] = val[i2];
+            key[i2] = tk;
+            val[i2] = tv;
+          }
+        }
+      }
     }
   }
+  // run heads, and each run's OR of query bits (a segmented scan towards the
+  // run's end; bit 31 of acc marks "a run end lies in the scanned range")
+  const uint32_t next0 = __shfl_down_sync(kFull, key[0], 1);
+  const uint32_t prev3 = __shfl_up_sync(kFull, key[3], 1);
+  uint32_t acc[4];
+  bool head[4];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    if (lead[m] && key[m] != 0xffffffffu) {
-      pl.blocks[rank[m]] = static_cast<int>(key[m] & 0xffffffu);
-      pl.segs[rank[m]] = static_cast<uint8_t>(key[m] >> 24);
-      pl.masks[rank[m]] = static_cast<uint8_t>(qmask[m]);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t nxt = i < 3 ? key[i + 1] : (lane < 31 ? next0 : kNone - 1);
+    const uint32_t prv = i > 0 ? key[i - 1] : (lane > 0 ? prev3 : kNone - 1);
+    const bool end = (i == 3 && lane == 31) || nxt != key[i];
+    head[i] = (i == 0 && lane == 0) || prv != key[i];
+    acc[i] = val[i] | (end ? 0x80000000u : 0u);
+  }
+#pragma unroll
+  for (int d = 1; d < 128; d <<= 1) {
+    uint32_t far[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tt = i + d;                          // element e + d, in lane + tt / 4
+      if (tt < 4) {
+        far[i] = acc[tt];
+      } else {
+        const uint32_t x = __shfl_down_sync(kFull, acc[tt & 3], tt >> 2);
+        far[i] = lane + (tt >> 2) < 32 ? x : 0x80000000u;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if ((acc[i] & 0x80000000u) == 0u) acc[i] |= far[i];
+  }
+  // places of the distinct valid keys
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mine += (head[i] && key[i] != kNone) ? 1 : 0;
+  int before = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(kFull, before, o);
+    if (lane >= o) before += x;
+  }
+  const int n = __shfl_sync(kFull, before, 31);
+  before -= mine;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (head[i] && key[i] != kNone) {
+      pl.blocks[before] = static_cast<int>(key[i] & 0xffffffu);
+      pl.segs[before] = static_cast<uint8_t>(key[i] >> 24);
+      pl.masks[before] = static_cast<uint8_t>(acc[i] & 0xffu);
+      ++before;
     }
   }
   if (lane == 0) pl.n = n;
   __syncwarp();
+}
+
+// The plan of every tile, one warp per tile, ahead of the attention kernel
+// (which reads them after its programmatic-dependent-launch wait): planning
+// inside the attention kernel starved for issue slots next to the softmax
+// warps (~50K cycles per tile).
+template <bool kPaged>
+__global__ void __launch_bounds__(256) plan_tiles_kernel(const Params P) {
+  pdl_trigger();
+  pdl_wait();                                          // the selections come from the kernel before
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t < P.G * P.n_tiles) build_plan<kPaged>(P, t, P.plans[t], threadIdx.x & 31);
 }
 
 template <bool kPaged>
@@ -272,10 +335,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tasks = P.G * P.n_tiles;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&B.plan_full[i], 1);
-      mbar_init(&B.plan_empty[i], 7);       // K loader, V loader, MMA, 4 softmax warps
-    }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&B.s_full[i], 1);
       mbar_init(&B.p_full[i], 4);
@@ -292,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&B.vempty[i], 1);
     }
     mbar_init(B.o_empty, 4);
-    mbar_init(B.mma_done, 1);
+    mbar_init(&B.mma_done[0], 1);
+    mbar_init(&B.mma_done[1], 1);
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(B.tmem_slot, kTmemCols);
@@ -302,37 +362,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   pdl_wait();
 
-  if (warp == 3) {
-    // ------------------------------ planner ------------------------------------
-    int tc = 0;
-    for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++tc) {
-      const int slot = tc & 1;
-      bool ok = true;
-      if (tc >= 2) ok = mbar_wait(&B.plan_empty[slot], ((tc >> 1) - 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      build_plan<kPaged>(P, t, plan_at(smem, slot), lane);
-      if (lane == 0) mbar_arrive(&B.plan_full[slot]);
-    }
-  } else if (warp == 0 || warp == 2) {
-    // ---------------- loaders: warp 0 the Q tile and K blocks, warp 2 V blocks ----
+  if (warp == 0) {
+    // ------------------------ the Q tile and the K blocks (lane 0) ---------------------
     if (lane == 0) {
-      const bool is_k = warp == 0;
-      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
-      uint64_t* rfull = is_k ? B.kfull : B.vfull;
-      uint64_t* rempty = is_k ? B.kempty : B.vempty;
-      uint8_t* rbase = smem + (is_k ? Layout::kKOff : Layout::kVOff);
-      const int ring_n = is_k ? kKRing : kVRing;
       int tc = 0, ring = 0, q_use = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
-        const int slot = tc & 1;
-        ok = mbar_wait(&B.plan_full[slot], (tc >> 1) & 1);
-        if (!ok) break;
-        const Plan& pl = plan_at(smem, slot);
+        const Plan& pl = P.plans[t];
         int g, q0;
         tile_coords(P, t, g, q0);
-        if (is_k && pl.n > 0) {
+        if (pl.n > 0) {
           // the previous tile's S MMAs have finished with the Q tile
           if (q_use > 0) ok = mbar_wait(B.q_empty, (q_use - 1) & 1);
           if (!ok) break;
@@ -348,58 +387,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++q_use;
         }
         for (int j = 0; j < pl.n && ok; ++j, ++ring) {
-          const int st = ring % ring_n;
-          const int use = ring / ring_n;
-          if (use > 0) ok = mbar_wait(&rempty[st], (use - 1) & 1);
+          const int st = ring % kKRing;
+          const int use = ring / kKRing;
+          if (use > 0) ok = mbar_wait(&B.kempty[st], (use - 1) & 1);
           if (!ok) break;
           const int s = pl.seg_stream[pl.segs[j]];
           const int row = kPaged ? static_cast<int>(kv_block_row(P.pages, s, g, pl.blocks[j], P.G, P.capacity))
                                  : (s * P.G + g) * P.capacity + pl.blocks[j] * kBlock;
-          uint8_t* dst = rbase + st * kTile;
-          mbar_arrive_expect_tx(&rfull[st], kTile);
-          tma_load_2d(dst, map, 0, row, &rfull[st]);
-          tma_load_2d(dst + kHalf, map, 64, row, &rfull[st]);
+          uint8_t* dst = smem + Layout::kKOff + st * kTile;
+          mbar_arrive_expect_tx(&B.kfull[st], kTile);
+          tma_load_2d(dst, &tm_k, 0, row, &B.kfull[st]);
+          tma_load_2d(dst + kHalf, &tm_k, 64, row, &B.kfull[st]);
         }
-        mbar_arrive(&B.plan_empty[slot]);
       }
       // no copy may still be landing when the CTA exits
-      for (int j = max(0, ring - ring_n); j < ring; ++j) mbar_wait(&rfull[j % ring_n], (j / ring_n) & 1);
-      if (is_k && q_use > 0) mbar_wait(B.q_full, (q_use - 1) & 1);
+      for (int j = max(0, ring - kKRing); j < ring; ++j) mbar_wait(&B.kfull[j % kKRing], (j / kKRing) & 1);
+      if (q_use > 0) mbar_wait(B.q_full, (q_use - 1) & 1);
+    }
+  } else if (warp == 2) {
+    // ------------------------------ V loader (lane 0) ------------------------------
+    if (lane == 0) {
+      int tc = 0, ring = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+        const Plan& pl = P.plans[t];
+        int g, q0;
+        tile_coords(P, t, g, q0);
+        for (int j = 0; j < pl.n && ok; ++j, ++ring) {
+          const int st = ring % kVRing;
+          const int use = ring / kVRing;
+          if (use > 0) ok = mbar_wait(&B.vempty[st], (use - 1) & 1);
+          if (!ok) break;
+          const int s = pl.seg_stream[pl.segs[j]];
+          const int row = kPaged ? static_cast<int>(kv_block_row(P.pages, s, g, pl.blocks[j], P.G, P.capacity))
+                                 : (s * P.G + g) * P.capacity + pl.blocks[j] * kBlock;
+          uint8_t* dst = smem + Layout::kVOff + st * kTile;
+          mbar_arrive_expect_tx(&B.vfull[st], kTile);
+          tma_load_2d(dst, &tm_v, 0, row, &B.vfull[st]);
+          tma_load_2d(dst + kHalf, &tm_v, 64, row, &B.vfull[st]);
+        }
+      }
+      for (int j = max(0, ring - kVRing); j < ring; ++j) mbar_wait(&B.vfull[j % kVRing], (j / kVRing) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer -----------------------------------
+    // ------------------------- S issuer: S = Q . K_b^T (lane 0) -------------------
+    // S and P . V come from two issuing threads: the tensor pipe drains when
+    // one thread switches operand configuration (shared-memory / tensor-memory
+    // A, K- / MN-major B), not when two threads' streams interleave.
     if (lane == 0) {
       const uint32_t q_base = smem_addr(smem + Layout::kQOff);
       const uint32_t k_base = smem_addr(smem + Layout::kKOff);
-      const uint32_t v_base = smem_addr(smem + Layout::kVOff);
-      int tc = 0, kr = 0, vr = 0, blk = 0, segs_done = 0, q_use = 0;
+      int tc = 0, kr = 0, blk = 0, q_use = 0;
       bool ok = true;
-      // O (+)= P . V for global block `b` (union position j of the current plan)
-      auto pv = [&](const Plan& pl, int j, int b) {
-        const bool seg_first = j == 0 || pl.segs[j] != pl.segs[j - 1];
-        const int sb = b % kSBufs;
-        if (ok) ok = mbar_wait(&B.p_full[sb], (b / kSBufs) & 1);
-        if (ok && seg_first && segs_done > 0) ok = mbar_wait(B.o_empty, (segs_done - 1) & 1);
-        const int st = vr % kVRing;
-        if (ok) ok = mbar_wait(&B.vfull[st], (vr / kVRing) & 1);
-        if (!ok) return;
-        tc_fence_after();
-        const uint32_t vb = v_base + st * kTile;
-        const uint32_t pa = tmem_base + kSCol + sb * 128;      // P: 64 columns of bf16 pairs
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ts(tmem_base + kOCol, pa + kk * 8, umma_desc_sw128_mn(vb + kk * 2048, kHalf), kIdescPV,
-                      (seg_first && kk == 0) ? 0u : 1u);
-        umma_commit(&B.vempty[st]);
-        umma_commit(&B.pv_done[sb]);
-        ++vr;
-        if (seg_first) ++segs_done;
-      };
       for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
-        const int slot = tc & 1;
-        ok = mbar_wait(&B.plan_full[slot], (tc >> 1) & 1);
-        if (!ok) break;
-        const Plan& pl = plan_at(smem, slot);
+        const Plan& pl = P.plans[t];
         if (pl.n > 0) {
           ok = mbar_wait(B.q_full, q_use & 1);
           ++q_use;
@@ -424,15 +465,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(&B.s_full[sb]);
             if (j == pl.n - 1) umma_commit(B.q_empty);         // the tile's last use of Q
             ++kr;
-            if (j >= kLag) pv(pl, j - kLag, b - kLag);
           }
-          for (int j = max(0, pl.n - kLag); j < pl.n && ok; ++j) pv(pl, j, blk + j);
           blk += pl.n;
         }
-        mbar_arrive(&B.plan_empty[slot]);
       }
-      umma_commit(B.mma_done);
-      mbar_wait(B.mma_done, 0);
+      umma_commit(&B.mma_done[0]);
+      mbar_wait(&B.mma_done[0], 0);
+    }
+  } else if (warp == 3) {
+    // ---------------------- P . V issuer: O (+)= P . V_b (lane 0) -----------------
+    if (lane == 0) {
+      const uint32_t v_base = smem_addr(smem + Layout::kVOff);
+      int tc = 0, vr = 0, blk = 0, segs_done = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+        const Plan& pl = P.plans[t];
+        for (int j = 0; j < pl.n && ok; ++j) {
+          const int b = blk + j;
+          const bool seg_first = j == 0 || pl.segs[j] != pl.segs[j - 1];
+          const int sb = b % kSBufs;
+          ok = mbar_wait(&B.p_full[sb], (b / kSBufs) & 1);
+          if (ok && seg_first && segs_done > 0) ok = mbar_wait(B.o_empty, (segs_done - 1) & 1);
+          const int st = vr % kVRing;
+          if (ok) ok = mbar_wait(&B.vfull[st], (vr / kVRing) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t vb = v_base + st * kTile;
+          const uint32_t pa = tmem_base + kSCol + sb * 128;      // P: 64 columns of bf16 pairs
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ts(tmem_base + kOCol, pa + kk * 8, umma_desc_sw128_mn(vb + kk * 2048, kHalf), kIdescPV,
+                        (seg_first && kk == 0) ? 0u : 1u);
+          umma_commit(&B.vempty[st]);
+          umma_commit(&B.pv_done[sb]);
+          ++vr;
+          if (seg_first) ++segs_done;
+        }
+        blk += pl.n;
+      }
+      umma_commit(&B.mma_done[1]);
+      mbar_wait(&B.mma_done[1], 0);
     }
   } else if (warp >= 4) {
     // ---------------- softmax and output: one thread per (query, head) row --------
@@ -443,11 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tc = 0, blk = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++tc) {
-      const int slot = tc & 1;
-      if (ok) ok = mbar_wait(&B.plan_full[slot], (tc >> 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const Plan& pl = plan_at(smem, slot);
+      const Plan& pl = P.plans[t];
       int g, q0;
       tile_coords(P, t, g, q0);
       const int qi = q0 + q;
@@ -589,8 +657,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(dst + i) = make_uint4(0u, 0u, 0u, 0u);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B.plan_empty[slot]);
     }
   }
   __syncthreads();
