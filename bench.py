@@ -532,11 +532,6 @@ def dsa_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches_per
     }
 
 
-# Prefill attention runs the union-tile kernel up to this cache capacity
-# (tokens per stream) and the per-pair kernel beyond it.
-UNION_MAX_CONTEXT = 32768
-
-
 def prefill_flops(w) -> tuple[int, int]:
     """Algorithmic FLOPs of one prefill step: the indexer contraction over
     each query's visible keys (2 * Di per key per group) and the attention
@@ -556,7 +551,7 @@ def prefill_line(args, w, world, ms, k_ms, e2e_ms, e2e_steps, h2d, d2h, launches
     tokens = w.n_queries * world
     tf = (ind + att) / (ms * 1e-3) / 1e12
     ktf = att / (k_ms * 1e-3) / 1e12                 # the attention kernel: its algorithmic FLOPs
-    kernel = "sparse_attn_prefill_union" if w.capacity <= UNION_MAX_CONTEXT else "sparse_attn_prefill_tc"
+    kernel = "sparse_attn_prefill_union"
     return {
         "metric": f"MSA prefill tokens/s ({w.name}); achieved TFLOP/s vs bf16 peak",
         "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -13,7 +13,6 @@
 #include "msa.h"
 #include "msa_append.cuh"
 #include "msa_attn_decode_sk.cuh"
-#include "msa_attn_prefill_tc.cuh"
 #include "msa_attn_prefill_union.cuh"
 #include "msa_common.cuh"
 #include "msa_decode_fused.cuh"
@@ -157,21 +156,15 @@ size_t scores_workspace(const msa_shape* sh, int32_t n_q) {
 // Decode attention workspace: two partial results per CTA of the persistent
 // grid (at most kMaxCtas CTAs, at most one per unit).  Depends only on the
 // pair count, so the workspace query and the launch always agree.
-// Prefill attention takes the union-tile kernel up to this cache capacity
-// (tokens per stream) and the per-pair kernel beyond it.
-constexpr int kUnionMaxContext = 32768;
 
-// Prefill attention on short contexts: the plan of every 8-query tile.
+// Prefill attention: the plan of every 8-query tile.
 int64_t union_tasks(const msa_shape* sh, int32_t n_q) {
   return static_cast<int64_t>(sh->n_kv_heads) * ((n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ);
 }
 
 size_t attn_workspace(const msa_shape* sh, int32_t n_q, int mode) {
   if (n_q == 0) return 0;
-  if (mode == MSA_MODE_PREFILL) {
-    if (sh->capacity > kUnionMaxContext) return 0;
-    return static_cast<size_t>(union_tasks(sh, n_q)) * sizeof(msa::uattn::Plan);
-  }
+  if (mode == MSA_MODE_PREFILL) return static_cast<size_t>(union_tasks(sh, n_q)) * sizeof(msa::uattn::Plan);
   const int64_t units = static_cast<int64_t>(n_q) * sh->n_kv_heads * msa::dattn::kTopK;
   const int64_t ctas = std::min<int64_t>(units, msa::dattn::kMaxCtas);
   return static_cast<size_t>(ctas) * 2 * msa::dattn::kPartial * sizeof(float);
@@ -207,65 +200,38 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   int sms = 0;
   if ((st = current_device_sms(&sms)) != MSA_OK) return st;
   if (mode == MSA_MODE_PREFILL) {
-    // tensor-core kernel, one persistent CTA per SM
+    // tensor-core kernels, one persistent CTA per SM: tiles of 8 queries over the
+    // union of their selected blocks; a first kernel plans every tile into the
+    // workspace, the attention kernel reads the plans after its dependent-launch wait
     CUtensorMap tm_q;
     if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q,
                              static_cast<int64_t>(n_q) * sh->n_q_heads, 16)) != MSA_OK)
       return st;
-    // Short contexts: tiles of 8 queries over the union of their blocks.  A
-    // union block costs ~1.1 us of a CTA and a per-pair (query, group) ~14 us,
-    // so the union wins while 8 queries' selections overlap enough: with
-    // selections spread over V visible blocks the union holds about
-    // V (1 - (1 - 16/V)^8) blocks, below the per-pair cost of 8 pairs up to
-    // V ~ 256.  The cache capacity bounds V.
-    if (sh->capacity <= kUnionMaxContext) {
-      const auto ukernel = pg.table != nullptr ? msa::uattn::sparse_attn_prefill_union_kernel<true>
-                                               : msa::uattn::sparse_attn_prefill_union_kernel<false>;
-      static std::atomic<uint64_t> u_smem_done[2] = {0, 0};
-      if ((st = ensure_smem(ukernel, msa::uattn::Layout::kBytes, u_smem_done[pg.table != nullptr])) != MSA_OK)
-        return st;
-      msa::uattn::Params U;
-      U.sel = sel;
-      U.q_stream = q_stream;
-      U.q_pos = q_pos;
-      U.out = reinterpret_cast<__nv_bfloat16*>(out);
-      U.n_q = n_q;
-      U.G = G;
-      U.n_streams = sh->n_streams;
-      U.capacity = sh->capacity;
-      U.n_tiles = (n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ;
-      U.scale_log2 = softmax_scale * 1.4426950408889634f;
-      U.pages = pg;
-      U.plans = static_cast<msa::uattn::Plan*>(workspace);
-      const int64_t tasks = static_cast<int64_t>(G) * U.n_tiles;
-      const int64_t ugrid = std::min<int64_t>(sms, tasks);
-      const auto pkernel_plan = pg.table != nullptr ? msa::uattn::plan_tiles_kernel<true>
-                                                    : msa::uattn::plan_tiles_kernel<false>;
-      launch(pkernel_plan, dim3(static_cast<unsigned>((tasks + 7) / 8)), dim3(256), 0, s, U);
-      launch(ukernel, dim3(static_cast<unsigned>(ugrid)), dim3(msa::uattn::kThreads), msa::uattn::Layout::kBytes, s, tm_q,
-             tm_k, tm_v, U);
-      return cuda_status(cudaGetLastError());
-    }
-    // long contexts: one (query, group) pair at a time, its 16 blocks only
-    const auto pkernel = pg.table != nullptr ? msa::pattn::sparse_attn_prefill_tc_kernel<true>
-                                             : msa::pattn::sparse_attn_prefill_tc_kernel<false>;
-    static std::atomic<uint64_t> tc_smem_done[2] = {0, 0};
-    if ((st = ensure_smem(pkernel, msa::pattn::Layout::kBytes, tc_smem_done[pg.table != nullptr])) != MSA_OK)
+    const auto ukernel = pg.table != nullptr ? msa::uattn::sparse_attn_prefill_union_kernel<true>
+                                             : msa::uattn::sparse_attn_prefill_union_kernel<false>;
+    static std::atomic<uint64_t> u_smem_done[2] = {0, 0};
+    if ((st = ensure_smem(ukernel, msa::uattn::Layout::kBytes, u_smem_done[pg.table != nullptr])) != MSA_OK)
       return st;
-    msa::pattn::Params Q;
-    Q.sel = sel;
-    Q.q_stream = q_stream;
-    Q.q_pos = q_pos;
-    Q.out = reinterpret_cast<__nv_bfloat16*>(out);
-    Q.n_q = n_q;
-    Q.G = G;
-    Q.n_streams = sh->n_streams;
-    Q.capacity = sh->capacity;
-    Q.scale_log2 = softmax_scale * 1.4426950408889634f;
-    Q.pages = pg;
-    const int64_t grid = std::min<int64_t>(sms, n_pairs);
-    launch(pkernel, dim3(static_cast<unsigned>(grid)), dim3(msa::pattn::kThreads), msa::pattn::Layout::kBytes, s, tm_q,
-           tm_k, tm_v, Q);
+    msa::uattn::Params U;
+    U.sel = sel;
+    U.q_stream = q_stream;
+    U.q_pos = q_pos;
+    U.out = reinterpret_cast<__nv_bfloat16*>(out);
+    U.n_q = n_q;
+    U.G = G;
+    U.n_streams = sh->n_streams;
+    U.capacity = sh->capacity;
+    U.n_tiles = (n_q + msa::uattn::kTileQ - 1) / msa::uattn::kTileQ;
+    U.scale_log2 = softmax_scale * 1.4426950408889634f;
+    U.pages = pg;
+    U.plans = static_cast<msa::uattn::Plan*>(workspace);
+    const int64_t tasks = static_cast<int64_t>(G) * U.n_tiles;
+    const int64_t ugrid = std::min<int64_t>(sms, tasks);
+    const auto pkernel_plan = pg.table != nullptr ? msa::uattn::plan_tiles_kernel<true>
+                                                  : msa::uattn::plan_tiles_kernel<false>;
+    launch(pkernel_plan, dim3(static_cast<unsigned>((tasks + 7) / 8)), dim3(256), 0, s, U);
+    launch(ukernel, dim3(static_cast<unsigned>(ugrid)), dim3(msa::uattn::kThreads), msa::uattn::Layout::kBytes, s, tm_q,
+           tm_k, tm_v, U);
     return cuda_status(cudaGetLastError());
   }
   // decode: persistent stream-K grid over (pair, selected block) units, or

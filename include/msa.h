@@ -194,9 +194,8 @@ MSA_API int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, co
  * MSA pull request, "Implementation", batch case: the query's block-level
  * selection combined with the token-level causal mask.  Workspace:
  * msa_workspace_bytes(shape, n_q, MSA_MODE_PREFILL) bytes, 16-byte aligned:
- * on caches of at most 32768 tokens per stream it holds the plan of every
- * tile of 8 queries (the union of their selected blocks), written by a
- * first kernel and read by the attention kernel; longer caches need none. */
+ * it holds the plan of every tile of 8 queries (the union of their selected
+ * blocks), written by a first kernel and read by the attention kernel. */
 MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
                             const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
                             const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,

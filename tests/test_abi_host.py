@@ -114,12 +114,11 @@ def test_attention_validation_and_workspace(lib):
     need = lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_DECODE)
     assert need == min(2 * 4 * 16, 256) * 2 * 16 * 130 * 4
     assert lib.msa_workspace_bytes(ctypes.byref(s), 1000, msa.MODE_DECODE) >= 256 * 2 * 16 * 130 * 4
-    # prefill attention on caches of at most 32K tokens per stream: the plan
-    # of every 8-query tile (844 bytes) per group; longer caches need none
+    # prefill attention: the plan of every 8-query tile (844 bytes) per group
     plans = lambda n_q, G=4: G * ((n_q + 7) // 8) * 844          # noqa: E731
     assert lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_PREFILL) == plans(2)
     long_cap = msa.Shape(n_streams=2, capacity=65536).c()
-    assert lib.msa_workspace_bytes(ctypes.byref(long_cap), 2, msa.MODE_PREFILL) == 0
+    assert lib.msa_workspace_bytes(ctypes.byref(long_cap), 2, msa.MODE_PREFILL) == plans(2)
     # 4096 queries over 2 streams: prefill-shaped, the block scores take the tile path
     big = lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_DECODE)
     assert big > 0 and big == lib.msa_workspace_bytes(ctypes.byref(s), 4096, msa.MODE_PREFILL)

@@ -57,8 +57,8 @@ def test_paged_prefill_ties_f16():
     assert rep["max_score_err"] == 0.0
 
 
-def test_paged_prefill_long_context_per_pair_path():
-    # caches above 32K tokens per stream: the per-pair prefill kernel on pages
+def test_paged_prefill_long_context():
+    # 33K-token caches on pages: long block tables, few blocks shared per tile
     w = W.Workload("paged_prefill_2x64_on_33000", 2, 33000, 33064, "new")
     inp = W.make_inputs(w, seed=49)
     rep = PT.full_parity(inp, prefill=True, paged=dict(seed=7, spare_pages=3, shared_prefix_blocks=4))
@@ -143,7 +143,7 @@ def test_unmapped_page_is_skipped_and_flagged():
     PT.check_attention(out.cpu(), o)
 
 
-@pytest.mark.parametrize("cap_blocks", [24, 260], ids=["union_path", "per_pair_path"])
+@pytest.mark.parametrize("cap_blocks", [24, 260], ids=["short_cache", "long_cache"])
 def test_unmapped_page_is_skipped_in_prefill(cap_blocks):
     """Prefill attention with a selected block on an unmapped page: the block
     drops out of that query's attention (bit-identical to dropping it from the

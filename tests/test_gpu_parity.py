@@ -140,9 +140,9 @@ def test_attention_given_selection(n_q, mode):
     report(f"attention n_q={n_q} {mode}", PT.check_attention(out.cpu(), want))
 
 
-def test_prefill_attention_long_context_per_pair_path():
-    """Caches above 32K tokens per stream take the per-pair prefill kernel
-    (shorter ones the union-tile kernel): the same oracle check there."""
+def test_prefill_attention_long_context():
+    """Caches of 38400 tokens per stream (300 blocks): few blocks shared
+    between the queries of a tile, the same oracle check."""
     g = torch.Generator().manual_seed(91)
     S, cap, G = 2, 128 * 300, 4
     lengths = [cap, 20000]
@@ -157,7 +157,7 @@ def test_prefill_attention_long_context_per_pair_path():
     report("prefill attention, 38400-token caches", PT.check_attention(out.cpu(), want))
 
 
-@pytest.mark.parametrize("cap", [1024, 128 * 260], ids=["union_path", "per_pair_path"])
+@pytest.mark.parametrize("cap", [1024, 128 * 260], ids=["short_cache", "long_cache"])
 def test_prefill_attention_edge_queries(cap):
     """Prefill attention on a ragged batch (21 queries: two 8-query tiles and
     a tail of 5) whose tiles mix streams, with shuffled selection lists (-1
