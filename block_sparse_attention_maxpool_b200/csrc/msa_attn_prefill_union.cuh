@@ -7,10 +7,11 @@
 // local block.
 //
 // A tile is 8 consecutive queries of one group: 8 x 16 = 128 query-head
-// rows, the M dimension of every MMA.  A planner warp builds the tile's
-// union of the 8 queries' selected blocks, each with an 8-bit mask
-// of the queries that selected it (queries of different streams form
-// separate segments of the union).  For every block b of the union:
+// rows, the M dimension of every MMA.  plan_tiles_kernel, launched just
+// before, builds each tile's union of the 8 queries' selected blocks, each
+// with an 8-bit mask of the queries that selected it (queries of different
+// streams form separate segments of the union).  For every block b of the
+// union:
 //   S = Q . K_b^T          M=128 rows, N=128 keys, K=128 dims (TMEM, f32)
 //   P = exp2(S - m)        masked: a row keeps only keys of blocks its query
 //                          selected and j <= its position; one thread per
@@ -43,9 +44,15 @@
 //
 // Warp roles: 0 loads the Q tile and the K blocks, 1 issues S, 2 loads the
 // V blocks, 3 issues P . V, 4-7 run the softmax and write the output (one
-// TMEM lane quarter each), 8 plans the tiles one tile ahead.  Shared
-// memory: Q 32 KB, K ring 3 x 32 KB, V ring 2 x 32 KB, two plans.  Tensor
-// memory: three S/P buffers and O (all 512 columns).
+// TMEM lane quarter each).  Shared memory: Q 32 KB, K ring 3 x 32 KB, V ring
+// 2 x 32 KB.  Tensor memory: three S/P buffers and O (all 512 columns).
+//
+// Per block, a softmax warp whose queries selected it spends ~1900 cycles
+// (S load ~250, row max ~280, 128 exponentials ~1330 against a floor of
+// 1024 on the special-function unit, which runs 4 per clock per SM
+// quarter), one whose queries did not ~400; the quarters are busy on about
+// half the blocks each, at random, and three S buffers let them drift at
+// most two blocks apart, so the slowest quarter sets the pace.
 #pragma once
 
 #include "msa_common.cuh"
@@ -132,6 +139,31 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed f32x2 arithmetic (sm_100 and later): two lanes per instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// max(a, b, c) in one instruction (three-input max.f32, sm_100 and later).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Tile t -> (group, first query).  Group-major, so the CTAs running at the
@@ -533,16 +565,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int sb = b % kSBufs;
         const uint32_t sbuf = tmem_base + lane_addr + kSCol + sb * 128;
+        // mask: the row's query selected this block (else its P row is
+        // exp2(-inf) = 0), and keys j <= its position (only its local block
+        // is cut).  Read before the wait, so that the plan's latency hides
+        // behind it.
+        const bool mine = ((pl.masks[j] >> q) & 1) != 0 && pq >= 0;
+        const int jmax = mine ? pq - pl.blocks[j] * kBlock : -1;       // last visible key in the block
+        const bool active = __any_sync(0xffffffffu, mine);
         ok = mbar_wait(&B.s_full[sb], (b / kSBufs) & 1);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        // mask: the row's query selected this block (else its P row is
-        // exp2(-inf) = 0), and keys j <= its position (only its local block
-        // is cut)
-        const bool mine = ((pl.masks[j] >> q) & 1) != 0 && pq >= 0;
-        const int jmax = mine ? pq - pl.blocks[j] * kBlock : -1;       // last visible key in the block
-        const bool active = __any_sync(0xffffffffu, mine);
         float s[kBlock];
         if (active) {
           float v0[32], v1[32], v2[32], v3[32];
@@ -560,13 +593,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         float mb = -INFINITY;
+        if (active && __any_sync(0xffffffffu, mine && jmax < kBlock - 1)) {
+#pragma unroll
+          for (int c = 0; c < kBlock; ++c) s[c] = c <= jmax ? s[c] : -INFINITY;
+        }
         if (active) {
-          if (__any_sync(0xffffffffu, mine && jmax < kBlock - 1)) {
+          // four independent chains of three-input maxima: 18 dependent steps
+          // instead of 128
+          float m4[4];
 #pragma unroll
-            for (int c = 0; c < kBlock; ++c) s[c] = c <= jmax ? s[c] : -INFINITY;
-          }
+          for (int i = 0; i < 4; ++i) m4[i] = fmax3(s[i], s[4 + i], s[8 + i]);
 #pragma unroll
-          for (int c = 0; c < kBlock; ++c) mb = fmaxf(mb, s[c]);
+          for (int c = 12; c < kBlock - 4; c += 8)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], s[c + i], s[c + 4 + i]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], s[kBlock - 4 + i]);
+          mb = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
           mb = mine ? mb * P.scale_log2 : -INFINITY;                     // max of the scaled scores
         }
         const bool raise = mb > m_ref + kRescale;
@@ -595,20 +638,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float neg_m = mine ? -m_ref : -INFINITY;
         // P = exp2(s - m_ref) as bf16 pairs over the first 64 columns of the buffer
         if (active) {
-          float rs = 0.f;
+          const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
+          const float2 nm2 = make_float2(neg_m, neg_m);
+          float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             float pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float a = ex2_approx(fmaf(s[h * 64 + 2 * i], P.scale_log2, neg_m));
-              const float c2 = ex2_approx(fmaf(s[h * 64 + 2 * i + 1], P.scale_log2, neg_m));
-              rs += a + c2;
-              pk[i] = __uint_as_float(pack_bf16(a, c2));
+              const float2 x = ffma2(make_float2(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]), sc2, nm2);
+              const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              rs = fadd2(rs, e);
+              pk[i] = __uint_as_float(pack_bf16(e.x, e.y));
             }
             tmem_st32(sbuf + h * 32, pk);
           }
-          l += rs;
+          l += rs.x + rs.y;
         } else {
           float z[32];
 #pragma unroll
