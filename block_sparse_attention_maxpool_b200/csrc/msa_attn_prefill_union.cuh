@@ -85,7 +85,7 @@ struct Plan {
   int pos[kTileQ];                // query positions (-1: no query / invalid)
   int seg_stream[kTileQ];         // stream of the segment whose id is this query index
   uint8_t seg_rows[kTileQ];       // queries of that segment
-  int blocks[kMaxUnion];          // ascending within each segment
+  int blocks[kMaxUnion];          // segments in order; within one, the order order_plan picks
   uint8_t masks[kMaxUnion];       // queries that selected the block
   uint8_t segs[kMaxUnion];        // segment id (index of its first query)
 };
@@ -173,6 +173,60 @@ __device__ __forceinline__ void tile_coords(const Params& P, int t, int& g, int&
   q0 = (t - g * P.n_tiles) * kTileQ;
 }
 
+// Order of the union within each segment.  The softmax warp of TMEM lane
+// quarter k serves queries 2k and 2k+1: on a block neither selected it only
+// writes zeros (~400 cycles), otherwise it computes a row of exponentials
+// (~1900), and with three S buffers the four quarters can drift only two
+// blocks apart, so runs of blocks busy on one quarter stall the others.
+// Greedily, the next block is one whose busy quarters overlap least with the
+// previous block's (ties: the lower block).  Any order gives the same
+// attention up to rounding (the online softmax does not depend on it).
+__device__ __forceinline__ void order_plan(Plan& pl, int n, int lane) {
+  constexpr uint32_t kFull = 0xffffffffu;
+  auto quarters = [](uint32_t m) { return (m | (m >> 1)) & 0x55u; };   // quarter k busy: bit 2k
+  uint32_t cm[4];
+  int cb[4], cs[4];
+  bool live[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e = lane + 32 * k;
+    live[k] = e < n;
+    cb[k] = live[k] ? pl.blocks[e] : 0;
+    cm[k] = live[k] ? pl.masks[e] : 0u;
+    cs[k] = live[k] ? pl.segs[e] : -1;
+  }
+  __syncwarp();
+  uint32_t prev = 0u;
+  for (int pos = 0; pos < n; ++pos) {
+    const int sg = pl.segs[pos];                   // segment ranges do not move
+    uint32_t best = 0xffffffffu;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (live[k] && cs[k] == sg) {
+        const uint32_t key = (static_cast<uint32_t>(__popc(quarters(cm[k]) & prev)) << 8) | static_cast<uint32_t>(lane + 32 * k);
+        best = min(best, key);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(kFull, best, o));
+    const int c = static_cast<int>(best & 0xffu);
+    uint32_t wq = 0u;
+    if ((c & 31) == lane) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k == (c >> 5)) {
+          live[k] = false;
+          pl.blocks[pos] = cb[k];
+          pl.masks[pos] = static_cast<uint8_t>(cm[k]);
+          wq = quarters(cm[k]);
+        }
+      }
+    }
+    prev = __shfl_sync(kFull, wq, c & 31);
+  }
+  __syncwarp();
+}
+
 // The planner warp: union of the tile's selections, by segment, into `pl`.
 // The 128 (query, slot) entries become sortable keys (segment << 24 |
 // block; ~0 for an empty or invalid entry), each carrying its query's bit;
@@ -184,7 +238,7 @@ __device__ __forceinline__ void tile_coords(const Params& P, int t, int& g, int&
 // whatever the order of a query's list, and a -1 or out-of-range entry
 // anywhere in it is simply left out.  With paged caches a selected block
 // whose page is missing is left out too (and MSA_DEVERR_PAGE_RANGE set), as
-// if the query had not selected it.
+// if the query had not selected it.  order_plan then reorders each segment.
 template <bool kPaged>
 __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, int lane) {
   constexpr uint32_t kFull = 0xffffffffu;
@@ -341,6 +395,7 @@ __device__ __forceinline__ void build_plan(const Params& P, int t, Plan& pl, int
   }
   if (lane == 0) pl.n = n;
   __syncwarp();
+  order_plan(pl, n, lane);
 }
 
 // The plan of every tile, one warp per tile, ahead of the attention kernel
