@@ -227,7 +227,7 @@ __device__ __forceinline__ void order_plan(Plan& pl, int n, int lane) {
   __syncwarp();
 }
 
-// The planner warp: union of the tile's selections, by segment, into `pl`.
+// One warp of plan_tiles_kernel: union of the tile's selections, by segment, into `pl`.
 // The 128 (query, slot) entries become sortable keys (segment << 24 |
 // block; ~0 for an empty or invalid entry), each carrying its query's bit;
 // lane l holds entries 4l .. 4l+3.  A bitonic sort of the 128 keys (28
