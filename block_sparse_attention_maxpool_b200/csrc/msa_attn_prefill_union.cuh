@@ -207,8 +207,7 @@ __device__ __forceinline__ void order_plan(Plan& pl, int n, int lane) {
         best = min(best, key);
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(kFull, best, o));
+    best = __reduce_min_sync(kFull, best);
     const int c = static_cast<int>(best & 0xffu);
     uint32_t wq = 0u;
     if ((c & 31) == lane) {
