@@ -451,9 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------ the Q tile and the K blocks (lane 0) ---------------------
     if (lane == 0) {
-      int tc = 0, ring = 0, q_use = 0;
+      int ring = 0, q_use = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x) {
         const Plan& pl = P.plans[t];
         int g, q0;
         tile_coords(P, t, g, q0);
@@ -493,9 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------ V loader (lane 0) ------------------------------
     if (lane == 0) {
-      int tc = 0, ring = 0;
+      int ring = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x) {
         const Plan& pl = P.plans[t];
         int g, q0;
         tile_coords(P, t, g, q0);
@@ -523,9 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t q_base = smem_addr(smem + Layout::kQOff);
       const uint32_t k_base = smem_addr(smem + Layout::kKOff);
-      int tc = 0, kr = 0, blk = 0, q_use = 0;
+      int kr = 0, blk = 0, q_use = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x) {
         const Plan& pl = P.plans[t];
         if (pl.n > 0) {
           ok = mbar_wait(B.q_full, q_use & 1);
@@ -562,9 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------- P . V issuer: O (+)= P . V_b (lane 0) -----------------
     if (lane == 0) {
       const uint32_t v_base = smem_addr(smem + Layout::kVOff);
-      int tc = 0, vr = 0, blk = 0, segs_done = 0;
+      int vr = 0, blk = 0, segs_done = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x, ++tc) {
+      for (int t = blockIdx.x; t < n_tasks && ok; t += gridDim.x) {
         const Plan& pl = P.plans[t];
         for (int j = 0; j < pl.n && ok; ++j) {
           const int b = blk + j;
@@ -598,9 +598,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;             // TMEM lane = MMA row
     const int q = r / kHpg;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    int tc = 0, blk = 0;
+    int blk = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++tc) {
+    for (int t = blockIdx.x; t < n_tasks; t += gridDim.x) {
       const Plan& pl = P.plans[t];
       int g, q0;
       tile_coords(P, t, g, q0);
