@@ -27,7 +27,7 @@ __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_bloc
            "msa_sparse_attn_prefill_paged", "DsaShape", "DSA_SEL_WIDTH", "msa_dsa_indexer_append",
            "msa_dsa_token_scores", "msa_dsa_select_topk", "msa_dsa_sparse_attn_decode", "dsa_decode_step",
            "msa_decode_step_fused", "msa_decode_step_fused_workspace_bytes", "decode_step_fused", "DecodeGraph",
-           "StepPipeline"]
+           "StepPipeline", "msa_wait_selftest", "WAIT_SELFTEST_WORKSPACE_BYTES"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa.so")
 MODE_DECODE = 0
@@ -158,6 +158,7 @@ _SIGS.update({
     "msa_decode_step_fused": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                                              _P, _P, _I, ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "msa_decode_step_fused_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(CShape), _I]),
+    "msa_wait_selftest": (ctypes.c_int, [ctypes.c_longlong, _P, ctypes.c_size_t, _P]),
 })
 
 
@@ -417,6 +418,19 @@ def msa_get_device_error(stream=None) -> int:
     v = ctypes.c_uint32(0)
     _check("msa_get_device_error", library().msa_get_device_error(ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+WAIT_SELFTEST_WORKSPACE_BYTES = 16
+
+
+def msa_wait_selftest(wait_cycles: int, workspace: torch.Tensor, stream=None) -> None:
+    """Run the library's bounded waits against conditions that never come
+    true (see include/msa.h); each gives up after ``wait_cycles`` SM clock
+    cycles and records the TIMEOUT bit of the device error word.
+    ``workspace``: a uint8 CUDA tensor of at least 16 bytes; its third
+    32-bit word is 0 afterwards when every wait ran out."""
+    _check("msa_wait_selftest", library().msa_wait_selftest(
+        int(wait_cycles), _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
 
 
 def msa_version() -> int:

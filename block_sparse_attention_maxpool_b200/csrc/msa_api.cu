@@ -533,19 +533,51 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[MSA_NOALLOC_SCR
 }  // extern "C"
 
 namespace {
+// The buffer's device address, per device, with the context it was looked up
+// in: a new context on the device (after cudaDeviceReset, or once the
+// primary context was released and re-created) holds a new copy of the
+// buffer, so the address is looked up again whenever the current context
+// differs from the recorded one.
+struct NoallocSlot {
+  CUcontext ctx;
+  void* ptr;
+};
 std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[64] = {};
+NoallocSlot g_noalloc[64] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
 
 int noalloc_scratch(void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MSA_ERR_CUDA;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (get_ctx == nullptr) return MSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return MSA_ERR_CUDA;
+  NoallocSlot& slot = g_noalloc[dev];
+  if (slot.ptr == nullptr || ctx == nullptr || slot.ctx != ctx) {
     void* p = nullptr;
+    // with that device current (it is): also makes the device's primary
+    // context current if no context was yet
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MSA_ERR_CUDA;
+    slot.ctx = ctx;
+    slot.ptr = p;
   }
-  *ptr = g_noalloc_ptr[dev];
+  *ptr = slot.ptr;
   return MSA_OK;
 }
 }  // namespace
@@ -822,6 +854,7 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
       static_cast<uint8_t*>(workspace) + msa::tc::align256(attn_workspace(shape, n_q, MSA_MODE_DECODE)));
   F.bar_count = bar;
   F.bar_gen = bar + 1;
+  F.wait_cycles = msa::kWaitCycles;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), cs) != cudaSuccess) return MSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -835,6 +868,32 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, F) != cudaSuccess) return MSA_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
+}
+
+int msa_wait_selftest(long long wait_cycles, void* workspace, size_t workspace_bytes, void* stream) {
+  if (wait_cycles < 1 || wait_cycles > msa::kWaitCycles) return MSA_ERR_RANGE;
+  if (workspace == nullptr) return MSA_ERR_NULL;
+  if (workspace_bytes < MSA_WAIT_SELFTEST_WORKSPACE_BYTES) return MSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MSA_ERR_ALIGN;
+  int sms = 0;
+  int st = current_device_sms(&sms);
+  if (st != MSA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  unsigned int* bar = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(bar, 0, MSA_WAIT_SELFTEST_WORKSPACE_BYTES, cs) != cudaSuccess) return MSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sms));
+  cfg.blockDim = dim3(32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = cs;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, msa::fused::wait_selftest_kernel, bar, wait_cycles) != cudaSuccess)
+    return MSA_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 

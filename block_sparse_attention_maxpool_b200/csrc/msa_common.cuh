@@ -52,8 +52,9 @@ __device__ __forceinline__ long long kv_block_row(const KvPages& pg, int s, int 
 }
 
 // A wait on an mbarrier gives up after this many SM clock cycles (about half
-// a second at the B200's boost clock), records MSA_DEVERR_TIMEOUT and lets
-// the kernel return instead of hanging the GPU.
+// a second at the B200's boost clock) unless the caller passes its own
+// limit, records MSA_DEVERR_TIMEOUT and lets the kernel return instead of
+// hanging the GPU.
 constexpr long long kWaitCycles = 1000000000LL;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -97,12 +98,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false (and records MSA_DEVERR_TIMEOUT) if it did not within kWaitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// false (and records MSA_DEVERR_TIMEOUT) if it did not within `limit` SM
+// clock cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       raise_error(MSA_DEVERR_TIMEOUT);
       return false;
     }

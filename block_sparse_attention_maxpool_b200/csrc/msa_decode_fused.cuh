@@ -58,6 +58,7 @@ struct Params {
   // grid barrier words (workspace, zeroed before the launch)
   unsigned int* bar_count;
   unsigned int* bar_gen;
+  long long wait_cycles;             // give-up limit of a grid-barrier wait (SM clock cycles)
 };
 
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
@@ -86,27 +87,29 @@ __device__ __forceinline__ void st_relaxed_gpu(unsigned int* p, unsigned int v) 
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Grid-wide barrier of the n_cta resident CTAs.  The CTA's threads meet at
-// __syncthreads, then thread 0 arrives with an acquire-release add on the counter;
-// the last arriver resets the counter and publishes the next generation
-// with a release store, the others poll it with acquire loads (bounded).
-// gen: the generation this CTA last saw.  proxy_fence: the phase wrote
-// global memory that async copies (bulk, TMA) read afterwards.  False, for
-// every thread of the CTA, when the wait timed out.
-__device__ __forceinline__ bool grid_barrier(const Params& F, unsigned int n_cta, unsigned int& gen, int* flag,
-                                             bool proxy_fence) {
+// Grid-wide barrier over `expected` arrivals (the n_cta resident CTAs).
+// The CTA's threads meet at __syncthreads, then thread 0 arrives with an
+// acquire-release add on the counter; the arrival that completes the count
+// resets the counter and publishes the next generation with a release
+// store, the others poll it with acquire loads for at most `limit` SM clock
+// cycles.  gen: the generation this CTA last saw.  proxy_fence: the phase
+// wrote global memory that async copies (bulk, TMA) read afterwards.  False,
+// for every thread of the CTA, when the wait timed out (MSA_DEVERR_TIMEOUT
+// recorded).
+__device__ __forceinline__ bool grid_barrier(unsigned int* bar_count, unsigned int* bar_gen, unsigned int expected,
+                                             long long limit, unsigned int& gen, int* flag, bool proxy_fence) {
   if (proxy_fence) fence_proxy_async_global();
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
     const unsigned int target = gen + 1;
-    if (atom_add_acq_rel_gpu(F.bar_count, 1u) == n_cta - 1) {
-      st_relaxed_gpu(F.bar_count, 0u);
-      st_release_gpu(F.bar_gen, target);
+    if (atom_add_acq_rel_gpu(bar_count, 1u) == expected - 1) {
+      st_relaxed_gpu(bar_count, 0u);
+      st_release_gpu(bar_gen, target);
     } else {
       const long long t0 = clock64();
-      while (ld_acquire_gpu(F.bar_gen) < target) {
-        if (clock64() - t0 > kWaitCycles) {
+      while (ld_acquire_gpu(bar_gen) < target) {
+        if (clock64() - t0 > limit) {
           raise_error(MSA_DEVERR_TIMEOUT);
           ok = false;
           break;
@@ -118,6 +121,11 @@ __device__ __forceinline__ bool grid_barrier(const Params& F, unsigned int n_cta
   }
   __syncthreads();
   return *flag != 0;
+}
+
+__device__ __forceinline__ bool grid_barrier(const Params& F, unsigned int n_cta, unsigned int& gen, int* flag,
+                                             bool proxy_fence) {
+  return grid_barrier(F.bar_count, F.bar_gen, n_cta, F.wait_cycles, gen, flag, proxy_fence);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -167,6 +175,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- 5. merge the partials of pairs cut between CTAs ----------------------
   for (long long w = gwarp; w < static_cast<long long>(n_pairs) * dattn::kHpg; w += n_gwarps)
     dattn::combine_pair_head(F.attn, w, lane);
+}
+
+// The library's bounded waits driven to their limit: every CTA of a
+// cooperative grid (one per SM) meets at the grid barrier above with one
+// more arrival expected than the grid gives, so no CTA sees the next
+// generation; then thread 0 of each CTA waits on an mbarrier nothing
+// arrives on.  Each wait gives up after `limit` cycles, records
+// MSA_DEVERR_TIMEOUT, and the kernel returns.  No copy or MMA is in flight
+// at either wait.  bar: two zeroed words (counter, generation).
+__global__ void __launch_bounds__(32, 1) wait_selftest_kernel(unsigned int* bar, long long limit) {
+  __shared__ int barrier_flag;
+  __shared__ __align__(8) uint64_t never;
+  unsigned int gen = 0;
+  const bool passed = grid_barrier(bar, bar + 1, gridDim.x + 1, limit, gen, &barrier_flag, false);
+  if (threadIdx.x == 0) {
+    mbar_init(&never, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const bool arrived = mbar_wait(&never, 0, limit);
+    mbar_inval(&never);
+    if (passed || arrived) bar[2] = 1u;          // a wait that should have run out did not
+  }
 }
 
 }  // namespace fused

@@ -221,7 +221,11 @@ MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, c
  * MSA_ERR_WORKSPACE; the decode partials need at most 256 CTAs x 2 x 8320
  * bytes = 4,259,840 bytes, so every batch fits.  The first call on each
  * device looks up the buffer's device address (with that device current);
- * make that first call before any stream capture.  All calls share the
+ * make that first call before any stream capture.  The address is looked up
+ * again when the device's current context is not the one it was found in
+ * (after cudaDeviceReset, or when the primary context was released and
+ * created anew), since each context holds its own copy of the buffer; that
+ * first call in a new context, too, belongs before any capture.  All calls share the
  * buffer: calls that can run at the same time on the GPU (different streams,
  * or different host threads on one device) race and must be serialised by
  * the caller.  Nothing in the buffer needs to start at zero: every call
@@ -387,6 +391,26 @@ MSA_API int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, ms
 /* Workspace bytes of msa_decode_step_fused, or (size_t)-1 for an
  * unsupported shape or batch. */
 MSA_API size_t msa_decode_step_fused_workspace_bytes(const msa_shape* shape, int32_t n_q);
+
+/* Bytes of device workspace msa_wait_selftest needs. */
+#define MSA_WAIT_SELFTEST_WORKSPACE_BYTES 16u
+
+/* msa_wait_selftest - drives the library's bounded device waits to their
+ * limit, so that a caller (or a test) can see that a wait which never ends
+ * gives up, records MSA_DEVERR_TIMEOUT and lets its kernel return with the
+ * context still usable.  The pages have no counterpart: it checks the
+ * library's own failure handling (no kernel here traps or spins without a
+ * limit).  One cooperative launch with one CTA per SM: every CTA meets at
+ * the grid barrier of msa_decode_step_fused set to expect one more arrival
+ * than the grid gives, then one thread per CTA waits on an mbarrier that
+ * nothing arrives on.  Each wait gives up after wait_cycles SM clock cycles
+ * (1 ..= 1e9; the library's own kernels use 1e9, about half a second).
+ * workspace: MSA_WAIT_SELFTEST_WORKSPACE_BYTES of device memory, 16-byte
+ * aligned, zeroed by the call on `stream`; afterwards its third 32-bit word
+ * is 0 when every wait ran out as it should.  Asynchronous on `stream`;
+ * read the result with msa_get_device_error.  MSA_ERR_RANGE for a limit out
+ * of range. */
+MSA_API int msa_wait_selftest(long long wait_cycles, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace that msa_block_scores and the attention call of `mode`
  * need for n_q queries (the larger of the two; one buffer serves both calls

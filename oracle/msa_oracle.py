@@ -42,7 +42,9 @@ Readings where the pages are silent (each also listed in the design notes):
 * query head h belongs to group h // (n_q_heads / n_kv_heads);
 * the query at position p attends to the rows j <= p of its selected blocks
   (only the local block can hold rows past p);
-* scores are plain dot products (no scale, activation or weights).
+* scores are plain dot products (no scale, activation or weights);
+* a NaN block score ranks as -inf (inputs never hold one; the rule only fixes
+  what the selection does if one appears).
 
 Every floating-point step runs in float64 on the CPU.  Tensors may be any
 float dtype; they are converted exactly (bf16/f32 -> f64) before use.
@@ -97,8 +99,26 @@ def indexer_append(idx_k_cache: torch.Tensor, idx_k_new: torch.Tensor,
 # block scores
 # ---------------------------------------------------------------------------
 def token_scores(idx_q_vec: torch.Tensor, idx_k_rows: torch.Tensor) -> torch.Tensor:
-    """s_j = idx_q . idx_k[j] for the given key rows, in float64."""
+    """s_j = idx_q . idx_k[j] for the given key rows, in float64.  With a
+    [Di][n] matrix of n query vectors the result is s[j][i]."""
     return _cpu64(idx_k_rows) @ _cpu64(idx_q_vec)
+
+
+def pool_visible(s: torch.Tensor, positions, block: int, n_blocks: int) -> torch.Tensor:
+    """maxpool_block over the causally masked token scores of n queries.
+
+    ``s`` [n][L] holds query i's scores over slots 0..L-1, and query i sees
+    the slots j <= positions[i] ("idx_q*idx_k^T + causal mask": every later
+    slot scores -inf).  Entry [i][b] is the largest masked score in slots
+    [b*block, (b+1)*block), so a block with no visible slot is -inf.
+    """
+    n, L = s.shape
+    pos = torch.as_tensor(positions, dtype=torch.long).reshape(n, 1)
+    masked = _cpu64(s).masked_fill(torch.arange(L).reshape(1, L) > pos, NEG_INF)   # causal mask
+    width = n_blocks * block
+    padded = torch.full((n, width), NEG_INF, dtype=F64)
+    padded[:, :min(L, width)] = masked[:, :width]
+    return padded.reshape(n, n_blocks, block).amax(dim=2)                          # maxpool_block
 
 
 def pooled_scores(idx_q_vec: torch.Tensor, idx_k_sg: torch.Tensor, pos: int, block: int,
@@ -107,31 +127,38 @@ def pooled_scores(idx_q_vec: torch.Tensor, idx_k_sg: torch.Tensor, pos: int, blo
 
     ``idx_k_sg`` is the [capacity][idx_dim] cache of the query's stream and
     group.  Entry b is max_{j in [b*block, (b+1)*block), j <= pos} s_j; blocks
-    with no visible token are -inf (the causal mask sets s_j = -inf for
-    j > pos before pooling).
+    with no visible token are -inf.
     """
-    s = token_scores(idx_q_vec, idx_k_sg[: pos + 1])          # visible tokens only
-    out = torch.full((n_blocks,), NEG_INF, dtype=F64)
-    for b in range(n_visible_blocks(pos, block)):
-        out[b] = s[b * block: min((b + 1) * block, pos + 1)].max()
-    return out
+    s = token_scores(idx_q_vec, idx_k_sg)                     # every slot of the cache
+    return pool_visible(s.reshape(1, -1), [pos], block, n_blocks)[0]
 
 
 def block_scores(idx_q: torch.Tensor, idx_k_cache: torch.Tensor, q_stream: torch.Tensor,
-                 q_pos: torch.Tensor, block: int, local_bias: float = LOCAL_BIAS) -> torch.Tensor:
+                 q_pos: torch.Tensor, block: int, local_bias: float = LOCAL_BIAS,
+                 chunk: int = 256) -> torch.Tensor:
     """bs[n_q][G][capacity/block]: pooled scores plus the local-force bias.
 
-    idx_q [n_q][G][Di], idx_k_cache [S][G][capacity][Di].
+    idx_q [n_q][G][Di], idx_k_cache [S][G][capacity][Di].  The queries of one
+    stream are scored ``chunk`` at a time as one matrix product against the
+    keys up to the chunk's last position (the same dot products as one query
+    at a time; only the number of queries per product differs).
     """
     n_q, G = idx_q.shape[0], idx_q.shape[1]
     n_blocks = idx_k_cache.shape[2] // block
     bs = torch.empty((n_q, G, n_blocks), dtype=F64)
-    for i in range(n_q):
-        s, p = int(q_stream[i]), int(q_pos[i])
+    streams = q_stream.to(torch.long)
+    positions = q_pos.to(torch.long)
+    for s in sorted(set(streams.tolist())):
+        mine = (streams == s).nonzero().flatten()
         for g in range(G):
-            row = pooled_scores(idx_q[i, g], idx_k_cache[s, g], p, block, n_blocks)
-            row[local_block(p, block)] += local_bias
-            bs[i, g] = row
+            keys = _cpu64(idx_k_cache[s, g])
+            for c0 in range(0, mine.numel(), chunk):
+                ii = mine[c0:c0 + chunk]
+                L = int(positions[ii].max()) + 1
+                sc = token_scores(idx_q[ii, g].T, keys[:L]).T                # [n][L]
+                bs[ii, g] = pool_visible(sc, positions[ii], block, n_blocks)
+    for i in range(n_q):
+        bs[i, :, local_block(int(positions[i]), block)] += local_bias
     return bs
 
 
@@ -139,10 +166,16 @@ def block_scores(idx_q: torch.Tensor, idx_k_cache: torch.Tensor, q_stream: torch
 # top-k block selection
 # ---------------------------------------------------------------------------
 def ranked_blocks(bs_row: torch.Tensor, pos: int, block: int) -> list[int]:
-    """Visible blocks ordered best first: higher score, then lower index."""
+    """Visible blocks ordered best first: higher score, then lower index.  A
+    NaN score ranks as -inf (below every finite score, tied with -inf and
+    ordered by index), and -0 equals +0."""
     nvis = n_visible_blocks(pos, block)
-    vals = [float(bs_row[b]) for b in range(nvis)]
-    return sorted(range(nvis), key=lambda b: (-vals[b], b))
+    vals = bs_row[:nvis].tolist()
+
+    def rank_key(b):
+        v = vals[b]
+        return (math.inf if v != v else -v, b)
+    return sorted(range(nvis), key=rank_key)
 
 
 def select_one(bs_row: torch.Tensor, pos: int, block: int, top_k: int) -> list[int]:

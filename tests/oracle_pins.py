@@ -168,6 +168,20 @@ def pin_selection_bruteforce(o, seed=3):
         assert got == want, (trial, pos, got, want)
 
 
+def pin_selection_nan_rule(o):
+    """A NaN block score ranks as -inf: below every finite score and tied
+    with -inf, ties going to the lower index; -0 equals +0.  The expected
+    orders are written out by hand from that rule."""
+    nan, inf = float("nan"), float("inf")
+    row = torch.tensor([nan, 0.5, -inf, -3.0, nan, 2.0, -0.0, 0.0], dtype=F64)
+    assert o.ranked_blocks(row, 7 * 4, 4) == [5, 1, 6, 7, 3, 0, 2, 4]
+    assert o.select_one(row, 7 * 4, 4, 6) == [0, 1, 3, 5, 6, 7]
+    row2 = torch.tensor([-inf, nan, nan, 1.0, -inf], dtype=F64)
+    assert o.ranked_blocks(row2, 4 * 4 + 2, 4) == [3, 0, 1, 2, 4]
+    sel, n_sel = o.select_blocks(row2.reshape(1, 1, 5), torch.tensor([4 * 4 + 2], dtype=torch.int32), 4, 3)
+    assert sel.tolist() == [[[0, 1, 3]]] and n_sel.tolist() == [[3]]
+
+
 def pin_selection_invariants(o, seed=4):
     g = torch.Generator().manual_seed(seed)
     block, top_k, Di, cap = 4, 3, 4, 48
@@ -509,7 +523,7 @@ def pin_dsa_mask_equivalence(o, seed=15):
 
 
 ALL_PINS = [pin_golden, pin_basis_query_pooling, pin_scores_bilinear, pin_selection_bruteforce,
-            pin_selection_invariants, pin_local_forced, pin_dense_equivalence,
+            pin_selection_nan_rule, pin_selection_invariants, pin_local_forced, pin_dense_equivalence,
             pin_block_mask_equivalence, pin_attention_closed_forms, pin_append_random,
             pin_paged_identity_layout, pin_paged_permutation_and_sharing, pin_paged_append_commutes,
             pin_dsa_scores_identities, pin_dsa_selection_bruteforce, pin_dsa_noop_exact, pin_dsa_mask_equivalence]

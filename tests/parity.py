@@ -16,8 +16,10 @@ Comparison rules
   * end-to-end selection: ids bit-exact, except (q, g) pairs whose oracle
     ranks top_k and top_k+1 are within 1e-5 relative (and not exactly equal);
     those are counted and the attention is checked with the GPU's selection;
-  * attention (bf16 out vs float64): elementwise |got - bf16(want)| <=
-    max(4e-3, one bf16 ulp of want), and mean |got - want| <= 5e-4.
+  * attention (bf16 out vs float64): elementwise |got - want| <= 4e-3 plus
+    half a bf16 ulp of want (the rounding of a correctly rounded bf16 output
+    is at most half an ulp, so only the output's own rounding is excused on
+    top of the 4e-3 bound), and mean |got - want| <= 5e-4.
 """
 from __future__ import annotations
 
@@ -70,19 +72,25 @@ def oracle_caches(inp, idx_f16=False):
     return idx, k, v
 
 
-def score_bounds(idx_q, idx_k_cache, q_stream, q_pos, block):
-    """Per (query, group, block): 64 u max_j sum_d |q_d k_jd| over visible j."""
+def score_bounds(idx_q, idx_k_cache, q_stream, q_pos, block, chunk=256):
+    """Per (query, group, block): 64 u max_j sum_d |q_d k_jd| over visible j
+    (the queries of one stream in chunks, as one product of absolute values)."""
     n_q, G = idx_q.shape[0], idx_q.shape[1]
     nblk = idx_k_cache.shape[2] // block
     out = torch.zeros((n_q, G, nblk), dtype=torch.float64)
-    for i in range(n_q):
-        s, p = int(q_stream[i]), int(q_pos[i])
+    streams, positions = q_stream.long(), q_pos.long()
+    for s in sorted(set(streams.tolist())):
+        mine = (streams == s).nonzero().flatten()
         for g in range(G):
-            a = idx_k_cache[s, g, :p + 1].double().abs() @ idx_q[i, g].double().abs()
-            nb = p // block + 1
-            pad = torch.full((nb * block,), 0.0, dtype=torch.float64)
-            pad[:p + 1] = a
-            out[i, g, :nb] = 64 * U32 * pad.view(nb, block).amax(dim=1)
+            keys = idx_k_cache[s, g].double().abs()
+            for c0 in range(0, mine.numel(), chunk):
+                ii = mine[c0:c0 + chunk]
+                L = int(positions[ii].max()) + 1
+                a = idx_q[ii, g].double().abs() @ keys[:L].T                     # [n][L]
+                a = a.masked_fill(torch.arange(L).view(1, L) > positions[ii].view(-1, 1), 0.0)
+                pad = torch.zeros((ii.numel(), nblk * block), dtype=torch.float64)
+                pad[:, :L] = a
+                out[ii, g] = 64 * U32 * pad.view(-1, nblk, block).amax(dim=2)
     return out
 
 
@@ -121,28 +129,35 @@ def check_selection(sel_gpu, nsel_gpu, bs_orc, q_pos, block, top_k):
 
 
 def bf16_ulp(x: torch.Tensor) -> torch.Tensor:
-    a = x.abs().clamp_min(2.0 ** -126)
-    return torch.exp2(torch.floor(torch.log2(a)) - 7)
+    """The spacing of bf16 numbers at |x| (8 significant bits): 2^(e-8) for
+    |x| in [2^(e-1), 2^e)."""
+    _, e = torch.frexp(x.abs().clamp_min(2.0 ** -126))
+    return torch.ldexp(torch.ones_like(x), e - 8)
 
 
 def check_attention(out_gpu, out_orc, rows=None):
+    """|got - want| <= 4e-3 + half a bf16 ulp of want for every element,
+    mean |got - want| <= 5e-4 (want: the float64 oracle).  Returns (max abs
+    error, mean abs error, largest error in bf16 ulps of want)."""
     g = out_gpu.double()
     w = out_orc
     if rows is not None:
         g, w = g[rows], w[rows]
-    w_bf = w.to(torch.bfloat16).double()
-    tol = torch.maximum(torch.full_like(w, ATTN_MAX_ABS), bf16_ulp(w))
-    d = (g - w_bf).abs()
+    ulp = bf16_ulp(w)
+    tol = ATTN_MAX_ABS + 0.5 * ulp
+    d = (g - w).abs()
     bad = d > tol
-    assert not bool(bad.any()), f"attention max err {d.max():.3e} (tol {tol[bad].min():.3e}) at {bad.nonzero()[0].tolist()}"
-    mean = float((g - w).abs().mean())
+    assert not bool(bad.any()), (f"attention max err {d.max():.3e} (tol {tol[bad].min():.3e}) "
+                                 f"at {bad.nonzero()[0].tolist()}")
+    mean = float(d.mean())
     assert mean <= ATTN_MEAN_ABS, f"attention mean abs err {mean:.3e}"
-    return float((g - w).abs().max()), mean
+    return float(d.max()), mean, float((d / ulp).max())
 
 
-def full_parity(inp, queries=None, prefill=False, dev="cuda", idx_f16=False, paged=None):
+def full_parity(inp, queries=None, prefill=False, dev="cuda", idx_f16=False, paged=None, attn_queries=None):
     """Run one step on the GPU and compare every part with the oracle on the
-    query indices ``queries`` (all when None).  With ``paged`` (keyword
+    query indices ``queries`` (all when None); the attention on
+    ``attn_queries`` only, when given (a subset of ``queries``).  With ``paged`` (keyword
     arguments of workloads.page_layout) the GPU runs the paged calls on
     shuffled page pools and the oracle reads the same pools through its own
     logical view.  Returns a small report."""
@@ -185,8 +200,13 @@ def full_parity(inp, queries=None, prefill=False, dev="cuda", idx_f16=False, pag
     bs_g, sel_g, nsel_g, out_g = bs.cpu()[qsub], sel.cpu()[qsub], n_sel.cpu()[qsub], out.cpu()[qsub]
     max_score_err = check_scores(bs_g, bs_o, bounds)
     merged, excused = check_selection(sel_g, nsel_g, bs_o, qp, w.block, w.top_k)
-    out_o = oracle.sparse_attention(inp.q[qsub], k_o, v_o, merged, qs, qp, w.block,
+    if attn_queries is not None:
+        pick = {int(x): j for j, x in enumerate(qsub.tolist())}
+        rows = torch.tensor([pick[int(x)] for x in attn_queries], dtype=torch.long)
+    else:
+        rows = torch.arange(qsub.numel())
+    out_o = oracle.sparse_attention(inp.q[qsub[rows]], k_o, v_o, merged[rows], qs[rows], qp[rows], w.block,
                                     1.0 / math.sqrt(w.head_dim))
-    max_err, mean_err = check_attention(out_g, out_o)
-    return dict(queries=len(qsub), near_ties=excused, max_score_err=max_score_err,
-                attn_max_abs=max_err, attn_mean_abs=mean_err)
+    max_err, mean_err, ulps = check_attention(out_g[rows], out_o)
+    return dict(queries=len(qsub), attn_queries=int(rows.numel()), near_ties=excused,
+                max_score_err=max_score_err, attn_max_abs=max_err, attn_mean_abs=mean_err, attn_max_ulps=ulps)

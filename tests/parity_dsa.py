@@ -117,6 +117,6 @@ def full_parity(dinp, top_k=2048, relu=True, queries=None, dev="cuda"):
     max_score_err = check_scores(sc.cpu()[qsub], sc_o, bounds)
     merged, excused = check_selection(sel.cpu()[qsub], n_sel.cpu()[qsub], sc_o, bounds, qp, top_k)
     out_o = oracle.dsa_sparse_attention(inp.q[qsub], k_o, v_o, merged, qs, qp, 1.0 / math.sqrt(w.head_dim))
-    max_err, mean_err = PT.check_attention(out.cpu()[qsub], out_o)
+    max_err, mean_err, _ = PT.check_attention(out.cpu()[qsub], out_o)
     return dict(queries=len(qsub), boundary_swaps=excused, max_score_err=max_score_err,
                 attn_max_abs=max_err, attn_mean_abs=mean_err)

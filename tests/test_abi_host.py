@@ -221,3 +221,13 @@ def test_fused_step_validation(lib):
     assert call(n_q=4096) == -3                       # prefill-shaped batch
     assert call(ws_ptr=0, ws_bytes=0) == -5
     assert call(ws_ptr=fake + 16) == -2               # workspace not 256-byte aligned
+
+
+def test_wait_selftest_validation(lib):
+    """Argument checks of msa_wait_selftest, made before any device work."""
+    fake = 0x10000
+    assert lib.msa_wait_selftest(0, fake, 16, None) == -4                 # limit out of range
+    assert lib.msa_wait_selftest(10 ** 9 + 1, fake, 16, None) == -4
+    assert lib.msa_wait_selftest(1000, None, 16, None) == -1
+    assert lib.msa_wait_selftest(1000, fake, 8, None) == -5               # too small
+    assert lib.msa_wait_selftest(1000, fake + 4, 16, None) == -2          # not 16-byte aligned

@@ -92,17 +92,28 @@ def test_select_bit_exact_from_identical_scores(nblk, ties):
 
 
 def test_select_nan_ranks_last_and_bad_positions():
+    """NaN scores rank as -inf (tied with -inf, lower index first), as the
+    oracle ranks them; a query past the capacity selects nothing."""
     sh = msa.Shape(n_streams=1, capacity=128 * 40)
-    bs = torch.zeros((2, 4, 40))
+    g = torch.Generator().manual_seed(40)
+    bs = torch.zeros((3, 4, 40))
     bs[:, :, 0] = float("nan")
     bs[:, :, 39] += 2.0 ** 100
-    q_pos = torch.tensor([128 * 40 - 1, 128 * 40], dtype=torch.int32)   # second is out of range
+    bs[2] = torch.randn((4, 40), generator=g)
+    bs[2, :, 5:30:3] = float("nan")                # many NaN blocks ...
+    bs[2, :, 7:33:4] = float("-inf")               # ... mixed with -inf ones
+    bs[2, 1, :] = float("nan")                     # a group with nothing but NaN and the local block
+    bs[2, :, 20] = 2.0 ** 100
+    q_pos = torch.tensor([128 * 40 - 1, 128 * 40, 128 * 20 + 3], dtype=torch.int32)   # second is out of range
     sel, n_sel = msa.msa_select_topk(sh, bs.cuda(), q_pos.cuda())
     assert msa.msa_get_device_error() & 0x1
-    sel = sel.cpu()
+    sel, n_sel = sel.cpu(), n_sel.cpu()
     assert 0 not in sel[0, 0].tolist()             # the NaN block loses to every finite one
     assert sel[0, 0].tolist() == list(range(1, 16)) + [39]
-    assert sel[1].eq(-1).all() and n_sel.cpu()[1].eq(0).all()
+    assert sel[1].eq(-1).all() and n_sel[1].eq(0).all()
+    good = torch.tensor([0, 2])
+    sel_o, nsel_o = oracle.select_blocks(bs[good].double(), q_pos[good], 128, 16)
+    assert torch.equal(sel[good], sel_o) and torch.equal(n_sel[good], nsel_o)
 
 
 def _random_selection(g, q_pos, G, top_k=16):
@@ -379,30 +390,45 @@ def test_workload_decode_1x4k_full():
     report(W.DECODE_4K.name, PT.full_parity(W.make_inputs(W.DECODE_4K)))
 
 
-def test_workload_decode_32x32k_sampled():
+def test_workload_decode_32x32k_full():
     inp = W.make_inputs(W.DECODE_32K_X32)
-    report(W.DECODE_32K_X32.name, PT.full_parity(inp, queries=[0, 7, 19, 31]))
+    report(W.DECODE_32K_X32.name, PT.full_parity(inp))
     report(W.DECODE_32K_X32.name + " f16 indexer cache", PT.full_parity(inp, queries=[3, 30], idx_f16=True))
 
 
-def test_workload_decode_8x128k_sampled():
+def test_workload_decode_8x128k_full():
     inp = W.make_inputs(W.DECODE_128K_X8)
-    report(W.DECODE_128K_X8.name, PT.full_parity(inp, queries=[0, 5]))
+    report(W.DECODE_128K_X8.name, PT.full_parity(inp))
 
 
-def test_workload_prefill_16k_sampled():
+def _spread_tiles(n_q, every=32, tile=8, extra=()):
+    """Queries of every ``every``-th attention tile (``tile`` consecutive
+    queries), plus ``extra``: a spread of whole tiles across the batch."""
+    q = set(extra)
+    for t0 in range(0, n_q, every * tile):
+        q.update(range(t0, min(t0 + tile, n_q)))
+    return sorted(q)
+
+
+def test_workload_prefill_16k_every_query():
+    """Block scores and selection of all 16384 queries against the oracle;
+    attention on every 32nd 8-query tile (512 queries) and the edges of the
+    dense/sparse boundary."""
     inp = W.make_inputs(W.PREFILL_16K)
-    g = torch.Generator().manual_seed(7)
-    q = sorted(set([0, 1, 2, 127, 128, 129, 2046, 2047, 2048, 2049, 4095, 4096, 8191, 16383]
-                   + torch.randint(0, 16384, (36,), generator=g).tolist()))
-    report(W.PREFILL_16K.name, PT.full_parity(inp, queries=q, prefill=True))
+    attn = _spread_tiles(16384, extra=[1, 127, 128, 129, 2046, 2047, 2048, 2049, 4095, 4096, 8191, 16383])
+    rep = PT.full_parity(inp, prefill=True, attn_queries=attn)
+    report(W.PREFILL_16K.name, rep)
+    assert rep["queries"] == 16384 and rep["attn_queries"] >= 256
 
 
-def test_workload_chunked_prefill_ties_sampled():
+def test_workload_chunked_prefill_ties_every_query():
+    """All 8192 queries of the tie workload: scores, and selection bit-exact
+    with no near-tie excused (every score is exact in float32); attention on
+    every 32nd 8-query tile of the four streams (256 queries) plus the
+    chunk edges."""
     inp = W.make_inputs(W.CHUNKED_PREFILL_TIES)
-    g = torch.Generator().manual_seed(8)
-    q = sorted(set([0, 1, 2047, 2048, 4095, 6143, 8191]
-                   + torch.randint(0, 8192, (25,), generator=g).tolist()))
-    rep = PT.full_parity(inp, queries=q, prefill=True)
+    attn = _spread_tiles(8192, extra=[1, 2047, 2048, 4095, 6143, 8191])
+    rep = PT.full_parity(inp, prefill=True, attn_queries=attn)
     report(W.CHUNKED_PREFILL_TIES.name, rep)
-    assert rep["near_ties"] == 0
+    assert rep["queries"] == 8192 and rep["attn_queries"] >= 256
+    assert rep["near_ties"] == 0 and rep["max_score_err"] == 0.0

@@ -24,22 +24,25 @@ def fresh_oracle(tag):
 
 
 def _mut_causal_off_by_one(o):
-    orig = o.pooled_scores
+    orig = o.pool_visible
 
-    def pooled_scores(q, k, pos, block, n_blocks):
-        out = orig(q, k, max(pos - 1, 0), block, n_blocks)
-        return out
-    o.pooled_scores = pooled_scores
+    def pool_visible(s, positions, block, n_blocks):
+        pos = torch.as_tensor(positions, dtype=torch.long).clamp_min(1) - 1
+        return orig(s, pos, block, n_blocks)
+    o.pool_visible = pool_visible
 
 
 def _mut_no_causal_mask(o):
-    def pooled_scores(q, k, pos, block, n_blocks):
-        s = o.token_scores(q, k)
-        out = torch.full((n_blocks,), float("-inf"), dtype=torch.float64)
-        for b in range(o.n_visible_blocks(pos, block)):
-            out[b] = s[b * block:(b + 1) * block].max()
+    orig = o.pool_visible
+
+    def pool_visible(s, positions, block, n_blocks):
+        # pools every slot of a visible block, including the ones past the query
+        pos = torch.as_tensor(positions, dtype=torch.long).reshape(-1)
+        out = orig(s, torch.full_like(pos, s.shape[1] - 1), block, n_blocks)
+        for i in range(out.shape[0]):
+            out[i, int(pos[i]) // block + 1:] = float("-inf")
         return out
-    o.pooled_scores = pooled_scores
+    o.pool_visible = pool_visible
 
 
 def _mut_tie_higher_index(o):
@@ -144,6 +147,14 @@ def _mut_lowest_scores(o):
     o.ranked_blocks = ranked_blocks
 
 
+def _mut_nan_unordered(o):
+    def ranked_blocks(row, pos, block):
+        nvis = o.n_visible_blocks(pos, block)
+        vals = [float(row[b]) for b in range(nvis)]
+        return sorted(range(nvis), key=lambda b: (-vals[b], b))     # NaN left as NaN
+    o.ranked_blocks = ranked_blocks
+
+
 def _mut_append_swapped(o):
     def indexer_append(cache, new, ts, tp):
         out = cache.clone()
@@ -232,7 +243,7 @@ def _mut_dsa_group_zero(o):
 MUTATIONS = [_mut_causal_off_by_one, _mut_no_causal_mask, _mut_tie_higher_index, _mut_no_bias,
              _mut_gqa_modulo, _mut_no_scale, _mut_nvis_off_by_one, _mut_transposed_scores,
              _mut_dropped_term, _mut_future_rows, _mut_sign, _mut_k_minus_one,
-             _mut_unsorted_ids, _mut_lowest_scores, _mut_append_swapped, _mut_paged_table_transposed,
+             _mut_unsorted_ids, _mut_lowest_scores, _mut_nan_unordered, _mut_append_swapped, _mut_paged_table_transposed,
              _mut_paged_slots_reversed, _mut_paged_append_next_slot, _mut_dsa_no_relu, _mut_dsa_unweighted,
              _mut_dsa_future_tokens, _mut_dsa_tie_higher_index, _mut_dsa_k_minus_one, _mut_dsa_group_zero]
 

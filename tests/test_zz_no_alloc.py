@@ -6,8 +6,8 @@ uses the library's fixed file-scope device buffer.
 
 The GPU test calls the new entry point through the C ABI twice in a row, with
 different batch sizes (so the second call runs over the first call's leftover
-buffer contents), and checks each output against the workspace entry point
-msa_sparse_attn_decode within the attention tolerance of the parity tests.
+buffer contents), and checks that each output is bit-identical to the
+workspace entry point msa_sparse_attn_decode (same kernels, same split).
 This file is collected last so a failure here never hides another test."""
 import ctypes
 
@@ -42,6 +42,16 @@ def test_noalloc_buffer_covers_every_batch_and_checks_shapes():
                                               ctypes.c_float(0.088), fake, None) == -3
 
 
+def test_binding_scratch_size_matches_header():
+    """The binding's copy of the buffer size is the header's constant."""
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "msa.h")).read()
+    m = re.search(r"#define\s+MSA_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", hdr)
+    assert m is not None
+    assert eval(m.group(1).replace("u", "").replace("ll", ""), {}) == msa.NOALLOC_SCRATCH_BYTES
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
     if not torch.cuda.is_available():
@@ -59,8 +69,6 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         msa.msa_sparse_attn_decode_noalloc(shape, d["q"], d["k_cache"], d["v_cache"], sel, d["q_stream"],
                                            d["q_pos"], out=out_na)
         assert msa.msa_get_device_error() == 0
-        a, b = out_na.cpu().double(), out_ws.cpu().double()
-        assert torch.isfinite(a).all(), f"call {call}: output not fully written"
-        diff = (a - b).abs()
-        assert float(diff.max()) <= PT.ATTN_MAX_ABS, f"call {call}: max abs diff {float(diff.max())}"
-        assert float(diff.mean()) <= PT.ATTN_MEAN_ABS, f"call {call}: mean abs diff {float(diff.mean())}"
+        # the same kernels with the same split: bit-identical, so a stale
+        # partial left in the shared buffer by the first call cannot hide
+        assert torch.equal(out_na, out_ws), f"call {call}: differs from the workspace entry point"
