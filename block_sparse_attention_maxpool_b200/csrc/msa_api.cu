@@ -368,6 +368,9 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
     Q.kscale = reinterpret_cast<float*>(ws + L.kscale);
     Q.khi = reinterpret_cast<__half*>(ws + L.khi);
     Q.klo = reinterpret_cast<__half*>(ws + L.klo);
+    Q.qlo_nz = reinterpret_cast<int*>(ws + L.qlo_nz);
+    Q.klo_nz = reinterpret_cast<int*>(ws + L.klo_nz);
+    Q.n_flags = G * L.n_tiles + S * G * Q.nblk;
     Q.pages = pg;
     const int64_t key_rows = static_cast<int64_t>(S) * G * cap;
     const int64_t q_rows = static_cast<int64_t>(G) * L.n_q_pad;
@@ -379,7 +382,7 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
     static std::atomic<uint64_t> tc_smem_done{0};
     if ((st = ensure_smem(T::block_scores_tc_kernel, T::SmemLayout::kBytes, tc_smem_done)) != MSA_OK) return st;
 
-    launch(T::tc_init_kernel, dim3(1), dim3(256), 0, cs, Q.counters, 1 + S);
+    launch(T::tc_init_kernel, dim3(1), dim3(1024), 0, cs, Q.counters, 1 + S, Q);
     launch(T::tc_tile_info_kernel, dim3((L.n_tiles * 32 + 255) / 256), dim3(256), 0, cs, Q);
     launch(T::tc_split_queries_kernel, dim3(static_cast<unsigned>((q_rows * 32 + 255) / 256)), dim3(256), 0, cs, Q);
     launch(T::tc_split_keys_kernel, dim3(static_cast<unsigned>((key_rows * 32 + 255) / 256)), dim3(256), 0, cs, Q);

@@ -400,12 +400,14 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
         alpha[h] = exp2f(m_run[h] - m_use[h]);
         m_run[h] = m_new;
       }
+      // P rounded to bf16 as the P . V product takes it, and the row sum of
+      // those rounded values, so the normalisation matches the weights used
       float rs[2] = {0.f, 0.f};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float pe = exp2f(sacc[nt][e] - m_use[e >> 1]);
+          const float pe = __bfloat162float(__float2bfloat16_rn(exp2f(sacc[nt][e] - m_use[e >> 1])));
           sacc[nt][e] = pe;
           rs[e >> 1] += pe;
         }

@@ -47,12 +47,12 @@
 // TMEM lane quarter each).  Shared memory: Q 32 KB, K ring 3 x 32 KB, V ring
 // 2 x 32 KB.  Tensor memory: three S/P buffers and O (all 512 columns).
 //
-// Per block, a softmax warp whose queries selected it spends ~1900 cycles
-// (S load ~250, row max ~280, 128 exponentials ~1330 against a floor of
-// 1024 on the special-function unit, which runs 4 per clock per SM
-// quarter), one whose queries did not ~400; the quarters are busy on about
-// half the blocks each, at random, and three S buffers let them drift at
-// most two blocks apart, so the slowest quarter sets the pace.
+// Per block, a softmax warp whose queries selected it loads S, takes the
+// row max and computes 128 exponentials per row; one whose queries did not
+// writes zeros.  The
+// quarters are busy on about half the blocks each, at random, and three S
+// buffers let them drift at most two blocks apart, so the slowest quarter
+// sets the pace when it is slower than the tensor pipe.
 #pragma once
 
 #include "msa_common.cuh"
@@ -141,6 +141,24 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Two floats rounded to bf16 (nearest even) and packed: `lo` into the low
+// half (the lower K index of a P pair), `hi` into the high half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// acc + both bf16 halves of `p`, in float32.
+__device__ __forceinline__ float add_bf16x2_f32(uint32_t p, float acc) {
+  float d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, lo, %2;\n\t"
+      "add.rn.f32.bf16 %0, hi, %0;\n}"
+      : "=f"(d)
+      : "r"(p), "f"(acc));
+  return d;
+}
+
 // Packed f32x2 arithmetic (sm_100 and later): two lanes per instruction.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   float2 d;
@@ -150,15 +168,6 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return d;
 }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
 // max(a, b, c) in one instruction (three-input max.f32, sm_100 and later).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -690,24 +699,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (raise) m_ref = mb;
         const float neg_m = mine ? -m_ref : -INFINITY;
-        // P = exp2(s - m_ref) as bf16 pairs over the first 64 columns of the buffer
+        // P = exp2(s - m_ref) as bf16 pairs over the first 64 columns of the
+        // buffer; the row sum adds the rounded P values the P . V product
+        // uses, so the normalisation matches the weights applied
         if (active) {
           const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
           const float2 nm2 = make_float2(neg_m, neg_m);
-          float2 rs = make_float2(0.f, 0.f);
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             float pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float2 x = ffma2(make_float2(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]), sc2, nm2);
-              const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-              rs = fadd2(rs, e);
-              pk[i] = __uint_as_float(pack_bf16(e.x, e.y));
+              const uint32_t pp = cvt_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+              acc[i & 3] = add_bf16x2_f32(pp, acc[i & 3]);
+              pk[i] = __uint_as_float(pp);
             }
             tmem_st32(sbuf + h * 32, pk);
           }
-          l += rs.x + rs.y;
+          l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         } else {
           float z[32];
 #pragma unroll

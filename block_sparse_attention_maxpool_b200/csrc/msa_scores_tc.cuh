@@ -16,6 +16,10 @@
 // dropped lo_q.lo_k term and the fp16 rounding of lo leave a relative error
 // near 2^-22 of sum |q_d k_d|, the same order as a float32 dot product.  The
 // epilogue multiplies each score by 2^-(e_q + e_k) (exact) before pooling.
+// The split kernels flag every 128-row tile with a nonzero lo part; a tile
+// whose lo half is all zero (rows that fit fp16 after scaling: keys of the
+// F16 cache, values on a coarse grid) is neither loaded nor multiplied, as
+// its products add exactly zero.
 //
 // Launch sequence (all on the caller's stream):
 //   tc_init_kernel         zero the per-call counters
@@ -57,7 +61,7 @@ struct SmemLayout {
 
 // Workspace carve-up of the prefill block-score path (byte offsets).
 struct Workspace {
-  size_t counters, tile_stream, tile_nb, leftover, qscale, qhi, qlo, kscale, khi, klo, total;
+  size_t counters, tile_stream, tile_nb, leftover, qscale, qhi, qlo, kscale, khi, klo, qlo_nz, klo_nz, total;
   int n_tiles, n_q_pad;
 };
 
@@ -78,6 +82,8 @@ __host__ inline Workspace workspace_layout(int n_q, int G, int S, int cap) {
   w.kscale = o;      o = align256(o + sizeof(float) * static_cast<size_t>(S) * G * cap);
   w.khi = o;         o = align256(o + sizeof(__half) * static_cast<size_t>(S) * G * cap * kDi);
   w.klo = o;         o = align256(o + sizeof(__half) * static_cast<size_t>(S) * G * cap * kDi);
+  w.qlo_nz = o;      o = align256(o + sizeof(int) * static_cast<size_t>(G) * w.n_tiles);
+  w.klo_nz = o;      o = align256(o + sizeof(int) * static_cast<size_t>(S) * G * (cap / kBlock));
   w.total = o;
   return w;
 }
@@ -100,6 +106,9 @@ struct Params {
   float* kscale;            // [S][G][cap]   2^-e_k
   __half* khi;              // [S][G][cap][Di]
   __half* klo;
+  int* qlo_nz;              // [G][n_tiles]       some query row of the tile has a nonzero lo part
+  int* klo_nz;              // [S][G][cap / 128]  some key row of the block has a nonzero lo part
+  int n_flags;              // entries of qlo_nz and klo_nz together (zeroed by tc_init_kernel)
   KvPages pages;            // block table of a paged key cache (table null: contiguous)
 };
 
@@ -109,10 +118,24 @@ __device__ __forceinline__ bool query_ok(const Params& P, int q, int& s, int& p)
   return s >= 0 && s < P.n_streams && p >= 0 && p < P.capacity;
 }
 
-__global__ void tc_init_kernel(int* counters, int n) {
+__global__ void tc_init_kernel(int* counters, int n, const Params P) {
   pdl_trigger();
   pdl_wait();
   for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0;
+  const int nq = P.G * P.n_tiles;
+  for (int i = threadIdx.x; i < P.n_flags; i += blockDim.x) {
+    if (i < nq) P.qlo_nz[i] = 0;
+    else P.klo_nz[i - nq] = 0;
+  }
+}
+
+// Flags the 128-row tile of a split row whose lo part is not all zero: the
+// products with that tile's lo half are then needed (an all-zero lo half
+// adds exactly zero, so its products are skipped).
+__device__ __forceinline__ void flag_lo(const __half2 (&lo)[2], int* flag) {
+  const uint32_t a = *reinterpret_cast<const uint32_t*>(&lo[0]) | *reinterpret_cast<const uint32_t*>(&lo[1]);
+  if (__any_sync(0xffffffffu, (a & 0x7fff7fffu) != 0u) && (threadIdx.x & 31) == 0 && *flag == 0)
+    atomicOr(flag, 1);
 }
 
 // One warp per tile of 128 consecutive queries.  The tile's stream is the
@@ -213,6 +236,7 @@ __global__ void __launch_bounds__(256) tc_split_queries_kernel(const Params P) {
   *reinterpret_cast<uint2*>(P.qlo + row * kDi + lane * 4) =
       make_uint2(*reinterpret_cast<uint32_t*>(&lo[0]), *reinterpret_cast<uint32_t*>(&lo[1]));
   if (lane == 0) P.qscale[row] = pow2f(-e);
+  flag_lo(lo, &P.qlo_nz[g * P.n_tiles + q / kTileQ]);
   if (!real) return;
   const int nvis = ok ? p / kBlock + 1 : 0;
   float* out = P.bs + (static_cast<size_t>(q) * P.G + g) * P.nblk;
@@ -267,6 +291,7 @@ __global__ void __launch_bounds__(256) tc_split_keys_kernel(const Params P) {
   *reinterpret_cast<uint2*>(P.klo + w * kDi + lane * 4) =
       make_uint2(*reinterpret_cast<uint32_t*>(&lo[0]), *reinterpret_cast<uint32_t*>(&lo[1]));
   if (lane == 0) P.kscale[w] = pow2f(-e);
+  flag_lo(lo, &P.klo_nz[w / kBlock]);
 }
 
 // Task t -> (group, key chunk, query tile); consecutive tasks share a key
@@ -341,24 +366,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = P.tile_stream[tile];
         if (a_use > 0 && !mbar_wait(a_empty, (a_use - 1) & 1)) { *abort_v = 1; break; }
         const int qrow = g * P.n_q_pad + tile * kTileQ;
-        mbar_arrive_expect_tx(a_full, kOperandBytes);
+        const bool q_lo = __ldcg(&P.qlo_nz[g * P.n_tiles + tile]) != 0;
+        mbar_arrive_expect_tx(a_full, q_lo ? kOperandBytes : kOperandBytes / 2);
         tma_load_2d(smem + SmemLayout::kA, &tm_qhi, 0, qrow, a_full);
         tma_load_2d(smem + SmemLayout::kA + kHalfBytes, &tm_qhi, 64, qrow, a_full);
-        tma_load_2d(smem + SmemLayout::kA + 2 * kHalfBytes, &tm_qlo, 0, qrow, a_full);
-        tma_load_2d(smem + SmemLayout::kA + 3 * kHalfBytes, &tm_qlo, 64, qrow, a_full);
+        if (q_lo) {
+          tma_load_2d(smem + SmemLayout::kA + 2 * kHalfBytes, &tm_qlo, 0, qrow, a_full);
+          tma_load_2d(smem + SmemLayout::kA + 3 * kHalfBytes, &tm_qlo, 64, qrow, a_full);
+        }
         ++a_use;
         const size_t krow0 = (static_cast<size_t>(s) * P.G + g) * P.capacity;
+        const int* klo_nz = P.klo_nz + (static_cast<size_t>(s) * P.G + g) * P.nblk;
         for (int b = b0; b < b1; ++b, ++kst) {
           const int st = kst % kStages;
           const int use = kst / kStages;
           if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1)) { *abort_v = 1; break; }
           uint8_t* dst = smem + SmemLayout::kB + st * kOperandBytes;
           const int krow = static_cast<int>(krow0) + b * kBlock;
-          mbar_arrive_expect_tx(&full[st], kOperandBytes);
+          const bool k_lo = __ldcg(klo_nz + b) != 0;
+          mbar_arrive_expect_tx(&full[st], k_lo ? kOperandBytes : kOperandBytes / 2);
           tma_load_2d(dst, &tm_khi, 0, krow, &full[st]);
           tma_load_2d(dst + kHalfBytes, &tm_khi, 64, krow, &full[st]);
-          tma_load_2d(dst + 2 * kHalfBytes, &tm_klo, 0, krow, &full[st]);
-          tma_load_2d(dst + 3 * kHalfBytes, &tm_klo, 64, krow, &full[st]);
+          if (k_lo) {
+            tma_load_2d(dst + 2 * kHalfBytes, &tm_klo, 0, krow, &full[st]);
+            tma_load_2d(dst + 3 * kHalfBytes, &tm_klo, 64, krow, &full[st]);
+          }
         }
       }
       // let copies still landing finish before the CTA can exit
@@ -377,6 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (b0 >= b1) continue;
         if (!mbar_wait(a_full, a_use & 1)) { *abort_v = 1; break; }
         tc_fence_after();
+        const int s = P.tile_stream[tile];
+        const bool q_lo = __ldcg(&P.qlo_nz[g * P.n_tiles + tile]) != 0;
+        const int* klo_nz = P.klo_nz + (static_cast<size_t>(s) * P.G + g) * P.nblk;
         for (int b = b0; b < b1; ++b, ++kst, ++acc) {
           const int st = kst % kStages;
           const int buf = acc & 1;
@@ -385,9 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t b_base = smem_addr(smem + SmemLayout::kB + st * kOperandBytes);
           const uint32_t d = tmem_base + static_cast<uint32_t>(buf * 128);
-          // three products: hi.hi, hi.lo, lo.hi; 8 K-steps of 16 each
+          // three products: hi.hi, hi.lo, lo.hi; 8 K-steps of 16 each; a
+          // product whose lo operand is all zero adds exactly zero and is skipped
+          const bool k_lo = __ldcg(klo_nz + b) != 0;
 #pragma unroll
           for (int pass = 0; pass < 3; ++pass) {
+            if ((pass == 1 && !k_lo) || (pass == 2 && !q_lo)) continue;
             const uint32_t a_off = pass == 2 ? 2 * kHalfBytes : 0;   // q lo for the last pass
             const uint32_t b_off = pass == 1 ? 2 * kHalfBytes : 0;   // k lo for the second pass
 #pragma unroll

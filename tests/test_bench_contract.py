@@ -26,8 +26,10 @@ def test_reference_arm_prints_one_contract_line():
     assert d["unit"] == "tokens/s" and d["value"] > 0
     assert d["n_gpus"] == 1 and d["warmup"] == 3 and 1 <= d["steps"] <= 3
     assert d["ms_per_step"] > 0
-    # value is the throughput of the timed steps: one stream's token per step
-    assert abs(d["value"] - 1e3 / d["ms_per_step"]) <= 1e-6 * d["value"]
+    # value is the throughput of the timed steps: one token per sampled stream per step
+    n = d["config"]["streams_per_step"]
+    assert n >= 1
+    assert abs(d["value"] - n * 1e3 / d["ms_per_step"]) <= 1e-6 * d["value"]
     assert d["higher_is_better"] is True and d["scaling"] == "weak"
     assert d["vs_baseline"] is None and d["dtype"] == "f64" and d["data"] == "synthetic"
     assert d["config"]["workload"] == "decode_32x32k"

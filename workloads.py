@@ -180,6 +180,32 @@ def make_inputs(w: Workload, seed: int = 0, streams: range | None = None) -> Inp
                   q_stream, q_pos, idx_q, q)
 
 
+def make_step_set(w: Workload, seed: int, streams: range | None = None) -> dict:
+    """Another draw of a decode step's new tokens and queries for the same
+    caches: idx_k_new, k_new, v_new [ns][G][dim] (one token per stream, at
+    its last slot), idx_q [ns][G][Di] and q [ns][Hq][D], from per-stream
+    generators seeded seed * 1000003 + stream + 9000000007.  Steps that
+    alternate between such sets append and query different values at the same
+    slot, so their block selections (and the K/V blocks they read) differ."""
+    if w.queries != "last" or w.n_new != 1:
+        raise ValueError("step sets are drawn for one-token decode steps")
+    S = w.n_streams
+    streams = range(S) if streams is None else streams
+    G, Di, D, Hq = w.n_kv_heads, w.idx_dim, w.head_dim, w.n_q_heads
+    ns = len(streams)
+    out = {"idx_k_new": torch.empty((ns, G, Di)), "k_new": torch.empty((ns, G, D), dtype=torch.bfloat16),
+           "v_new": torch.empty((ns, G, D), dtype=torch.bfloat16), "idx_q": torch.empty((ns, G, Di)),
+           "q": torch.empty((ns, Hq, D), dtype=torch.bfloat16)}
+    for i, s in enumerate(streams):
+        g = torch.Generator().manual_seed(seed * 1_000_003 + s + 9_000_000_007)
+        out["idx_k_new"][i] = _idx_draw(g, (G, Di), Di, w.quantize_idx)
+        out["k_new"][i] = _bf16_draw(g, (G, D))
+        out["v_new"][i] = _bf16_draw(g, (G, D))
+        out["idx_q"][i] = _idx_draw(g, (G, Di), Di, w.quantize_idx)
+        out["q"][i] = _bf16_draw(g, (Hq, D))
+    return out
+
+
 def make_custom(n_streams: int, capacity: int, lengths, q_positions, *, seed: int = 0,
                 n_q_heads: int = N_Q_HEADS, n_kv_heads: int = N_KV_HEADS,
                 head_dim: int = HEAD_DIM, idx_dim: int = IDX_DIM, quantize_idx: bool = False,
