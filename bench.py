@@ -58,11 +58,11 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM traffic of one block-scores launch on the 32-stream workload, per key
 # type: dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of
 # the 8-stream case (one launch), scaled by 4 to 32 streams (the reads grow
-# in proportion to the keys scanned).  Valid only for the kernel source it
-# was taken on (sha256 prefix of msa_scores_gemv.cuh); any other source
-# reports null.
-SCORES_TRAFFIC = {"source_sha": "b9bc1ca3c5d4d5a4",
-                  "bytes_per_launch": {"f32": 4 * (536_911_872 + 3_886_848), "f16": 4 * (268_474_112 + 2_967_040)}}
+# in proportion to the keys scanned).  Each figure is valid only for the
+# kernel source it was taken on (sha256 prefix of msa_scores_gemv.cuh); any
+# other source reports null.
+SCORES_TRAFFIC = {"f32": {"source_sha": "0c7e835ccd50eea6", "bytes_per_launch": 4 * (536_926_720 + 3_099_392)},
+                  "f16": {"source_sha": "b9bc1ca3c5d4d5a4", "bytes_per_launch": 4 * (268_474_112 + 2_967_040)}}
 
 # The same for the token-score kernel of the token-level variant, from a
 # capture of the 16-stream case, scaled by 2 to 32 streams (sha256 prefix
@@ -684,9 +684,10 @@ def roofline_decode(w, step: Step, k_ms: float, peaks: dict, key_bytes: int) -> 
         sbytes, kernel = scores_bytes(w, key_bytes), "block_scores_gemv"
     achieved = sbytes / (k_ms * 1e-3) / 1e9
     traffic = None
-    if not step.fused and not step.dsa and SCORES_TRAFFIC["source_sha"] == scores_source_sha() \
+    cap = SCORES_TRAFFIC["f16" if key_bytes == 2 else "f32"]
+    if not step.fused and not step.dsa and cap["source_sha"] == scores_source_sha() \
             and w == WORKLOAD and step.pages is None:
-        traffic = SCORES_TRAFFIC["bytes_per_launch"]["f16" if key_bytes == 2 else "f32"]
+        traffic = cap["bytes_per_launch"]
     if step.dsa and DSA_SCORES_TRAFFIC["source_sha"] == scores_source_sha("msa_dsa_scores.cuh") and w == WORKLOAD:
         traffic = DSA_SCORES_TRAFFIC["bytes_per_launch"]
     return {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -496,17 +496,18 @@ int msa_select_topk(const msa_shape* shape, const float* block_scores, const int
   const int nblk = shape->capacity / 128;
   const int64_t warps = static_cast<int64_t>(n_q) * G;
   if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
-  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  using msa::sel::SelectLaunch;
+  auto grid_of = [&](int threads) { return dim3(static_cast<unsigned>((warps * 32 + threads - 1) / threads)); };
   if (nblk <= 32 * 8) {
-    launch(msa::sel::select_topk_kernel<8>, dim3(grid), dim3(256), 0, s, block_scores, q_pos, n_q, G, nblk, shape->capacity,
-                                                          sel, n_sel);
+    launch(msa::sel::select_topk_kernel<8>, grid_of(SelectLaunch<8>::kThreads), dim3(SelectLaunch<8>::kThreads),
+           SelectLaunch<8>::kSmem, s, block_scores, q_pos, n_q, G, nblk, shape->capacity, sel, n_sel);
   } else if (nblk <= 32 * 32) {
-    launch(msa::sel::select_topk_kernel<32>, dim3(grid), dim3(256), 0, s, block_scores, q_pos, n_q, G, nblk, shape->capacity,
-                                                           sel, n_sel);
+    launch(msa::sel::select_topk_kernel<32>, grid_of(SelectLaunch<32>::kThreads), dim3(SelectLaunch<32>::kThreads),
+           SelectLaunch<32>::kSmem, s, block_scores, q_pos, n_q, G, nblk, shape->capacity, sel, n_sel);
   } else {
-    launch(msa::sel::select_topk_kernel<0>, dim3(grid), dim3(256), 0, s, block_scores, q_pos, n_q, G, nblk, shape->capacity,
-                                                          sel, n_sel);
+    launch(msa::sel::select_topk_kernel<0>, grid_of(SelectLaunch<0>::kThreads), dim3(SelectLaunch<0>::kThreads),
+           SelectLaunch<0>::kSmem, s, block_scores, q_pos, n_q, G, nblk, shape->capacity, sel, n_sel);
   }
   return cuda_status(cudaGetLastError());
 }

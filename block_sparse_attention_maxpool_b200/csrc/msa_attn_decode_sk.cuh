@@ -468,24 +468,40 @@ __device__ __forceinline__ void combine_pair_head(const Params& P, long long w, 
   const int c_lo = cta_of(U, P.n_cta, pair * kTopK);
   const int c_hi = cta_of(U, P.n_cta, pair * kTopK + kTopK - 1);
   if (c_lo == c_hi) return;                              // written directly by its CTA
-  float M = -INFINITY;
-  for (int c = c_lo; c <= c_hi; ++c) {
-    const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
-    M = fmaxf(M, __ldcg(P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial + kHpg * kD + head));
-  }
-  const float Mu = M == -INFINITY ? 0.f : M;
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = c_lo; c <= c_hi; ++c) {
+  // every CTA in [c_lo, c_hi] holds at least one of the pair's 16 units, so
+  // there are at most 16 partials: lane j reads partial j's max and sum, and
+  // the warp reduces them, then sums the scaled O slices
+  const int n = c_hi - c_lo + 1;
+  float mj = -INFINITY, lj = 0.f;
+  if (lane < n) {
+    const int c = c_lo + lane;
     const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
     const float* part = P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial;
-    const float sc = exp2f(__ldcg(part + kHpg * kD + head) - Mu);
-    L += __ldcg(part + kHpg * kD + kHpg + head) * sc;
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(part + head * kD + lane * 4));
-    acc.x += v.x * sc;
-    acc.y += v.y * sc;
-    acc.z += v.z * sc;
-    acc.w += v.w * sc;
+    mj = __ldcg(part + kHpg * kD + head);
+    lj = __ldcg(part + kHpg * kD + kHpg + head);
+  }
+  float M = mj;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float Mu = M == -INFINITY ? 0.f : M;
+  const float scj = lane < n ? exp2f(mj - Mu) : 0.f;
+  float L = lj * scj;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < kTopK; ++j) {
+    const float sc = __shfl_sync(0xffffffffu, scj, j);
+    if (j < n) {
+      const int c = c_lo + j;
+      const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
+      const float* part = P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(part + head * kD + lane * 4));
+      acc.x += v.x * sc;
+      acc.y += v.y * sc;
+      acc.z += v.z * sc;
+      acc.w += v.w * sc;
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + lane * 4;

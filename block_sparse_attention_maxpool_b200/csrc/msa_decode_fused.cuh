@@ -38,6 +38,7 @@ constexpr int kThreads = dattn::kThreads;                      // the widest pha
 constexpr size_t kScoreSmem = sizeof(gemv::Smem<ScoreKey, kScoreStages, kScoreWarps>);
 constexpr size_t kSmemBytes = dattn::Layout::kBytes > kScoreSmem + 1024 ? dattn::Layout::kBytes : kScoreSmem + 1024;
 static_assert(kThreads >= (kScoreWarps + 1) * 32, "the score body needs its producer warp");
+static_assert((kThreads / 32) * sel::KeySmem<32>::kBytesPerWarp <= kSmemBytes, "the top-16 keys of every warp");
 
 struct Params {
   // phase 1: appends of the new tokens
@@ -163,9 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- 3. top-16 per (query, group) ----------------------------------------
   const int n_pairs = F.scores.n_q * G;
+  uint64_t* wsm = reinterpret_cast<uint64_t*>(smem + warp * sel::select_smem_per_warp(F.scores.nblk));
   for (long long w = gwarp; w < n_pairs; w += n_gwarps)
     sel::select_pair_any(F.scores.bs, F.scores.q_pos, G, F.scores.nblk, F.scores.capacity, F.sel, F.n_sel,
-                         static_cast<int>(w), lane);
+                         static_cast<int>(w), lane, wsm);
   if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
 
   // ---- 4. attention over the selected blocks -------------------------------

@@ -28,7 +28,9 @@
 //   tc_split_queries_kernel  hi/lo/scale of every (query, group) row, -inf
 //                          for the blocks a query cannot see
 //   tc_split_keys_kernel   hi/lo/scale of the keys the tiles will read
-//   block_scores_tc_kernel persistent, warp-specialised tile kernel
+//   block_scores_tc_kernel persistent, warp-specialised tile kernel (one
+//                          TMA producer with a ring of five 32 KB key
+//                          slots, one MMA issuer, four epilogue warps)
 //   block_scores_gemv_kernel (list mode) for the leftover queries
 #pragma once
 
@@ -45,19 +47,24 @@ constexpr int kTileQ = 128;                 // queries per tile (MMA M)
 constexpr int kChunk = 32;                  // key blocks per task
 constexpr uint32_t kHalfBytes = 128 * 128;  // [128 rows][64 fp16] = 16 KB (one swizzle-128B box)
 constexpr uint32_t kOperandBytes = 4 * kHalfBytes;   // hi (2 halves) + lo (2 halves) = 64 KB
-constexpr int kStages = 2;
-constexpr int kThreads = 6 * 32;            // producer, MMA, 4 epilogue warps
+constexpr uint32_t kSlotBytes = 2 * kHalfBytes;      // the hi or the lo half of a key block = 32 KB
+constexpr int kSlots = 5;                            // key ring: a block takes 1 slot (hi) or 2 (hi, lo)
+constexpr int kEpiGroups = 1;               // epilogue groups (group e drains accumulators acc % kEpiGroups == e)
+constexpr int kThreads = (2 + 4 * kEpiGroups) * 32;   // producer, MMA, 2 x 4 epilogue warps
 constexpr uint32_t kTmemCols = 256;         // two 128-column fp32 accumulators
 constexpr uint32_t kIdesc = umma_idesc_f16_f32(128, 128);
 
 struct SmemLayout {
   // all operand tiles 1024-byte aligned (swizzle atom)
   static constexpr uint32_t kA = 0;                                     // q hi|lo
-  static constexpr uint32_t kB = kA + kOperandBytes;                    // stages of k hi|lo
-  static constexpr uint32_t kBars = kB + kStages * kOperandBytes;
+  static constexpr uint32_t kB = kA + kOperandBytes;                    // key ring: kSlots x 32 KB
+  static constexpr uint32_t kBars = kB + kSlots * kSlotBytes;
   static constexpr uint32_t kEnd = kBars + 256;
   static constexpr size_t kBytes = kEnd + 1024;                         // + alignment slack
 };
+
+static_assert(SmemLayout::kBytes <= 232448, "shared memory budget");
+static_assert(2 * kSlots + 7 <= 32, "barrier slots");
 
 // Workspace carve-up of the prefill block-score path (byte offsets).
 struct Workspace {
@@ -111,6 +118,23 @@ struct Params {
   int n_flags;              // entries of qlo_nz and klo_nz together (zeroed by tc_init_kernel)
   KvPages pages;            // block table of a paged key cache (table null: contiguous)
 };
+
+// Packed f32x2 multiply (sm_100 and later): two lanes per instruction.
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// max(a, b, c) in one instruction (three-input max.f32, sm_100 and later).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 __device__ __forceinline__ bool query_ok(const Params& P, int q, int& s, int& p) {
   s = P.q_stream[q];
@@ -317,22 +341,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBars);
-  uint64_t* full = bars;                  // [kStages]  key tile landed
-  uint64_t* empty = bars + 2;             // [kStages]  MMAs done reading the key tile
-  uint64_t* a_full = bars + 4;            // query tile landed
-  uint64_t* a_empty = bars + 5;           // MMAs done reading the query tile
-  uint64_t* acc_full = bars + 6;          // [2] accumulator ready
-  uint64_t* acc_empty = bars + 8;         // [2] accumulator drained
-  uint64_t* mma_done = bars + 10;         // every MMA of this CTA finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
-  int* abort_flag = reinterpret_cast<int*>(bars + 12);
+  uint64_t* full = bars;                  // [kSlots]  key half-tile landed
+  uint64_t* empty = full + kSlots;        // [kSlots]  MMAs done reading it
+  uint64_t* a_full = empty + kSlots;      // query tile landed
+  uint64_t* a_empty = a_full + 1;         // MMAs done reading the query tile
+  uint64_t* acc_full = a_empty + 1;       // [2] accumulator ready
+  uint64_t* acc_empty = acc_full + 2;     // [2] accumulator drained
+  uint64_t* mma_done = acc_empty + 2;     // every MMA of this CTA finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  int* abort_flag = reinterpret_cast<int*>(mma_done + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tasks = P.G * P.n_chunks * P.n_tiles;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -357,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
-      int kst = 0, a_use = 0;
+      int slot = 0, a_use = 0;
       for (int t = blockIdx.x; t < n_tasks && !*abort_v; t += gridDim.x) {
         int g, chunk, tile, b0, b1;
         task_coords(P, t, g, chunk, tile);
@@ -377,30 +401,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++a_use;
         const size_t krow0 = (static_cast<size_t>(s) * P.G + g) * P.capacity;
         const int* klo_nz = P.klo_nz + (static_cast<size_t>(s) * P.G + g) * P.nblk;
-        for (int b = b0; b < b1; ++b, ++kst) {
-          const int st = kst % kStages;
-          const int use = kst / kStages;
-          if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1)) { *abort_v = 1; break; }
-          uint8_t* dst = smem + SmemLayout::kB + st * kOperandBytes;
+        bool stop = false;
+        for (int b = b0; b < b1 && !stop; ++b) {
           const int krow = static_cast<int>(krow0) + b * kBlock;
           const bool k_lo = __ldcg(klo_nz + b) != 0;
-          mbar_arrive_expect_tx(&full[st], k_lo ? kOperandBytes : kOperandBytes / 2);
-          tma_load_2d(dst, &tm_khi, 0, krow, &full[st]);
-          tma_load_2d(dst + kHalfBytes, &tm_khi, 64, krow, &full[st]);
-          if (k_lo) {
-            tma_load_2d(dst + 2 * kHalfBytes, &tm_klo, 0, krow, &full[st]);
-            tma_load_2d(dst + 3 * kHalfBytes, &tm_klo, 64, krow, &full[st]);
+          // the hi half of the key block, then (when nonzero) its lo half, one slot each
+          for (int h = 0; h < (k_lo ? 2 : 1); ++h, ++slot) {
+            const int st = slot % kSlots;
+            const int use = slot / kSlots;
+            if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1)) { *abort_v = 1; stop = true; break; }
+            uint8_t* dst = smem + SmemLayout::kB + st * kSlotBytes;
+            const CUtensorMap* map = h == 0 ? &tm_khi : &tm_klo;
+            mbar_arrive_expect_tx(&full[st], kSlotBytes);
+            tma_load_2d(dst, map, 0, krow, &full[st]);
+            tma_load_2d(dst + kHalfBytes, map, 64, krow, &full[st]);
           }
         }
+        if (stop) break;
       }
       // let copies still landing finish before the CTA can exit
-      for (int j = max(0, kst - kStages); j < kst; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
+      for (int j = max(0, slot - kSlots); j < slot; ++j) mbar_wait(&full[j % kSlots], (j / kSlots) & 1);
       if (a_use > 0) mbar_wait(a_full, (a_use - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
-      int kst = 0, a_use = 0, acc = 0;
+      int slot = 0, a_use = 0, acc = 0;
       const uint32_t a_base = smem_addr(smem + SmemLayout::kA);
       for (int t = blockIdx.x; t < n_tasks && !*abort_v; t += gridDim.x) {
         int g, chunk, tile, b0, b1;
@@ -412,31 +438,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = P.tile_stream[tile];
         const bool q_lo = __ldcg(&P.qlo_nz[g * P.n_tiles + tile]) != 0;
         const int* klo_nz = P.klo_nz + (static_cast<size_t>(s) * P.G + g) * P.nblk;
-        for (int b = b0; b < b1; ++b, ++kst, ++acc) {
-          const int st = kst % kStages;
+        for (int b = b0; b < b1; ++b, ++acc) {
+          const bool k_lo = __ldcg(klo_nz + b) != 0;
+          const int st_hi = slot % kSlots;
+          const int st_lo = (slot + 1) % kSlots;
           const int buf = acc & 1;
-          if (!mbar_wait(&full[st], (kst / kStages) & 1)) { *abort_v = 1; break; }
+          if (!mbar_wait(&full[st_hi], (slot / kSlots) & 1)) { *abort_v = 1; break; }
+          if (k_lo && !mbar_wait(&full[st_lo], ((slot + 1) / kSlots) & 1)) { *abort_v = 1; break; }
           if (acc >= 2 && !mbar_wait(&acc_empty[buf], ((acc >> 1) - 1) & 1)) { *abort_v = 1; break; }
           tc_fence_after();
-          const uint32_t b_base = smem_addr(smem + SmemLayout::kB + st * kOperandBytes);
+          const uint32_t b_hi = smem_addr(smem + SmemLayout::kB + st_hi * kSlotBytes);
+          const uint32_t b_lo = smem_addr(smem + SmemLayout::kB + st_lo * kSlotBytes);
           const uint32_t d = tmem_base + static_cast<uint32_t>(buf * 128);
           // three products: hi.hi, hi.lo, lo.hi; 8 K-steps of 16 each; a
           // product whose lo operand is all zero adds exactly zero and is skipped
-          const bool k_lo = __ldcg(klo_nz + b) != 0;
 #pragma unroll
           for (int pass = 0; pass < 3; ++pass) {
             if ((pass == 1 && !k_lo) || (pass == 2 && !q_lo)) continue;
             const uint32_t a_off = pass == 2 ? 2 * kHalfBytes : 0;   // q lo for the last pass
-            const uint32_t b_off = pass == 1 ? 2 * kHalfBytes : 0;   // k lo for the second pass
+            const uint32_t bb = pass == 1 ? b_lo : b_hi;              // k lo for the second pass
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-              umma_f16_ss(d, umma_desc_sw128(a_base + a_off + koff), umma_desc_sw128(b_base + b_off + koff),
-                          kIdesc, (pass | kk) != 0);
+              umma_f16_ss(d, umma_desc_sw128(a_base + a_off + koff), umma_desc_sw128(bb + koff), kIdesc,
+                          (pass | kk) != 0);
             }
           }
-          umma_commit(&empty[st]);       // key tile may be overwritten once these MMAs finish
+          umma_commit(&empty[st_hi]);    // key slots may be overwritten once these MMAs finish
+          if (k_lo) umma_commit(&empty[st_lo]);
           umma_commit(&acc_full[buf]);   // accumulator ready for the epilogue
+          slot += k_lo ? 2 : 1;
         }
         umma_commit(a_empty);            // query tile free after the task's last MMA
         ++a_use;
@@ -446,8 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0);
     }
   } else {
-    // ------------------------------ epilogue (4 warps) -----------------------
+    // ---------------- epilogue: kEpiGroups groups of 4 warps ----------------
+    // Group e drains the accumulators of blocks acc with acc % kEpiGroups == e.
     const int quarter = warp & 3;                 // TMEM lane quarter this warp may read
+    const int group = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;          // query row within the tile
     int acc = 0;
     bool ok = true;
@@ -466,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* ksc_base = P.kscale + (static_cast<size_t>(ts < 0 ? 0 : ts) * P.G + g) * P.capacity;
       for (int b = b0; b < b1; ++b, ++acc) {
         const int buf = acc & 1;
+        if (kEpiGroups > 1 && (acc % kEpiGroups) != group) continue;
         if (ok && !*abort_v) ok = mbar_wait(&acc_full[buf], (acc >> 1) & 1);
         ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
         if (!ok) *abort_v = 1;
@@ -474,23 +508,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4* ksc = reinterpret_cast<const float4*>(ksc_base + static_cast<size_t>(b) * kBlock);
         const int jmax = p - b * kBlock;   // last visible key of this block (row-local)
         if (ok) {
+          float v[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + c * 32, v[c]);
+          tmem_ld_wait();
+          // scale each key's score by its exact power of two, then the max over
+          // the visible keys (only a row's local block is cut)
+          const bool cut = __any_sync(0xffffffffu, active && jmax < kBlock - 1);
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float v[32];
-            tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + c * 32, v);
-            tmem_ld_wait();
 #pragma unroll
             for (int i4 = 0; i4 < 8; ++i4) {
               const float4 k4 = __ldg(ksc + c * 8 + i4);
-              const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+              const float2 x01 = fmul2(make_float2(v[c][i4 * 4], v[c][i4 * 4 + 1]), make_float2(k4.x, k4.y));
+              const float2 x23 = fmul2(make_float2(v[c][i4 * 4 + 2], v[c][i4 * 4 + 3]), make_float2(k4.z, k4.w));
+              float x[4] = {x01.x, x01.y, x23.x, x23.y};
+              if (cut) {
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int j = c * 32 + i4 * 4 + u;
-                const float x = v[i4 * 4 + u] * kv[u];
-                if (j <= jmax) m = fmaxf(m, x);
+                for (int u = 0; u < 4; ++u) x[u] = c * 32 + i4 * 4 + u <= jmax ? x[u] : -INFINITY;
               }
+              m4[i4 & 3] = fmax3(m4[i4 & 3], fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
             }
           }
+          m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         tc_fence_before();
         __syncwarp();
