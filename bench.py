@@ -337,7 +337,8 @@ class Step:
         elif variant == "shared":
             self.launches = 1 + 2                # K/V append, attention + combine
         else:
-            self.launches = 2 + (6 if tiles else 1) + 1 + (2 if self.prefill else 2)
+            appends = 2 if args.idx_f16 else 1
+            self.launches = appends + (6 if tiles else 1) + 1 + 2
         self.parts = self._parts()
 
     def switch(self, variant: str):
@@ -355,10 +356,14 @@ class Step:
 
         def append(st, i):
             d = self.sets[i]
-            fn = msa.msa_indexer_append_f16 if self.idx_f16 else msa.msa_indexer_append
-            fn(sh, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st, pages)
-            msa.msa_kv_append(sh, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
-                              d["tok_pos"], st, pages)
+            if self.idx_f16:
+                msa.msa_indexer_append_f16(sh, d["idx_k_cache"], d["idx_k_new"], d["tok_stream"], d["tok_pos"], st,
+                                           pages)
+                msa.msa_kv_append(sh, d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["tok_stream"],
+                                  d["tok_pos"], st, pages)
+            else:                                   # one launch for the three caches
+                msa.msa_step_append(sh, d["idx_k_cache"], d["k_cache"], d["v_cache"], d["idx_k_new"], d["k_new"],
+                                    d["v_new"], d["tok_stream"], d["tok_pos"], st, pages)
 
         def scores(st, i):
             d = self.sets[i]

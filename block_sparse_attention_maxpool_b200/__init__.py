@@ -17,7 +17,7 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_block_scores",
+__all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_step_append", "msa_block_scores",
            "msa_indexer_append_f16",
            "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
            "msa_workspace_bytes", "msa_get_device_error", "msa_sparse_attn_decode_noalloc", "msa_version", "library", "LIB_PATH",
@@ -119,6 +119,7 @@ _I = ctypes.c_int32
 _SIGS = {
     "msa_indexer_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P]),
     "msa_kv_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I, _P]),
+    "msa_step_append": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     "msa_block_scores": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t,
                                         _P]),
     "msa_block_scores_f16": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _I, _P, _P,
@@ -142,6 +143,7 @@ _SIGS.update({
     "msa_indexer_append_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P]),
     "msa_indexer_append_f16_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P]),
     "msa_kv_append_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "msa_step_append_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     "msa_block_scores_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P, _P,
                                               ctypes.c_size_t, _P]),
     "msa_block_scores_f16_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _I, _P, _P,
@@ -242,6 +244,22 @@ def msa_kv_append(shape: Shape, k_cache, v_cache, k_new, v_new, tok_stream, tok_
     ns = (n, shape.n_kv_heads, shape.head_dim)
     _call("msa_kv_append", shape, pages,
           _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+          _ptr(k_new, torch.bfloat16, ns, "k_new"), _ptr(v_new, torch.bfloat16, ns, "v_new"),
+          _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
+          n, _stream(stream))
+
+
+def msa_step_append(shape: Shape, idx_k_cache, k_cache, v_cache, idx_k_new, k_new, v_new, tok_stream, tok_pos,
+                    stream=None, pages=None):
+    """The step's appends in one launch: F32 indexer keys and K/V rows
+    (msa_indexer_append + msa_kv_append)."""
+    n = _n(tok_stream, "tok_stream")
+    cs = _cache_shape(shape, pages, shape.head_dim)
+    ns = (n, shape.n_kv_heads, shape.head_dim)
+    _call("msa_step_append", shape, pages,
+          _ptr(idx_k_cache, torch.float32, _cache_shape(shape, pages, shape.idx_dim), "idx_k_cache"),
+          _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+          _ptr(idx_k_new, torch.float32, (n, shape.n_kv_heads, shape.idx_dim), "idx_k_new"),
           _ptr(k_new, torch.bfloat16, ns, "k_new"), _ptr(v_new, torch.bfloat16, ns, "v_new"),
           _ptr(tok_stream, torch.int32, (n,), "tok_stream"), _ptr(tok_pos, torch.int32, (n,), "tok_pos"),
           n, _stream(stream))
@@ -450,10 +468,14 @@ def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None,
     Returns (out, sel, n_sel, block_scores).
     """
     b = bufs or {}
-    append = msa_indexer_append_f16 if caches["idx_k_cache"].dtype == torch.float16 else msa_indexer_append
-    append(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"], new["tok_pos"], stream, pages)
-    msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
-                  new["tok_stream"], new["tok_pos"], stream, pages)
+    if caches["idx_k_cache"].dtype == torch.float16:
+        msa_indexer_append_f16(shape, caches["idx_k_cache"], new["idx_k_new"], new["tok_stream"], new["tok_pos"],
+                               stream, pages)
+        msa_kv_append(shape, caches["k_cache"], caches["v_cache"], new["k_new"], new["v_new"],
+                      new["tok_stream"], new["tok_pos"], stream, pages)
+    else:
+        msa_step_append(shape, caches["idx_k_cache"], caches["k_cache"], caches["v_cache"], new["idx_k_new"],
+                        new["k_new"], new["v_new"], new["tok_stream"], new["tok_pos"], stream, pages)
     n = new["q_pos"].shape[0]
     mode = MODE_PREFILL if prefill else MODE_DECODE
     if b.get("workspace") is None and msa_workspace_bytes(shape, n, mode) > 0:

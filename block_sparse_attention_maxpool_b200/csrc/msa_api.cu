@@ -289,6 +289,32 @@ int append_rows(const msa_shape* sh, void* cache0, const void* src0, void* cache
   return cuda_status(cudaGetLastError());
 }
 
+// The appends of one step (F32 indexer keys, K, V) in one launch.
+int step_append(const msa_shape* sh, float* idx_k_cache, msa_bf16* k_cache, msa_bf16* v_cache,
+                const float* idx_k_new, const msa_bf16* k_new, const msa_bf16* v_new, const int32_t* tok_stream,
+                const int32_t* tok_pos, int32_t n_tok, void* stream, const msa_pages* pages) {
+  int st = check_shape(sh);
+  if (st != MSA_OK) return st;
+  if (n_tok < 0) return MSA_ERR_RANGE;
+  if (n_tok == 0) return MSA_OK;
+  if (!idx_k_cache || !k_cache || !v_cache || !idx_k_new || !k_new || !v_new || !tok_stream || !tok_pos)
+    return MSA_ERR_NULL;
+  if (!aligned16(idx_k_cache) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(idx_k_new) ||
+      !aligned16(k_new) || !aligned16(v_new))
+    return MSA_ERR_ALIGN;
+  msa::KvPages pg;
+  int64_t rows = 0;
+  if ((st = pages_of(sh, pages, &pg, &rows)) != MSA_OK) return st;
+  const int64_t warps = static_cast<int64_t>(n_tok) * sh->n_kv_heads;
+  if (warps * 32 >= (int64_t{1} << 31)) return MSA_ERR_RANGE;
+  const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
+  launch(msa::append_step_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), idx_k_cache,
+         idx_k_new, reinterpret_cast<uint8_t*>(k_cache), reinterpret_cast<const uint8_t*>(k_new),
+         reinterpret_cast<uint8_t*>(v_cache), reinterpret_cast<const uint8_t*>(v_new), tok_stream, tok_pos, n_tok,
+         sh->n_streams, sh->n_kv_heads, sh->capacity, pg);
+  return cuda_status(cudaGetLastError());
+}
+
 template <typename KeyT>
 int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* idx_k_cache,
                       const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float* block_scores,
@@ -369,8 +395,8 @@ int block_scores_impl(const msa_shape* shape, const float* idx_q, const KeyT* id
     Q.khi = reinterpret_cast<__half*>(ws + L.khi);
     Q.klo = reinterpret_cast<__half*>(ws + L.klo);
     Q.qlo_nz = reinterpret_cast<int*>(ws + L.qlo_nz);
-    Q.klo_nz = reinterpret_cast<int*>(ws + L.klo_nz);
-    Q.n_flags = G * L.n_tiles + S * G * Q.nblk;
+    Q.klo_mask = reinterpret_cast<uint32_t*>(ws + L.klo_mask);
+    Q.n_flags = G * L.n_tiles + S * G * Q.n_chunks;
     Q.pages = pg;
     const int64_t key_rows = static_cast<int64_t>(S) * G * cap;
     const int64_t q_rows = static_cast<int64_t>(G) * L.n_q_pad;
@@ -463,6 +489,21 @@ int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v_cache, 
   if (n_tok > 0 && (!v_cache || !v_new)) return MSA_ERR_NULL;
   return append_rows(shape, k_cache, k_new, v_cache, v_new, tok_stream, tok_pos, n_tok,
                      128 * static_cast<int>(sizeof(msa_bf16)), stream, nullptr);
+}
+
+int msa_step_append(const msa_shape* shape, float* idx_k_cache, msa_bf16* k_cache, msa_bf16* v_cache,
+                    const float* idx_k_new, const msa_bf16* k_new, const msa_bf16* v_new, const int32_t* tok_stream,
+                    const int32_t* tok_pos, int32_t n_tok, void* stream) {
+  return step_append(shape, idx_k_cache, k_cache, v_cache, idx_k_new, k_new, v_new, tok_stream, tok_pos, n_tok,
+                     stream, nullptr);
+}
+
+int msa_step_append_paged(const msa_shape* shape, const msa_pages* pages, float* idx_k_pool, msa_bf16* k_pool,
+                          msa_bf16* v_pool, const float* idx_k_new, const msa_bf16* k_new, const msa_bf16* v_new,
+                          const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  return step_append(shape, idx_k_pool, k_pool, v_pool, idx_k_new, k_new, v_new, tok_stream, tok_pos, n_tok, stream,
+                     pages);
 }
 
 int msa_block_scores(const msa_shape* shape, const float* idx_q, const float* idx_k_cache,

@@ -60,6 +60,43 @@ __global__ void __launch_bounds__(256) append_rows_kernel(
              warp, threadIdx.x & 31);
 }
 
+// All of a step's appends in one launch: one warp per (token, group) writes
+// the F32 indexer key (512 B, one 16-byte vector per lane), then the K row
+// (lanes 0-15) and the V row (lanes 16-31), 256 B each, at the slot the
+// separate appends use, with the same checks and error bits.
+__global__ void __launch_bounds__(256) append_step_kernel(
+    float* __restrict__ idx_cache, const float* __restrict__ idx_src, uint8_t* __restrict__ k_cache,
+    const uint8_t* __restrict__ k_src, uint8_t* __restrict__ v_cache, const uint8_t* __restrict__ v_src,
+    const int32_t* __restrict__ tok_stream, const int32_t* __restrict__ tok_pos, int n_tok, int n_streams,
+    int n_groups, int capacity, const KvPages pages) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_tok * n_groups) return;
+  const int t = warp / n_groups;
+  const int g = warp - t * n_groups;
+  const int s = tok_stream[t];
+  const int p = tok_pos[t];
+  if (s < 0 || s >= n_streams || p < 0 || p >= capacity) {
+    if (g == 0 && lane == 0) raise_error(MSA_DEVERR_TOKEN_RANGE);
+    return;
+  }
+  const long long blk = kv_block_row(pages, s, g, p / 128, n_groups, capacity);
+  if (blk < 0) {
+    if (lane == 0) raise_error(MSA_DEVERR_PAGE_RANGE);
+    return;
+  }
+  const size_t dst_row = static_cast<size_t>(blk) + (p & 127);
+  const size_t src_row = static_cast<size_t>(t) * n_groups + g;
+  reinterpret_cast<int4*>(idx_cache + dst_row * 128)[lane] =
+      __ldg(reinterpret_cast<const int4*>(idx_src + src_row * 128) + lane);
+  const int h = lane & 15;
+  uint8_t* cache = lane < 16 ? k_cache : v_cache;
+  const uint8_t* src = lane < 16 ? k_src : v_src;
+  reinterpret_cast<int4*>(cache + dst_row * 256)[h] = __ldg(reinterpret_cast<const int4*>(src + src_row * 256) + h);
+}
+
 // F16 indexer-key cache variant: each F32 key of 128 values is rounded to
 // fp16 (nearest even) as it is written.  One warp per (token, group) row,
 // four values per lane.

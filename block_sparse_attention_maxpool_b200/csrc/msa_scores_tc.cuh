@@ -68,7 +68,7 @@ static_assert(2 * kSlots + 7 <= 32, "barrier slots");
 
 // Workspace carve-up of the prefill block-score path (byte offsets).
 struct Workspace {
-  size_t counters, tile_stream, tile_nb, leftover, qscale, qhi, qlo, kscale, khi, klo, qlo_nz, klo_nz, total;
+  size_t counters, tile_stream, tile_nb, leftover, qscale, qhi, qlo, kscale, khi, klo, qlo_nz, klo_mask, total;
   int n_tiles, n_q_pad;
 };
 
@@ -90,7 +90,7 @@ __host__ inline Workspace workspace_layout(int n_q, int G, int S, int cap) {
   w.khi = o;         o = align256(o + sizeof(__half) * static_cast<size_t>(S) * G * cap * kDi);
   w.klo = o;         o = align256(o + sizeof(__half) * static_cast<size_t>(S) * G * cap * kDi);
   w.qlo_nz = o;      o = align256(o + sizeof(int) * static_cast<size_t>(G) * w.n_tiles);
-  w.klo_nz = o;      o = align256(o + sizeof(int) * static_cast<size_t>(S) * G * (cap / kBlock));
+  w.klo_mask = o;    o = align256(o + sizeof(uint32_t) * static_cast<size_t>(S) * G * ((cap / kBlock + kChunk - 1) / kChunk));
   w.total = o;
   return w;
 }
@@ -114,8 +114,8 @@ struct Params {
   __half* khi;              // [S][G][cap][Di]
   __half* klo;
   int* qlo_nz;              // [G][n_tiles]       some query row of the tile has a nonzero lo part
-  int* klo_nz;              // [S][G][cap / 128]  some key row of the block has a nonzero lo part
-  int n_flags;              // entries of qlo_nz and klo_nz together (zeroed by tc_init_kernel)
+  uint32_t* klo_mask;       // [S][G][n_chunks]   bit b % 32: some key row of block b has a nonzero lo part
+  int n_flags;              // entries of qlo_nz and klo_mask together (zeroed by tc_init_kernel)
   KvPages pages;            // block table of a paged key cache (table null: contiguous)
 };
 
@@ -149,17 +149,17 @@ __global__ void tc_init_kernel(int* counters, int n, const Params P) {
   const int nq = P.G * P.n_tiles;
   for (int i = threadIdx.x; i < P.n_flags; i += blockDim.x) {
     if (i < nq) P.qlo_nz[i] = 0;
-    else P.klo_nz[i - nq] = 0;
+    else P.klo_mask[i - nq] = 0u;
   }
 }
 
-// Flags the 128-row tile of a split row whose lo part is not all zero: the
-// products with that tile's lo half are then needed (an all-zero lo half
-// adds exactly zero, so its products are skipped).
-__device__ __forceinline__ void flag_lo(const __half2 (&lo)[2], int* flag) {
+// Sets `bit` of *flags when this warp's split row has a lo part that is not
+// all zero: the products with that 128-row tile's lo half are then needed
+// (an all-zero lo half adds exactly zero, so its products are skipped).
+__device__ __forceinline__ void flag_lo(const __half2 (&lo)[2], uint32_t* flags, uint32_t bit) {
   const uint32_t a = *reinterpret_cast<const uint32_t*>(&lo[0]) | *reinterpret_cast<const uint32_t*>(&lo[1]);
-  if (__any_sync(0xffffffffu, (a & 0x7fff7fffu) != 0u) && (threadIdx.x & 31) == 0 && *flag == 0)
-    atomicOr(flag, 1);
+  if (__any_sync(0xffffffffu, (a & 0x7fff7fffu) != 0u) && (threadIdx.x & 31) == 0 && (*flags & bit) == 0u)
+    atomicOr(flags, bit);
 }
 
 // One warp per tile of 128 consecutive queries.  The tile's stream is the
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(256) tc_split_queries_kernel(const Params P) {
   *reinterpret_cast<uint2*>(P.qlo + row * kDi + lane * 4) =
       make_uint2(*reinterpret_cast<uint32_t*>(&lo[0]), *reinterpret_cast<uint32_t*>(&lo[1]));
   if (lane == 0) P.qscale[row] = pow2f(-e);
-  flag_lo(lo, &P.qlo_nz[g * P.n_tiles + q / kTileQ]);
+  flag_lo(lo, reinterpret_cast<uint32_t*>(&P.qlo_nz[g * P.n_tiles + q / kTileQ]), 1u);
   if (!real) return;
   const int nvis = ok ? p / kBlock + 1 : 0;
   float* out = P.bs + (static_cast<size_t>(q) * P.G + g) * P.nblk;
@@ -315,7 +315,10 @@ __global__ void __launch_bounds__(256) tc_split_keys_kernel(const Params P) {
   *reinterpret_cast<uint2*>(P.klo + w * kDi + lane * 4) =
       make_uint2(*reinterpret_cast<uint32_t*>(&lo[0]), *reinterpret_cast<uint32_t*>(&lo[1]));
   if (lane == 0) P.kscale[w] = pow2f(-e);
-  flag_lo(lo, &P.klo_nz[w / kBlock]);
+  {
+    const int blk = j / kBlock;
+    flag_lo(lo, &P.klo_mask[sg * P.n_chunks + blk / kChunk], 1u << (blk % kChunk));
+  }
 }
 
 // Task t -> (group, key chunk, query tile); consecutive tasks share a key
@@ -388,9 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         task_range(P, tile, chunk, b0, b1);
         if (b0 >= b1) continue;
         const int s = P.tile_stream[tile];
+        // the task's lo flags, loaded before the wait so their latency hides behind it
+        const bool q_lo = __ldcg(&P.qlo_nz[g * P.n_tiles + tile]) != 0;
+        const uint32_t kmask = __ldcg(P.klo_mask + (static_cast<size_t>(s) * P.G + g) * P.n_chunks + chunk);
         if (a_use > 0 && !mbar_wait(a_empty, (a_use - 1) & 1)) { *abort_v = 1; break; }
         const int qrow = g * P.n_q_pad + tile * kTileQ;
-        const bool q_lo = __ldcg(&P.qlo_nz[g * P.n_tiles + tile]) != 0;
         mbar_arrive_expect_tx(a_full, q_lo ? kOperandBytes : kOperandBytes / 2);
         tma_load_2d(smem + SmemLayout::kA, &tm_qhi, 0, qrow, a_full);
         tma_load_2d(smem + SmemLayout::kA + kHalfBytes, &tm_qhi, 64, qrow, a_full);
@@ -400,11 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++a_use;
         const size_t krow0 = (static_cast<size_t>(s) * P.G + g) * P.capacity;
-        const int* klo_nz = P.klo_nz + (static_cast<size_t>(s) * P.G + g) * P.nblk;
         bool stop = false;
         for (int b = b0; b < b1 && !stop; ++b) {
           const int krow = static_cast<int>(krow0) + b * kBlock;
-          const bool k_lo = __ldcg(klo_nz + b) != 0;
+          const bool k_lo = ((kmask >> (b - b0)) & 1u) != 0u;
           // the hi half of the key block, then (when nonzero) its lo half, one slot each
           for (int h = 0; h < (k_lo ? 2 : 1); ++h, ++slot) {
             const int st = slot % kSlots;
@@ -433,13 +437,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         task_coords(P, t, g, chunk, tile);
         task_range(P, tile, chunk, b0, b1);
         if (b0 >= b1) continue;
-        if (!mbar_wait(a_full, a_use & 1)) { *abort_v = 1; break; }
-        tc_fence_after();
         const int s = P.tile_stream[tile];
         const bool q_lo = __ldcg(&P.qlo_nz[g * P.n_tiles + tile]) != 0;
-        const int* klo_nz = P.klo_nz + (static_cast<size_t>(s) * P.G + g) * P.nblk;
+        const uint32_t kmask = __ldcg(P.klo_mask + (static_cast<size_t>(s) * P.G + g) * P.n_chunks + chunk);
+        if (!mbar_wait(a_full, a_use & 1)) { *abort_v = 1; break; }
+        tc_fence_after();
         for (int b = b0; b < b1; ++b, ++acc) {
-          const bool k_lo = __ldcg(klo_nz + b) != 0;
+          const bool k_lo = ((kmask >> (b - b0)) & 1u) != 0u;
           const int st_hi = slot % kSlots;
           const int st_lo = (slot + 1) % kSlots;
           const int buf = acc & 1;

@@ -117,6 +117,17 @@ MSA_API int msa_kv_append(const msa_shape* shape, msa_bf16* k_cache, msa_bf16* v
                   const msa_bf16* k_new, const msa_bf16* v_new, const int32_t* tok_stream,
                   const int32_t* tok_pos, int32_t n_tok, void* stream);
 
+/* msa_step_append - msa_indexer_append and msa_kv_append in one launch: each
+ * new token's F32 indexer key and its K and V rows are written at the same
+ * slots, with the same arguments, layouts, checks and error bits as the two
+ * calls (the indexer keeps its own key cache beside K/V: MSA pull request,
+ * "Implementation").  One kernel instead of two per step, which matters
+ * when a step is launch-bound (a decode batch of a few streams).  All six
+ * cache and row pointers are required and 16-byte aligned. */
+MSA_API int msa_step_append(const msa_shape* shape, float* idx_k_cache, msa_bf16* k_cache, msa_bf16* v_cache,
+                            const float* idx_k_new, const msa_bf16* k_new, const msa_bf16* v_new,
+                            const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream);
+
 /* msa_block_scores - fused indexer score, causal mask, max-pool and local
  * bias: block_scores[i][g][b] = max over slots j of block b with j <= q_pos[i]
  * of idx_q[i][g] . idx_k_cache[q_stream[i]][g][j], accumulated in float32
@@ -277,6 +288,10 @@ MSA_API int msa_indexer_append_f16_paged(const msa_shape* shape, const msa_pages
 MSA_API int msa_kv_append_paged(const msa_shape* shape, const msa_pages* pages, msa_bf16* k_pool,
                                 msa_bf16* v_pool, const msa_bf16* k_new, const msa_bf16* v_new,
                                 const int32_t* tok_stream, const int32_t* tok_pos, int32_t n_tok, void* stream);
+MSA_API int msa_step_append_paged(const msa_shape* shape, const msa_pages* pages, float* idx_k_pool,
+                                  msa_bf16* k_pool, msa_bf16* v_pool, const float* idx_k_new,
+                                  const msa_bf16* k_new, const msa_bf16* v_new, const int32_t* tok_stream,
+                                  const int32_t* tok_pos, int32_t n_tok, void* stream);
 MSA_API int msa_block_scores_paged(const msa_shape* shape, const msa_pages* pages, const float* idx_q,
                                    const float* idx_k_pool, const int32_t* q_stream, const int32_t* q_pos,
                                    int32_t n_q, float* block_scores, void* workspace, size_t workspace_bytes,

@@ -231,3 +231,24 @@ def test_wait_selftest_validation(lib):
     assert lib.msa_wait_selftest(1000, None, 16, None) == -1
     assert lib.msa_wait_selftest(1000, fake, 8, None) == -5               # too small
     assert lib.msa_wait_selftest(1000, fake + 4, 16, None) == -2          # not 16-byte aligned
+
+
+def test_step_append_validation(lib):
+    """msa_step_append (indexer keys + K/V in one launch): null, alignment,
+    count and shape errors before any device work."""
+    s = msa.Shape(n_streams=1, capacity=256).c()
+    fake = 0x10000
+    args = [fake] * 6 + [fake, fake]
+    assert lib.msa_step_append(ctypes.byref(s), *args, 0, None) == 0            # nothing to append
+    assert lib.msa_step_append(ctypes.byref(s), *args, -1, None) == -4
+    for i in range(8):
+        bad = list(args)
+        bad[i] = None
+        assert lib.msa_step_append(ctypes.byref(s), *bad, 3, None) == -1, i
+    for i in range(6):
+        bad = list(args)
+        bad[i] = fake + 8
+        assert lib.msa_step_append(ctypes.byref(s), *bad, 3, None) == -2, i
+    bad_shape = msa.Shape(n_streams=1, capacity=200).c()
+    assert lib.msa_step_append(ctypes.byref(bad_shape), *args, 3, None) == -3
+    assert lib.msa_step_append_paged(ctypes.byref(s), None, *args, 3, None) == -1
