@@ -61,6 +61,32 @@ def test_append_bit_exact_and_range_errors():
     assert torch.equal(di, before)
 
 
+def test_step_append_matches_the_separate_appends_and_flags_bad_tokens():
+    """msa_step_append (indexer keys + K/V in one launch) writes what
+    msa_indexer_append and msa_kv_append write, bit for bit, skips a token
+    outside the cache and sets the same error bit."""
+    g = torch.Generator().manual_seed(12)
+    sh = msa.Shape(n_streams=3, capacity=384, n_kv_heads=2, n_q_heads=32)
+    idx = torch.randn((3, 2, 384, 128), generator=g)
+    k = torch.randn((3, 2, 384, 128), generator=g).to(torch.bfloat16)
+    v = torch.randn((3, 2, 384, 128), generator=g).to(torch.bfloat16)
+    n = 60
+    ts = torch.randint(0, 3, (n,), generator=g, dtype=torch.int32)
+    tp = torch.randperm(384, generator=g)[:n].to(torch.int32)
+    ts[7], tp[9] = 3, 384                       # no such stream; past the capacity
+    new_i = torch.randn((n, 2, 128), generator=g)
+    new_k = torch.randn((n, 2, 128), generator=g).to(torch.bfloat16)
+    new_v = torch.randn((n, 2, 128), generator=g).to(torch.bfloat16)
+    di, dk, dv = idx.cuda(), k.cuda(), v.cuda()
+    msa.msa_step_append(sh, di, dk, dv, new_i.cuda(), new_k.cuda(), new_v.cuda(), ts.cuda(), tp.cuda())
+    assert msa.msa_get_device_error() == 0x2
+    ok = torch.ones(n, dtype=torch.bool)
+    ok[7] = ok[9] = False
+    assert torch.equal(di.cpu(), oracle.indexer_append(idx, new_i[ok], ts[ok], tp[ok]))
+    assert torch.equal(dk.cpu(), oracle.indexer_append(k, new_k[ok], ts[ok], tp[ok]))
+    assert torch.equal(dv.cpu(), oracle.indexer_append(v, new_v[ok], ts[ok], tp[ok]))
+
+
 def _rand_scores(g, n_q, G, nblk, q_pos, ties):
     bs = torch.randn((n_q, G, nblk), generator=g)
     if ties:
