@@ -774,6 +774,42 @@ int msa_dsa_select_topk(const msa_dsa_shape* shape, const float* scores, const i
   if (!scores || !q_pos || !sel) return MSA_ERR_NULL;
   if (!aligned16(scores) || !aligned16(sel)) return MSA_ERR_ALIGN;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int sms = 0;
+  if ((st = current_device_sms(&sms)) != MSA_OK) return st;
+  // fewer queries than SMs: a cluster of four CTAs per query, each staging a
+  // quarter of the row, so a small batch of long rows uses four times the SMs
+  if (n_q < sms && shape->capacity <= msa::dsa::kClusterKeys &&
+      static_cast<int64_t>(n_q) * msa::dsa::kClusterCtas < (int64_t{1} << 31)) {
+    const auto ck = msa::dsa::dsa_select_topk_cluster_kernel;
+    static std::atomic<uint64_t> csmem_done{0};
+    static std::atomic<int> cluster_ok{-1};           // can a cluster of this size be scheduled
+    if ((st = ensure_smem(ck, msa::dsa::kClusterSmemBytes, csmem_done)) != MSA_OK) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_q * msa::dsa::kClusterCtas));
+    cfg.blockDim = dim3(msa::dsa::kSelThreads);
+    cfg.dynamicSmemBytes = msa::dsa::kClusterSmemBytes;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = msa::dsa::kClusterCtas;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cluster_ok.load() < 0) {
+      int clusters = 0;
+      cluster_ok.store(cudaOccupancyMaxActiveClusters(&clusters, ck, &cfg) == cudaSuccess && clusters > 0 ? 1 : 0);
+      (void)cudaGetLastError();
+    }
+    if (cluster_ok.load() == 1) {
+      if (cudaLaunchKernelEx(&cfg, ck, scores, q_pos, n_q, shape->capacity, shape->top_k, sel, n_sel) !=
+          cudaSuccess)
+        return MSA_ERR_CUDA;
+      return cuda_status(cudaGetLastError());
+    }
+  }
   if (shape->capacity <= msa::dsa::kSmemKeys) {
     static std::atomic<uint64_t> smem_done{0};
     if ((st = ensure_smem(msa::dsa::dsa_select_topk_kernel<true>, msa::dsa::kSelSmemStaged, smem_done)) != MSA_OK)

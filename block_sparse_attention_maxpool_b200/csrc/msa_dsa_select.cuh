@@ -23,7 +23,16 @@
 // The radix select is most-significant-digit first, 8 bits per pass, with
 // shared-memory atomic histograms; the filter and emit passes take four
 // keys per lane per step and place them with warp scans.
+//
+// A batch with fewer queries than SMs (a decode step) would leave most SMs
+// idle with one CTA per query, so it runs on clusters of four CTAs per query
+// instead (dsa_select_topk_cluster_kernel, rows up to 192K tokens): the
+// quarters of a row are staged by the four CTAs, and the radix select and
+// the emit offsets are combined through distributed shared memory.
 #pragma once
+
+#include <cooperative_groups.h>
+#include <cstddef>
 
 #include "msa_common.cuh"
 
@@ -50,6 +59,9 @@ struct SelSmem {
   uint32_t cands[kMaxCands];
   uint32_t keys[kSmemKeys];    // last: the unstaged kernel is launched without it
 };
+static_assert(offsetof(SelSmem, keys) % 16 == 0 && offsetof(SelSmem, cands) % 16 == 0 &&
+                  offsetof(SelSmem, samples) % 16 == 0,
+              "key vectors must be 16-byte aligned");
 constexpr size_t kSelSmemStaged = sizeof(SelSmem);
 constexpr size_t kSelSmemUnstaged = sizeof(SelSmem) - sizeof(uint32_t) * kSmemKeys;
 static_assert(kSelSmemStaged <= 232448, "shared memory budget");
@@ -217,22 +229,27 @@ __device__ bool sample_kth(SelSmem& sm, Get get, int n, int k, uint32_t* T, int*
   return true;
 }
 
-// Write, in index order, every token with key > T and the first need_eq
-// tokens with key == T (k tokens in all).  Each warp owns a contiguous range
-// and walks it 128 keys at a time, four consecutive keys per lane: a count
-// pass, one block-wide exchange of the warps' counts, then an emit pass
-// whose positions come from one warp scan per 128 keys.
+// Per-warp key counts of the emit pass: warp w owns the contiguous range
+// [w0, w1) of the n keys (whole spans of 128) and counts its keys above T
+// and equal to T into warp_gt[w] / warp_eq[w].  Called by the whole CTA;
+// ends with a barrier.
+constexpr int kEmitSpan = 4 * 32;
+
+__device__ __forceinline__ void warp_range(int n, int warp, int& w0, int& w1) {
+  const int per_warp = (n + kSelWarps * kEmitSpan - 1) / (kSelWarps * kEmitSpan) * kEmitSpan;
+  w0 = min(n, warp * per_warp);
+  w1 = min(n, w0 + per_warp);
+}
+
 template <typename Get>
-__device__ void emit_topk(SelSmem& sm, Get get, int n, uint32_t T, int need_eq, int32_t* out) {
-  constexpr int kSpan = 4 * 32;
+__device__ void count_gt_eq(Get get, int n, uint32_t T, int* warp_gt, int* warp_eq) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int per_warp = (n + kSelWarps * kSpan - 1) / (kSelWarps * kSpan) * kSpan;
-  const int w0 = min(n, warp * per_warp);
-  const int w1 = min(n, w0 + per_warp);
+  int w0, w1;
+  warp_range(n, warp, w0, w1);
   int gt = 0, eq = 0;
-  for (int b0 = w0; b0 < w1; b0 += kSpan) {
+  for (int b0 = w0; b0 < w1; b0 += kEmitSpan) {
     const int i0 = b0 + 4 * lane;
     const uint4 kv = i0 < w1 ? get.get4(i0) : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t key[4] = {kv.x, kv.y, kv.z, kv.w};
@@ -248,16 +265,31 @@ __device__ void emit_topk(SelSmem& sm, Get get, int n, uint32_t T, int need_eq, 
     eq += __shfl_xor_sync(0xffffffffu, eq, o);
   }
   if (lane == 0) {
-    sm.warp_gt[warp] = gt;
-    sm.warp_eq[warp] = eq;
+    warp_gt[warp] = gt;
+    warp_eq[warp] = eq;
   }
   __syncthreads();
-  int gt_before = 0, eq_before = 0;
+}
+
+// Write, in index order, every token with key > T and the first need_eq
+// tokens with key == T.  Key i is token tok0 + i; gt0 / eq0 keys above /
+// equal to T come before key 0 (other CTAs' ranges).  Each warp walks its
+// range 128 keys at a time, four consecutive keys per lane, placing them
+// with one warp scan per 128 keys after the counts of count_gt_eq.
+template <typename Get>
+__device__ void emit_counted(Get get, int n, uint32_t T, int need_eq, int32_t* out, const int* warp_gt,
+                             const int* warp_eq, int tok0, int gt0, int eq0) {
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  int w0, w1;
+  warp_range(n, warp, w0, w1);
+  int gt_before = gt0, eq_before = eq0;
   for (int w = 0; w < warp; ++w) {
-    gt_before += sm.warp_gt[w];
-    eq_before += sm.warp_eq[w];
+    gt_before += warp_gt[w];
+    eq_before += warp_eq[w];
   }
-  for (int b0 = w0; b0 < w1; b0 += kSpan) {
+  for (int b0 = w0; b0 < w1; b0 += kEmitSpan) {
     bool is_gt[4], is_eq[4];
     int packed = 0;                                   // gt count | eq count << 16
     const int i0 = b0 + 4 * lane;
@@ -281,7 +313,7 @@ __device__ void emit_topk(SelSmem& sm, Get get, int n, uint32_t T, int need_eq, 
     int e = eq_before + (excl >> 16);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int i = b0 + 4 * lane + j;
+      const int i = tok0 + b0 + 4 * lane + j;
       if (is_gt[j]) {
         out[g + min(e, need_eq)] = i;
         ++g;
@@ -294,6 +326,13 @@ __device__ void emit_topk(SelSmem& sm, Get get, int n, uint32_t T, int need_eq, 
     gt_before += tot & 0xffff;
     eq_before += tot >> 16;
   }
+}
+
+// The emit pass of one CTA over all n keys.
+template <typename Get>
+__device__ void emit_topk(SelSmem& sm, Get get, int n, uint32_t T, int need_eq, int32_t* out) {
+  count_gt_eq(get, n, T, sm.warp_gt, sm.warp_eq);
+  emit_counted(get, n, T, need_eq, out, sm.warp_gt, sm.warp_eq, 0, 0, 0);
 }
 
 template <bool kStaged>
@@ -340,6 +379,172 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   }
   for (int i = top_k + tid; i < kMaxTopK; i += kSelThreads) out[i] = -1;
   if (tid == 0 && n_sel != nullptr) n_sel[t] = top_k;
+}
+
+// ---- the same selection on a cluster of CTAs per query ----------------------
+// One query's keys split into kClusterCtas contiguous quarters, one per CTA
+// of a thread-block cluster (so a small batch of long rows uses four times
+// the SMs).  Each CTA stages its quarter in shared memory.  The radix select
+// of the k-th key runs over the whole row: per 8-bit digit, every CTA
+// counts its own keys into a local histogram and adds it into rank 0's
+// histogram through distributed shared memory; after a cluster barrier rank
+// 0 picks the digit (as radix_kth does) and clears its histogram; after a
+// second barrier every CTA reads the decided prefix.  The emit pass then
+// counts each CTA's keys above and equal to T, exchanges the four totals
+// through rank 0, and each CTA writes its quarter's tokens at their global
+// places: the output is the same ascending list as the one-CTA kernels'.
+constexpr int kClusterCtas = 4;
+constexpr int kClusterKeys = kClusterCtas * kSmemKeys;   // longest row the cluster path stages
+
+struct ClusterSmem {
+  unsigned int hist[256];          // this CTA's digit histogram
+  unsigned int chist[256];         // rank 0: the cluster's histogram
+  int warp_gt[kSelWarps];
+  int warp_eq[kSelWarps];
+  uint32_t prefix;                 // rank 0: the decided key prefix
+  int need;                        // rank 0: how many keys of that prefix are still needed
+  int cta_gt[kClusterCtas];        // rank 0: each CTA's keys above T
+  int cta_eq[kClusterCtas];        // rank 0: each CTA's keys equal to T
+  alignas(16) uint32_t keys[kSmemKeys];   // read four at a time (16-byte vectors)
+};
+constexpr size_t kClusterSmemBytes = sizeof(ClusterSmem);
+static_assert(kClusterSmemBytes <= 232448, "shared memory budget");
+static_assert(offsetof(ClusterSmem, keys) % 16 == 0, "key vectors must be 16-byte aligned");
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+    dsa_select_topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int n_q,
+                                   int capacity, int top_k, int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  ClusterSmem& sm = *reinterpret_cast<ClusterSmem*>(smem_raw);
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int t = blockIdx.x / kClusterCtas;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  pdl_trigger();
+  pdl_wait();
+  // every branch below that returns before the cluster barriers is taken by
+  // the whole cluster (it depends on the query only)
+  if (t >= n_q) return;
+  const int p = q_pos[t];
+  int32_t* out = sel + static_cast<size_t>(t) * kMaxTopK;
+  if (p < 0 || p >= capacity) {
+    if (rank == 0) {
+      for (int i = tid; i < kMaxTopK; i += kSelThreads) out[i] = -1;
+      if (tid == 0) {
+        if (n_sel != nullptr) n_sel[t] = 0;
+        raise_error(MSA_DEVERR_QUERY_RANGE);
+      }
+    }
+    return;
+  }
+  const int n = p + 1;
+  if (n <= top_k) {                                   // every visible token is kept
+    if (rank == 0) {
+      for (int i = tid; i < kMaxTopK; i += kSelThreads) out[i] = i < n ? i : -1;
+      if (tid == 0 && n_sel != nullptr) n_sel[t] = n;
+    }
+    return;
+  }
+  const int lo = static_cast<int>(static_cast<long long>(n) * rank / kClusterCtas);
+  const int hi = static_cast<int>(static_cast<long long>(n) * (rank + 1) / kClusterCtas);
+  const int m = hi - lo;
+  const float* row = scores + static_cast<size_t>(t) * capacity + lo;
+#pragma unroll 8
+  for (int i = tid; i < m; i += kSelThreads) sm.keys[i] = score_key(__ldg(row + i));
+  for (int i = m + tid; i < ((m + 3) & ~3); i += kSelThreads) sm.keys[i] = 0u;   // whole vectors for get4
+  if (rank == 0) {
+    for (int b = tid; b < 256; b += kSelThreads) sm.chist[b] = 0;
+    if (tid == 0) {
+      sm.prefix = 0;
+      sm.need = top_k;
+    }
+  }
+  cluster.sync();                                     // keys staged; rank 0's histogram and decision ready
+  unsigned int* chist0 = cluster.map_shared_rank(sm.chist, 0);
+  uint32_t prefix = 0, mask = 0;
+  int need = top_k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 256; b += kSelThreads) sm.hist[b] = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += kSelThreads) {
+      const uint32_t key = sm.keys[i];
+      if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    for (int b = tid; b < 256; b += kSelThreads) {
+      const unsigned int c = sm.hist[b];
+      if (c != 0u) atomicAdd(chist0 + b, c);
+    }
+    cluster.sync();                                   // every CTA's counts are in rank 0's histogram
+    if (rank == 0) {
+      if (warp == 0) {
+        // lane l holds bins 255-8l .. 248-8l (descending); find the bin where
+        // the count from the top reaches `need`
+        const int need0 = sm.need;
+        unsigned int c[8];
+        unsigned int local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c[j] = sm.chist[255 - 8 * lane - j];
+          local += c[j];
+        }
+        unsigned int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const unsigned int excl = incl - local;
+        if (excl < static_cast<unsigned int>(need0) && incl >= static_cast<unsigned int>(need0)) {
+          unsigned int cum = excl;
+          int bin = 255 - 8 * lane;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (cum + c[j] >= static_cast<unsigned int>(need0)) {
+              bin = 255 - 8 * lane - j;
+              break;
+            }
+            cum += c[j];
+          }
+          sm.prefix = sm.prefix | (static_cast<uint32_t>(bin) << shift);
+          sm.need = need0 - static_cast<int>(cum);
+        }
+      }
+      __syncthreads();                                // the decision is made: clear for the next digit
+      for (int b = tid; b < 256; b += kSelThreads) sm.chist[b] = 0;
+    }
+    cluster.sync();                                   // the decided prefix is visible to every CTA
+    prefix = *cluster.map_shared_rank(&sm.prefix, 0);
+    need = *cluster.map_shared_rank(&sm.need, 0);
+    mask |= 255u << shift;
+  }
+  const uint32_t T = prefix;
+  const SmemKeys get{sm.keys};
+  count_gt_eq(get, m, T, sm.warp_gt, sm.warp_eq);
+  if (tid == 0) {
+    int gt = 0, eq = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      gt += sm.warp_gt[w];
+      eq += sm.warp_eq[w];
+    }
+    *cluster.map_shared_rank(&sm.cta_gt[rank], 0) = gt;
+    *cluster.map_shared_rank(&sm.cta_eq[rank], 0) = eq;
+  }
+  cluster.sync();                                     // every CTA's totals are at rank 0
+  int gt0 = 0, eq0 = 0;
+  for (int r = 0; r < rank; ++r) {
+    gt0 += *cluster.map_shared_rank(&sm.cta_gt[r], 0);
+    eq0 += *cluster.map_shared_rank(&sm.cta_eq[r], 0);
+  }
+  emit_counted(get, m, T, need, out, sm.warp_gt, sm.warp_eq, lo, gt0, eq0);
+  if (rank == 0) {
+    for (int i = top_k + tid; i < kMaxTopK; i += kSelThreads) out[i] = -1;
+    if (tid == 0 && n_sel != nullptr) n_sel[t] = top_k;
+  }
+  cluster.sync();                                     // no CTA leaves while another reads its shared memory
 }
 
 }  // namespace dsa
