@@ -71,3 +71,22 @@ def test_quantised_indexer_keys_make_ties():
     inp = W.make_inputs(w, seed=2)
     vals = inp.idx_k_cache[:, :, :w.l_existing].flatten()
     assert vals.unique().numel() < vals.numel() // 100
+
+
+def test_step_sets_redraw_the_new_token_and_query_only():
+    """The benchmark's second decode input set: same layouts and
+    distributions as the workload's own new token and query, different
+    values, deterministic, and the same per stream whatever streams are
+    drawn."""
+    w = W.Workload("small_decode", 5, 299, 300, "last", n_q_heads=32, n_kv_heads=2)
+    inp = W.make_inputs(w, seed=0)
+    a, b = W.make_step_set(w, seed=1001), W.make_step_set(w, seed=1001)
+    for name in ("idx_k_new", "k_new", "v_new", "idx_q", "q"):
+        got, base = a[name], getattr(inp, name)
+        assert got.shape == base.shape and got.dtype == base.dtype, name
+        assert torch.equal(got, b[name]), name
+        assert not torch.equal(got, base), name
+    part = W.make_step_set(w, seed=1001, streams=range(2, 4))
+    assert torch.equal(part["q"], a["q"][2:4]) and torch.equal(part["idx_k_new"], a["idx_k_new"][2:4])
+    with pytest.raises(ValueError):
+        W.make_step_set(_small("new"), seed=1)
