@@ -62,7 +62,7 @@ NOMINAL_HBM_GBS = 7700.0       # B200 HBM3e, HGX figure (context beside the meas
 # in proportion to the keys scanned).  Each figure is valid only for the
 # kernel source it was taken on (sha256 prefix of msa_scores_gemv.cuh); any
 # other source reports null.
-SCORES_TRAFFIC = {"f32": {"source_sha": "0c7e835ccd50eea6", "bytes_per_launch": 4 * (536_926_720 + 3_099_392)},
+SCORES_TRAFFIC = {"f32": {"source_sha": "fbcb00edc6a2593a", "bytes_per_launch": 4 * (536_912_896 + 3_008_000)},
                   "f16": {"source_sha": "b9bc1ca3c5d4d5a4", "bytes_per_launch": 4 * (268_474_112 + 2_967_040)}}
 
 # The same for the token-score kernel of the token-level variant, from a
@@ -339,7 +339,8 @@ class Step:
             self.launches = 1 + 2                # K/V append, attention + combine
         else:
             appends = 2 if args.idx_f16 else 1
-            self.launches = appends + (6 if tiles else 1) + 1 + 2
+            # decode: selection inside the attention kernel (+ combine); prefill: top-k, plan, attention
+            self.launches = appends + (6 if tiles else 1) + (3 if self.prefill else 2)
         self.parts = self._parts()
 
     def switch(self, variant: str):
@@ -406,6 +407,13 @@ class Step:
             def fused(st, i):
                 msa.decode_step_fused(sh, self.caches, self.sets[i], b, st)
             return [fused]
+        if not self.prefill and self.variant == "full":
+            def select_attend(st, i):               # the top-16 inside the attention kernel
+                d = self.sets[i]
+                msa.msa_select_attn_decode(sh, b["block_scores"], d["q"], d["k_cache"], d["v_cache"],
+                                           d["q_stream"], d["q_pos"], self.scale, b["sel"], b["n_sel"], b["out"],
+                                           b["workspace"], st, pages)
+            return [append, scores, select_attend]
         if self.variant == "shared":
             def kv_append(st, i):
                 d = self.sets[i]

@@ -19,7 +19,8 @@ import torch
 
 __all__ = ["MsaError", "Shape", "msa_indexer_append", "msa_kv_append", "msa_step_append", "msa_block_scores",
            "msa_indexer_append_f16",
-           "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
+           "msa_select_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill", "msa_select_attn_decode",
+           "msa_select_attn_decode_paged",
            "msa_workspace_bytes", "msa_get_device_error", "msa_sparse_attn_decode_noalloc", "msa_version", "library", "LIB_PATH",
            "MODE_DECODE", "MODE_PREFILL", "LOCAL_BIAS", "decode_step",
            "Pages", "msa_indexer_append_paged", "msa_indexer_append_f16_paged", "msa_kv_append_paged",
@@ -130,6 +131,8 @@ _SIGS = {
                                               ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "msa_sparse_attn_prefill": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
                                                ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_select_attn_decode": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _I,
+                                              ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "msa_sparse_attn_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P,
                                                       _I, ctypes.c_float, _P, _P]),
     "msa_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(CShape), _I, _I]),
@@ -152,6 +155,8 @@ _SIGS.update({
                                                     ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
     "msa_sparse_attn_prefill_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
                                                      ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "msa_select_attn_decode_paged": (ctypes.c_int, [ctypes.POINTER(CShape), _PG, _P, _P, _P, _P, _P, _P, _I,
+                                                    ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "msa_dsa_indexer_append": (ctypes.c_int, [_DS, _PG, _P, _P, _P, _P, _I, _P]),
     "msa_dsa_token_scores": (ctypes.c_int, [_DS, _PG, _P, _P, _P, _P, _P, _I, _P, _P]),
     "msa_dsa_select_topk": (ctypes.c_int, [_DS, _P, _P, _I, _P, _P, _P]),
@@ -363,6 +368,40 @@ def msa_sparse_attn_prefill(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_
                  q_pos, softmax_scale, out, workspace, stream, pages)
 
 
+def msa_select_attn_decode(shape: Shape, block_scores, q, k_cache, v_cache, q_stream, q_pos, softmax_scale=None,
+                           sel=None, n_sel=None, out=None, workspace=None, stream=None, pages=None):
+    """Top-16 selection and decode attention in one call (msa_select_attn_decode,
+    or its _paged form with ``pages``).  Returns (out, sel, n_sel)."""
+    n = _n(q_pos, "q_pos")
+    dev = q.device
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(shape.head_dim)
+    if sel is None:
+        sel = torch.empty((n, shape.n_kv_heads, shape.top_k), dtype=torch.int32, device=dev)
+    if n_sel is None:
+        n_sel = torch.empty((n, shape.n_kv_heads), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((n, shape.n_q_heads, shape.head_dim), dtype=torch.bfloat16, device=dev)
+    ws_ptr, ws_bytes, _keep = _workspace(shape, n, MODE_DECODE, workspace, dev)
+    cs = _cache_shape(shape, pages, shape.head_dim)
+    _call("msa_select_attn_decode", shape, pages,
+          _ptr(block_scores, torch.float32, (n, shape.n_kv_heads, shape.n_blocks), "block_scores"),
+          _ptr(q, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "q"),
+          _ptr(k_cache, torch.bfloat16, cs, "k_cache"), _ptr(v_cache, torch.bfloat16, cs, "v_cache"),
+          _ptr(q_stream, torch.int32, (n,), "q_stream"), _ptr(q_pos, torch.int32, (n,), "q_pos"), n,
+          float(softmax_scale), _ptr(sel, torch.int32, (n, shape.n_kv_heads, shape.top_k), "sel"),
+          _ptr(n_sel, torch.int32, (n, shape.n_kv_heads), "n_sel"),
+          _ptr(out, torch.bfloat16, (n, shape.n_q_heads, shape.head_dim), "out"), ws_ptr, ws_bytes,
+          _stream(stream))
+    return out, sel, n_sel
+
+
+def msa_select_attn_decode_paged(shape: Shape, pages: Pages, block_scores, q, k_pool, v_pool, q_stream, q_pos,
+                                 softmax_scale=None, sel=None, n_sel=None, out=None, workspace=None, stream=None):
+    return msa_select_attn_decode(shape, block_scores, q, k_pool, v_pool, q_stream, q_pos, softmax_scale, sel,
+                                  n_sel, out, workspace, stream, pages)
+
+
 # ---- paged caches: the C ABI's *_paged calls --------------------------------
 def msa_indexer_append_paged(shape: Shape, pages: Pages, idx_k_pool, idx_k_new, tok_stream, tok_pos,
                              stream=None):
@@ -483,10 +522,14 @@ def decode_step(shape: Shape, caches: dict, new: dict, bufs: dict | None = None,
                                           device=new["q"].device))
     bs = msa_block_scores(shape, new["idx_q"], caches["idx_k_cache"], new["q_stream"], new["q_pos"],
                           b.get("block_scores"), stream, b.get("workspace"), pages)
+    if not prefill:                         # the top-16 inside the attention kernel
+        out, sel, n_sel = msa_select_attn_decode(shape, bs, new["q"], caches["k_cache"], caches["v_cache"],
+                                                 new["q_stream"], new["q_pos"], None, b.get("sel"), b.get("n_sel"),
+                                                 b.get("out"), b.get("workspace"), stream, pages)
+        return out, sel, n_sel, bs
     sel, n_sel = msa_select_topk(shape, bs, new["q_pos"], b.get("sel"), b.get("n_sel"), stream)
-    attn = msa_sparse_attn_prefill if prefill else msa_sparse_attn_decode
-    out = attn(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
-               new["q_pos"], None, b.get("out"), b.get("workspace"), stream, pages)
+    out = msa_sparse_attn_prefill(shape, new["q"], caches["k_cache"], caches["v_cache"], sel, new["q_stream"],
+                                  new["q_pos"], None, b.get("out"), b.get("workspace"), stream, pages)
     return out, sel, n_sel, bs
 
 

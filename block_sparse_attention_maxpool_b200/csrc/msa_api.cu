@@ -170,10 +170,25 @@ size_t attn_workspace(const msa_shape* sh, int32_t n_q, int mode) {
   return static_cast<size_t>(ctas) * 2 * msa::dattn::kPartial * sizeof(float);
 }
 
+// Most pairs one CTA's share of the decode units touches.
+int64_t max_pairs_per_cta(int64_t units, int n_cta) {
+  int64_t most = 0;
+  for (int c = 0; c < n_cta; ++c) {
+    const int64_t u0 = msa::dattn::unit_begin(units, n_cta, c), u1 = msa::dattn::unit_begin(units, n_cta, c + 1);
+    if (u1 > u0) most = std::max(most, (u1 - 1) / msa::dattn::kTopK - u0 / msa::dattn::kTopK + 1);
+  }
+  return most;
+}
+
+// Decode and prefill attention over a selection.  Decode with block_scores
+// set: the top-16 is taken inside the attention kernel (or, when a CTA's
+// share would touch more than kSelPairs pairs, by the selection kernel
+// first) and written to sel_out / n_sel_out; `sel` is then sel_out.
 int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache, const msa_bf16* v_cache,
                 const int32_t* sel, const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
                 float softmax_scale, msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream,
-                int mode, const msa_pages* pages, const int32_t* tok_sel = nullptr) {
+                int mode, const msa_pages* pages, const int32_t* tok_sel = nullptr,
+                const float* block_scores = nullptr, int32_t* sel_out = nullptr, int32_t* n_sel_out = nullptr) {
   int st = check_shape(sh);
   if (st != MSA_OK) return st;
   if (n_q < 0) return MSA_ERR_RANGE;
@@ -236,10 +251,26 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   }
   // decode: persistent stream-K grid over (pair, selected block) units, or
   // (pair, chunk of 128 kept tokens) units for the token-level variant
-  const auto kernel = tok_sel != nullptr ? msa::dattn::sparse_attn_decode_sk_kernel<true>
-                                         : msa::dattn::sparse_attn_decode_sk_kernel<false>;
-  static std::atomic<uint64_t> smem_done[2] = {0, 0};
-  if ((st = ensure_smem(kernel, msa::dattn::Layout::kBytes, smem_done[tok_sel != nullptr])) != MSA_OK) return st;
+  if (n_pairs * msa::dattn::kHpg >= (int64_t{1} << 31)) return MSA_ERR_RANGE;   // Q rows: TMA coordinates
+  CUtensorMap tm_q;
+  if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, n_pairs * msa::dattn::kHpg,
+                           msa::dattn::kHpg)) != MSA_OK)
+    return st;
+  const int64_t n_units = n_pairs * msa::dattn::kTopK;
+  const int n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), n_units,
+                                                        static_cast<int64_t>(msa::dattn::kMaxCtas)}));
+  bool fuse_sel = false;
+  if (block_scores != nullptr) {
+    fuse_sel = max_pairs_per_cta(n_units, n_cta) <= msa::dattn::kSelPairs;
+    if (!fuse_sel && (st = msa_select_topk(sh, block_scores, q_pos, n_q, sel_out, n_sel_out, stream)) != MSA_OK)
+      return st;
+  }
+  const int variant = tok_sel != nullptr ? 1 : (fuse_sel ? 2 : 0);
+  const auto kernel = variant == 1 ? msa::dattn::sparse_attn_decode_sk_kernel<true, false>
+                                   : (variant == 2 ? msa::dattn::sparse_attn_decode_sk_kernel<false, true>
+                                                   : msa::dattn::sparse_attn_decode_sk_kernel<false, false>);
+  static std::atomic<uint64_t> smem_done[3] = {0, 0, 0};
+  if ((st = ensure_smem(kernel, msa::dattn::Layout::kBytes, smem_done[variant])) != MSA_OK) return st;
   msa::dattn::Params P;
   P.q = reinterpret_cast<const __nv_bfloat16*>(q);
   P.sel = sel;
@@ -251,15 +282,19 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   P.G = G;
   P.n_streams = sh->n_streams;
   P.capacity = sh->capacity;
-  P.n_units = n_pairs * msa::dattn::kTopK;
-  P.n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), P.n_units,
-                                                static_cast<int64_t>(msa::dattn::kMaxCtas)}));
+  P.n_units = n_units;
+  P.n_cta = n_cta;
   P.scale_log2 = softmax_scale * 1.4426950408889634f;
   P.pages = pg;
   P.tok_sel = tok_sel;
   P.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
   P.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
-  launch(kernel, dim3(static_cast<unsigned>(P.n_cta)), dim3(msa::dattn::kThreads), msa::dattn::Layout::kBytes, s, tm_k, tm_v, P);
+  P.bs = fuse_sel ? block_scores : nullptr;
+  P.nblk = sh->capacity / msa::dattn::kBlock;
+  P.sel_out = fuse_sel ? sel_out : nullptr;
+  P.n_sel_out = fuse_sel ? n_sel_out : nullptr;
+  launch(kernel, dim3(static_cast<unsigned>(P.n_cta)), dim3(msa::dattn::kThreads), msa::dattn::Layout::kBytes, s,
+         tm_k, tm_v, tm_q, P);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
   const int64_t warps = n_pairs * msa::dattn::kHpg;
   launch(msa::dattn::attn_sk_combine_kernel, dim3(static_cast<unsigned>((warps * 32 + 255) / 256)), dim3(256), 0, s, P);
@@ -553,6 +588,16 @@ int msa_select_topk(const msa_shape* shape, const float* block_scores, const int
   return cuda_status(cudaGetLastError());
 }
 
+int msa_select_attn_decode(const msa_shape* shape, const float* block_scores, const msa_bf16* q,
+                           const msa_bf16* k_cache, const msa_bf16* v_cache, const int32_t* q_stream,
+                           const int32_t* q_pos, int32_t n_q, float softmax_scale, int32_t* sel, int32_t* n_sel,
+                           msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_q > 0 && (block_scores == nullptr || sel == nullptr)) return MSA_ERR_NULL;
+  if (n_q > 0 && !aligned16(block_scores)) return MSA_ERR_ALIGN;
+  return sparse_attn(shape, q, k_cache, v_cache, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_DECODE, nullptr, nullptr, block_scores, sel, n_sel);
+}
+
 int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
                            const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
@@ -702,6 +747,18 @@ int msa_sparse_attn_decode_paged(const msa_shape* shape, const msa_pages* pages,
   if (pages == nullptr) return MSA_ERR_NULL;
   return sparse_attn(shape, q, k_pool, v_pool, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
                      workspace_bytes, stream, MSA_MODE_DECODE, pages);
+}
+
+int msa_select_attn_decode_paged(const msa_shape* shape, const msa_pages* pages, const float* block_scores,
+                                 const msa_bf16* q, const msa_bf16* k_pool, const msa_bf16* v_pool,
+                                 const int32_t* q_stream, const int32_t* q_pos, int32_t n_q, float softmax_scale,
+                                 int32_t* sel, int32_t* n_sel, msa_bf16* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (pages == nullptr) return MSA_ERR_NULL;
+  if (n_q > 0 && (block_scores == nullptr || sel == nullptr)) return MSA_ERR_NULL;
+  if (n_q > 0 && !aligned16(block_scores)) return MSA_ERR_ALIGN;
+  return sparse_attn(shape, q, k_pool, v_pool, sel, q_stream, q_pos, n_q, softmax_scale, out, workspace,
+                     workspace_bytes, stream, MSA_MODE_DECODE, pages, nullptr, block_scores, sel, n_sel);
 }
 
 int msa_sparse_attn_prefill_paged(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
@@ -881,9 +938,12 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
     return MSA_ERR_CUDA;
   const int grid = sms;                                      // one resident CTA per SM, as the separate kernels use
   const int64_t rows = static_cast<int64_t>(shape->n_streams) * G * shape->capacity;
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_k, tm_v, tm_q;
   if ((st = make_kv_map(&tm_k, k_cache, rows)) != MSA_OK) return st;
   if ((st = make_kv_map(&tm_v, v_cache, rows)) != MSA_OK) return st;
+  if ((st = make_map_16bit(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, n_pairs * msa::dattn::kHpg,
+                           msa::dattn::kHpg)) != MSA_OK)
+    return st;
 
   msa::fused::Params F;
   F.idx_k_cache = idx_k_cache;
@@ -931,6 +991,10 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   A.tok_sel = nullptr;
   A.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
   A.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
+  A.bs = nullptr;
+  A.nblk = S.nblk;
+  A.sel_out = nullptr;
+  A.n_sel_out = nullptr;
   unsigned int* bar = reinterpret_cast<unsigned int*>(
       static_cast<uint8_t*>(workspace) + msa::tc::align256(attn_workspace(shape, n_q, MSA_MODE_DECODE)));
   F.bar_count = bar;
@@ -948,7 +1012,7 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, F) != cudaSuccess) return MSA_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, tm_q, F) != cudaSuccess) return MSA_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 

@@ -9,15 +9,27 @@
 // V (1 MB).  The work units are (pair, selected block); every CTA of a
 // persistent grid (at most one per SM) takes one contiguous, equal share of
 // the units, so all SMs stream K/V for the whole kernel with no wave tail.
-// One producer thread TMA-loads each unit's K and V tiles (four 16 KB boxes,
-// 128-byte swizzle) into a two-stage ring; eight consumer warps each own 16
-// key rows of the block and compute S = Q K^T (16 heads x 16 rows) and
+// One producer thread resolves each unit (query position, selected block,
+// cache row), writes what the consumers need into a small per-stage record
+// and TMA-loads the unit's K and V tiles (four 16 KB boxes, 128-byte
+// swizzle) into a two-stage ring, plus the pair's Q (16 heads x 128 dims)
+// when the unit is the first of its pair in this CTA; the consumers so make
+// no global-memory round trip between units.  Eight consumer warps each own
+// 16 key rows of the block and compute S = Q K^T (16 heads x 16 rows) and
 // O += P V with bf16 m16n8k16 MMAs, fp32 accumulation and a streaming base-2
 // softmax.  Consecutive units of one pair accumulate in registers; when the
 // pair changes the eight warps merge through shared memory.  A pair whose
 // units all lie in one CTA's share is written out directly; a pair cut by a
 // share boundary leaves one partial (max, sum, unnormalised O) per CTA,
 // merged by attn_sk_combine_kernel.
+//
+// Fused selection (Params::bs set): before the ring starts, the CTA's
+// consumer warps rank the block scores of the (at most kSelPairs) pairs its
+// units touch, one warp per pair with the top-16 routine of the selection
+// kernel, keys staged in the stage ring (idle until the first load); the
+// producer then reads the selection from shared memory, and the CTA holding
+// a pair's first unit writes that pair's selection and count for the caller.
+// The result is the selection kernel's, bit for bit, without its launch.
 //
 // Token-level variant ("deepseek2 : GLM-DSA sparse attention (lightning
 // indexer)": top-k tokens per query, the same set for every group): a unit
@@ -27,11 +39,13 @@
 // straight into the same 128-byte-swizzled tile layout the TMA path
 // produces, each lane arriving on the stage's barrier when its copies land;
 // rows of padding or of an unmapped page are copied from a zero row and
-// masked.  Random 256-byte rows bound this path near 2 TB/s on B200 (a TMA
-// tile::gather4 form measured slower).
+// masked through a 128-bit row mask in the stage record.  Random 256-byte
+// rows bound this path near 2 TB/s on B200 (a TMA tile::gather4 form
+// measured slower).
 #pragma once
 
 #include "msa_common.cuh"
+#include "msa_select.cuh"
 
 namespace msa {
 namespace dattn {
@@ -46,19 +60,40 @@ constexpr int kThreads = (kWarps + kGatherWarps) * 32;   // block path: one prod
 constexpr int kRowsPerWarp = kBlock / kWarps;       // 16
 constexpr uint32_t kTileBytes = kBlock * 64 * 2;    // [128 rows][64 dims] bf16 = 16 KB
 constexpr uint32_t kStageBytes = 4 * kTileBytes;    // K lo, K hi, V lo, V hi
+constexpr uint32_t kQBytes = kHpg * kD * 2;         // Q of one pair: two [16 heads][64 dims] boxes, 4 KB
 constexpr int kStages = 2;
 constexpr int kOStride = kD + 4;                    // padded fp32 row of the merge buffer
 constexpr int kMaxCtas = 256;                       // grid cap (bounds the workspace)
 constexpr int kPartial = kHpg * (kD + 2);           // floats of one partial: O[16][128], m[16], l[16]
+constexpr int kSelPairs = 8;                        // fused selection: pairs one CTA may touch
+
+// What the producer tells the consumers about the unit in a stage.
+struct UnitInfo {
+  int32_t flags;      // kUnitData: K/V rows landed; kUnitQ: the pair's Q landed
+  int32_t p;          // query position
+  int32_t slot0;      // first slot of the block in its stream (block path)
+  int32_t pad;
+  uint32_t mask[4];   // token path: bit r set = row r of the unit is attended
+};
+constexpr int32_t kUnitData = 1;
+constexpr int32_t kUnitQ = 2;
 
 struct Layout {
   static constexpr uint32_t kStageOff = 0;
-  static constexpr uint32_t kMergeOff = kStages * kStageBytes;
+  static constexpr uint32_t kQOff = kStages * kStageBytes;
+  static constexpr uint32_t kMergeOff = kQOff + kStages * kQBytes;
   static constexpr uint32_t kMlOff = kMergeOff + kWarps * kHpg * kOStride * 4;
-  static constexpr uint32_t kBarOff = kMlOff + kWarps * kHpg * 2 * 4;
+  static constexpr uint32_t kInfoOff = kMlOff + kWarps * kHpg * 2 * 4;
+  static constexpr uint32_t kSelOff = kInfoOff + kStages * sizeof(UnitInfo);
+  static constexpr uint32_t kBarOff = kSelOff + kSelPairs * (kTopK + 1) * 4 + 16;
   static constexpr uint32_t kEnd = kBarOff + 64;
   static constexpr size_t kBytes = kEnd + 1024;
 };
+static_assert(Layout::kQOff % 1024 == 0 && kQBytes % 1024 == 0, "128-byte-swizzled TMA boxes start on 1 KB");
+static_assert(Layout::kBarOff % 8 == 0 && Layout::kInfoOff % 16 == 0, "barrier and record alignment");
+static_assert(kWarps * sel::KeySmem<32>::kBytesPerWarp <= Layout::kQOff - Layout::kStageOff,
+              "fused selection: every consumer warp's keys fit the stage ring");
+static_assert(Layout::kBytes <= 227 * 1024, "shared memory of one CTA");
 
 struct Params {
   const __nv_bfloat16* q;     // [n_q][Hq][D]
@@ -74,6 +109,10 @@ struct Params {
   const int32_t* tok_sel;     // token-level variant: [n_q][16 * 128] ascending token ids (else null)
   const __nv_bfloat16* k_cache;   // token-level variant: the K and V caches (or pools) the gathers read
   const __nv_bfloat16* v_cache;
+  const float* bs;            // fused selection: block scores [n_q][G][nblk] (else null)
+  int nblk;
+  int32_t* sel_out;           // fused selection: the selection and its counts, written for the caller
+  int32_t* n_sel_out;         // (nullable)
 };
 
 // 256 zero bytes: the source of the K and V rows of masked token slots.
@@ -128,7 +167,10 @@ __device__ inline int cta_of(long long U, int C, long long u) {
 // Cache row of unit u's block, or -1 when the unit has nothing to attend
 // (padding, an invalid selection, an invalid query or a block with no valid
 // page).  p: query position; slot0: first slot of the block in its stream.
-__device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, int& slot0, bool report) {
+// sel_s: the CTA's fused selection (rows of pairs pf, pf + 1, ...), else null
+// and the selection is read from P.sel.
+__device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, int& slot0, bool report,
+                                        const int32_t* sel_s, long long pf) {
   const long long pair = u / kTopK;
   const int j = static_cast<int>(u - pair * kTopK);
   const int qi = static_cast<int>(pair / P.G);
@@ -139,7 +181,13 @@ __device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, in
     if (report && j == 0 && g == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
     return -1;
   }
-  const int b = __ldcg(P.sel + pair * kTopK + j);   // L2 only: may come from other CTAs of this grid
+  int b;
+  if (sel_s != nullptr) {
+    if (pair - pf >= kSelPairs) return -1;            // the host never launches such a share
+    b = sel_s[(pair - pf) * kTopK + j];
+  } else {
+    b = __ldcg(P.sel + pair * kTopK + j);             // L2 only: the selection may come from the previous kernel
+  }
   if (b < 0) return -1;
   if (b > p / kBlock) {
     if (report) raise_error(MSA_DEVERR_SEL_RANGE);
@@ -223,14 +271,46 @@ __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long 
   }
 }
 
+// The top-16 of the pairs this CTA's units touch (fused selection), into
+// sel_s: consumer warp w ranks pairs pf + w, pf + w + kWarps, ... with its
+// keys in its slice of the stage ring; the CTA holding a pair's first unit
+// writes the pair's selection and count to the caller's buffers.
+__device__ __forceinline__ void select_share(const Params& P, uint8_t* smem, int32_t* sel_s, long long u0,
+                                             long long u1, int warp, int lane) {
+  const long long pf = u0 / kTopK;
+  const int np = u1 > u0 ? static_cast<int>((u1 - 1) / kTopK - pf + 1) : 0;
+  int32_t* cnt_s = sel_s + kSelPairs * kTopK;
+  uint64_t* wsm = reinterpret_cast<uint64_t*>(smem + Layout::kStageOff) +
+                  warp * (sel::KeySmem<32>::kBytesPerWarp / sizeof(uint64_t));
+  for (int i = warp; i < np && i < kSelPairs; i += kWarps) {
+    const long long pair = pf + i;
+    int32_t* row = sel_s + i * kTopK;
+    sel::select_pair_any(P.bs, P.q_pos, P.G, P.nblk, P.capacity, row, cnt_s + i, static_cast<int>(pair), lane,
+                         wsm);
+    __syncwarp();
+    if (pair * kTopK >= u0) {
+      if (lane < kTopK) P.sel_out[pair * kTopK + lane] = row[lane];
+      if (lane == 0 && P.n_sel_out != nullptr) P.n_sel_out[pair] = cnt_s[i];
+    }
+    __syncwarp();
+  }
+  // the keys were stored to the stage ring, which TMA writes next
+  fence_proxy_async_smem();
+}
+
 // The kernel body for CTA `cta` of the P.n_cta sharing the units.  tm_k, tm_v:
-// tensor maps of the K and V caches (block path); smem: Layout::kBytes,
-// 1024-byte aligned; the CTA has kThreads threads.
-template <bool kTok>
+// tensor maps of the K and V caches (block path); tm_q: of Q, [n_q * Hq][128]
+// with [16][64] boxes; smem: Layout::kBytes, 1024-byte aligned; the CTA has
+// kThreads threads.  kSel: rank the block scores first (P.bs).
+template <bool kTok, bool kSel>
 __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                                           const Params& P, uint8_t* smem, int cta) {
+                                                           const CUtensorMap* tm_q, const Params& P, uint8_t* smem,
+                                                           int cta) {
+  static_assert(!(kTok && kSel), "the token-level variant takes its selection from the caller");
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Layout::kBarOff);
   uint64_t* empty = full + kStages;
+  UnitInfo* info = reinterpret_cast<UnitInfo*>(smem + Layout::kInfoOff);
+  int32_t* sel_s = reinterpret_cast<int32_t*>(smem + Layout::kSelOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -240,10 +320,15 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(&full[st], kTok ? 32 * kGatherWarps : 1);   // token gathers: one arrival per producer lane
+      // token gathers: one arrival per producer lane (its copies landed) and
+      // one per producer warp (its record written); TMA: the producer's one
+      mbar_init(&full[st], kTok ? (32 + 1) * kGatherWarps : 1);
       mbar_init(&empty[st], kWarps);
     }
     mbar_fence_init();
+  }
+  if constexpr (kSel) {
+    if (warp < kWarps) select_share(P, smem, sel_s, u0, u1, warp, lane);
   }
   __syncthreads();
 
@@ -251,37 +336,64 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
     // ----------------------- producer: token gathers (whole warp) -----------------------
     const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(P.k_cache);
     const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(P.v_cache);
+    const int pw = warp - kWarps;
     int k = 0;
     bool ok = true;
-    for (long long u = u0; u < u1 && ok; ++u) {
-      int s, g, p;
-      const int32_t* toks;
-      if (!tok_unit(P, u, s, g, p, toks, false)) continue;
+    for (long long u = u0; u < u1; ++u, ++k) {
       const int st = k % kStages;
       const int use = k / kStages;
       if (use > 0) ok = mbar_wait(&empty[st], (use - 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
+      int s = 0, g = 0, p = 0;
+      const int32_t* toks = nullptr;
+      const bool any = tok_unit(P, u, s, g, p, toks, pw == 0 && lane == 0);
+      const bool qstart = u == u0 || u % kTopK == 0;
       const uint32_t dst = smem_addr(smem + Layout::kStageOff + st * kStageBytes);
-      // one row per lane (two producer warps: 64 rows each), all 16 chunks of
-      // K and V; measured faster than spreading a row over 16 lanes
+      uint32_t m[2] = {0u, 0u};
+      if (any) {
+        // one row per lane (two producer warps: 64 rows each), all 16 chunks
+        // of K and V; measured faster than spreading a row over 16 lanes
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = (warp - kWarps) * 64 + lane + 32 * i;
-        const int tok = __ldg(toks + r);
-        const long long row = tok_row(P, s, g, p, tok);
-        if (row < 0 && tok >= 0) raise_error(tok > p ? MSA_DEVERR_SEL_RANGE : MSA_DEVERR_PAGE_RANGE);
-        const uint8_t* ksrc = row < 0 ? g_zero_row : reinterpret_cast<const uint8_t*>(kc + row * kD);
-        const uint8_t* vsrc = row < 0 ? g_zero_row : reinterpret_cast<const uint8_t*>(vc + row * kD);
+        for (int i = 0; i < 2; ++i) {
+          const int r = pw * 64 + lane + 32 * i;
+          const int tok = __ldg(toks + r);
+          const long long row = tok_row(P, s, g, p, tok);
+          if (row < 0 && tok >= 0) raise_error(tok > p ? MSA_DEVERR_SEL_RANGE : MSA_DEVERR_PAGE_RANGE);
+          m[i] = __ballot_sync(0xffffffffu, row >= 0);
+          const uint8_t* ksrc = row < 0 ? g_zero_row : reinterpret_cast<const uint8_t*>(kc + row * kD);
+          const uint8_t* vsrc = row < 0 ? g_zero_row : reinterpret_cast<const uint8_t*>(vc + row * kD);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t off = (c >> 3) * kTileBytes + swz128(r, c & 7);
-          cp_async16(dst + off, ksrc + 16 * c);
-          cp_async16(dst + 2 * kTileBytes + off, vsrc + 16 * c);
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t off = (c >> 3) * kTileBytes + swz128(r, c & 7);
+            cp_async16(dst + off, ksrc + 16 * c);
+            cp_async16(dst + 2 * kTileBytes + off, vsrc + 16 * c);
+          }
+        }
+      }
+      if (lane == 0) {
+        UnitInfo& in = info[st];
+        in.mask[2 * pw] = m[0];
+        in.mask[2 * pw + 1] = m[1];
+        if (pw == 0) {
+          in.flags = (any ? kUnitData : 0) | (qstart ? kUnitQ : 0);
+          in.p = p;
+          in.slot0 = 0;
+          if (qstart) {
+            // the record's arrival also announces the pair's Q
+            const int qrow = static_cast<int>(u / kTopK) * kHpg;
+            uint8_t* qdst = smem + Layout::kQOff + st * kQBytes;
+            mbar_arrive_expect_tx(&full[st], kQBytes);
+            tma_load_2d(qdst, tm_q, 0, qrow, &full[st]);
+            tma_load_2d(qdst + kQBytes / 2, tm_q, 64, qrow, &full[st]);
+          } else {
+            mbar_arrive(&full[st]);
+          }
+        } else {
+          mbar_arrive(&full[st]);
         }
       }
       cp_async_arrive(&full[st]);
-      ++k;
     }
     // no copy may still be landing when the CTA exits
     for (int j = max(0, k - kStages); j < k; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
@@ -290,23 +402,35 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
   if (!kTok && warp >= kWarps) {
     // -------------------------------- producer --------------------------------
     if (warp != kWarps || lane != 0) return;
+    const long long pf = u0 / kTopK;
     int k = 0;
     bool ok = true;
-    for (long long u = u0; u < u1 && ok; ++u) {
-      int p, slot0;
-      const int row = unit_row(P, u, p, slot0, false);
-      if (row < 0) continue;
+    for (long long u = u0; u < u1; ++u, ++k) {
       const int st = k % kStages;
       const int use = k / kStages;
       if (use > 0) ok = mbar_wait(&empty[st], (use - 1) & 1);
       if (!ok) break;
-      uint8_t* dst = smem + Layout::kStageOff + st * kStageBytes;
-      mbar_arrive_expect_tx(&full[st], kStageBytes);
-      tma_load_2d(dst, tm_k, 0, row, &full[st]);
-      tma_load_2d(dst + kTileBytes, tm_k, 64, row, &full[st]);
-      tma_load_2d(dst + 2 * kTileBytes, tm_v, 0, row, &full[st]);
-      tma_load_2d(dst + 3 * kTileBytes, tm_v, 64, row, &full[st]);
-      ++k;
+      int p = 0, slot0 = 0;
+      const int row = unit_row(P, u, p, slot0, true, kSel ? sel_s : nullptr, pf);
+      const bool qstart = u == u0 || u % kTopK == 0;
+      UnitInfo& in = info[st];
+      in.flags = (row >= 0 ? kUnitData : 0) | (qstart ? kUnitQ : 0);
+      in.p = p;
+      in.slot0 = slot0;
+      mbar_arrive_expect_tx(&full[st], (row >= 0 ? kStageBytes : 0u) + (qstart ? kQBytes : 0u));
+      if (qstart) {
+        const int qrow = static_cast<int>(u / kTopK) * kHpg;
+        uint8_t* qdst = smem + Layout::kQOff + st * kQBytes;
+        tma_load_2d(qdst, tm_q, 0, qrow, &full[st]);
+        tma_load_2d(qdst + kQBytes / 2, tm_q, 64, qrow, &full[st]);
+      }
+      if (row >= 0) {
+        uint8_t* dst = smem + Layout::kStageOff + st * kStageBytes;
+        tma_load_2d(dst, tm_k, 0, row, &full[st]);
+        tma_load_2d(dst + kTileBytes, tm_k, 64, row, &full[st]);
+        tma_load_2d(dst + 2 * kTileBytes, tm_v, 0, row, &full[st]);
+        tma_load_2d(dst + 3 * kTileBytes, tm_v, 64, row, &full[st]);
+      }
     }
     // no copy may still be landing when the CTA exits
     for (int j = max(0, k - kStages); j < k; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1);
@@ -314,7 +438,6 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
   }
 
   // -------------------------------- consumers --------------------------------
-  const int gr = lane >> 2;   // fragment row group
   const int tq = lane & 3;    // thread in quad
   const int wr = warp * kRowsPerWarp;
   uint32_t qa[8][4];
@@ -323,7 +446,10 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
   long long cur = -1;
   int k = 0;
   bool ok = true;
-  for (long long u = u0; u < u1; ++u) {
+  for (long long u = u0; u < u1; ++u, ++k) {
+    const int st = k % kStages;
+    if (ok) ok = mbar_wait(&full[st], (k / kStages) & 1);
+    ok = __all_sync(0xffffffffu, ok);     // warp-uniform: the MMAs below take the whole warp
     const long long pair = u / kTopK;
     if (pair != cur) {
       if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane);
@@ -332,29 +458,21 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
       for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
       m_run[0] = m_run[1] = -INFINITY;
       l_run[0] = l_run[1] = 0.f;
-      // Q of the pair's 16 heads as the A operand, straight from global memory
-      const __nv_bfloat16* qb = P.q + static_cast<size_t>(pair) * kHpg * kD;
-      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qb + gr * kD);
-      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qb + (gr + 8) * kD);
+      // Q of the pair's 16 heads as the A operand, from the Q boxes that
+      // landed with this unit
+      const uint32_t qbase = smem_addr(smem + Layout::kQOff + st * kQBytes);
+      const int mi = lane >> 3;
+      const int qr = (mi & 1) * 8 + (lane & 7);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const int c = ks * 8 + tq;   // 32-bit word of dims 16ks + 2tq
-        qa[ks][0] = __ldg(r0 + c);
-        qa[ks][1] = __ldg(r1 + c);
-        qa[ks][2] = __ldg(r0 + c + 4);
-        qa[ks][3] = __ldg(r1 + c + 4);
+        const int kc = ks * 2 + (mi >> 1);    // 16-byte chunk of dims 8kc .. 8kc + 7
+        ldmatrix_x4(qa[ks], qbase + (kc >> 3) * (kQBytes / 2) + swz128(qr, kc & 7));
       }
     }
-    int p, slot0 = 0, s = 0, g = 0;
-    const int32_t* toks = nullptr;
-    if constexpr (kTok) {
-      if (!tok_unit(P, u, s, g, p, toks, warp == 0 && lane == 0)) continue;
-    } else {
-      if (unit_row(P, u, p, slot0, warp == 0 && lane == 0) < 0) continue;
-    }
-    const int st = k % kStages;
-    if (ok) ok = mbar_wait(&full[st], (k / kStages) & 1);
-    if (ok) {
+    const int flags = info[st].flags;
+    if (ok && (flags & kUnitData)) {
+      const int p = info[st].p;
+      const int slot0 = info[st].slot0;
       const uint32_t kbase = smem_addr(smem + Layout::kStageOff + st * kStageBytes);
       const uint32_t vbase = kbase + 2 * kTileBytes;
       // S = Q K^T: two n-tiles of 8 key rows
@@ -371,19 +489,21 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
         mma_bf16_16816(sacc[0], qa[ks], b[0], b[1]);
         mma_bf16_16816(sacc[1], qa[ks], b[2], b[3]);
       }
-      // causal mask inside the block, base-2 scaling, online softmax
-      const int jb = slot0 + wr;    // slot (in the stream) of this warp's first key
+      // causal mask inside the block (token path: the unit's row mask),
+      // base-2 scaling, online softmax
+      uint32_t rmask = 0u;
+      if constexpr (kTok) rmask = info[st].mask[warp >> 1] >> ((warp & 1) * 16);   // this warp's 16 rows
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int j = jb + nt * 8 + tq * 2 + (e & 1);
+          const int rr = nt * 8 + tq * 2 + (e & 1);    // row within this warp's 16
           bool valid;
           if constexpr (kTok) {
-            valid = tok_row(P, s, g, p, __ldg(toks + (j - slot0))) >= 0;   // j - slot0: row in the unit
+            valid = (rmask >> rr) & 1u;
           } else {
-            valid = j <= p;
+            valid = slot0 + wr + rr <= p;
           }
           const float x = valid ? sacc[nt][e] * P.scale_log2 : -INFINITY;
           sacc[nt][e] = x;
@@ -443,20 +563,19 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
-    ++k;
   }
   if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane);
 }
 
-template <bool kTok>
+template <bool kTok, bool kSel>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                                 const Params P) {
+                                 const __grid_constant__ CUtensorMap tm_q, const Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   pdl_trigger();
   pdl_wait();
-  sparse_attn_decode_sk_body<kTok>(&tm_k, &tm_v, P, smem, blockIdx.x);
+  sparse_attn_decode_sk_body<kTok, kSel>(&tm_k, &tm_v, &tm_q, P, smem, blockIdx.x);
 }
 
 // Pairs cut by a share boundary: merge the partials of every CTA whose share

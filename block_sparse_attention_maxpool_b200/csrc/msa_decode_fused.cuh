@@ -131,7 +131,7 @@ __device__ __forceinline__ bool grid_barrier(const Params& F, unsigned int n_cta
 
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                             const Params F) {
+                             const __grid_constant__ CUtensorMap tm_q, const Params F) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ int barrier_flag;
@@ -166,12 +166,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_pairs = F.scores.n_q * G;
   uint64_t* wsm = reinterpret_cast<uint64_t*>(smem + warp * sel::select_smem_per_warp(F.scores.nblk));
   for (long long w = gwarp; w < n_pairs; w += n_gwarps)
-    sel::select_pair_any(F.scores.bs, F.scores.q_pos, G, F.scores.nblk, F.scores.capacity, F.sel, F.n_sel,
+    sel::select_pair_any(F.scores.bs, F.scores.q_pos, G, F.scores.nblk, F.scores.capacity,
+                         F.sel + static_cast<size_t>(w) * sel::kTopK, F.n_sel != nullptr ? F.n_sel + w : nullptr,
                          static_cast<int>(w), lane, wsm);
   if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
 
   // ---- 4. attention over the selected blocks -------------------------------
-  if (cta < F.attn.n_cta) dattn::sparse_attn_decode_sk_body<false>(&tm_k, &tm_v, F.attn, smem, cta);
+  if (cta < F.attn.n_cta) dattn::sparse_attn_decode_sk_body<false, false>(&tm_k, &tm_v, &tm_q, F.attn, smem, cta);
   if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
 
   // ---- 5. merge the partials of pairs cut between CTAs ----------------------

@@ -267,6 +267,7 @@ __device__ __forceinline__ void block_scores_gemv_body(const Params<KeyT>& P, ui
     for (int c = 0; c < n_chunks; ++c, ++k) {
       const int st = k % kStages;
       if (ok) ok = mbar_wait(&sm.full[st], (k / kStages) & 1);
+      ok = __all_sync(0xffffffffu, ok);   // warp-uniform: the row sums below shuffle across the warp
       if (ok) {
         const KeyT* base = sm.stage[st] + (warp * R::kPerWarp + lane / R::kLanesPerRow) * kDi;
         float part[R::kPartials];

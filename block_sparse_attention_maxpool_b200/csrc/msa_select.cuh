@@ -8,17 +8,20 @@
 // Every visible block gets a unique 64-bit key: the float32 score mapped to
 // an order-preserving unsigned integer in the high word, the complemented
 // block index in the low word.  One unsigned compare then orders by score
-// descending and index ascending, exactly.  Lane l owns the blocks l + 32 j;
-// it keeps its keys in shared memory and its best remaining key in a
-// register.  Round r takes the warp maximum of the lanes' best keys (two
-// 32-bit warp reductions: the high words, then the low words of the lanes
-// that hold the highest high word), which is the r-th ranked block; only the
-// lane that owned it needs a new best, the largest of its keys below the
-// winner, and the warp reads that lane's keys from shared memory in parallel
-// (one per lane) and reduces them the same way.  k rounds give the top-k in
-// rank order; the k ids are then placed in ascending order with a 16-lane
-// rank count.  Above 1024 blocks the keys are re-read from global memory
-// every round instead.
+// descending and index ascending, exactly.  Lane l owns the blocks l + 32 j
+// and keeps its keys in shared memory and its best key in a register.
+//
+// With more than 16 visible blocks the top 16 are found in one pass: the
+// 16th largest of the 32 lanes' best keys bounds the 16th largest key from
+// below, the keys at or above it (typically about 20) are gathered and
+// ranked against each other all at once (31 independent shuffles per lane),
+// and the chosen ids are placed in ascending order the same way.  When more
+// than 32 keys pass the bound, k exact rounds run instead: round r takes
+// the warp maximum of the lanes' best keys (two 32-bit warp reductions: the
+// high words, then the low words of the lanes that hold the highest high
+// word), the r-th ranked block; only the lane that owned it needs a new
+// best, which the warp finds among that lane's keys in parallel.  Above
+// 1024 blocks the keys are re-read from global memory every round.
 #pragma once
 
 #include "msa_common.cuh"
@@ -49,27 +52,92 @@ __device__ __forceinline__ uint64_t warp_max_key(uint64_t x) {
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// Shared memory of one warp's keys (kPerLane > 0): a padded row per lane.
+// Shared memory of one warp's keys (kPerLane > 0): a padded row per lane,
+// then 32 slots for the candidates of the threshold pass.
 template <int kPerLane>
 struct KeySmem {
   static constexpr int kStride = kPerLane + 1;
-  static constexpr size_t kBytesPerWarp = 32 * kStride * sizeof(uint64_t);
+  static constexpr int kCandOff = 32 * kStride;
+  static constexpr size_t kBytesPerWarp = (32 * kStride + 32) * sizeof(uint64_t);
 };
 
+// Number of the warp's 32 values (one per lane, unique among the nonzero
+// ones) that are larger than this lane's: 31 independent shuffles.
+__device__ __forceinline__ int rank_in_warp(uint64_t x, int lane) {
+  const uint32_t hi = static_cast<uint32_t>(x >> 32), lo = static_cast<uint32_t>(x);
+  int r = 0;
+#pragma unroll
+  for (int d = 1; d < 32; ++d) {
+    const int src = (lane + d) & 31;
+    const uint32_t oh = __shfl_sync(0xffffffffu, hi, src);
+    const uint32_t ol = __shfl_sync(0xffffffffu, lo, src);
+    r += (oh > hi || (oh == hi && ol > lo)) ? 1 : 0;
+  }
+  return r;
+}
+
+// The top k = kTopK keys when more than kTopK blocks are visible, without
+// k serial rounds: the kTopK-th largest of the lanes' best keys, T, is a
+// lower bound of the kTopK-th largest key overall (kTopK lanes each hold a
+// key >= T), so the top k are among the keys >= T.  Those candidates
+// (typically about 20) are gathered into shared memory and ranked all at
+// once, one per lane.  False, with nothing written, when there are more
+// than 32 candidates; the caller then runs the exact rounds.
+template <int kPerLane>
+__device__ __forceinline__ bool select_by_threshold(uint64_t* wsm, uint64_t best, int lane, int32_t* out) {
+  constexpr int kStride = KeySmem<kPerLane>::kStride;
+  const int rb = rank_in_warp(best, lane);
+  const int tl = __ffs(__ballot_sync(0xffffffffu, rb == kTopK - 1)) - 1;
+  const uint64_t t = __shfl_sync(0xffffffffu, best, tl);
+  int cnt = 0;
+#pragma unroll
+  for (int j = 0; j < kPerLane; ++j) cnt += wsm[lane * kStride + j] >= t ? 1 : 0;
+  const int total = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt));
+  if (total > 32) return false;
+  int off = cnt;                                   // inclusive prefix of the counts
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, off, d);
+    if (lane >= d) off += o;
+  }
+  off -= cnt;
+  uint64_t* cand = wsm + KeySmem<kPerLane>::kCandOff;
+#pragma unroll
+  for (int j = 0; j < kPerLane; ++j) {
+    const uint64_t x = wsm[lane * kStride + j];
+    if (x >= t) cand[off++] = x;
+  }
+  __syncwarp();
+  const uint64_t c = lane < total ? cand[lane] : 0ull;
+  __syncwarp();
+  const int rc = rank_in_warp(c, lane);          // every lane: the shuffles take the whole warp
+  const bool chosen = lane < total && rc < kTopK;
+  // ascending block order: a chosen block's place is the number of chosen
+  // blocks with a smaller index
+  const int id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(c));
+  const int key = chosen ? id : 0x7fffffff;
+  int pos = 0;
+#pragma unroll
+  for (int d = 1; d < 32; ++d) pos += __shfl_sync(0xffffffffu, key, (lane + d) & 31) < key ? 1 : 0;
+  if (chosen) out[pos] = id;
+  return true;
+}
+
+// The top-k of (query, group) pair `wid` into `out` (k ids, ascending, -1
+// padded to kTopK) and its count into *count (nullable).
 // kPerLane > 0: at most 32 * kPerLane visible blocks, keys in `wsm` (this
 // warp's KeySmem<kPerLane>::kBytesPerWarp bytes of shared memory);
 // kPerLane == 0: any count, re-read from global memory each round.
 template <int kPerLane>
 __device__ __forceinline__ void select_pair(const float* __restrict__ bs, const int32_t* __restrict__ q_pos,
-                                            int G, int nblk, int capacity, int32_t* __restrict__ sel,
-                                            int32_t* __restrict__ n_sel, int wid, int lane, uint64_t* wsm) {
+                                            int G, int nblk, int capacity, int32_t* out, int32_t* count, int wid,
+                                            int lane, uint64_t* wsm) {
   const int qi = wid / G;
   const int p = q_pos[qi];
-  int32_t* out = sel + static_cast<size_t>(wid) * kTopK;
   if (p < 0 || p >= capacity) {
     if (lane < kTopK) out[lane] = -1;
     if (lane == 0) {
-      if (n_sel != nullptr) n_sel[wid] = 0;
+      if (count != nullptr) *count = 0;
       if (wid % G == 0) raise_error(MSA_DEVERR_QUERY_RANGE);
     }
     return;
@@ -82,14 +150,28 @@ __device__ __forceinline__ void select_pair(const float* __restrict__ bs, const 
   if constexpr (kPerLane > 0) {
     constexpr int kStride = KeySmem<kPerLane>::kStride;
     uint64_t best = 0ull;                          // every real key is > 0
+    // all of this lane's scores in flight at once: with the shared-memory
+    // stores in the same loop, the compiler (which cannot tell the two
+    // pointers apart) would issue one load per store, each a full round trip
+    float v[kPerLane];
 #pragma unroll
     for (int j = 0; j < kPerLane; ++j) {
       const int b = lane + 32 * j;
-      const uint64_t x = b < nvis ? block_key(__ldcg(row + b), b) : 0ull;
+      v[j] = b < nvis ? __ldcg(row + b) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+      const int b = lane + 32 * j;
+      const uint64_t x = b < nvis ? block_key(v[j], b) : 0ull;
       wsm[lane * kStride + j] = x;
       best = x > best ? x : best;
     }
     __syncwarp();
+    if (nvis > kTopK && select_by_threshold<kPerLane>(wsm, best, lane, out)) {
+      __syncwarp();
+      if (lane == 0 && count != nullptr) *count = kTopK;
+      return;
+    }
     for (int r = 0; r < k; ++r) {
       const uint64_t win = warp_max_key(best);
       const int b = static_cast<int>(0xffffffffu - static_cast<uint32_t>(win));
@@ -130,7 +212,7 @@ __device__ __forceinline__ void select_pair(const float* __restrict__ bs, const 
   } else if (lane < kTopK) {
     out[lane] = -1;
   }
-  if (lane == 0 && n_sel != nullptr) n_sel[wid] = k;
+  if (lane == 0 && count != nullptr) *count = k;
 }
 
 
@@ -147,7 +229,8 @@ __global__ void __launch_bounds__(256) select_topk_kernel(const float* __restric
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (wid >= n_q * G) return;
   uint64_t* wsm = kPerLane > 0 ? key_smem + (threadIdx.x >> 5) * (KeySmem<kPerLane>::kBytesPerWarp / 8) : nullptr;
-  select_pair<kPerLane>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, threadIdx.x & 31, wsm);
+  select_pair<kPerLane>(bs, q_pos, G, nblk, capacity, sel + static_cast<size_t>(wid) * kTopK,
+                        n_sel != nullptr ? n_sel + wid : nullptr, wid, threadIdx.x & 31, wsm);
 }
 
 // The warp count of a select_topk_kernel block and its dynamic shared memory.
@@ -165,14 +248,14 @@ __host__ __device__ constexpr size_t select_smem_per_warp(int nblk) {
 // The same for any block count, choosing the shared-memory variant when the
 // keys fit; wsm: select_smem_per_warp(nblk) bytes of this warp's shared memory.
 __device__ __forceinline__ void select_pair_any(const float* bs, const int32_t* q_pos, int G, int nblk,
-                                                int capacity, int32_t* sel, int32_t* n_sel, int wid, int lane,
+                                                int capacity, int32_t* out, int32_t* count, int wid, int lane,
                                                 uint64_t* wsm) {
   if (nblk <= 32 * 8) {
-    select_pair<8>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, lane, wsm);
+    select_pair<8>(bs, q_pos, G, nblk, capacity, out, count, wid, lane, wsm);
   } else if (nblk <= 32 * 32) {
-    select_pair<32>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, lane, wsm);
+    select_pair<32>(bs, q_pos, G, nblk, capacity, out, count, wid, lane, wsm);
   } else {
-    select_pair<0>(bs, q_pos, G, nblk, capacity, sel, n_sel, wid, lane, wsm);
+    select_pair<0>(bs, q_pos, G, nblk, capacity, out, count, wid, lane, wsm);
   }
 }
 

@@ -200,6 +200,24 @@ MSA_API int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, co
                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* msa_select_attn_decode - msa_select_topk followed by
+ * msa_sparse_attn_decode in one call, bit-identical to the two: block_scores
+ * [n_q][G][capacity/128] f32 in, the selection written to sel [n_q][G][16]
+ * and n_sel [n_q][G] (n_sel may be NULL), the attention to out.  MSA pull
+ * request, "Implementation": the block scores are ranked for the top-k and
+ * attention runs over the kept blocks.  Each CTA of the persistent attention
+ * grid ranks the pairs its units touch before it starts loading K/V, so a
+ * decode step has one launch fewer; when a CTA's share would touch more
+ * than 8 pairs (more than about 900 (query, group) pairs on 148 SMs) the
+ * call runs the selection kernel first instead, with the same results.
+ * Same arguments, layouts, workspace (msa_workspace_bytes(shape, n_q,
+ * MSA_MODE_DECODE)) and device errors as the two calls. */
+MSA_API int msa_select_attn_decode(const msa_shape* shape, const float* block_scores, const msa_bf16* q,
+                                   const msa_bf16* k_cache, const msa_bf16* v_cache, const int32_t* q_stream,
+                                   const int32_t* q_pos, int32_t n_q, float softmax_scale, int32_t* sel,
+                                   int32_t* n_sel, msa_bf16* out, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /* msa_sparse_attn_prefill - the same computation as msa_sparse_attn_decode,
  * for batches of many queries (prefill: every appended token is a query).
  * MSA pull request, "Implementation", batch case: the query's block-level
@@ -305,6 +323,11 @@ MSA_API int msa_sparse_attn_decode_paged(const msa_shape* shape, const msa_pages
                                          const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
                                          float softmax_scale, msa_bf16* out, void* workspace,
                                          size_t workspace_bytes, void* stream);
+MSA_API int msa_select_attn_decode_paged(const msa_shape* shape, const msa_pages* pages,
+                                         const float* block_scores, const msa_bf16* q, const msa_bf16* k_pool,
+                                         const msa_bf16* v_pool, const int32_t* q_stream, const int32_t* q_pos,
+                                         int32_t n_q, float softmax_scale, int32_t* sel, int32_t* n_sel,
+                                         msa_bf16* out, void* workspace, size_t workspace_bytes, void* stream);
 MSA_API int msa_sparse_attn_prefill_paged(const msa_shape* shape, const msa_pages* pages, const msa_bf16* q,
                                           const msa_bf16* k_pool, const msa_bf16* v_pool, const int32_t* sel,
                                           const int32_t* q_stream, const int32_t* q_pos, int32_t n_q,
