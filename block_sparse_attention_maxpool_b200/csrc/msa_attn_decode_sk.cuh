@@ -318,7 +318,8 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
   const long long u0 = unit_begin(U, P.n_cta, cta);
   const long long u1 = unit_begin(U, P.n_cta, cta + 1);
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == kWarps * 32) {
+    // the producer thread sets up the ring while the consumer warps rank
     for (int st = 0; st < kStages; ++st) {
       // token gathers: one arrival per producer lane (its copies landed) and
       // one per producer warp (its record written); TMA: the producer's one
@@ -326,6 +327,11 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
       mbar_init(&empty[st], kWarps);
     }
     mbar_fence_init();
+    if (u1 > u0) {                                 // the first unit's query, into L1
+      const int qi = static_cast<int>(u0 / kTopK / P.G);
+      prefetch_l1(P.q_stream + qi);
+      prefetch_l1(P.q_pos + qi);
+    }
   }
   if constexpr (kSel) {
     if (warp < kWarps) select_share(P, smem, sel_s, u0, u1, warp, lane);
@@ -573,6 +579,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  const __grid_constant__ CUtensorMap tm_q, const Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (threadIdx.x == kWarps * 32 && !kTok) {       // descriptors fetched before the dependency wait
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_q);
+  }
   pdl_trigger();
   pdl_wait();
   sparse_attn_decode_sk_body<kTok, kSel>(&tm_k, &tm_v, &tm_q, P, smem, blockIdx.x);

@@ -132,6 +132,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 // 2-D tiled tensor copy global -> shared (TMA).  x is the inner coordinate
 // in elements (kept a multiple of 16 bytes by every caller), y the row.
+// Fetch a tensor map (a __grid_constant__ kernel parameter) ahead of its
+// first TMA use.
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Bring the line holding p into L1 (no value returned, nothing waits).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
   asm volatile(

@@ -9,19 +9,21 @@
 // an order-preserving unsigned integer in the high word, the complemented
 // block index in the low word.  One unsigned compare then orders by score
 // descending and index ascending, exactly.  Lane l owns the blocks l + 32 j
-// and keeps its keys in shared memory and its best key in a register.
+// and holds their keys in registers.
 //
-// With more than 16 visible blocks the top 16 are found in one pass: the
-// 16th largest of the 32 lanes' best keys bounds the 16th largest key from
-// below, the keys at or above it (typically about 20) are gathered and
-// ranked against each other all at once (31 independent shuffles per lane),
-// and the chosen ids are placed in ascending order the same way.  When more
-// than 32 keys pass the bound, k exact rounds run instead: round r takes
-// the warp maximum of the lanes' best keys (two 32-bit warp reductions: the
-// high words, then the low words of the lanes that hold the highest high
-// word), the r-th ranked block; only the lane that owned it needs a new
-// best, which the warp finds among that lane's keys in parallel.  Above
-// 1024 blocks the keys are re-read from global memory every round.
+// With at most 16 visible blocks all of them are kept.  With more, the top
+// 16 are found in one pass: the 16th largest of the 32 lanes' best keys
+// bounds the 16th largest key from below; the keys at or above it
+// (typically about 20) are compacted into shared memory in ascending block
+// order with one ballot per column, each is ranked against the others by
+// broadcast reads, and a chosen key's place in the ascending output is a
+// ballot count.  When more than 32 keys pass the bound, k exact rounds run
+// instead: round r takes the warp maximum of the lanes' best keys (two
+// 32-bit warp reductions: the high words, then the low words of the lanes
+// that hold the highest high word), the r-th ranked block; only the lane
+// that owned it needs a new best, which the warp finds among that lane's
+// keys (now in shared memory) in parallel.  Above 1024 blocks the keys are
+// re-read from global memory every round.
 #pragma once
 
 #include "msa_common.cuh"
@@ -61,65 +63,47 @@ struct KeySmem {
   static constexpr size_t kBytesPerWarp = (32 * kStride + 32) * sizeof(uint64_t);
 };
 
-// Number of the warp's 32 values (one per lane, unique among the nonzero
-// ones) that are larger than this lane's: 31 independent shuffles.
-__device__ __forceinline__ int rank_in_warp(uint64_t x, int lane) {
-  const uint32_t hi = static_cast<uint32_t>(x >> 32), lo = static_cast<uint32_t>(x);
-  int r = 0;
-#pragma unroll
-  for (int d = 1; d < 32; ++d) {
-    const int src = (lane + d) & 31;
-    const uint32_t oh = __shfl_sync(0xffffffffu, hi, src);
-    const uint32_t ol = __shfl_sync(0xffffffffu, lo, src);
-    r += (oh > hi || (oh == hi && ol > lo)) ? 1 : 0;
-  }
-  return r;
-}
-
-// The top k = kTopK keys when more than kTopK blocks are visible, without
-// k serial rounds: the kTopK-th largest of the lanes' best keys, T, is a
-// lower bound of the kTopK-th largest key overall (kTopK lanes each hold a
-// key >= T), so the top k are among the keys >= T.  Those candidates
-// (typically about 20) are gathered into shared memory and ranked all at
-// once, one per lane.  False, with nothing written, when there are more
-// than 32 candidates; the caller then runs the exact rounds.
+// The top kTopK keys when more than kTopK blocks are visible, without
+// kTopK serial rounds.  x: this lane's keys (block lane + 32 j, 0 when not
+// visible); best: the largest of them; cand: 32 slots of this warp's shared
+// memory.  The kTopK-th largest of the 32 lanes' best keys, t, bounds the
+// kTopK-th largest key from below (kTopK lanes each hold a key >= t), so the
+// top keys are among those >= t.  They are compacted into cand column by
+// column (one ballot per column), which leaves them in ascending block
+// order, then each is ranked against the others by broadcast reads; a
+// chosen key's place in the ascending output is then one ballot count.
+// False, with nothing written, when more than 32 keys pass the bound (the
+// caller then runs the exact rounds).
 template <int kPerLane>
-__device__ __forceinline__ bool select_by_threshold(uint64_t* wsm, uint64_t best, int lane, int32_t* out) {
-  constexpr int kStride = KeySmem<kPerLane>::kStride;
-  const int rb = rank_in_warp(best, lane);
+__device__ __forceinline__ bool select_by_threshold(const uint64_t (&x)[kPerLane], uint64_t best, int lane,
+                                                    uint64_t* cand, int32_t* out) {
+  const uint32_t lt = (1u << lane) - 1u;
+  cand[lane] = best;
+  __syncwarp();
+  int rb = 0;
+#pragma unroll
+  for (int d = 0; d < 32; ++d) rb += cand[d] > best ? 1 : 0;
+  __syncwarp();
   const int tl = __ffs(__ballot_sync(0xffffffffu, rb == kTopK - 1)) - 1;
   const uint64_t t = __shfl_sync(0xffffffffu, best, tl);
-  int cnt = 0;
-#pragma unroll
-  for (int j = 0; j < kPerLane; ++j) cnt += wsm[lane * kStride + j] >= t ? 1 : 0;
-  const int total = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt));
-  if (total > 32) return false;
-  int off = cnt;                                   // inclusive prefix of the counts
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, off, d);
-    if (lane >= d) off += o;
-  }
-  off -= cnt;
-  uint64_t* cand = wsm + KeySmem<kPerLane>::kCandOff;
+  int total = 0;
 #pragma unroll
   for (int j = 0; j < kPerLane; ++j) {
-    const uint64_t x = wsm[lane * kStride + j];
-    if (x >= t) cand[off++] = x;
+    const bool pass = x[j] >= t;
+    const uint32_t m = __ballot_sync(0xffffffffu, pass);
+    const int slot = total + __popc(m & lt);
+    if (pass && slot < 32) cand[slot] = x[j];
+    total += __popc(m);
   }
   __syncwarp();
+  if (total > 32) return false;
   const uint64_t c = lane < total ? cand[lane] : 0ull;
-  __syncwarp();
-  const int rc = rank_in_warp(c, lane);          // every lane: the shuffles take the whole warp
+  int rc = 0;
+  for (int d = 0; d < total; ++d) rc += cand[d] > c ? 1 : 0;
   const bool chosen = lane < total && rc < kTopK;
-  // ascending block order: a chosen block's place is the number of chosen
-  // blocks with a smaller index
-  const int id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(c));
-  const int key = chosen ? id : 0x7fffffff;
-  int pos = 0;
-#pragma unroll
-  for (int d = 1; d < 32; ++d) pos += __shfl_sync(0xffffffffu, key, (lane + d) & 31) < key ? 1 : 0;
-  if (chosen) out[pos] = id;
+  const int pos = __popc(__ballot_sync(0xffffffffu, chosen) & lt);
+  if (chosen) out[pos] = static_cast<int>(0xffffffffu - static_cast<uint32_t>(c));
+  __syncwarp();
   return true;
 }
 
@@ -133,6 +117,17 @@ __device__ __forceinline__ void select_pair(const float* __restrict__ bs, const 
                                             int G, int nblk, int capacity, int32_t* out, int32_t* count, int wid,
                                             int lane, uint64_t* wsm) {
   const int qi = wid / G;
+  const float* row = bs + static_cast<size_t>(wid) * nblk;
+  // the row's scores are requested before the query position arrives (the
+  // two round trips overlap); blocks past the position are masked after
+  float v[kPerLane > 0 ? kPerLane : 1];
+  if constexpr (kPerLane > 0) {
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+      const int b = lane + 32 * j;
+      v[j] = b < nblk ? __ldcg(row + b) : 0.f;
+    }
+  }
   const int p = q_pos[qi];
   if (p < 0 || p >= capacity) {
     if (lane < kTopK) out[lane] = -1;
@@ -144,46 +139,43 @@ __device__ __forceinline__ void select_pair(const float* __restrict__ bs, const 
   }
   const int nvis = p / kBlock + 1;
   const int k = min(kTopK, nvis);
-  const float* row = bs + static_cast<size_t>(wid) * nblk;
+  if (nvis <= kTopK) {                              // every visible block is kept
+    if (lane < kTopK) out[lane] = lane < nvis ? lane : -1;
+    if (lane == 0 && count != nullptr) *count = nvis;
+    return;
+  }
   int my_id = -1;
 
   if constexpr (kPerLane > 0) {
     constexpr int kStride = KeySmem<kPerLane>::kStride;
+    uint64_t x[kPerLane];
     uint64_t best = 0ull;                          // every real key is > 0
-    // all of this lane's scores in flight at once: with the shared-memory
-    // stores in the same loop, the compiler (which cannot tell the two
-    // pointers apart) would issue one load per store, each a full round trip
-    float v[kPerLane];
 #pragma unroll
     for (int j = 0; j < kPerLane; ++j) {
       const int b = lane + 32 * j;
-      v[j] = b < nvis ? __ldcg(row + b) : 0.f;
+      x[j] = b < nvis ? block_key(v[j], b) : 0ull;
+      best = x[j] > best ? x[j] : best;
     }
-#pragma unroll
-    for (int j = 0; j < kPerLane; ++j) {
-      const int b = lane + 32 * j;
-      const uint64_t x = b < nvis ? block_key(v[j], b) : 0ull;
-      wsm[lane * kStride + j] = x;
-      best = x > best ? x : best;
-    }
-    __syncwarp();
-    if (nvis > kTopK && select_by_threshold<kPerLane>(wsm, best, lane, out)) {
-      __syncwarp();
+    if (select_by_threshold<kPerLane>(x, best, lane, wsm + KeySmem<kPerLane>::kCandOff, out)) {
       if (lane == 0 && count != nullptr) *count = kTopK;
       return;
     }
+    // more than 32 keys at or above the bound: k exact rounds over the keys
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) wsm[lane * kStride + j] = x[j];
+    __syncwarp();
     for (int r = 0; r < k; ++r) {
       const uint64_t win = warp_max_key(best);
       const int b = static_cast<int>(0xffffffffu - static_cast<uint32_t>(win));
       if (lane == r) my_id = b;
       // the owner of the winner (lane b % 32) takes its largest key below it
       const int owner = b & 31;
-      uint64_t x = 0ull;
+      uint64_t y = 0ull;
       if (lane < kPerLane) {
-        x = wsm[owner * kStride + lane];
-        if (x >= win) x = 0ull;
+        y = wsm[owner * kStride + lane];
+        if (y >= win) y = 0ull;
       }
-      const uint64_t next = warp_max_key(x);
+      const uint64_t next = warp_max_key(y);
       if (lane == owner) best = next;
     }
     __syncwarp();
@@ -192,8 +184,8 @@ __device__ __forceinline__ void select_pair(const float* __restrict__ bs, const 
     for (int r = 0; r < k; ++r) {
       uint64_t best = 0ull;
       for (int b = lane; b < nvis; b += 32) {
-        const uint64_t x = block_key(__ldcg(row + b), b);
-        if (x < prev && x > best) best = x;
+        const uint64_t y = block_key(__ldcg(row + b), b);
+        if (y < prev && y > best) best = y;
       }
       best = warp_max_key(best);
       prev = best;
