@@ -12,7 +12,7 @@
 // One producer thread resolves each unit (query position, selected block,
 // cache row), writes what the consumers need into a small per-stage record
 // and TMA-loads the unit's K and V tiles (four 16 KB boxes, 128-byte
-// swizzle) into a two-stage ring, plus the pair's Q (16 heads x 128 dims)
+// swizzle) into a three-stage ring, plus the pair's Q (16 heads x 128 dims)
 // when the unit is the first of its pair in this CTA; the consumers so make
 // no global-memory round trip between units.  Eight consumer warps each own
 // 16 key rows of the block and compute S = Q K^T (16 heads x 16 rows) and
@@ -61,8 +61,9 @@ constexpr int kRowsPerWarp = kBlock / kWarps;       // 16
 constexpr uint32_t kTileBytes = kBlock * 64 * 2;    // [128 rows][64 dims] bf16 = 16 KB
 constexpr uint32_t kStageBytes = 4 * kTileBytes;    // K lo, K hi, V lo, V hi
 constexpr uint32_t kQBytes = kHpg * kD * 2;         // Q of one pair: two [16 heads][64 dims] boxes, 4 KB
-constexpr int kStages = 2;
-constexpr int kOStride = kD + 4;                    // padded fp32 row of the merge buffer
+constexpr int kStages = 3;
+constexpr int kMergeCols = 32;                      // dims of O merged per round (four rounds)
+constexpr int kMStride = kMergeCols + 4;            // padded fp32 row of the merge buffer
 constexpr int kMaxCtas = 256;                       // grid cap (bounds the workspace)
 constexpr int kPartial = kHpg * (kD + 2);           // floats of one partial: O[16][128], m[16], l[16]
 constexpr int kSelPairs = 8;                        // fused selection: pairs one CTA may touch
@@ -82,7 +83,7 @@ struct Layout {
   static constexpr uint32_t kStageOff = 0;
   static constexpr uint32_t kQOff = kStages * kStageBytes;
   static constexpr uint32_t kMergeOff = kQOff + kStages * kQBytes;
-  static constexpr uint32_t kMlOff = kMergeOff + kWarps * kHpg * kOStride * 4;
+  static constexpr uint32_t kMlOff = kMergeOff + kWarps * kHpg * kMStride * 4;
   static constexpr uint32_t kInfoOff = kMlOff + kWarps * kHpg * 2 * 4;
   static constexpr uint32_t kSelOff = kInfoOff + kStages * sizeof(UnitInfo);
   static constexpr uint32_t kBarOff = kSelOff + kSelPairs * (kTopK + 1) * 4 + 16;
@@ -93,7 +94,7 @@ static_assert(Layout::kQOff % 1024 == 0 && kQBytes % 1024 == 0, "128-byte-swizzl
 static_assert(Layout::kBarOff % 8 == 0 && Layout::kInfoOff % 16 == 0, "barrier and record alignment");
 static_assert(kWarps * sel::KeySmem<32>::kBytesPerWarp <= Layout::kQOff - Layout::kStageOff,
               "fused selection: every consumer warp's keys fit the stage ring");
-static_assert(Layout::kBytes <= 227 * 1024, "shared memory of one CTA");
+static_assert(Layout::kBytes + 256 <= 227 * 1024, "shared memory of one CTA (and of the one-kernel step)");
 
 struct Params {
   const __nv_bfloat16* q;     // [n_q][Hq][D]
@@ -203,7 +204,10 @@ __device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, in
 }
 
 // Merge the eight warps' states of one pair and write the output rows (or
-// this CTA's partial for a pair shared with a neighbouring CTA).
+// this CTA's partial for a pair shared with a neighbouring CTA).  O goes
+// through shared memory in four rounds of 32 dims (a quarter-size buffer,
+// which leaves room for a third stage of the ring); thread (head, 2 dims)
+// sums the eight warps' slices, scaled to the common maximum.
 __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long long pair, long long u0,
                                            long long u1, int slot_cta, float (&o)[16][4], float (&m_run)[2],
                                            float (&l_run)[2], int warp, int lane) {
@@ -214,60 +218,64 @@ __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long 
     l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
     l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
   }
-  float* so = reinterpret_cast<float*>(smem + Layout::kMergeOff);   // [8][16][kOStride]
+  float* so = reinterpret_cast<float*>(smem + Layout::kMergeOff);   // [8][16][kMStride]
   float* sml = reinterpret_cast<float*>(smem + Layout::kMlOff);     // [8][16][2]
-  named_barrier_sync(1, kWarps * 32);                                 // previous merge fully read
-  {
-    float* ow = so + warp * kHpg * kOStride;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const int col = n * 8 + tq * 2;
-      *reinterpret_cast<float2*>(ow + gr * kOStride + col) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(ow + (gr + 8) * kOStride + col) = make_float2(o[n][2], o[n][3]);
-    }
-    if (tq == 0) {
-      sml[(warp * kHpg + gr) * 2 + 0] = m_run[0];
-      sml[(warp * kHpg + gr) * 2 + 1] = l_run[0];
-      sml[(warp * kHpg + gr + 8) * 2 + 0] = m_run[1];
-      sml[(warp * kHpg + gr + 8) * 2 + 1] = l_run[1];
-    }
-  }
-  named_barrier_sync(1, kWarps * 32);
   const int head = tid >> 4;            // 16 heads x 16 threads
-  const int d0 = (tid & 15) * 8;        // 8 dims per thread
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sml[(w * kHpg + head) * 2]);
-  const float Mu = M == -INFINITY ? 0.f : M;
-  float L = 0.f;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const float sc = exp2f(sml[(w * kHpg + head) * 2] - Mu);
-    L += sml[(w * kHpg + head) * 2 + 1] * sc;
-    const float4* src = reinterpret_cast<const float4*>(so + (w * kHpg + head) * kOStride + d0);
-    const float4 a = src[0], b = src[1];
-    acc[0] += a.x * sc; acc[1] += a.y * sc; acc[2] += a.z * sc; acc[3] += a.w * sc;
-    acc[4] += b.x * sc; acc[5] += b.y * sc; acc[6] += b.z * sc; acc[7] += b.w * sc;
-  }
+  const int dd = (tid & 15) * 2;        // 2 dims of the round's 32 per thread
   const bool complete = pair * kTopK >= u0 && pair * kTopK + kTopK <= u1;
-  if (complete) {
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint32_t pk[4];
+  float* part = complete ? nullptr
+                         : P.ws + (static_cast<size_t>(slot_cta) * 2 + (pair * kTopK < u0 ? 0 : 1)) * kPartial;
+  float sc[kWarps];
+  float M = -INFINITY, L = 0.f, inv = 0.f;
 #pragma unroll
-    for (int d = 0; d < 4; ++d) pk[d] = pack_bf16(acc[2 * d] * inv, acc[2 * d + 1] * inv);
-    __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + d0;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  } else {
-    const int slot = pair * kTopK < u0 ? 0 : 1;
-    float* part = P.ws + (static_cast<size_t>(slot_cta) * 2 + slot) * kPartial;
-    float* dst = part + head * kD + d0;
-    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    if ((tid & 15) == 0) {
-      part[kHpg * kD + head] = M;
-      part[kHpg * kD + kHpg + head] = L;
+  for (int r = 0; r < kD / kMergeCols; ++r) {
+    named_barrier_sync(1, kWarps * 32);                               // the previous round fully read
+    {
+      float* ow = so + warp * kHpg * kMStride;
+#pragma unroll
+      for (int nn = 0; nn < kMergeCols / 8; ++nn) {
+        const int n = r * (kMergeCols / 8) + nn;
+        const int col = nn * 8 + tq * 2;
+        *reinterpret_cast<float2*>(ow + gr * kMStride + col) = make_float2(o[n][0], o[n][1]);
+        *reinterpret_cast<float2*>(ow + (gr + 8) * kMStride + col) = make_float2(o[n][2], o[n][3]);
+      }
+      if (r == 0 && tq == 0) {
+        sml[(warp * kHpg + gr) * 2 + 0] = m_run[0];
+        sml[(warp * kHpg + gr) * 2 + 1] = l_run[0];
+        sml[(warp * kHpg + gr + 8) * 2 + 0] = m_run[1];
+        sml[(warp * kHpg + gr + 8) * 2 + 1] = l_run[1];
+      }
     }
+    named_barrier_sync(1, kWarps * 32);
+    if (r == 0) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sml[(w * kHpg + head) * 2]);
+      const float Mu = M == -INFINITY ? 0.f : M;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        sc[w] = exp2f(sml[(w * kHpg + head) * 2] - Mu);
+        L += sml[(w * kHpg + head) * 2 + 1] * sc[w];
+      }
+      inv = L > 0.f ? 1.f / L : 0.f;
+    }
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float2 v = *reinterpret_cast<const float2*>(so + (w * kHpg + head) * kMStride + dd);
+      a0 += v.x * sc[w];
+      a1 += v.y * sc[w];
+    }
+    const int d = r * kMergeCols + dd;
+    if (complete) {
+      __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + d;
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16(a0 * inv, a1 * inv);
+    } else {
+      *reinterpret_cast<float2*>(part + head * kD + d) = make_float2(a0, a1);
+    }
+  }
+  if (!complete && (tid & 15) == 0) {
+    part[kHpg * kD + head] = M;
+    part[kHpg * kD + kHpg + head] = L;
   }
 }
 
