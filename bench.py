@@ -332,15 +332,15 @@ class Step:
         self.scale = 1.0 / math.sqrt(sh.head_dim)
         tiles = n_q >= 256 and n_q >= 64 * w.n_streams
         if self.dsa:
-            self.launches = 2 + 1 + 1 + 2        # appends, token scores, top-k, attention + combine
+            self.launches = 2 + 1 + 1 + 1        # appends, token scores, top-k, attention
         elif self.fused:
             self.launches = 1
         elif variant == "shared":
-            self.launches = 1 + 2                # K/V append, attention + combine
+            self.launches = 1 + 1                # K/V append, attention
         else:
             appends = 2 if args.idx_f16 else 1
-            # decode: selection inside the attention kernel (+ combine); prefill: top-k, plan, attention
-            self.launches = appends + (6 if tiles else 1) + (3 if self.prefill else 2)
+            # decode: selection and merges inside the attention kernel; prefill: top-k, plan, attention
+            self.launches = appends + (6 if tiles else 1) + (3 if self.prefill else 1)
         self.parts = self._parts()
 
     def switch(self, variant: str):
@@ -348,7 +348,7 @@ class Step:
         step ("full" or "shared"); graphs are captured again."""
         self.variant = variant
         self.set_sel = [torch.empty_like(self.bufs["sel"]) for _ in self.sets] if variant == "shared" else None
-        self.launches = 1 + 2 if variant == "shared" else self.launches
+        self.launches = 1 + 1 if variant == "shared" else self.launches
         self.whole, self.split = [], []
         self.parts = self._parts()
 
@@ -921,7 +921,7 @@ def run_ours(args, rank, world, dev):
         line["step_hbm"] = {"achieved_gbs": sb / (ms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
                             "frac": sb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "bytes_per_step": sb}
         a = kv_bytes_per_stream(w) * w.n_streams / (k_ms * 1e-3) / 1e9
-        line["roofline"] = {"kernel": "sparse_attn_decode_sk + combine", "bound": "hbm", "achieved": a,
+        line["roofline"] = {"kernel": "sparse_attn_decode_sk", "bound": "hbm", "achieved": a,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": a / peaks["hbm_gbs"], "traffic": None,
                             "algorithmic_bytes": kv_bytes_per_stream(w) * w.n_streams, "ms_per_launch": k_ms,
                             "peak_src": peaks["src"]}

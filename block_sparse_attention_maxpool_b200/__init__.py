@@ -449,8 +449,8 @@ NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 def msa_sparse_attn_decode_noalloc(shape: Shape, q, k_cache, v_cache, sel, q_stream, q_pos,
                                    softmax_scale=None, out=None, stream=None):
     """Decode attention for callers that cannot allocate device memory: the
-    split partials go to the library's fixed 8 MiB device buffer instead of
-    a workspace.  ``out`` is still the caller's (allocated here only when
+    merge bookkeeping and partials go to the library's fixed 8 MiB device
+    buffer instead of a workspace.  ``out`` is still the caller's (allocated here only when
     None, for convenience).  Calls sharing the buffer at the same time on the
     GPU race; see include/msa.h."""
     n = _n(q_pos, "q_pos")

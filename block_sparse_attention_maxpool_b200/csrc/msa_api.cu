@@ -153,9 +153,10 @@ size_t scores_workspace(const msa_shape* sh, int32_t n_q) {
   return msa::tc::workspace_layout(n_q, sh->n_kv_heads, sh->n_streams, sh->capacity).total;
 }
 
-// Decode attention workspace: two partial results per CTA of the persistent
-// grid (at most kMaxCtas CTAs, at most one per unit).  Depends only on the
-// pair count, so the workspace query and the launch always agree.
+// Decode attention workspace: the merge bookkeeping of kMaxCtas CTA slots
+// (kept from call to call), then one partial result per CTA of the
+// persistent grid (at most kMaxCtas CTAs, at most one per unit).  Depends
+// only on the pair count, so the workspace query and the launch always agree.
 
 // Prefill attention: the plan of every 8-query tile.
 int64_t union_tasks(const msa_shape* sh, int32_t n_q) {
@@ -167,7 +168,7 @@ size_t attn_workspace(const msa_shape* sh, int32_t n_q, int mode) {
   if (mode == MSA_MODE_PREFILL) return static_cast<size_t>(union_tasks(sh, n_q)) * sizeof(msa::uattn::Plan);
   const int64_t units = static_cast<int64_t>(n_q) * sh->n_kv_heads * msa::dattn::kTopK;
   const int64_t ctas = std::min<int64_t>(units, msa::dattn::kMaxCtas);
-  return static_cast<size_t>(ctas) * 2 * msa::dattn::kPartial * sizeof(float);
+  return msa::dattn::kSyncBytes + static_cast<size_t>(ctas) * msa::dattn::kPartial * sizeof(float);
 }
 
 // Most pairs one CTA's share of the decode units touches.
@@ -277,7 +278,8 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   P.q_stream = q_stream;
   P.q_pos = q_pos;
   P.out = reinterpret_cast<__nv_bfloat16*>(out);
-  P.ws = static_cast<float*>(workspace);
+  P.sync = static_cast<msa::dattn::SyncSlot*>(workspace);
+  P.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + msa::dattn::kSyncBytes);
   P.n_q = n_q;
   P.G = G;
   P.n_streams = sh->n_streams;
@@ -295,9 +297,6 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
   P.n_sel_out = fuse_sel ? n_sel_out : nullptr;
   launch(kernel, dim3(static_cast<unsigned>(P.n_cta)), dim3(msa::dattn::kThreads), msa::dattn::Layout::kBytes, s,
          tm_k, tm_v, tm_q, P);
-  if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
-  const int64_t warps = n_pairs * msa::dattn::kHpg;
-  launch(msa::dattn::attn_sk_combine_kernel, dim3(static_cast<unsigned>((warps * 32 + 255) / 256)), dim3(256), 0, s, P);
   return cuda_status(cudaGetLastError());
 }
 
@@ -978,7 +977,8 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   A.q_stream = q_stream;
   A.q_pos = q_pos;
   A.out = reinterpret_cast<__nv_bfloat16*>(out);
-  A.ws = static_cast<float*>(workspace);
+  A.sync = static_cast<msa::dattn::SyncSlot*>(workspace);
+  A.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + msa::dattn::kSyncBytes);
   A.n_q = n_q;
   A.G = G;
   A.n_streams = shape->n_streams;

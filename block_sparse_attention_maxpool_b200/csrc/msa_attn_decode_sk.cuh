@@ -20,8 +20,10 @@
 // softmax.  Consecutive units of one pair accumulate in registers; when the
 // pair changes the eight warps merge through shared memory.  A pair whose
 // units all lie in one CTA's share is written out directly; a pair cut by a
-// share boundary leaves one partial (max, sum, unnormalised O) per CTA,
-// merged by attn_sk_combine_kernel.
+// share boundary is merged inside the kernel by the CTA holding its first
+// unit, which reaches it last (at the end of its share), from the partials
+// (max, sum, unnormalised O) the later CTAs published; no merge kernel
+// follows.
 //
 // Fused selection (Params::bs set): before the ring starts, the CTA's
 // consumer warps rank the block scores of the (at most kSelPairs) pairs its
@@ -68,6 +70,23 @@ constexpr int kMaxCtas = 256;                       // grid cap (bounds the work
 constexpr int kPartial = kHpg * (kD + 2);           // floats of one partial: O[16][128], m[16], l[16]
 constexpr int kSelPairs = 8;                        // fused selection: pairs one CTA may touch
 
+// One CTA slot of the workspace's merge bookkeeping (kMaxCtas slots at the
+// start of the workspace, kept from call to call).  A pair cut by share
+// boundaries is merged by the CTA holding its first unit (its "merger"),
+// which reaches that pair last, at the end of its share; every later CTA
+// holding some of its units publishes a partial and sets `flag` to
+// kFlagTag | merger << 32 | (merger's epoch + 1).  The merger waits for
+// exactly that value, merges, and then raises its own epoch, so a flag left
+// from an earlier call (or any other contents of a reused buffer) never
+// matches, and the slots need no zeroing.
+struct SyncSlot {
+  unsigned long long flag;
+  unsigned int epoch;
+  unsigned int pad;
+};
+constexpr unsigned long long kFlagTag = 0x4d53ull << 48;
+constexpr size_t kSyncBytes = kMaxCtas * sizeof(SyncSlot);
+
 // What the producer tells the consumers about the unit in a stage.
 struct UnitInfo {
   int32_t flags;      // kUnitData: K/V rows landed; kUnitQ: the pair's Q landed
@@ -86,7 +105,8 @@ struct Layout {
   static constexpr uint32_t kMlOff = kMergeOff + kWarps * kHpg * kMStride * 4;
   static constexpr uint32_t kInfoOff = kMlOff + kWarps * kHpg * 2 * 4;
   static constexpr uint32_t kSelOff = kInfoOff + kStages * sizeof(UnitInfo);
-  static constexpr uint32_t kBarOff = kSelOff + kSelPairs * (kTopK + 1) * 4 + 16;
+  static constexpr uint32_t kMiscOff = kSelOff + kSelPairs * (kTopK + 1) * 4 + 16;   // the CTA's epoch
+  static constexpr uint32_t kBarOff = kMiscOff + 16;
   static constexpr uint32_t kEnd = kBarOff + 64;
   static constexpr size_t kBytes = kEnd + 1024;
 };
@@ -102,7 +122,8 @@ struct Params {
   const int32_t* q_stream;
   const int32_t* q_pos;
   __nv_bfloat16* out;         // [n_q][Hq][D]
-  float* ws;                  // [n_cta][2][kPartial]
+  float* ws;                  // [n_cta][kPartial]: the partial of each CTA's first pair when it began earlier
+  SyncSlot* sync;             // [kMaxCtas], kept between calls
   int n_q, G, n_streams, capacity, n_cta;
   long long n_units;          // n_q * G * 16
   float scale_log2;
@@ -203,14 +224,28 @@ __device__ __forceinline__ int unit_row(const Params& P, long long u, int& p, in
   return static_cast<int>(row);   // the host checks that every row fits 31 bits
 }
 
-// Merge the eight warps' states of one pair and write the output rows (or
-// this CTA's partial for a pair shared with a neighbouring CTA).  O goes
-// through shared memory in four rounds of 32 dims (a quarter-size buffer,
-// which leaves room for a third stage of the ring); thread (head, 2 dims)
-// sums the eight warps' slices, scaled to the common maximum.
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Merge the eight warps' states of one pair and write the output rows.  O
+// goes through shared memory in four rounds of 32 dims (a quarter-size
+// buffer, which leaves room for a third stage of the ring); thread (head,
+// 2 dims) sums the eight warps' slices, scaled to the common maximum.  A
+// pair this CTA holds only the tail of (it began in an earlier CTA) is
+// published as this CTA's partial instead (`pub`: the flag value, thread
+// 0).  A pair that begins here and ends in later CTAs is the CTA's last, so
+// the ring is idle: its merged state goes to the stage area, and once the
+// later CTAs' flags read this CTA's next epoch, thread (head, 8 dims) folds
+// their partials in, all loads in flight at once, and writes the rows.
 __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long long pair, long long u0,
-                                           long long u1, int slot_cta, float (&o)[16][4], float (&m_run)[2],
-                                           float (&l_run)[2], int warp, int lane) {
+                                           long long u1, int cta, float (&o)[16][4], float (&m_run)[2],
+                                           float (&l_run)[2], int warp, int lane, unsigned long long pub) {
   const int gr = lane >> 2, tq = lane & 3;
   const int tid = warp * 32 + lane;
 #pragma unroll
@@ -220,11 +255,12 @@ __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long 
   }
   float* so = reinterpret_cast<float*>(smem + Layout::kMergeOff);   // [8][16][kMStride]
   float* sml = reinterpret_cast<float*>(smem + Layout::kMlOff);     // [8][16][2]
+  float* mine = reinterpret_cast<float*>(smem + Layout::kStageOff); // merger: [16][128] own merged O
   const int head = tid >> 4;            // 16 heads x 16 threads
   const int dd = (tid & 15) * 2;        // 2 dims of the round's 32 per thread
-  const bool complete = pair * kTopK >= u0 && pair * kTopK + kTopK <= u1;
-  float* part = complete ? nullptr
-                         : P.ws + (static_cast<size_t>(slot_cta) * 2 + (pair * kTopK < u0 ? 0 : 1)) * kPartial;
+  const bool tail = pair * kTopK < u0;                               // began in an earlier CTA
+  const bool merger = !tail && pair * kTopK + kTopK > u1;            // begins here, ends later
+  float* part = P.ws + static_cast<size_t>(cta) * kPartial;
   float sc[kWarps];
   float M = -INFINITY, L = 0.f, inv = 0.f;
 #pragma unroll
@@ -266,17 +302,97 @@ __device__ __forceinline__ void flush_pair(const Params& P, uint8_t* smem, long 
       a1 += v.y * sc[w];
     }
     const int d = r * kMergeCols + dd;
-    if (complete) {
+    if (tail) {
+      *reinterpret_cast<float2*>(part + head * kD + d) = make_float2(a0, a1);
+    } else if (merger) {
+      *reinterpret_cast<float2*>(mine + head * kD + d) = make_float2(a0, a1);
+    } else {
       __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + d;
       *reinterpret_cast<uint32_t*>(dst) = pack_bf16(a0 * inv, a1 * inv);
-    } else {
-      *reinterpret_cast<float2*>(part + head * kD + d) = make_float2(a0, a1);
     }
   }
-  if (!complete && (tid & 15) == 0) {
-    part[kHpg * kD + head] = M;
-    part[kHpg * kD + kHpg + head] = L;
+  if (tail) {
+    if ((tid & 15) == 0) {
+      part[kHpg * kD + head] = M;
+      part[kHpg * kD + kHpg + head] = L;
+    }
+    __syncwarp();
+    named_barrier_sync(1, kWarps * 32);    // every thread's share of the partial written
+    if (tid == 0) st_release_u64(&P.sync[cta].flag, pub);   // releases what the barrier ordered before it
+    return;
   }
+  if (!merger) return;
+  // the later CTAs holding some of this pair publish their partials early
+  // in their shares; by now they are normally there
+  const int n_later = cta_of(P.n_units, P.n_cta, pair * kTopK + kTopK - 1) - cta;
+  const unsigned int epoch = *reinterpret_cast<const unsigned int*>(smem + Layout::kMiscOff);
+  if (tid < n_later) {
+    const unsigned long long want = kFlagTag | (static_cast<unsigned long long>(cta) << 32) | (epoch + 1u);
+    const unsigned long long* f = &P.sync[cta + 1 + tid].flag;
+    if (ld_acquire_u64(f) != want) {
+      const long long t0 = clock64();
+      while (ld_acquire_u64(f) != want) {
+        if (clock64() - t0 > kWaitCycles) {
+          raise_error(MSA_DEVERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  named_barrier_sync(1, kWarps * 32);      // the flags seen, the own state in `mine`
+  const int d8 = (tid & 15) * 8;           // thread (head, 8 dims)
+  // fold the later partials in, eight at a time with all their loads in
+  // flight, rescaling the running state to each batch's maximum
+  float acc[8];
+  {
+    const float4 x = *reinterpret_cast<const float4*>(mine + head * kD + d8);
+    const float4 y = *reinterpret_cast<const float4*>(mine + head * kD + d8 + 4);
+    acc[0] = x.x; acc[1] = x.y; acc[2] = x.z; acc[3] = x.w;
+    acc[4] = y.x; acc[5] = y.y; acc[6] = y.z; acc[7] = y.w;
+  }
+  float Mrun = M, Lrun = L;
+  for (int base = 0; base < n_later; base += 8) {
+    float mj[8], lj[8];
+    float4 xj[8], yj[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      mj[t] = -INFINITY;
+      lj[t] = 0.f;
+      xj[t] = yj[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (base + t < n_later) {
+        const float* pj = P.ws + static_cast<size_t>(cta + 1 + base + t) * kPartial;
+        mj[t] = __ldcg(pj + kHpg * kD + head);
+        lj[t] = __ldcg(pj + kHpg * kD + kHpg + head);
+        xj[t] = __ldcg(reinterpret_cast<const float4*>(pj + head * kD + d8));
+        yj[t] = __ldcg(reinterpret_cast<const float4*>(pj + head * kD + d8 + 4));
+      }
+    }
+    float Mnew = Mrun;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) Mnew = fmaxf(Mnew, mj[t]);
+    const float Mu = Mnew == -INFINITY ? 0.f : Mnew;
+    const float sr = exp2f(Mrun - Mu);
+    Lrun *= sr;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= sr;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const float sj = exp2f(mj[t] - Mu);
+      Lrun += lj[t] * sj;
+      acc[0] += xj[t].x * sj; acc[1] += xj[t].y * sj; acc[2] += xj[t].z * sj; acc[3] += xj[t].w * sj;
+      acc[4] += yj[t].x * sj; acc[5] += yj[t].y * sj; acc[6] += yj[t].z * sj; acc[7] += yj[t].w * sj;
+    }
+    Mrun = Mnew;
+  }
+  const float iall = Lrun > 0.f ? 1.f / Lrun : 0.f;
+  uint32_t pk[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(acc[2 * e] * iall, acc[2 * e + 1] * iall);
+  *reinterpret_cast<uint4*>(P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + d8) =
+      make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  named_barrier_sync(1, kWarps * 32);      // every later partial read
+  if (tid == 0) P.sync[cta].epoch = epoch + 1u;   // read by the next call's CTAs, after this kernel ends
 }
 
 // The top-16 of the pairs this CTA's units touch (fused selection), into
@@ -339,6 +455,17 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
       const int qi = static_cast<int>(u0 / kTopK / P.G);
       prefetch_l1(P.q_stream + qi);
       prefetch_l1(P.q_pos + qi);
+    }
+  }
+  // merges of cut pairs: this CTA's epoch (as a merger), and the flag value
+  // it publishes with its first pair's partial when that pair began earlier
+  unsigned long long pub = 0ull;
+  if (threadIdx.x == 0) {
+    *reinterpret_cast<unsigned int*>(smem + Layout::kMiscOff) = __ldcg(&P.sync[cta].epoch);
+    const long long first = u0 / kTopK * kTopK;
+    if (u1 > u0 && first < u0) {
+      const int m = cta_of(U, P.n_cta, first);
+      pub = kFlagTag | (static_cast<unsigned long long>(m) << 32) | (__ldcg(&P.sync[m].epoch) + 1u);
     }
   }
   if constexpr (kSel) {
@@ -466,7 +593,7 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
     ok = __all_sync(0xffffffffu, ok);     // warp-uniform: the MMAs below take the whole warp
     const long long pair = u / kTopK;
     if (pair != cur) {
-      if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane);
+      if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane, pub);
       cur = pair;
 #pragma unroll
       for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -578,7 +705,7 @@ __device__ __forceinline__ void sparse_attn_decode_sk_body(const CUtensorMap* tm
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
   }
-  if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane);
+  if (cur >= 0) flush_pair(P, smem, cur, u0, u1, cta, o, m_run, l_run, warp, lane, pub);
 }
 
 template <bool kTok, bool kSel>
@@ -595,63 +722,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   pdl_wait();
   sparse_attn_decode_sk_body<kTok, kSel>(&tm_k, &tm_v, &tm_q, P, smem, blockIdx.x);
-}
-
-// Pairs cut by a share boundary: merge the partials of every CTA whose share
-// touches the pair.  One warp per (pair, head), four dims per lane.
-__device__ __forceinline__ void combine_pair_head(const Params& P, long long w, int lane) {
-  const long long pair = w / kHpg;
-  const int head = static_cast<int>(w - pair * kHpg);
-  const long long U = P.n_units;
-  const int c_lo = cta_of(U, P.n_cta, pair * kTopK);
-  const int c_hi = cta_of(U, P.n_cta, pair * kTopK + kTopK - 1);
-  if (c_lo == c_hi) return;                              // written directly by its CTA
-  // every CTA in [c_lo, c_hi] holds at least one of the pair's 16 units, so
-  // there are at most 16 partials: lane j reads partial j's max and sum, and
-  // the warp reduces them, then sums the scaled O slices
-  const int n = c_hi - c_lo + 1;
-  float mj = -INFINITY, lj = 0.f;
-  if (lane < n) {
-    const int c = c_lo + lane;
-    const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
-    const float* part = P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial;
-    mj = __ldcg(part + kHpg * kD + head);
-    lj = __ldcg(part + kHpg * kD + kHpg + head);
-  }
-  float M = mj;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float Mu = M == -INFINITY ? 0.f : M;
-  const float scj = lane < n ? exp2f(mj - Mu) : 0.f;
-  float L = lj * scj;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < kTopK; ++j) {
-    const float sc = __shfl_sync(0xffffffffu, scj, j);
-    if (j < n) {
-      const int c = c_lo + j;
-      const int slot = pair * kTopK < unit_begin(U, P.n_cta, c) ? 0 : 1;
-      const float* part = P.ws + (static_cast<size_t>(c) * 2 + slot) * kPartial;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(part + head * kD + lane * 4));
-      acc.x += v.x * sc;
-      acc.y += v.y * sc;
-      acc.z += v.z * sc;
-      acc.w += v.w * sc;
-    }
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  __nv_bfloat16* dst = P.out + (static_cast<size_t>(pair) * kHpg + head) * kD + lane * 4;
-  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-}
-
-__global__ void __launch_bounds__(256) attn_sk_combine_kernel(const Params P) {
-  pdl_trigger();
-  pdl_wait();
-  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (w >= P.n_units / kTopK * kHpg) return;
-  combine_pair_head(P, w, threadIdx.x & 31);
 }
 
 }  // namespace dattn

@@ -4,14 +4,14 @@
 // new token's indexer key and K/V rows, scores the blocks
 // (maxpool_128(idx_q * idx_k^T + causal mask) + local bias), keeps the
 // top-16 per group and attends over the selected blocks.  The same step
-// runs here as five phases of one cooperative launch (one CTA per SM, all
+// runs here as four phases of one cooperative launch (one CTA per SM, all
 // resident), separated by grid-wide barriers instead of kernel boundaries:
 //
 //   1. append      one warp per (token, group) row, grid-stride
 //   2. scores      the streaming block-score body (F32 keys), every CTA
 //   3. select      one warp per (query, group), grid-stride
-//   4. attention   the stream-K decode body over (pair, block) units
-//   5. combine     one warp per (pair, head) cut between CTAs, grid-stride
+//   4. attention   the stream-K decode body over (pair, block) units, pairs
+//                  cut between CTAs merged by the CTA holding their first unit
 //
 // Each phase computes exactly what its standalone kernel computes, with the
 // same launch shape where it matters (the score body's task split and the
@@ -51,7 +51,7 @@ struct Params {
   const int32_t* tok_stream;
   const int32_t* tok_pos;
   int n_tok;
-  // phases 2-5
+  // phases 2-4
   gemv::Params<ScoreKey> scores;     // writes block_scores
   int32_t* sel;
   int32_t* n_sel;
@@ -172,12 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
 
   // ---- 4. attention over the selected blocks -------------------------------
+  // (pairs cut between CTAs are merged inside the attention body)
   if (cta < F.attn.n_cta) dattn::sparse_attn_decode_sk_body<false, false>(&tm_k, &tm_v, &tm_q, F.attn, smem, cta);
-  if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
-
-  // ---- 5. merge the partials of pairs cut between CTAs ----------------------
-  for (long long w = gwarp; w < static_cast<long long>(n_pairs) * dattn::kHpg; w += n_gwarps)
-    dattn::combine_pair_head(F.attn, w, lane);
 }
 
 // The library's bounded waits driven to their limit: every CTA of a

@@ -192,9 +192,20 @@ MSA_API int msa_select_topk(const msa_shape* shape, const float* block_scores, c
  * token-level causal mask applies inside the local block).  Softmax and
  * accumulation in float32, output rounded to bf16 (nearest even).  A query
  * with no attended row writes zeros.  A persistent grid splits the (pair,
- * selected block) units evenly over the SMs; `workspace` holds the partial
- * results of pairs cut between two CTAs (at most 2 per CTA, 256 CTAs) and
- * must be at least msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE) bytes. */
+ * selected block) units evenly over the SMs, in one launch: a pair cut
+ * between CTAs is merged by the CTA holding its first unit from the partial
+ * results the later CTAs publish.  `workspace` (at least
+ * msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE) bytes, 16-byte aligned)
+ * holds, in its first 4096 bytes, the merge bookkeeping of 256 CTA slots
+ * (per slot: a 64-bit publication flag and a 32-bit epoch that the merging
+ * CTA raises), then one partial result per CTA (16 x 130 floats).  The
+ * bookkeeping carries over from call to call and needs no initial value: a
+ * merger waits for a flag equal to a tag, its own index and its epoch + 1,
+ * which no earlier call (and, short of that exact 64-bit pattern, no other
+ * contents of a reused buffer) leaves behind.  Calls that may run at the
+ * same time on the GPU need separate workspaces.  A merge whose partial
+ * never appears gives up after the library's bounded wait and sets
+ * MSA_DEVERR_TIMEOUT. */
 MSA_API int msa_sparse_attn_decode(const msa_shape* shape, const msa_bf16* q, const msa_bf16* k_cache,
                            const msa_bf16* v_cache, const int32_t* sel, const int32_t* q_stream,
                            const int32_t* q_pos, int32_t n_q, float softmax_scale, msa_bf16* out,
@@ -243,12 +254,12 @@ MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, c
  * start-up, or a program driving the C ABI from a language that has no CUDA
  * allocator of its own.  Such a caller still owns q, the caches, sel and out.
  *
- * The partial results go to one file-scope device buffer of
- * MSA_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
- * the process exits.  A call whose msa_workspace_bytes(shape, n_q,
- * MSA_MODE_DECODE) exceeded that size would be rejected with
- * MSA_ERR_WORKSPACE; the decode partials need at most 256 CTAs x 2 x 8320
- * bytes = 4,259,840 bytes, so every batch fits.  The first call on each
+ * The workspace (merge bookkeeping and partial results) is one file-scope
+ * device buffer of MSA_NOALLOC_SCRATCH_BYTES that every GPU loading this
+ * library holds until the process exits.  A call whose
+ * msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE) exceeded that size would
+ * be rejected with MSA_ERR_WORKSPACE; decode needs at most 4096 + 256 CTAs x
+ * 8320 bytes = 2,134,016 bytes, so every batch fits.  The first call on each
  * device looks up the buffer's device address (with that device current);
  * make that first call before any stream capture.  The address is looked up
  * again when the device's current context is not the one it was found in
@@ -258,8 +269,8 @@ MSA_API int msa_sparse_attn_prefill(const msa_shape* shape, const msa_bf16* q, c
  * buffer: calls that can run at the same time on the GPU (different streams,
  * or different host threads on one device) race and must be serialised by
  * the caller.  Nothing in the buffer needs to start at zero: every call
- * writes each partial it reads.  Allocates nothing, on the host or the
- * device. */
+ * writes each partial it reads, and the bookkeeping needs no initial value.
+ * Allocates nothing, on the host or the device. */
 MSA_API int msa_sparse_attn_decode_noalloc(const msa_shape* shape, const msa_bf16* q,
                                            const msa_bf16* k_cache, const msa_bf16* v_cache,
                                            const int32_t* sel, const int32_t* q_stream,
@@ -415,7 +426,7 @@ MSA_API int msa_dsa_sparse_attn_decode(const msa_shape* shape, const msa_pages* 
  * than 256 queries, or fewer than 64 per stream on average; otherwise
  * MSA_ERR_SHAPE).  n_sel may be NULL.  workspace: at least
  * msa_decode_step_fused_workspace_bytes(shape, n_q) bytes, 256-byte aligned
- * (partials of pairs cut between CTAs, and the barrier words, which the call
+ * (the attention's merge bookkeeping and partials, and the barrier words, which the call
  * zeroes on `stream` before the launch).  A barrier wait that gives up sets
  * MSA_DEVERR_TIMEOUT and leaves the outputs incomplete.  n_q == 0 only
  * appends. */

@@ -109,11 +109,12 @@ def test_select_and_append_validation(lib):
 
 def test_attention_validation_and_workspace(lib):
     s = GOOD.c()
-    # decode: 2 partials (16 heads x (128 + 2) floats) per CTA, one CTA per
-    # (pair, block) unit at most, 256 CTAs at most
+    # decode: the merge bookkeeping of 256 CTA slots (16 bytes each), then one
+    # partial (16 heads x (128 + 2) floats) per CTA, one CTA per (pair,
+    # block) unit at most, 256 CTAs at most
     need = lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_DECODE)
-    assert need == min(2 * 4 * 16, 256) * 2 * 16 * 130 * 4
-    assert lib.msa_workspace_bytes(ctypes.byref(s), 1000, msa.MODE_DECODE) >= 256 * 2 * 16 * 130 * 4
+    assert need == 256 * 16 + min(2 * 4 * 16, 256) * 16 * 130 * 4
+    assert lib.msa_workspace_bytes(ctypes.byref(s), 1000, msa.MODE_DECODE) >= 256 * 16 + 256 * 16 * 130 * 4
     # prefill attention: the plan of every 8-query tile (844 bytes) per group
     plans = lambda n_q, G=4: G * ((n_q + 7) // 8) * 844          # noqa: E731
     assert lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_PREFILL) == plans(2)
@@ -125,7 +126,7 @@ def test_attention_validation_and_workspace(lib):
     # 600 decode queries over 600 streams keep the streaming score kernel (no
     # score workspace): only the attention partials remain
     many = msa.Shape(n_streams=600, capacity=1024).c()
-    assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_DECODE) == 256 * 2 * 16 * 130 * 4
+    assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_DECODE) == 256 * 16 + 256 * 16 * 130 * 4
     assert lib.msa_workspace_bytes(ctypes.byref(many), 600, msa.MODE_PREFILL) == plans(600)
     bad = msa.Shape(n_streams=2, capacity=1000).c()
     assert lib.msa_workspace_bytes(ctypes.byref(bad), 2, 0) == ctypes.c_size_t(-1).value

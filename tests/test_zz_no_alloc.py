@@ -21,12 +21,12 @@ from tests import parity as PT
 
 
 def test_noalloc_buffer_covers_every_batch_and_checks_shapes():
-    """Host-side checks (no GPU needed): the decode partials of any batch fit
-    the fixed buffer (at most 256 CTAs x 2 partials), and bad arguments are
-    rejected before any device work."""
+    """Host-side checks (no GPU needed): the decode workspace of any batch
+    (merge bookkeeping and at most 256 CTAs x 1 partial) fits the fixed
+    buffer, and bad arguments are rejected before any device work."""
     msa_build.build()
     lib = msa.library()
-    # many streams: decode-shaped batches, so the query measures the attention partials only
+    # many streams: decode-shaped batches, so the query measures the attention workspace only
     many = msa.Shape(n_streams=20000, capacity=128).c()
     for n_q in (1, 3, 127, 128, 4096, 1 << 20):
         assert 0 < lib.msa_workspace_bytes(ctypes.byref(many), n_q, msa.MODE_DECODE) <= msa.NOALLOC_SCRATCH_BYTES
