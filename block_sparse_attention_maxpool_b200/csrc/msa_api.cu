@@ -991,10 +991,13 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   A.tok_sel = nullptr;
   A.k_cache = reinterpret_cast<const __nv_bfloat16*>(k_cache);
   A.v_cache = reinterpret_cast<const __nv_bfloat16*>(v_cache);
-  A.bs = nullptr;
+  // the top-16 inside the attention phase when every CTA's share touches at
+  // most kSelPairs pairs (no barrier between ranking and attention)
+  const bool fuse_sel = max_pairs_per_cta(A.n_units, A.n_cta) <= msa::dattn::kSelPairs;
+  A.bs = fuse_sel ? block_scores : nullptr;
   A.nblk = S.nblk;
-  A.sel_out = nullptr;
-  A.n_sel_out = nullptr;
+  A.sel_out = fuse_sel ? sel : nullptr;
+  A.n_sel_out = fuse_sel ? n_sel : nullptr;
   unsigned int* bar = reinterpret_cast<unsigned int*>(
       static_cast<uint8_t*>(workspace) + msa::tc::align256(attn_workspace(shape, n_q, MSA_MODE_DECODE)));
   F.bar_count = bar;

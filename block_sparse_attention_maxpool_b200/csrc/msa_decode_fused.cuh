@@ -4,12 +4,15 @@
 // new token's indexer key and K/V rows, scores the blocks
 // (maxpool_128(idx_q * idx_k^T + causal mask) + local bias), keeps the
 // top-16 per group and attends over the selected blocks.  The same step
-// runs here as four phases of one cooperative launch (one CTA per SM, all
+// runs here as three or four phases of one cooperative launch (one CTA per SM, all
 // resident), separated by grid-wide barriers instead of kernel boundaries:
 //
 //   1. append      one warp per (token, group) row, grid-stride
 //   2. scores      the streaming block-score body (F32 keys), every CTA
-//   3. select      one warp per (query, group), grid-stride
+//   3. select      each attention CTA ranks the pairs its units touch, at
+//                  the start of phase 4 (no barrier); for batches whose
+//                  CTA shares touch more than 8 pairs, one warp per
+//                  (query, group), grid-stride, then a barrier
 //   4. attention   the stream-K decode body over (pair, block) units, pairs
 //                  cut between CTAs merged by the CTA holding their first unit
 //
@@ -162,7 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) gemv::block_scores_gemv_release<ScoreKey, kScoreStages, kScoreWarps>(smem);
   if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
 
-  // ---- 3. top-16 per (query, group) ----------------------------------------
+  // ---- 3 + 4. top-16 and attention over the selected blocks ---------------
+  // (pairs cut between CTAs are merged inside the attention body)
+  if (F.attn.bs != nullptr) {
+    // every CTA ranks the pairs its units touch, as the attention kernel
+    // of msa_select_attn_decode does: no grid barrier between the two
+    if (cta < F.attn.n_cta) dattn::sparse_attn_decode_sk_body<false, true>(&tm_k, &tm_v, &tm_q, F.attn, smem, cta);
+    return;
+  }
   const int n_pairs = F.scores.n_q * G;
   uint64_t* wsm = reinterpret_cast<uint64_t*>(smem + warp * sel::select_smem_per_warp(F.scores.nblk));
   for (long long w = gwarp; w < n_pairs; w += n_gwarps)
@@ -170,9 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                          F.sel + static_cast<size_t>(w) * sel::kTopK, F.n_sel != nullptr ? F.n_sel + w : nullptr,
                          static_cast<int>(w), lane, wsm);
   if (!grid_barrier(F, n_cta, gen, &barrier_flag, false)) return;
-
-  // ---- 4. attention over the selected blocks -------------------------------
-  // (pairs cut between CTAs are merged inside the attention body)
   if (cta < F.attn.n_cta) dattn::sparse_attn_decode_sk_body<false, false>(&tm_k, &tm_v, &tm_q, F.attn, smem, cta);
 }
 
