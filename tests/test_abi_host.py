@@ -143,6 +143,30 @@ def test_attention_validation_and_workspace(lib):
     assert lib.msa_sparse_attn_prefill(ctypes.byref(s), *args[:6], 0, args[7], FAKE, 0, 0, None) == 0
 
 
+def test_select_attn_validation(lib):
+    """msa_select_attn_decode checks its block scores and selection buffer on
+    top of the decode attention's arguments, before any device work."""
+    s = GOOD.c()
+    need = lib.msa_workspace_bytes(ctypes.byref(s), 2, msa.MODE_DECODE)
+    scale = ctypes.c_float(0.088)
+
+    def call(bs=FAKE, q=FAKE, sel=FAKE, n_q=2, scale=scale, ws=FAKE, ws_bytes=need):
+        return lib.msa_select_attn_decode(ctypes.byref(s), bs, q, FAKE, FAKE, FAKE, FAKE, n_q, scale, sel, 0,
+                                          FAKE, ws, ws_bytes, None)
+    assert call(bs=0) == -1
+    assert call(sel=0) == -1
+    assert call(q=0) == -1
+    assert call(bs=FAKE + 4) == -2
+    assert call(sel=FAKE + 8) == -2
+    assert call(ws_bytes=need - 1) == -5
+    assert call(ws=0) == -5
+    assert call(scale=ctypes.c_float(float("nan"))) == -4
+    assert call(n_q=-1) == -4
+    assert call(bs=0, sel=0, n_q=0) == 0
+    assert lib.msa_select_attn_decode_paged(ctypes.byref(s), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, scale,
+                                            FAKE, 0, FAKE, FAKE, need, None) == -1
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     sh = msa.Shape(n_streams=1, capacity=128)
