@@ -68,7 +68,7 @@ SCORES_TRAFFIC = {"f32": {"source_sha": "fbcb00edc6a2593a", "bytes_per_launch": 
 # The same for the token-score kernel of the token-level variant, from a
 # capture of the 16-stream case, scaled by 2 to 32 streams (sha256 prefix
 # of msa_dsa_scores.cuh).
-DSA_SCORES_TRAFFIC = {"source_sha": "6c6fa9e892144930", "bytes_per_launch": 2 * (134_557_696 + 5_160_960)}
+DSA_SCORES_TRAFFIC = {"source_sha": "1f3f0fc92a3f7ca2", "bytes_per_launch": 2 * (134_548_480 + 3_636_992)}
 
 
 def variant_metric(metric: str, args) -> str:
