@@ -171,6 +171,25 @@ size_t attn_workspace(const msa_shape* sh, int32_t n_q, int mode) {
   return msa::dattn::kSyncBytes + static_cast<size_t>(ctas) * msa::dattn::kPartial * sizeof(float);
 }
 
+// CTAs of the decode attention grid.  The even split (one CTA per SM, equal
+// shares) cuts pairs at arbitrary units, and a pair's merger then waits for
+// CTAs that hold a different amount of that pair.  When the pairs fit, k
+// CTAs per pair (k dividing 16, as many as the SMs allow) gives shares that
+// line up with pair boundaries: the CTAs of a pair finish together, and
+// with k = 1 nothing is merged.  Measured on 148 SMs: 128 pairs, 128 CTAs
+// instead of 148: 4 us less per step; 32 pairs, 128 instead of 148: 2 us.
+// It is taken unless its shares are more than two units longer.
+int decode_attn_ctas(int64_t n_pairs, int sms) {
+  const int64_t units = n_pairs * msa::dattn::kTopK;
+  const int64_t cap = std::min<int64_t>(sms, msa::dattn::kMaxCtas);
+  const int64_t even = std::min<int64_t>(cap, units);
+  const int64_t even_units = (units + even - 1) / even;
+  for (int k = msa::dattn::kTopK; k >= 1; k /= 2) {
+    if (n_pairs * k <= cap) return static_cast<int>(msa::dattn::kTopK / k <= even_units + 2 ? n_pairs * k : even);
+  }
+  return static_cast<int>(even);
+}
+
 // Most pairs one CTA's share of the decode units touches.
 int64_t max_pairs_per_cta(int64_t units, int n_cta) {
   int64_t most = 0;
@@ -258,8 +277,7 @@ int sparse_attn(const msa_shape* sh, const msa_bf16* q, const msa_bf16* k_cache,
                            msa::dattn::kHpg)) != MSA_OK)
     return st;
   const int64_t n_units = n_pairs * msa::dattn::kTopK;
-  const int n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), n_units,
-                                                        static_cast<int64_t>(msa::dattn::kMaxCtas)}));
+  const int n_cta = decode_attn_ctas(n_pairs, sms);
   bool fuse_sel = false;
   if (block_scores != nullptr) {
     fuse_sel = max_pairs_per_cta(n_units, n_cta) <= msa::dattn::kSelPairs;
@@ -984,8 +1002,7 @@ int msa_decode_step_fused(const msa_shape* shape, float* idx_k_cache, msa_bf16* 
   A.n_streams = shape->n_streams;
   A.capacity = shape->capacity;
   A.n_units = n_pairs * msa::dattn::kTopK;
-  A.n_cta = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(grid), A.n_units,
-                                                static_cast<int64_t>(msa::dattn::kMaxCtas)}));
+  A.n_cta = decode_attn_ctas(n_pairs, grid);                 // the separate calls' split
   A.scale_log2 = softmax_scale * 1.4426950408889634f;
   A.pages = msa::KvPages{nullptr, 0};
   A.tok_sel = nullptr;
