@@ -191,10 +191,12 @@ MSA_API int msa_select_topk(const msa_shape* shape, const float* block_scores, c
  * section "Overview": attention runs only over the selected blocks; the
  * token-level causal mask applies inside the local block).  Softmax and
  * accumulation in float32, output rounded to bf16 (nearest even).  A query
- * with no attended row writes zeros.  A persistent grid splits the (pair,
- * selected block) units evenly over the SMs, in one launch: a pair cut
- * between CTAs is merged by the CTA holding its first unit from the partial
- * results the later CTAs publish.  `workspace` (at least
+ * with no attended row writes zeros.  A persistent grid of at most one CTA
+ * per SM splits the (pair, selected block) units into equal contiguous
+ * shares, in one launch (when the pairs fit, k CTAs per pair, so that the
+ * shares line up with the pairs); a pair cut between CTAs is merged by the
+ * CTA holding its first unit from the partial results the later CTAs
+ * publish.  `workspace` (at least
  * msa_workspace_bytes(shape, n_q, MSA_MODE_DECODE) bytes, 16-byte aligned)
  * holds, in its first 4096 bytes, the merge bookkeeping of 256 CTA slots
  * (per slot: a 64-bit publication flag and a 32-bit epoch that the merging
